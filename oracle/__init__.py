@@ -1,0 +1,205 @@
+"""fp64 CPU oracle for exact attention: TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product library never loads it and
+shares no code with it: the only thing both sides share are the seeded
+input generators, which hold no attention arithmetic.
+
+Contents
+--------
+``attn_oracle.c``  the plain definition in C (fp64, OpenMP): one full row of
+                   scores per query, two-pass safe softmax, P.V, L = m + ln l,
+                   and the exact analytic backward. Built by :func:`build`.
+``numpy_ref.py``   an independent whole-matrix numpy version for tiny shapes.
+``online.py``      the tiled online-softmax forward written from the pages'
+                   step list, used only to pin "online == two-pass".
+
+Every function here works on float64 numpy arrays in the layouts documented
+in ``attn_oracle.c`` (q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d], lse [B,Hq,Nq]).
+Parity of every function is pinned by ``tests/test_oracle.py`` against
+closed forms, invariants, brute force and finite differences.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import time
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "liboracle.so")
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int)
+_up = ctypes.POINTER(ctypes.c_ubyte)
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle (plain gcc, -O2, OpenMP) into oracle/_build."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", _SRC,
+                               "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.ora_attn_fwd.restype = ctypes.c_int
+        lib.ora_attn_fwd.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
+                                                                            _up, _ip, ctypes.c_int, _dp, _dp]
+        lib.ora_attn_probs.restype = ctypes.c_int
+        lib.ora_attn_probs.argtypes = [_dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
+                                                                         _up, ctypes.c_int, ctypes.c_int, _dp]
+        lib.ora_attn_bwd.restype = ctypes.c_int
+        lib.ora_attn_bwd.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
+                                                                                 _up, _dp, _dp, _dp]
+        lib.ora_attn_bwd_sampled.restype = ctypes.c_int
+        lib.ora_attn_bwd_sampled.argtypes = ([_dp, _dp, _dp, _dp] + [ctypes.c_int] * 6 +
+                                             [ctypes.c_double, ctypes.c_int, _up, ctypes.c_int, ctypes.c_int,
+                                              _ip, ctypes.c_int, _ip, ctypes.c_int, _dp, _dp, _dp])
+        lib.ora_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().ora_num_threads())
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast of a bf16/fp16/fp32 tensor or array to contiguous float64."""
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().to("cpu").to(torch.float64).numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a: np.ndarray, t=_dp):
+    return a.ctypes.data_as(t)
+
+
+def _mask_ptr(key_keep, B, Nk):
+    if key_keep is None:
+        return None, None
+    kk = np.ascontiguousarray(np.asarray(key_keep, dtype=np.uint8).reshape(B, Nk))
+    return kk, _ptr(kk, _up)
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool = False, key_keep=None, rows=None):
+    """O [B,Nq,Hq,d] and L [B,Hq,Nq] in fp64 by the plain definition.
+
+    ``rows`` (sequence of query indices) restricts the work to those rows;
+    the other entries of the returned arrays are NaN.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    o = np.full((B, Nq, Hq, d), np.nan)
+    lse = np.full((B, Hq, Nq), np.nan)
+    kk, kp = _mask_ptr(key_keep, B, Nk)
+    if rows is not None:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        assert r.size == 0 or (r.min() >= 0 and r.max() < Nq)
+        rp, nr = _ptr(r, _ip), int(r.size)
+    else:
+        r, rp, nr = None, None, 0
+    if B * Hq * (nr if rows is not None else Nq) > 0:
+        err = _load().ora_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                   int(bool(causal)), kp, rp, nr, _ptr(o), _ptr(lse))
+        if err:
+            raise RuntimeError(f"ora_attn_fwd failed with code {err}")
+    return o, lse
+
+
+def attn_probs(q, k, scale: float, b: int, h: int, causal: bool = False, key_keep=None):
+    """The Nq x Nk probability matrix of one (batch, query head)."""
+    q, k = _f64(q), _f64(k)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    P = np.zeros((Nq, Nk))
+    kk, kp = _mask_ptr(key_keep, B, Nk)
+    err = _load().ora_attn_probs(_ptr(q), _ptr(k), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                 int(bool(causal)), kp, b, h, _ptr(P))
+    if err:
+        raise RuntimeError(f"ora_attn_probs failed with code {err}")
+    return P
+
+
+def attn_bwd(q, k, v, do, scale: float, causal: bool = False, key_keep=None):
+    """dQ, dK, dV in fp64 by the exact gradient of the definition."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    kk, kp = _mask_ptr(key_keep, B, Nk)
+    err = _load().ora_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, Hq, Hkv, Nq, Nk, d,
+                               float(scale), int(bool(causal)), kp, _ptr(dq), _ptr(dk), _ptr(dv))
+    if err:
+        raise RuntimeError(f"ora_attn_bwd failed with code {err}")
+    return dq, dk, dv
+
+
+def attn_bwd_sampled(q, k, v, do, scale: float, b: int, hk: int, qrows, krows,
+                     causal: bool = False, key_keep=None):
+    """Gradients of sampled rows of one (batch, KV head) group.
+
+    Returns (dq_rows [len(qrows), group, d], dk_rows [len(krows), d],
+    dv_rows [len(krows), d]) where group = Hq/Hkv query heads hk*group...
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    group = Hq // Hkv
+    qr = np.ascontiguousarray(np.asarray(qrows, dtype=np.int32))
+    kr = np.ascontiguousarray(np.asarray(krows, dtype=np.int32))
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    kk, kp = _mask_ptr(key_keep, B, Nk)
+    err = _load().ora_attn_bwd_sampled(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, Hq, Hkv, Nq, Nk, d,
+                                       float(scale), int(bool(causal)), kp, b, hk, _ptr(qr, _ip),
+                                       int(qr.size), _ptr(kr, _ip), int(kr.size), _ptr(dq), _ptr(dk),
+                                       _ptr(dv))
+    if err:
+        raise RuntimeError(f"ora_attn_bwd_sampled failed with code {err}")
+    return (dq[b][qr][:, hk * group:(hk + 1) * group, :], dk[b, kr, hk, :], dv[b, kr, hk, :])
+
+
+def varlen_fwd(q, k, v, cu_q, cu_k, scale: float, causal: bool = False):
+    """Packed variable-length forward: each sequence is an independent B=1 problem.
+
+    q [total_q,Hq,d], k/v [total_k,Hkv,d]; returns O [total_q,Hq,d] and
+    L [Hq,total_q]. This follows the cu_seqlens addressing of the packed path
+    on the InternViT page: sequence s owns rows cu[s] .. cu[s+1]-1.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu_q = [int(x) for x in np.asarray(cu_q)]
+    cu_k = [int(x) for x in np.asarray(cu_k)]
+    T, Hq, d = q.shape
+    o = np.zeros((T, Hq, d))
+    lse = np.zeros((Hq, T))
+    for s in range(len(cu_q) - 1):
+        a, e = cu_q[s], cu_q[s + 1]
+        ka, ke = cu_k[s], cu_k[s + 1]
+        if e == a:
+            continue
+        os_, ls = attn_fwd(q[None, a:e], k[None, ka:ke], v[None, ka:ke], scale, causal)
+        o[a:e] = os_[0]
+        lse[:, a:e] = ls[0]
+    return o, lse
+
+
+def timed(fn, *args, **kw):
+    """(result, seconds) of one call."""
+    t0 = time.perf_counter()
+    r = fn(*args, **kw)
+    return r, time.perf_counter() - t0
