@@ -1,0 +1,179 @@
+"""Thin ctypes binding of libfa.so.
+
+The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_bwd_workspace_size``,
+``fa_bwd``, ``fa_status_string`` and ``fa_get_last_device_error`` have the
+names, argument order and meaning of the C ABI in ``include/fa.h``: pointers
+are passed as integers (device addresses), streams as integers (0 = default
+stream), and the return value is the ``fa_status`` code. They only marshal
+arguments; every step of the computation runs in the library's kernels.
+
+``attention_fwd``, ``attention_varlen_fwd`` and ``attention_bwd`` are the
+same calls on torch CUDA tensors: torch allocates the outputs and workspace,
+the library fills them. There is no fallback: if ``libfa.so`` is missing or
+a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
+FA_BF16, FA_FP16 = 0, 1
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+
+_SIGS = {
+    "fa_fwd": ([_P, _P, _P, _P, _P] + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_varlen_fwd": ([_P, _P, _P, _P, _P, _P, _P] + [_I] * 8 + [_F, _I, _I, _P], _I),
+    "fa_bwd_workspace_size": ([_I] * 4, ctypes.c_size_t),
+    "fa_bwd": ([_P] * 10 + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_status_string": ([_I], ctypes.c_char_p),
+    "fa_get_last_device_error": ([_P], _I),
+    "fa_get_last_device_error_site": ([], _I),
+    "fa_version": ([], ctypes.c_char_p),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {fa_status_string(status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m exact_tiled_attention_36_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(l, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = l
+    return _lib
+
+
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream)
+
+
+def fa_varlen_fwd(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream) -> int:
+    return lib().fa_varlen_fwd(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q, total_k,
+                               max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream)
+
+
+def fa_bwd_workspace_size(B, Hq, Nq, d) -> int:
+    return int(lib().fa_bwd_workspace_size(B, Hq, Nq, d))
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype,
+           stream) -> int:
+    return lib().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                        dtype, stream)
+
+
+def fa_status_string(s: int) -> str:
+    return lib().fa_status_string(s).decode()
+
+
+def fa_get_last_device_error(stream) -> int:
+    return lib().fa_get_last_device_error(stream)
+
+
+def fa_get_last_device_error_site() -> int:
+    return lib().fa_get_last_device_error_site()
+
+
+def fa_version() -> str:
+    return lib().fa_version().decode()
+
+
+# ----------------------------------------------------------------------------- torch tensors
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise TypeError(f"q/k/v must be bfloat16 or float16, got {t.dtype}")
+
+
+def _dev(t):
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    return t.contiguous()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int, what: str):
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+def attention_fwd(q, k, v, scale: float | None = None, causal: bool = False, out=None, lse=None, stream=None):
+    """O, L = attention(q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]); L is float32 [B,Hq,Nq]."""
+    import torch
+    q, k, v = _dev(q), _dev(k), _dev(v)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty_like(q) if out is None else out
+    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                  float(scale), int(bool(causal)), _dtype_code(q), _stream(stream)), "fa_fwd")
+    return o, L
+
+
+def attention_varlen_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                         scale: float | None = None, causal: bool = False, out=None, lse=None, stream=None):
+    """Packed varlen forward: q [total_q,Hq,d], k/v [total_k,Hkv,d]; L is float32 [Hq,total_q]."""
+    import torch
+    q, k, v = _dev(q), _dev(k), _dev(v)
+    cu_q = _dev(cu_seqlens_q).to(torch.int32)
+    cu_k = _dev(cu_seqlens_k).to(torch.int32)
+    Tq, Hq, d = q.shape
+    Tk, Hkv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty_like(q) if out is None else out
+    L = torch.empty((Hq, Tq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(fa_varlen_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), cu_q.data_ptr(),
+                         cu_k.data_ptr(), cu_q.numel() - 1, Tq, Tk, int(max_seqlen_q), int(max_seqlen_k), Hq, Hkv,
+                         d, float(scale), int(bool(causal)), _dtype_code(q), _stream(stream)), "fa_varlen_fwd")
+    return o, L
+
+
+def attention_bwd(q, k, v, o, lse, dout, scale: float | None = None, causal: bool = False, workspace=None,
+                  stream=None):
+    """dQ, dK, dV of the fixed-length forward (same layouts as q, k, v)."""
+    import torch
+    q, k, v, o, dout = _dev(q), _dev(k), _dev(v), _dev(o), _dev(dout)
+    lse = _dev(lse)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    ws_bytes = fa_bwd_workspace_size(B, Hq, Nq, d)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    _check(fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                  dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                  int(bool(causal)), _dtype_code(q), _stream(stream)), "fa_bwd")
+    return dq, dk, dv

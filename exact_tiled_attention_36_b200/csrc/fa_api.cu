@@ -1,0 +1,311 @@
+// fa_api.cu: the C ABI of libfa.so (declared in include/fa.h).
+//
+// Host side only: argument validation, TMA descriptor encoding and kernel
+// launches. Every step of the attention computation runs in the kernels of
+// fa_fwd.cuh and fa_bwd.cuh; nothing here touches tensor data.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd.cuh"
+#include "fa_bwd.cuh"
+
+namespace {
+
+__device__ int g_fa_error = 0;  // first timeout site of any kernel (0 = none)
+int g_last_site = 0;
+
+constexpr float kLog2e = 1.4426950408889634074f;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map of a [batches, rows, H, d] 16-bit tensor, box = 128 rows x 64
+// columns of one head, 128-byte swizzle. Rows past `rows` read as zero.
+fa_status make_map(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16) {
+    auto enc = encode_tiled();
+    if (!enc) return FA_ERR_CUDA;
+    if (rows < 1) rows = 1;
+    if (batches < 1) batches = 1;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batches)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
+                                   static_cast<cuuint64_t>(rows) * H * d * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int* error_word() {
+    static int* ptr = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fa_error) == cudaSuccess) ptr = static_cast<int*>(p);
+    });
+    return ptr;
+}
+
+fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype) {
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (Hq > 65535) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+template <int D, bool BF16, bool CAUSAL, bool VARLEN>
+fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
+                       dim3 grid, cudaStream_t stream) {
+    auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, VARLEN>;
+    constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
+    static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+    if (!attr_ok) return FA_ERR_CUDA;
+    kern<<<grid, 256, smem, stream>>>(mq, mk, mv, a);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_fwd_d(bool bf16, bool causal, bool varlen, const CUtensorMap& mq, const CUtensorMap& mk,
+                       const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
+    if (bf16) {
+        if (causal) return varlen ? launch_fwd_t<D, true, true, true>(mq, mk, mv, a, grid, s)
+                                  : launch_fwd_t<D, true, true, false>(mq, mk, mv, a, grid, s);
+        return varlen ? launch_fwd_t<D, true, false, true>(mq, mk, mv, a, grid, s)
+                      : launch_fwd_t<D, true, false, false>(mq, mk, mv, a, grid, s);
+    }
+    if (causal) return varlen ? launch_fwd_t<D, false, true, true>(mq, mk, mv, a, grid, s)
+                              : launch_fwd_t<D, false, true, false>(mq, mk, mv, a, grid, s);
+    return varlen ? launch_fwd_t<D, false, false, true>(mq, mk, mv, a, grid, s)
+                  : launch_fwd_t<D, false, false, false>(mq, mk, mv, a, grid, s);
+}
+
+fa_status launch_fwd(int d, bool bf16, bool causal, bool varlen, const CUtensorMap& mq, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
+    return d == 64 ? launch_fwd_d<64>(bf16, causal, varlen, mq, mk, mv, a, grid, s)
+                   : launch_fwd_d<128>(bf16, causal, varlen, mq, mk, mv, a, grid, s);
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <int D, bool BF16, bool CAUSAL>
+fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                       const fa::BwdArgs& a, dim3 grid, cudaStream_t stream) {
+    auto kern = fa::fa_bwd_kernel<D, BF16, CAUSAL>;
+    constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
+    static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+    if (!attr_ok) return FA_ERR_CUDA;
+    kern<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, a);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_bwd_d(bool bf16, bool causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& mdo, const fa::BwdArgs& a, dim3 grid, cudaStream_t s) {
+    if (bf16) return causal ? launch_bwd_t<D, true, true>(mq, mk, mv, mdo, a, grid, s)
+                            : launch_bwd_t<D, true, false>(mq, mk, mv, mdo, a, grid, s);
+    return causal ? launch_bwd_t<D, false, true>(mq, mk, mv, mdo, a, grid, s)
+                  : launch_bwd_t<D, false, false>(mq, mk, mv, mdo, a, grid, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_version(void) { return "0.1.0"; }
+
+const char* fa_status_string(fa_status s) {
+    switch (s) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dim, dtype or size";
+        case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: tensor pointer not 16-byte aligned";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call failed";
+        case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a bounded device wait ran out";
+    }
+    return "unknown fa_status";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                 int Nq, int Nk, int d, float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
+    if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    if ((Nq > 0 && (!q || !o || !lse)) || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+    fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_MISALIGNED;
+    if (B > 65535) return FA_ERR_UNSUPPORTED;
+    if (Nq == 0) return FA_OK;
+    int* err = error_word();
+    if (!err) return FA_ERR_CUDA;
+    const bool bf16 = dtype == FA_BF16;
+    CUtensorMap mq, mk{}, mv{};  // K/V maps stay unused (zero) when there is no key
+    if ((st = make_map(&mq, q, d, Hq, Nq, B, bf16)) != FA_OK) return st;
+    if (Nk > 0 && (st = make_map(&mk, k, d, Hkv, Nk, B, bf16)) != FA_OK) return st;
+    if (Nk > 0 && (st = make_map(&mv, v, d, Hkv, Nk, B, bf16)) != FA_OK) return st;
+    fa::FwdArgs a{};
+    a.o = o;
+    a.lse = lse;
+    a.num_batches = B;
+    a.Hq = Hq;
+    a.group = Hq / Hkv;
+    a.Nq = Nq;
+    a.Nk = Nk;
+    a.scale_log2 = scale * kLog2e;
+    a.err = err;
+    dim3 grid((Nq + 127) / 128, Hq, B);
+    return launch_fwd(d, bf16, causal != 0, false, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
+                        int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
+                        fa_stream_t stream) {
+    if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+        return FA_ERR_INVALID_ARG;
+    if (!cu_seqlens_q || !cu_seqlens_k || (total_q > 0 && (!q || !o || !lse)) || (total_k > 0 && (!k || !v)))
+        return FA_ERR_INVALID_ARG;
+    fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+        return FA_ERR_MISALIGNED;
+    if (num_seqs > 65535) return FA_ERR_UNSUPPORTED;
+    if (max_seqlen_q == 0 || total_q == 0) return FA_OK;
+    int* err = error_word();
+    if (!err) return FA_ERR_CUDA;
+    const bool bf16 = dtype == FA_BF16;
+    // The maps span exactly the caller's buffers: a tile that runs past the
+    // last packed row reads zeros instead of memory beyond the allocation.
+    CUtensorMap mq, mk{}, mv{};
+    if ((st = make_map(&mq, q, d, Hq, total_q, 1, bf16)) != FA_OK) return st;
+    if (total_k > 0 && (st = make_map(&mk, k, d, Hkv, total_k, 1, bf16)) != FA_OK) return st;
+    if (total_k > 0 && (st = make_map(&mv, v, d, Hkv, total_k, 1, bf16)) != FA_OK) return st;
+    fa::FwdArgs a{};
+    a.o = o;
+    a.lse = lse;
+    a.cu_q = cu_seqlens_q;
+    a.cu_k = cu_seqlens_k;
+    a.num_batches = num_seqs;
+    a.total_q = total_q;
+    a.Hq = Hq;
+    a.group = Hq / Hkv;
+    a.Nq = max_seqlen_q;
+    a.Nk = max_seqlen_k;
+    a.scale_log2 = scale * kLog2e;
+    a.err = err;
+    dim3 grid((max_seqlen_q + 127) / 128, Hq, num_seqs);
+    return launch_fwd(d, bf16, causal != 0, true, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {
+    if (B < 1 || Hq < 1 || Nq < 0 || (d != 64 && d != 128)) return 0;
+    const size_t rows = static_cast<size_t>(B) * Hq * Nq;
+    return round256(rows * sizeof(float)) + round256(rows * d * sizeof(float));
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                 float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
+    if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    if ((Nq > 0 && (!q || !o || !lse || !dout || !dq)) || (Nk > 0 && (!k || !v || !dk || !dv)) || !workspace)
+        return FA_ERR_INVALID_ARG;
+    fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return FA_ERR_MISALIGNED;
+    if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+    int* err = error_word();
+    if (!err) return FA_ERR_CUDA;
+    const bool bf16 = dtype == FA_BF16;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t rows = static_cast<size_t>(B) * Nq * Hq;
+    float* Dvec = static_cast<float*>(workspace);
+    float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256(rows * sizeof(float)));
+    if (rows > 0) {
+        const size_t threads = rows * (d / 8);
+        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        if (d == 64)
+            fa::fa_bwd_preprocess<64><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
+                                                             static_cast<const uint16_t*>(dout), Dvec, dq_acc, B, Nq,
+                                                             Hq, bf16);
+        else
+            fa::fa_bwd_preprocess<128><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
+                                                              static_cast<const uint16_t*>(dout), Dvec, dq_acc, B,
+                                                              Nq, Hq, bf16);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    if (Nk > 0) {
+        CUtensorMap mq{}, mdo{}, mk, mv;
+        if (Nq > 0 && (st = make_map(&mq, q, d, Hq, Nq, B, bf16)) != FA_OK) return st;
+        if (Nq > 0 && (st = make_map(&mdo, dout, d, Hq, Nq, B, bf16)) != FA_OK) return st;
+        if ((st = make_map(&mk, k, d, Hkv, Nk, B, bf16)) != FA_OK) return st;
+        if ((st = make_map(&mv, v, d, Hkv, Nk, B, bf16)) != FA_OK) return st;
+        fa::BwdArgs a{};
+        a.lse = lse;
+        a.D = Dvec;
+        a.dq_acc = dq_acc;
+        a.dk = dk;
+        a.dv = dv;
+        a.Hq = Hq;
+        a.Hkv = Hkv;
+        a.group = Hq / Hkv;
+        a.Nq = Nq;
+        a.Nk = Nk;
+        a.scale = scale;
+        a.scale_log2 = scale * kLog2e;
+        a.err = err;
+        dim3 grid((Nk + 127) / 128, Hkv, B);
+        st = d == 64 ? launch_bwd_d<64>(bf16, causal != 0, mq, mk, mv, mdo, a, grid, s)
+                     : launch_bwd_d<128>(bf16, causal != 0, mq, mk, mv, mdo, a, grid, s);
+        if (st != FA_OK) return st;
+    }
+    if (rows > 0) {
+        const size_t n8 = rows * d / 8;
+        fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
+            dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
+fa_status fa_get_last_device_error(fa_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_fa_error, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    if (v == 0) return FA_OK;
+    g_last_site = v;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fa_error, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return (v >= fa::kErrTimeoutBase && v < fa::kErrSmemAlign) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+}
+
+int fa_get_last_device_error_site(void) { return g_last_site; }
+
+}  // extern "C"
+

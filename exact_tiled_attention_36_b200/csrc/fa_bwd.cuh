@@ -1,0 +1,449 @@
+// fa_bwd.cuh: tiled exact attention backward for sm_100a.
+//
+// The backward recomputes S and P from the saved log-sum-exp L and dO, so no
+// N x N matrix is stored ("FlashAttention/zh", section "backward pass and
+// recomputation"). With P = exp(scale Q K^T - L) the kernels compute the exact
+// gradient of the definition:
+//     D_i = sum_c dO_ic O_ic           (equals sum_j P_ij dP_ij)
+//     dP = dO V^T,  dS = P o (dP - D),  dV = P^T dO,
+//     dK = scale dS^T Q,  dQ = scale dS K,
+// and with grouped KV heads dK, dV of a KV head sum over its query heads.
+//
+// Three kernels run in order on the caller's stream:
+//   fa_bwd_preprocess  D = rowsum(dO o O) (fp32) and dQ_acc = 0.
+//   fa_bwd_kernel      one CTA per (128-key tile j, KV head, batch). K_j and V_j
+//                      stay in shared memory; for every query head of the
+//                      group and every 128-query tile i it recomputes
+//                        S^T = K_j Q_i^T and dP^T = V_j dO_i^T   (TMEM, fp32)
+//                      turns them into P^T and dS^T (16-bit, written back over
+//                      the same TMEM columns, dS also to shared memory), then
+//                        dV += P^T dO_i,  dK += dS^T Q_i          (TMEM, fp32)
+//                        dQ_i = dS K_j                             (TMEM, fp32)
+//                      and adds dQ_i into the fp32 accumulator with vector
+//                      reductions. dK, dV leave TMEM once, at the end.
+//   fa_bwd_dq_convert  dQ = dtype(scale * dQ_acc).
+//
+// Warp roles of fa_bwd_kernel (384 threads): warp 0 TMA producer, warp 1 TMEM
+// allocation and the single MMA-issuing thread, warps 2-3 idle, warps 4-11 two
+// compute warpgroups (each owns half of the 128 query columns of S^T / dP^T,
+// half of the dQ columns while draining, and one of dV / dK at the end).
+//
+// TMEM columns: [0,128) S^T, later P^T, later dQ_i; [128,256) dP^T, later dS^T;
+// [256,256+d) dV; [256+d,256+2d) dK.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+struct BwdArgs {
+    const float* lse;  // [B, Hq, Nq]
+    const float* D;    // [B, Hq, Nq]
+    float* dq_acc;     // [B, Nq, Hq, d]
+    void* dk;          // [B, Nk, Hkv, d]
+    void* dv;
+    int Hq, Hkv, group, Nq, Nk;
+    float scale;
+    float scale_log2;
+    int* err;
+};
+
+template <int D>
+struct BwdCfg {
+    static constexpr int kSlabBytes = 128 * 128;
+    static constexpr int kTileBytes = (D / 64) * kSlabBytes;  // 128 rows x d, 16-bit
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kKOff + kTileBytes;
+    static constexpr int kQOff = kVOff + kTileBytes;     // 2 stages
+    static constexpr int kDOOff = kQOff + 2 * kTileBytes;  // 2 stages
+    static constexpr int kDSOff = kDOOff + 2 * kTileBytes;  // dS [128 q x 128 keys], MN-major for the dQ MMA
+    static constexpr int kLDOff = kDSOff + 2 * kSlabBytes;  // 2 stages of L*log2e [128] and D [128], fp32
+    static constexpr int kBarOff = kLDOff + 2048;
+    static constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1 + 1 + 1 + 1 + 2;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 16;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+constexpr int kBwdThreads = 384;
+
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdArgs args) {
+    using C = BwdCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (!smem_base_ok(smem, args.err)) return;  // the 128-byte swizzle needs 1024-byte aligned tiles
+
+    const int kt = blockIdx.x;  // key tile
+    const int hk = blockIdx.y;
+    const int b = blockIdx.z;
+    const int k0 = kt * 128;
+    const int Nq = args.Nq, Nk = args.Nk;
+    const int n_qt = (Nq + 127) / 128;
+    // Causal: query q sees key k iff k <= q + (Nk - Nq). The first query tile
+    // that sees any key of this tile:
+    int i0 = 0;
+    if (CAUSAL) {
+        const int qmin = k0 - (Nk - Nq);
+        i0 = qmin <= 0 ? 0 : qmin / 128;
+    }
+    const int n_i = n_qt > i0 ? n_qt - i0 : 0;
+    const int n_it = args.group * n_i;
+
+    using T16 = uint16_t;
+    const int warp = warp_id();
+    const int lane = lane_id();
+
+    if (n_it == 0) {  // no query sees this key tile: dK = dV = 0
+        if (threadIdx.x < 128) {
+            const int key = k0 + static_cast<int>(threadIdx.x);
+            if (key < Nk) {
+                const size_t off = ((static_cast<size_t>(b) * Nk + key) * args.Hkv + hk) * D;
+                uint4* a = reinterpret_cast<uint4*>(static_cast<T16*>(args.dk) + off);
+                uint4* c = reinterpret_cast<uint4*>(static_cast<T16*>(args.dv) + off);
+#pragma unroll
+                for (int i = 0; i < D / 8; ++i) a[i] = c[i] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        return;
+    }
+
+    uint8_t* sK = smem + C::kKOff;
+    uint8_t* sV = smem + C::kVOff;
+    uint8_t* sQ = smem + C::kQOff;
+    uint8_t* sDO = smem + C::kDOOff;
+    uint8_t* sDS = smem + C::kDSOff;
+    float* sLD = reinterpret_cast<float*>(smem + C::kLDOff);  // stage st: L2 at [256 st], D at [256 st + 128]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* kv_full = bars;
+    uint64_t* q_full = bars + 1;   // [2]
+    uint64_t* q_empty = bars + 3;  // [2]
+    uint64_t* s_full = bars + 5;
+    uint64_t* ds_ready = bars + 6;
+    uint64_t* mm_done = bars + 7;
+    uint64_t* dq_full = bars + 8;
+    uint64_t* dq_free = bars + 9;
+    uint64_t* fin = bars + 10;
+    uint64_t* ld_full = bars + 11;  // [2]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+    int* abort_flag = reinterpret_cast<int*>(smem + C::kMiscOff + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(ds_ready, 256);
+        mbar_init(mm_done, 1);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_free, 256);
+        mbar_init(fin, 1);
+        mbar_init(&ld_full[0], 128);
+        mbar_init(&ld_full[1], 128);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+    const WaitCtx wc{abort_flag, args.err};
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+#pragma unroll
+            for (int s = 0; s < D / 64; ++s) {
+                tma_load_4d(sK + s * C::kSlabBytes, &tm_k, kv_full, s * 64, hk, k0, b);
+                tma_load_4d(sV + s * C::kSlabBytes, &tm_v, kv_full, s * 64, hk, k0, b);
+            }
+            int issued = 0;
+            for (int it = 0; it < n_it; ++it) {
+                const int st = it & 1;
+                const int h = hk * args.group + it / n_i;
+                const int q0 = (i0 + it % n_i) * 128;
+                if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1u, wc, 21)) break;
+                mbar_arrive_expect_tx(&q_full[st], 2 * C::kTileBytes);
+#pragma unroll
+                for (int s = 0; s < D / 64; ++s) {
+                    tma_load_4d(sQ + st * C::kTileBytes + s * C::kSlabBytes, &tm_q, &q_full[st], s * 64, h, q0, b);
+                    tma_load_4d(sDO + st * C::kTileBytes + s * C::kSlabBytes, &tm_do, &q_full[st], s * 64, h, q0, b);
+                }
+                ++issued;
+            }
+            mbar_wait_drain(kv_full, 0);
+            for (int st = 0; st < 2; ++st)
+                if (issued > st) mbar_wait_drain(&q_full[st], (((issued - 1 - st) / 2 * 2 + st) >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_kk = idesc_f16(128, 128, BF16, false, false);  // S^T, dP^T
+            constexpr uint32_t id_tm = idesc_f16(128, D, BF16, false, true);     // dV, dK (A in TMEM)
+            constexpr uint32_t id_dq = idesc_f16(128, D, BF16, true, true);      // dQ (A = dS, MN-major)
+            const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), ds_addr = smem_u32(sDS);
+            bool ok = mbar_wait(kv_full, 0, wc, 22);
+            for (int it = 0; ok && it < n_it; ++it) {
+                const int st = it & 1;
+                if (it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, 23))) break;  // dQ_{it-1} drained
+                if (!(ok = mbar_wait(&q_full[st], (it >> 1) & 1, wc, 24))) break;
+                tc_fence_after();
+                const uint32_t q_addr = smem_u32(sQ + st * C::kTileBytes);
+                const uint32_t do_addr = smem_u32(sDO + st * C::kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
+                    mma_ss(tmem + C::kColS, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024),
+                           id_kk, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
+                    mma_ss(tmem + C::kColDP, sdesc_sw128(v_addr + off, 16, 1024),
+                           sdesc_sw128(do_addr + off, 16, 1024), id_kk, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(s_full);
+                if (!(ok = mbar_wait(ds_ready, it & 1, wc, 25))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+                           sdesc_sw128(do_addr + kk * 2048, C::kSlabBytes, 1024), id_tm, (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + C::kColDK, tmem + C::kColDP + kk * 8,
+                           sdesc_sw128(q_addr + kk * 2048, C::kSlabBytes, 1024), id_tm, (it > 0 || kk > 0) ? 1u : 0u);
+                // dQ_i overwrites the P^T columns and the next dP^T the dS^T
+                // columns; both are different accumulators, so wait explicitly.
+                tc_commit(mm_done);
+                if (!(ok = mbar_wait(mm_done, it & 1, wc, 26))) break;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + C::kColS, sdesc_sw128(ds_addr + kk * 2048, C::kSlabBytes, 1024),
+                           sdesc_sw128(k_addr + kk * 2048, C::kSlabBytes, 1024), id_dq, kk > 0 ? 1u : 0u);
+                tc_commit(&q_empty[st]);
+                tc_commit(dq_full);
+            }
+            tc_commit(fin);
+            mbar_wait_drain(fin, 0);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ compute warpgroups
+        const int wg = (warp - 4) >> 2;  // 0 or 1
+        const int w4 = warp & 3;
+        const int r = w4 * 32 + lane;  // TMEM lane: key row for S^T / dP^T / dV / dK, query row for dQ
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
+        const int key = k0 + r;
+        const bool key_ok = key < Nk;
+        const float sl2 = args.scale_log2;
+        constexpr float kLog2eF = 1.4426950408889634074f;
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int h = hk * args.group + it / n_i;
+            const int q0 = (i0 + it % n_i) * 128;
+            // Per-query L (in log2 units) and D of this tile, shared through a
+            // 2-stage smem buffer. Stage it&1 is rewritten at it+2, when every
+            // compute thread has arrived on ds_ready for it+1, so no reader of
+            // iteration it is left.
+            float* sL = sLD + (it & 1) * 256;
+            float* sD = sL + 128;
+            if (wg == 0) {
+                const int q = q0 + r;
+                float l2 = INFINITY, dd = 0.f;
+                if (q < Nq) {
+                    const size_t row = (static_cast<size_t>(b) * args.Hq + h) * Nq + q;
+                    const float L = args.lse[row];
+                    l2 = (L == -INFINITY) ? INFINITY : L * kLog2eF;  // a row that saw no key has P = 0
+                    dd = args.D[row];
+                }
+                sL[r] = l2;
+                sD[r] = dd;
+                mbar_arrive(&ld_full[it & 1]);
+            }
+            ok = warp_all(mbar_wait(&ld_full[it & 1], (it >> 1) & 1, wc, 30));
+            if (!ok) break;
+            ok = warp_all(mbar_wait(s_full, it & 1, wc, 27));
+            if (!ok) break;
+            tc_fence_after();
+            // Query q sees this thread's key iff key <= q + (Nk - Nq) (and key < Nk).
+            const int qlim = key - (Nk - Nq);  // smallest query that sees the key
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = wg * 2 + cc;  // 32-column chunk of the 128 queries
+                uint32_t sv[32], pv[32];
+                tmem_ld32(lane_base + C::kColS + c * 32, sv);
+                tmem_ld32(lane_base + C::kColDP + c * 32, pv);
+                tmem_ld_wait(sv);
+                tmem_ld_wait(pv);
+                uint32_t pk[16], dk16[16];
+#pragma unroll
+                for (int t = 0; t < 32; t += 2) {
+                    float p[2], ds[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int qq = c * 32 + t + e;
+                        bool vis = key_ok;
+                        if (CAUSAL) vis = vis && (q0 + qq >= qlim);
+                        const float pe = ex2_approx(fmaf(__uint_as_float(sv[t + e]), sl2, -sL[qq]));
+                        p[e] = vis ? pe : 0.f;
+                        ds[e] = p[e] * (__uint_as_float(pv[t + e]) - sD[qq]);
+                    }
+                    pk[t >> 1] = pack2<BF16>(p[0], p[1]);
+                    dk16[t >> 1] = pack2<BF16>(ds[0], ds[1]);
+                }
+                tmem_st16(lane_base + C::kColS + c * 16, pk);
+                tmem_st16(lane_base + C::kColDP + c * 16, dk16);
+                // dS row of this key into the MN-major dQ operand: 64-query slabs,
+                // key rows of 128 B, 16-byte chunks swizzled by key % 8.
+                uint8_t* row = sDS + (c >> 1) * C::kSlabBytes + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int chunk = ((c & 1) * 4 + u) ^ (r & 7);
+                    *reinterpret_cast<uint4*>(row + chunk * 16) =
+                        make_uint4(dk16[4 * u], dk16[4 * u + 1], dk16[4 * u + 2], dk16[4 * u + 3]);
+                }
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(ds_ready);
+            // Drain dQ_i = dS K_j: lane r is query q0 + r; this warpgroup adds d/2 columns.
+            ok = warp_all(mbar_wait(dq_full, it & 1, wc, 28));
+            if (!ok) break;
+            tc_fence_after();
+            const int q = q0 + r;
+            float* dst = args.dq_acc + ((static_cast<size_t>(b) * Nq + q) * args.Hq + h) * D;
+#pragma unroll
+            for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(lane_base + C::kColS + c0, v);
+                tmem_ld_wait(v);
+                if (q < Nq) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        red_add_v4(dst + c0 + i, __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                   __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(dq_free);
+        }
+        if (ok) ok = warp_all(mbar_wait(fin, 0, wc, 29));
+        if (ok) {
+            tc_fence_after();
+            // Warpgroup 0 writes dV, warpgroup 1 writes dK = scale * (dS^T Q).
+            const uint32_t col = wg == 0 ? C::kColDV : C::kColDK;
+            const float mul = wg == 0 ? 1.f : args.scale;
+            T16* dst = static_cast<T16*>(wg == 0 ? args.dv : args.dk) +
+                       ((static_cast<size_t>(b) * Nk + key) * args.Hkv + hk) * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(lane_base + col + c0, v);
+                tmem_ld_wait(v);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack2<BF16>(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+                if (key_ok) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// D[b,h,q] = sum_c dO[b,q,h,c] O[b,q,h,c] in fp32, and dQ_acc[b,q,h,:] = 0.
+// A group of D/8 lanes handles one (b, q, h) row, 8 elements per lane.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float* Dvec,
+                                                          float* dq_acc, int B, int Nq, int Hq, bool bf16) {
+    constexpr int kLanes = D / 8;
+    const size_t rows = static_cast<size_t>(B) * Nq * Hq;
+    const size_t row = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / kLanes;
+    const int sub = threadIdx.x % kLanes;
+    float acc = 0.f;
+    if (row < rows) {
+        const uint4 a = reinterpret_cast<const uint4*>(o + row * D)[sub];
+        const uint4 c = reinterpret_cast<const uint4*>(dout + row * D)[sub];
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float a0, a1, c0, c1;
+            if (bf16) {
+                a0 = __uint_as_float(av[i] << 16);
+                a1 = __uint_as_float(av[i] & 0xFFFF0000u);
+                c0 = __uint_as_float(cv[i] << 16);
+                c1 = __uint_as_float(cv[i] & 0xFFFF0000u);
+            } else {
+                a0 = __half2float(__ushort_as_half(static_cast<unsigned short>(av[i] & 0xFFFFu)));
+                a1 = __half2float(__ushort_as_half(static_cast<unsigned short>(av[i] >> 16)));
+                c0 = __half2float(__ushort_as_half(static_cast<unsigned short>(cv[i] & 0xFFFFu)));
+                c1 = __half2float(__ushort_as_half(static_cast<unsigned short>(cv[i] >> 16)));
+            }
+            acc = fmaf(a0, c0, acc);
+            acc = fmaf(a1, c1, acc);
+        }
+        float4* z = reinterpret_cast<float4*>(dq_acc + row * D) + sub * 2;
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && sub == 0) {
+        // row = (b * Nq + q) * Hq + h  ->  D layout [B, Hq, Nq]
+        const size_t h = row % Hq;
+        const size_t bq = row / Hq;
+        const size_t q = bq % Nq;
+        const size_t bb = bq / Nq;
+        Dvec[(bb * Hq + h) * Nq + q] = acc;
+    }
+}
+
+// dq[i] = dtype(scale * dq_acc[i]), 8 elements per thread.
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert(const float* dq_acc, uint16_t* dq, size_t n8, float scale,
+                                                          bool bf16) {
+    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * i];
+    const float4 c = reinterpret_cast<const float4*>(dq_acc)[2 * i + 1];
+    uint4 out;
+    if (bf16) {
+        out = make_uint4(pack2<true>(a.x * scale, a.y * scale), pack2<true>(a.z * scale, a.w * scale),
+                         pack2<true>(c.x * scale, c.y * scale), pack2<true>(c.z * scale, c.w * scale));
+    } else {
+        out = make_uint4(pack2<false>(a.x * scale, a.y * scale), pack2<false>(a.z * scale, a.w * scale),
+                         pack2<false>(c.x * scale, c.y * scale), pack2<false>(c.z * scale, c.w * scale));
+    }
+    reinterpret_cast<uint4*>(dq)[i] = out;
+}
+
+}  // namespace fa

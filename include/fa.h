@@ -1,0 +1,152 @@
+/*
+ * fa.h: C ABI of the exact tiled attention library (libfa.so), sm_100a.
+ *
+ * The library computes exact scaled dot-product attention
+ *     O = softmax(scale * Q K^T) V
+ * tile by tile with the online-softmax recurrence (a running row max m and
+ * normaliser l; the partial output is rescaled by exp(m_old - m_new) each
+ * time the max grows), writing only O and the log-sum-exp L = m + ln(l).
+ * The backward pass recomputes S and P from L and dO, so no N x N matrix is
+ * ever written to device memory. Sources: "FlashAttention/zh", sections
+ * "why standard attention is slow" (the definition), "online softmax trick",
+ * "FlashAttention algorithm" (the tiled forward and L), and "backward pass
+ * and recomputation"; the varlen interface (cu_seqlens, max_s, fp16/bf16
+ * only, no attention-weights output) follows the FlashAttention wrapper on
+ * "InternViT-6B-448px-V1-2 ... FlashAttention v1/v2" (its three execution
+ * paths).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every pointer is a DEVICE pointer owned by the caller. The
+ *           library allocates no device memory per call; its only state is
+ *           a device error word. Tensors are contiguous, row-major.
+ * Layouts.  Fixed length uses BSHD: q, o, dO [B, Nq, Hq, d]; k, v
+ *           [B, Nk, Hkv, d]. lse is float32 [B, Hq, Nq], natural log, of the
+ *           SCALED scores: lse[b,h,i] = log sum_j exp(scale * q_i . k_j).
+ * Heads.    Grouped KV heads: query head h reads KV head h / (Hq / Hkv).
+ * Causal.   causal = 1 masks key j for query i when j > i + (Nk - Nq)
+ *           (bottom-right alignment; the pages name the causal mask but not
+ *           its alignment). A query row that sees no key gets O = 0 and
+ *           lse = -inf.
+ * Types.    dtype selects bf16 or fp16 for q, k, v, o, dO, dq, dk, dv;
+ *           accumulation is fp32; P is rounded to dtype before P V.
+ * Sizes.    d must be 64 or 128. B, Hq, Hkv >= 1; Nq, Nk >= 0 (0 gives no
+ *           work); Hq % Hkv == 0.
+ * Alignment Every tensor pointer must be 16-byte aligned.
+ * Streams.  Work is enqueued on `stream` (may be 0 = legacy default stream)
+ *           and runs asynchronously; nothing is written to host memory and
+ *           no call synchronises, except fa_get_last_device_error.
+ * Errors.   Invalid arguments are reported before anything is launched and
+ *           nothing is launched then. Launch failures give FA_ERR_CUDA.
+ *           Every wait inside a kernel is bounded; a wait that runs out sets
+ *           the device error word and the kernel returns early, which the
+ *           host sees through fa_get_last_device_error (FA_ERR_TIMEOUT).
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1, /* null pointer, bad size, Hq % Hkv != 0, bad scale */
+    FA_ERR_UNSUPPORTED = 2, /* head dim other than 64 / 128, unknown dtype, too large */
+    FA_ERR_MISALIGNED = 3,  /* a tensor pointer not 16-byte aligned */
+    FA_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed */
+    FA_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see fa_get_last_device_error) */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/*
+ * Forward, fixed length ("FlashAttention/zh", section "FlashAttention
+ * algorithm": tiled online softmax, O_i / l_i and L_i = m_i + log l_i).
+ *   q [B,Nq,Hq,d], k and v [B,Nk,Hkv,d]  (inputs, dtype)
+ *   o [B,Nq,Hq,d] (output, dtype), lse [B,Hq,Nq] (output, float32)
+ *   scale: multiplies Q K^T; pass 1/sqrt(d) for the standard definition.
+ *          Must be finite and > 0.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                 float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
+ * Forward, packed variable length (the cu_seqlens / max_s varlen path of
+ * the InternViT FlashAttention wrapper; key padding is handled by unpadding
+ * K/V and passing their own cu_seqlens_k).
+ *   q, o [total_q, Hq, d]; k, v [total_k, Hkv, d] (dtype)
+ *   cu_seqlens_q, cu_seqlens_k: DEVICE int32 [num_seqs + 1], cu[0] = 0,
+ *       non-decreasing; sequence s owns query rows cu_q[s] .. cu_q[s+1]-1
+ *       and key rows cu_k[s] .. cu_k[s+1]-1. Lengths may be 0.
+ *   total_q, total_k: the number of rows of the q/o and k/v buffers (the
+ *       host-side extents of the packed tensors; cu_seqlens live on the
+ *       device, so the library cannot read them without a synchronisation).
+ *       No row at or past total_q is written and no row at or past total_k
+ *       is read, whatever cu_seqlens hold.
+ *   max_seqlen_q, max_seqlen_k: upper bounds of the lengths (grid sizing
+ *       only; a length above its bound is not processed past the bound).
+ *   lse [Hq, total_q] float32.
+ *   Causal alignment is bottom-right within each sequence.
+ */
+fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                        int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                        int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
+                        fa_stream_t stream);
+
+/*
+ * Size in bytes of the caller-owned workspace fa_bwd needs: the per-row
+ * D_i = sum_c dO_ic O_ic (float32 [B,Hq,Nq]) and the float32 dQ accumulator
+ * ([B,Nq,Hq,d]), each rounded up to 256 bytes. Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
+
+/*
+ * Backward, fixed length ("FlashAttention/zh", section "backward pass and
+ * recomputation": S and P are recomputed from the saved L and dO). With
+ * P = exp(scale Q K^T - L) the gradients are the exact derivatives of the
+ * definition: dV = P^T dO, dP = dO V^T, D_i = sum_c dO_ic O_ic,
+ * dS = P o (dP - D), dQ = scale dS K, dK = scale dS^T Q; with grouped KV
+ * heads dK and dV of a KV head sum over its query heads.
+ *   q, k, v, o, lse: exactly as given to / returned by fa_fwd.
+ *   dout [B,Nq,Hq,d] (input, dtype).
+ *   dq [B,Nq,Hq,d], dk and dv [B,Nk,Hkv,d] (outputs, dtype; overwritten).
+ *   workspace: device buffer of fa_bwd_workspace_size(B,Hq,Nq,d) bytes,
+ *       16-byte aligned, owned by the caller; its contents on entry do not
+ *       matter and on exit are unspecified.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                 float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/* A static description of a status code. Never NULL. */
+const char* fa_status_string(fa_status s);
+
+/*
+ * Synchronises `stream`, then reports and clears the device error word:
+ * FA_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last call,
+ * FA_ERR_CUDA if the synchronisation failed or a kernel refused to run,
+ * FA_OK otherwise.
+ */
+fa_status fa_get_last_device_error(fa_stream_t stream);
+
+/* The raw device error code behind the last non-OK fa_get_last_device_error:
+ * 0x1000 + site for a wait that ran out, 0x2000 for a shared-memory window
+ * that was not 1024-byte aligned (the kernel then does nothing); 0 if none. */
+int fa_get_last_device_error_site(void);
+
+/* Library version, "major.minor.patch". */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,126 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, and rejects invalid arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_tiled_attention_36_b200 import binding as fb
+from exact_tiled_attention_36_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fbuild.build()
+    return fb.lib()
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(fa_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"fa_fwd", "fa_varlen_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string",
+            "fa_get_last_device_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert fb.fa_status_string(s).startswith("FA_")
+    assert "unknown" in fb.fa_status_string(77)
+    assert re.match(r"\d+\.\d+\.\d+", fb.fa_version())
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced on these paths
+
+
+def fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=64, scale=0.125,
+             causal=0, dtype=fb.FA_BF16, stream=None)
+    a.update(kw)
+    return fb.fa_fwd(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), fb.FA_ERR_INVALID_ARG),
+    (dict(lse=None), fb.FA_ERR_INVALID_ARG),
+    (dict(B=0), fb.FA_ERR_INVALID_ARG),
+    (dict(Nq=-1), fb.FA_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), fb.FA_ERR_INVALID_ARG),
+    (dict(Hkv=0), fb.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fb.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fb.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), fb.FA_ERR_INVALID_ARG),
+    (dict(causal=2), fb.FA_ERR_INVALID_ARG),
+    (dict(d=96), fb.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fb.FA_ERR_UNSUPPORTED),
+    (dict(dtype=7), fb.FA_ERR_UNSUPPORTED),
+    (dict(k=FAKE + 8), fb.FA_ERR_MISALIGNED),
+    (dict(lse=FAKE + 4), fb.FA_ERR_MISALIGNED),
+    (dict(Nq=0), fb.FA_OK),  # no work: nothing is launched
+])
+def test_fwd_rejects_before_launch(lib, kw, code):
+    assert fwd(**kw) == code
+
+
+def varlen(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, cu_q=FAKE, cu_k=FAKE, num_seqs=2, total_q=10, total_k=10,
+             max_q=5, max_k=5, Hq=2, Hkv=2, d=128, scale=0.1, causal=0, dtype=fb.FA_FP16, stream=None)
+    a.update(kw)
+    return fb.fa_varlen_fwd(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu_q=None), fb.FA_ERR_INVALID_ARG),
+    (dict(num_seqs=0), fb.FA_ERR_INVALID_ARG),
+    (dict(total_k=-1), fb.FA_ERR_INVALID_ARG),
+    (dict(max_q=-3), fb.FA_ERR_INVALID_ARG),
+    (dict(d=32), fb.FA_ERR_UNSUPPORTED),
+    (dict(cu_k=FAKE + 2), fb.FA_ERR_MISALIGNED),
+    (dict(o=FAKE + 2), fb.FA_ERR_MISALIGNED),
+    (dict(max_q=0), fb.FA_OK),
+    (dict(total_q=0), fb.FA_OK),
+])
+def test_varlen_rejects_before_launch(lib, kw, code):
+    assert varlen(**kw) == code
+
+
+def bwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, ws=FAKE, B=1, Hq=4,
+             Hkv=2, Nq=8, Nk=8, d=128, scale=0.1, causal=1, dtype=fb.FA_BF16, stream=None)
+    a.update(kw)
+    return fb.fa_bwd(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), fb.FA_ERR_INVALID_ARG),
+    (dict(dq=None), fb.FA_ERR_INVALID_ARG),
+    (dict(Hq=5), fb.FA_ERR_INVALID_ARG),
+    (dict(d=80), fb.FA_ERR_UNSUPPORTED),
+    (dict(ws=FAKE + 8), fb.FA_ERR_MISALIGNED),
+    (dict(dv=FAKE + 1), fb.FA_ERR_MISALIGNED),
+])
+def test_bwd_rejects_before_launch(lib, kw, code):
+    assert bwd(**kw) == code
+
+
+def test_workspace_size(lib):
+    B, Hq, Nq, d = 2, 32, 8192, 128
+    rows = B * Hq * Nq
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert fb.fa_bwd_workspace_size(B, Hq, Nq, d) == r256(rows * 4) + r256(rows * d * 4)
+    assert fb.fa_bwd_workspace_size(1, 1, 3, 64) == 256 + r256(3 * 64 * 4)
+    assert fb.fa_bwd_workspace_size(0, 1, 1, 64) == 0
+    assert fb.fa_bwd_workspace_size(1, 1, 1, 96) == 0

@@ -1,0 +1,101 @@
+"""Backward parity: fa_bwd (through the C ABI) against the fp64 oracle's exact gradients."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_tiled_attention_36_b200 import binding as fb
+from exact_tiled_attention_36_b200 import inputs
+from tests.gpu_util import RTOL_GRAD, f64, guarded
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    fb.lib()
+    yield
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+
+
+def run_fwd_bwd(fi, causal, scale):
+    q, k, v, do = fi.q.cuda(), fi.k.cuda(), fi.v.cuda(), fi.do.cuda()
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    dt = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device="cuda")
+    assert fb.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                     scale, int(causal), dt, 0) == fb.FA_OK
+    ws = torch.full((fb.fa_bwd_workspace_size(B, Hq, Nq, d),), 255, dtype=torch.uint8, device="cuda")
+    dq, dq_ok = guarded((B, Nq, Hq, d), q.dtype)
+    dk, dk_ok = guarded((B, Nk, Hkv, d), q.dtype)
+    dv, dv_ok = guarded((B, Nk, Hkv, d), q.dtype)
+    st = fb.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                   dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale,
+                   int(causal), dt, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    torch.cuda.synchronize()
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    assert dq_ok() and dk_ok() and dv_ok(), "write outside dQ / dK / dV"
+    return dq, dk, dv
+
+
+def rel_l2(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+SMALL = [
+    # B, Hq, Hkv, Nq, Nk, d, causal, dtype
+    (1, 2, 2, 128, 128, 64, False, "bf16"),
+    (1, 2, 2, 256, 256, 128, False, "bf16"),
+    (2, 4, 2, 129, 129, 128, True, "bf16"),
+    (1, 2, 1, 300, 200, 64, True, "fp16"),
+    (1, 2, 2, 200, 333, 128, True, "bf16"),
+    (2, 3, 1, 97, 250, 64, False, "fp16"),
+    (1, 4, 4, 1, 5, 128, False, "bf16"),
+    (1, 8, 2, 520, 520, 128, True, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "-".join(map(str, c)))
+def test_bwd_small_shapes(case):
+    B, Hq, Hkv, Nq, Nk, d, causal, dt = case
+    fi = inputs.make_fixed(inputs.CAUSAL_GQA, B=B, Hq=Hq, Hkv=Hkv, Nq=Nq, Nk=Nk, d=d, dtype=dt, causal=causal,
+                           seed=23)
+    scale = d ** -0.5
+    dq, dk, dv = run_fwd_bwd(fi, causal, scale)
+    rq, rk, rv = oracle.attn_bwd(fi.q, fi.k, fi.v, fi.do, scale, causal)
+    errs = [rel_l2(f64(x), r) for x, r in ((dq, rq), (dk, rk), (dv, rv))]
+    assert max(errs) <= RTOL_GRAD, errs
+
+
+def test_bwd_causal_gqa_full_size():
+    """The causal GQA prefill workload at full size: sampled rows against the oracle,
+    and two identities that hold at any size on every row of dK and dV."""
+    cfg = inputs.CAUSAL_GQA
+    fi = inputs.make_fixed(cfg)
+    dq, dk, dv = run_fwd_bwd(fi, cfg.causal, cfg.scale)
+    dq, dk, dv = f64(dq), f64(dk), f64(dv)
+    g = cfg.Hq // cfg.Hkv
+    qrows = [0, 1, 127, 128, 4095, 8000, 8191]
+    krows = [7936, 8000, 8100, 8190, 8191]
+    for (b, hk) in [(0, 0), (1, 7)]:
+        sq, sk, sv = oracle.attn_bwd_sampled(fi.q, fi.k, fi.v, fi.do, cfg.scale, b, hk, qrows, krows, True)
+        gq = dq[b][qrows][:, hk * g:(hk + 1) * g]
+        assert rel_l2(gq, sq) <= RTOL_GRAD
+        assert rel_l2(dk[b, krows, hk], sk) <= RTOL_GRAD
+        assert rel_l2(dv[b, krows, hk], sv) <= RTOL_GRAD
+    # sum over keys of dK is 0 (rows of dS sum to 0); sum over keys of dV equals the
+    # sum of dO over the group's query rows (rows of P sum to 1).
+    do = f64(fi.do)
+    for b in range(cfg.B):
+        for hk in range(cfg.Hkv):
+            sdk = dk[b, :, hk].sum(0)
+            assert np.abs(sdk).max() <= 2e-2 * np.abs(dk[b, :, hk]).sum(0).max() + 1e-3
+            sdv = dv[b, :, hk].sum(0)
+            ref = do[b, :, hk * g:(hk + 1) * g].sum((0, 1))
+            assert rel_l2(sdv, ref) <= RTOL_GRAD
