@@ -29,7 +29,8 @@
 // half of the dQ columns while draining, and one of dV / dK at the end).
 //
 // TMEM columns: [0,128) S^T, later P^T, later dQ_i; [128,256) dP^T, later dS^T;
-// [256,256+d) dV; [256+d,256+2d) dK.
+// [256,256+d) dV; [256+d,256+2d) dK. Each compute warpgroup writes its packed
+// 16-bit P^T / dS^T over the first half of its own 64 columns.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -224,13 +225,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tc_commit(s_full);
                 if (!(ok = mbar_wait(ds_ready, it & 1, wc, 25))) break;
                 tc_fence_after();
+                // P^T / dS^T of queries 16 kk .. 16 kk + 15 sit at column
+                // 64 (kk / 4) + 8 (kk % 4) of their region (see the compute warps).
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+                    mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
                            sdesc_sw128(do_addr + kk * 2048, C::kSlabBytes, 1024), id_tm, (it > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + C::kColDK, tmem + C::kColDP + kk * 8,
+                    mma_ts(tmem + C::kColDK, tmem + C::kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
                            sdesc_sw128(q_addr + kk * 2048, C::kSlabBytes, 1024), id_tm, (it > 0 || kk > 0) ? 1u : 0u);
                 // dQ_i overwrites the P^T columns and the next dP^T the dS^T
                 // columns; both are different accumulators, so wait explicitly.
@@ -310,8 +313,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     pk[t >> 1] = pack2<BF16>(p[0], p[1]);
                     dk16[t >> 1] = pack2<BF16>(ds[0], ds[1]);
                 }
-                tmem_st16(lane_base + C::kColS + c * 16, pk);
-                tmem_st16(lane_base + C::kColDP + c * 16, dk16);
+                // Packed 16-bit pairs go over columns this warpgroup has already
+                // read itself: queries 64 wg + 32 cc + t land in column
+                // 64 wg + 16 cc + t / 2 (the other warpgroup may still be reading
+                // its own half).
+                tmem_st16(lane_base + C::kColS + wg * 64 + cc * 16, pk);
+                tmem_st16(lane_base + C::kColDP + wg * 64 + cc * 16, dk16);
                 // dS row of this key into the MN-major dQ operand: 64-query slabs,
                 // key rows of 128 B, 16-byte chunks swizzled by key % 8.
                 uint8_t* row = sDS + (c >> 1) * C::kSlabBytes + (r >> 3) * 1024 + (r & 7) * 128;
