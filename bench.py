@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the exact tiled attention hot path on B200.
+
+One step is the whole path on one batch of the causal GQA prefill workload
+(B=2, N=8192, Hq=32, Hkv=8, d=128, bf16, causal): fa_fwd (O and L), then
+fa_bwd (D = rowsum(dO o O), the recompute kernel, dQ convert). Inputs are
+seeded synthetic N(0,1) tensors, resident in device memory before timing.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). FLOPs follow the FlashAttention convention:
+fwd = 4 Nq Nk d per (batch, query head), halved for causal; bwd = 2.5 fwd.
+With N > 1 (torchrun, one rank per GPU) every rank runs its own independent
+batch (the path has no exchange step: replicas, weak scaling); the time is the
+max over ranks.
+
+--impl reference times the fp64 CPU oracle (the plain definition) on a
+bounded sample of the same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(name="causal_gqa_prefill_fwd_bwd", B=2, N=8192, Hq=32, Hkv=8, d=128, dtype="bf16", causal=True)
+METRIC = "attention fwd+bwd TFLOPS on 1 B200 (FlashAttention FLOP convention) and % of dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# CPU sample for the oracle: batch 0, every query head, the first T tokens.
+# Under the causal mask these tokens form exactly the top-left block of the
+# full problem, i.e. a causal attention problem of length T. The CPU-baseline
+# leg of the GPU run takes one larger sample; the reference arm repeats a
+# smaller one per step so that a whole --steps/--warmup run stays short.
+CPU_SAMPLE_TOKENS = 2048
+REF_STEP_TOKENS = 1024
+# Small case of the same kernels for profiler captures (inputs still > L2).
+PROFILE_CASE = dict(B=1, N=4096)
+
+
+def flops_fwd(B, N, Hq, d, causal):
+    f = 4.0 * N * N * d * B * Hq
+    return f / 2 if causal else f
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "exact_tiled_attention_36_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was
+    captured from the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}.txt")
+    try:
+        kv = {}
+        for line in open(path):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("csrc_sha256_16") == csrc_digest():
+            return float(kv["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle (reference arm)
+def cpu_oracle_sample(n_steps, tokens):
+    """Time the fp64 oracle (fwd + bwd) on the bounded sample, n_steps times."""
+    import oracle
+    from exact_tiled_attention_36_b200 import inputs
+    w = WORKLOAD
+    cfg = inputs.CAUSAL_GQA
+    fi = inputs.make_fixed(cfg, B=1, Nq=tokens, Nk=tokens)
+    args = [oracle._f64(t) for t in (fi.q, fi.k, fi.v, fi.do)]
+    oracle.build()
+    flops = 3.5 * flops_fwd(1, tokens, w["Hq"], w["d"], w["causal"])
+    times = []
+    for _ in range(n_steps):
+        t0 = time.perf_counter()
+        oracle.attn_fwd(args[0], args[1], args[2], cfg.scale, True)
+        oracle.attn_bwd(args[0], args[1], args[2], args[3], cfg.scale, True)
+        times.append(time.perf_counter() - t0)
+    return flops, times, oracle.num_threads()
+
+
+def cpu_sample_desc(tokens):
+    w = WORKLOAD
+    return (f"oracle fwd+bwd (fp64, OpenMP) on batch 0, all {w['Hq']} query heads / {w['Hkv']} KV heads, "
+            f"first {tokens} of {w['N']} tokens (the top-left causal block), d={w['d']}")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    if args.warmup > 0:
+        cpu_oracle_sample(args.warmup, REF_STEP_TOKENS)
+    flops, times, cores = cpu_oracle_sample(args.steps, REF_STEP_TOKENS)
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD["name"], "sample_tokens": REF_STEP_TOKENS,
+                   **{k: WORKLOAD[k] for k in ("Hq", "Hkv", "d", "causal")}},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": cpu_sample_desc(REF_STEP_TOKENS) + ", once per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from exact_tiled_attention_36_b200 import binding as fb
+    from exact_tiled_attention_36_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    fb.lib()
+    w = dict(WORKLOAD)
+    if args.profile_small:
+        w.update(PROFILE_CASE)
+    cfg = inputs.CAUSAL_GQA
+    # each rank draws its own batch (independent replicas of the workload)
+    fi = inputs.make_fixed(cfg, seed=cfg.seed + 1000 * rank, B=w["B"], Nq=w["N"], Nk=w["N"])
+    B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
+    scale = d ** -0.5
+    dt = fb.FA_BF16
+    q, k, v, do = (t.cuda() for t in (fi.q, fi.k, fi.v, fi.do))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, N, d), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def step():
+        st = fb.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d,
+                       scale, 1, dt, sh)
+        if st != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(st))
+        st = fb.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, N, N, d, scale, 1, dt,
+                       sh)
+        if st != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(st))
+
+    f_fwd = flops_fwd(B, N, Hq, d, True)
+    f_step = 3.5 * f_fwd
+    warm = max(args.warmup, 3)
+    K = args.steps
+
+    def timed_region():
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+        for e in ev:
+            for x in e:
+                x.record(stream)  # create the underlying events
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(K):
+            e0, e1, e2, eb0, eb1 = ev[i]
+            fb.fa_bwd_set_timing_events(eb0.cuda_event, eb1.cuda_event)
+            e0.record(stream)
+            st = fb.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N,
+                           d, scale, 1, dt, sh)
+            e1.record(stream)
+            st2 = fb.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, N, N, d, scale,
+                            1, dt, sh)
+            e2.record(stream)
+            if st != fb.FA_OK or st2 != fb.FA_OK:
+                raise RuntimeError(fb.fa_status_string(st or st2))
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        fb.fa_bwd_set_timing_events(None, None)
+        total_ms = start.elapsed_time(end)
+        fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
+        bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
+        bwd_main_ms = [e[3].elapsed_time(e[4]) for e in ev]
+        return total_ms, fwd_ms, bwd_ms, bwd_main_ms
+
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+    if fb.fa_get_last_device_error(None) != fb.FA_OK:
+        raise RuntimeError("device error during warm-up")
+    if args.profile_small:  # profiler driver: the warm-up launches are the capture targets
+        print(f"profile case B={B} N={N}: {warm} fwd+bwd steps done", flush=True)
+        return 0
+
+    sampler = ClockSampler(local)
+    result = None
+    clocks = None
+    for attempt in range(2):
+        sampler.start()
+        time.sleep(0.3)
+        result = timed_region()
+        clocks = sampler.stop()
+        if not clocks or not (set(clocks["reasons"]) & BAD_REASONS):
+            break
+    total_ms, fwd_ms, bwd_ms, bwd_main_ms = result
+    if fb.fa_get_last_device_error(None) != fb.FA_OK:
+        raise RuntimeError("device error during the timed region")
+    total_ms = max_over_ranks(total_ms)
+
+    # end to end through the C ABI with host buffers: H2D of q, k, v, dO from
+    # pinned memory, fwd + bwd, D2H of dq, dk, dv, every step.
+    hq, hk, hv, hdo = (t.pin_memory() for t in (fi.q, fi.k, fi.v, fi.do))
+    hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in (hdq, hdk, hdv))
+    K_e2e = max(3, min(K, 20))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        do.copy_(hdo, non_blocking=True)
+        step()
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(K_e2e):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1))
+
+    peaks, peak_src = load_peaks()
+    value = world * f_step * K / (total_ms / 1e3) / 1e12
+    e2e_value = world * f_step * K_e2e / (e2e_ms / 1e3) / 1e12
+    fwd_avg = statistics.mean(fwd_ms)
+    bwd_avg = statistics.mean(bwd_ms)
+    main_avg = statistics.mean(bwd_main_ms)
+    f_bwd = 2.5 * f_fwd
+    # dominant kernel: the longer of the forward kernel and the backward main kernel
+    if main_avg >= fwd_avg:
+        kname, kflops, kms = "fa_bwd_kernel", f_bwd, main_avg
+    else:
+        kname, kflops, kms = "fa_fwd_kernel", f_fwd, fwd_avg
+    achieved = kflops / (kms / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w["name"], "B": B, "seq_len": N, "Hq": Hq, "Hkv": Hkv, "d": d, "causal": True,
+                   "parallelism": f"replicas x{world} (no exchange step)",
+                   "l2": "inputs larger than L2: ~1.0 GB of tensors touched per step vs 126 MB L2"},
+        "fwd_tflops": f_fwd / (fwd_avg / 1e3) / 1e12,
+        "bwd_tflops": f_bwd / (bwd_avg / 1e3) / 1e12,
+        "fwd_ms": fwd_avg, "bwd_ms": bwd_avg, "bwd_main_kernel_ms": main_avg,
+        "roofline": {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_kind": f"bf16_tflops_sustained ({peak_src})",
+                     "peak_burst": peak_burst, "frac_of_burst": achieved / peak_burst,
+                     "traffic": profiled_traffic(kname)},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": K_e2e},
+        "gpu_launches": K * 4,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops, times, cores = cpu_oracle_sample(1, CPU_SAMPLE_TOKENS)
+        cpu_v = flops / times[0] / 1e12
+        line["cpu_baseline"] = {"value": cpu_v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": cpu_sample_desc(CPU_SAMPLE_TOKENS), "seconds": times[0]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-small", action="store_true",
+                    help="run only the warm-up steps on a smaller case (B=1, N=4096) for ncu captures")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

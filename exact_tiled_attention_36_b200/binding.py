@@ -38,6 +38,7 @@ _SIGS = {
     "fa_get_last_device_error": ([_P], _I),
     "fa_get_last_device_error_site": ([], _I),
     "fa_version": ([], ctypes.c_char_p),
+    "fa_bwd_set_timing_events": ([_P, _P], None),
 }
 
 
@@ -92,6 +93,10 @@ def fa_get_last_device_error(stream) -> int:
 
 def fa_get_last_device_error_site() -> int:
     return lib().fa_get_last_device_error_site()
+
+
+def fa_bwd_set_timing_events(before, after) -> None:
+    lib().fa_bwd_set_timing_events(before, after)
 
 
 def fa_version() -> str:

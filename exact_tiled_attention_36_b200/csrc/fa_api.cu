@@ -20,6 +20,7 @@ namespace {
 
 __device__ int g_fa_error = 0;  // first timeout site of any kernel (0 = none)
 int g_last_site = 0;
+cudaEvent_t g_bwd_ev_before = nullptr, g_bwd_ev_after = nullptr;  // fa_bwd_set_timing_events
 
 constexpr float kLog2e = 1.4426950408889634074f;
 
@@ -281,9 +282,12 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
         a.scale_log2 = scale * kLog2e;
         a.err = err;
         dim3 grid((Nk + 127) / 128, Hkv, B);
+        const bool timed = g_bwd_ev_before && g_bwd_ev_after;
+        if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;
         st = d == 64 ? launch_bwd_d<64>(bf16, causal != 0, mq, mk, mv, mdo, a, grid, s)
                      : launch_bwd_d<128>(bf16, causal != 0, mq, mk, mv, mdo, a, grid, s);
         if (st != FA_OK) return st;
+        if (timed && cudaEventRecord(g_bwd_ev_after, s) != cudaSuccess) return FA_ERR_CUDA;
     }
     if (rows > 0) {
         const size_t n8 = rows * d / 8;
@@ -306,6 +310,11 @@ fa_status fa_get_last_device_error(fa_stream_t stream) {
 }
 
 int fa_get_last_device_error_site(void) { return g_last_site; }
+
+void fa_bwd_set_timing_events(void* before, void* after) {
+    g_bwd_ev_before = static_cast<cudaEvent_t>(before);
+    g_bwd_ev_after = static_cast<cudaEvent_t>(after);
+}
 
 }  // extern "C"
 

@@ -126,6 +126,16 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int B, int Hq, int Hkv, int Nq, int Nk, int d,
                  float scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
+/*
+ * Profiling aid: when `before` and `after` are both non-NULL CUDA event
+ * handles (cudaEvent_t), every later fa_bwd call records `before` on its
+ * stream right before it launches its main kernel and `after` right after,
+ * so a caller can time that kernel alone with cudaEventElapsedTime. Passing
+ * NULL turns it off. The setting is process-wide and not synchronised
+ * between host threads; the events must stay valid while it is set.
+ */
+void fa_bwd_set_timing_events(void* before, void* after);
+
 /* A static description of a status code. Never NULL. */
 const char* fa_status_string(fa_status s);
 
