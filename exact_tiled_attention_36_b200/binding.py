@@ -39,6 +39,7 @@ _SIGS = {
     "fa_get_last_device_error_site": ([], _I),
     "fa_version": ([], ctypes.c_char_p),
     "fa_bwd_set_timing_events": ([_P, _P], None),
+    "fa_bwd_noalloc": ([_P] * 9 + [_I] * 6 + [_F, _I, _I, _P], _I),
 }
 
 
@@ -81,6 +82,12 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, 
            stream) -> int:
     return lib().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal,
                         dtype, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    """fa_bwd with the library's own fixed-size workspace (for callers that cannot allocate)."""
+    return lib().fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype,
+                                stream)
 
 
 def fa_status_string(s: int) -> str:

@@ -2,8 +2,8 @@
 
     python -m exact_tiled_attention_36_b200.build
 
-Compiles csrc/fa_api.cu (which includes the kernel headers) into
-exact_tiled_attention_36_b200/libfa.so, with the CUDA runtime linked
+Compiles csrc/fa_api.cu (which includes the kernel headers) and
+csrc/fa_noalloc.cu into exact_tiled_attention_36_b200/libfa.so, with the CUDA runtime linked
 statically so the library loads on a machine without a GPU driver (the
 driver is reached at run time through the runtime's entry-point query).
 """
@@ -15,7 +15,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "csrc", "fa_api.cu")
+SRCS = [os.path.join(HERE, "csrc", "fa_api.cu"), os.path.join(HERE, "csrc", "fa_noalloc.cu")]
 DEPS = [os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))] + \
        [os.path.join(ROOT, "include", "fa.h")]
 LIB = os.path.join(HERE, "libfa.so")
@@ -35,7 +35,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         return LIB
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [NVCC, *FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc"),
-           SRC, "-o", tmp]
+           *SRCS, "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)

@@ -127,6 +127,36 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  float scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * Backward without a caller-provided workspace. This entry point has no
+ * counterpart in the pages; it exists for callers that cannot allocate
+ * device memory themselves (a host framework that owns every allocation,
+ * a loop that must not pay for cudaMalloc's device-wide synchronisation, a
+ * plugin with a fixed memory budget).
+ *
+ * Same arguments, results and errors as fa_bwd, minus `workspace`: the
+ * workspace is a device array of FA_BWD_NOALLOC_MAX_BYTES bytes inside the
+ * library, which every GPU that loads this part of the library keeps until
+ * the process exits. Nothing is allocated per call: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *   - Sizes whose fa_bwd_workspace_size(B, Hq, Nq, d) exceeds
+ *     FA_BWD_NOALLOC_MAX_BYTES are rejected with FA_ERR_UNSUPPORTED before
+ *     anything runs (with d = 128: B * Hq * Nq up to about 130,000 rows).
+ *   - The first call on a device looks up the array's device address (a
+ *     one-time set-up per device, done with that device current); make that
+ *     first call before any stream capture.
+ *   - All calls share the one array: calls whose work overlaps on the GPU
+ *     (different streams, or different host threads, without ordering
+ *     between them) race on it and give wrong gradients. Calls ordered on
+ *     one stream are safe; each call re-initialises what it reads.
+ */
+#define FA_BWD_NOALLOC_MAX_BYTES (64u << 20)
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Profiling aid: when `before` and `after` are both non-NULL CUDA event
  * handles (cudaEvent_t), every later fa_bwd call records `before` on its
  * stream right before it launches its main kernel and `after` right after,
