@@ -140,6 +140,28 @@ class ClockSampler:
 BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 
 
+# ----------------------------------------------------------------------------- multi-rank plumbing
+def rank_seed(base_seed, rank):
+    """Each rank draws its own batch: independent replicas of the workload."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(x, world, device):
+    """The largest of every rank's `x` (the job's time is its slowest rank's)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world, flops_per_step, steps, max_ms):
+    """Whole-job throughput: every rank's FLOPs over the slowest rank's time."""
+    return world * flops_per_step * steps / (max_ms / 1e3) / 1e12
+
+
 # ----------------------------------------------------------------------------- CPU oracle (reference arm)
 def cpu_oracle_sample(n_steps, tokens):
     """Time the fp64 oracle (fwd + bwd) on the bounded sample, n_steps times."""
@@ -210,12 +232,6 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     fb.lib()
     w = dict(WORKLOAD)
@@ -223,7 +239,7 @@ def run_ours(args):
         w.update(PROFILE_CASE)
     cfg = inputs.CAUSAL_GQA
     # each rank draws its own batch (independent replicas of the workload)
-    fi = inputs.make_fixed(cfg, seed=cfg.seed + 1000 * rank, B=w["B"], Nq=w["N"], Nk=w["N"])
+    fi = inputs.make_fixed(cfg, seed=rank_seed(cfg.seed, rank), B=w["B"], Nq=w["N"], Nk=w["N"])
     B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
     scale = d ** -0.5
     dt = fb.FA_BF16
@@ -308,7 +324,7 @@ def run_ours(args):
     total_ms, fwd_ms, bwd_ms, bwd_main_ms = result
     if fb.fa_get_last_device_error(None) != fb.FA_OK:
         raise RuntimeError("device error during the timed region")
-    total_ms = max_over_ranks(total_ms)
+    total_ms = max_over_ranks(total_ms, world, "cuda")
 
     # end to end through the C ABI with host buffers: H2D of q, k, v, dO from
     # pinned memory, fwd + bwd, D2H of dq, dk, dv, every step.
@@ -341,11 +357,11 @@ def run_ours(args):
     s1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(s0.elapsed_time(s1))
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1), world, "cuda")
 
     peaks, peak_src = load_peaks()
-    value = world * f_step * K / (total_ms / 1e3) / 1e12
-    e2e_value = world * f_step * K_e2e / (e2e_ms / 1e3) / 1e12
+    value = job_tflops(world, f_step, K, total_ms)
+    e2e_value = job_tflops(world, f_step, K_e2e, e2e_ms)
     fwd_avg = statistics.mean(fwd_ms)
     bwd_avg = statistics.mean(bwd_ms)
     main_avg = statistics.mean(bwd_main_ms)

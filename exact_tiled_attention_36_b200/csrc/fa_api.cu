@@ -178,7 +178,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     a.Nk = Nk;
     a.scale_log2 = scale * kLog2e;
     a.err = err;
-    dim3 grid((Nq + 127) / 128, Hq, B);
+    const unsigned nqt = static_cast<unsigned>((Nq + 127) / 128);
+    if (nqt > 65535u) return FA_ERR_UNSUPPORTED;
+    const dim3 grid = causal ? dim3(Hq, B, nqt) : dim3(nqt, Hq, B);
     return launch_fwd(d, bf16, causal != 0, false, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -219,7 +221,9 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
     a.Nk = max_seqlen_k;
     a.scale_log2 = scale * kLog2e;
     a.err = err;
-    dim3 grid((max_seqlen_q + 127) / 128, Hq, num_seqs);
+    const unsigned nqt = static_cast<unsigned>((max_seqlen_q + 127) / 128);
+    if (nqt > 65535u) return FA_ERR_UNSUPPORTED;
+    const dim3 grid = causal ? dim3(Hq, num_seqs, nqt) : dim3(nqt, Hq, num_seqs);
     return launch_fwd(d, bf16, causal != 0, true, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -281,7 +285,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
         a.scale = scale;
         a.scale_log2 = scale * kLog2e;
         a.err = err;
-        dim3 grid((Nk + 127) / 128, Hkv, B);
+        const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
+        if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
+        const dim3 grid = causal ? dim3(Hkv, B, nkt) : dim3(nkt, Hkv, B);
         const bool timed = g_bwd_ev_before && g_bwd_ev_after;
         if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;
         st = d == 64 ? launch_bwd_d<64>(bf16, causal != 0, mq, mk, mv, mdo, a, grid, s)

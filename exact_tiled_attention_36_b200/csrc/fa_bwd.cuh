@@ -81,9 +81,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     if (!smem_base_ok(smem, args.err)) return;  // the 128-byte swizzle needs 1024-byte aligned tiles
 
-    const int kt = blockIdx.x;  // key tile
-    const int hk = blockIdx.y;
-    const int b = blockIdx.z;
+    // Non-causal grid (key tiles, Hkv, batches); causal grid (Hkv, batches, key
+    // tiles) so that the first key tiles, which see the most query tiles, are
+    // dispatched first.
+    const int kt = CAUSAL ? static_cast<int>(blockIdx.z) : static_cast<int>(blockIdx.x);
+    const int hk = CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
+    const int b = CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
     const int k0 = kt * 128;
     const int Nq = args.Nq, Nk = args.Nk;
     const int n_qt = (Nq + 127) / 128;

@@ -19,7 +19,8 @@
 //               row of S_j, masks, takes the row max, forms
 //               P = 2^(S * scale * log2 e - m) with the scale folded into one
 //               FFMA, writes P as 16-bit pairs over the first half of the same
-//               TMEM columns, keeps l, rescales its O row in TMEM when m has
+//               TMEM columns, keeps l (for L) and the sum of the rounded P
+//               (which normalises O), rescales its O row in TMEM when m has
 //               grown by more than 2^8 since the last rescale (exact: O and l
 //               share the stale reference max), and finally writes O / l and L.
 //   warps 2-3   idle.
@@ -87,9 +88,13 @@ __global__ void __launch_bounds__(256, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     if (!smem_base_ok(smem, args.err)) return;  // the 128-byte swizzle needs 1024-byte aligned tiles
 
-    const int h = blockIdx.y;
-    const int bidx = blockIdx.z;
-    const int q_tile = CAUSAL ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
+    // Non-causal grid (q tiles, Hq, batches): neighbouring CTAs share K/V in L2.
+    // Causal grid (Hq, batches, q tiles), the last query tile first: CTAs are
+    // dispatched heaviest first (longest-processing-time order), so the long
+    // tiles do not start in the last wave.
+    const int h = CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
+    const int bidx = CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
+    const int q_tile = CAUSAL ? static_cast<int>(gridDim.z - 1 - blockIdx.z) : static_cast<int>(blockIdx.x);
     const int q0 = q_tile * 128;
 
     int q_len, k_len, q_row0, k_row0, tma_b;
@@ -289,7 +294,7 @@ __global__ void __launch_bounds__(256, 1)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
         const int row_limit = CAUSAL ? min(k_len, q + k_len - q_len + 1) : k_len;
         const float sl2 = args.scale_log2;
-        float m = -INFINITY, l = 0.f;
+        float m = -INFINITY, l = 0.f, lr = 0.f;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
             ok = warp_all(mbar_wait(&s_full[j & 1], (j >> 1) & 1, wc, 7));
@@ -325,14 +330,22 @@ __global__ void __launch_bounds__(256, 1)
                 m = m_new;
             }
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            float rs = 0.f;
+            // P is rounded to 16 bits for the P V product. l (exact fp32 sum)
+            // gives L; lr, the sum of the ROUNDED values, normalises O, so the
+            // weights applied to V sum to exactly one.
+            float rs = 0.f, rsr = 0.f;
+            uint32_t pk[2][32];
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                const float p = ex2_approx(fmaf(__uint_as_float(s[c >> 5][c & 31]), sl2, neg_m));
-                rs += p;
-                s[c >> 5][c & 31] = __float_as_uint(p);
+            for (int i = 0; i < 64; ++i) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(s[(2 * i) >> 5][(2 * i) & 31]), sl2, neg_m));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(s[(2 * i + 1) >> 5][(2 * i + 1) & 31]), sl2, neg_m));
+                rs += p0 + p1;
+                const uint32_t u = pack2<BF16>(p0, p1);
+                rsr += unpack_lo<BF16>(u) + unpack_hi<BF16>(u);
+                pk[i >> 5][i & 31] = u;
             }
             l = l * alpha + rs;
+            lr = lr * alpha + rsr;
             if (j > 0 && __any_sync(0xffffffffu, resc)) {
                 ok = warp_all(mbar_wait(o_done, (j - 1) & 1, wc, 8));
                 if (!ok) break;
@@ -348,11 +361,6 @@ __global__ void __launch_bounds__(256, 1)
                 }
                 tmem_st_wait();
             }
-            uint32_t pk[2][32];
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-                pk[i >> 5][i & 31] = pack2<BF16>(__uint_as_float(s[(2 * i) >> 5][(2 * i) & 31]),
-                                                 __uint_as_float(s[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
             tmem_st32(s_addr + 0, pk[0]);
             tmem_st32(s_addr + 32, pk[1]);
             tmem_st_wait();
@@ -365,7 +373,7 @@ __global__ void __launch_bounds__(256, 1)
         if (ok) {
             tc_fence_after();
             const bool row_ok = row_valid(q);
-            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+            const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
             T16* dst = row_ok ? o_row(q) : nullptr;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {

@@ -288,4 +288,26 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return r;
 }
 
+// The element of a packed 16-bit pair as fp32 (exact).
+template <bool BF16>
+__device__ __forceinline__ float unpack_lo(uint32_t u) {
+    if constexpr (BF16) {
+        return __uint_as_float(u << 16);
+    } else {
+        float f;
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, lo;\n\t}" : "=f"(f) : "r"(u));
+        return f;
+    }
+}
+template <bool BF16>
+__device__ __forceinline__ float unpack_hi(uint32_t u) {
+    if constexpr (BF16) {
+        return __uint_as_float(u & 0xFFFF0000u);
+    } else {
+        float f;
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, hi;\n\t}" : "=f"(f) : "r"(u));
+        return f;
+    }
+}
+
 }  // namespace fa

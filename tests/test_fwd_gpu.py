@@ -6,7 +6,7 @@ import torch
 import oracle
 from exact_tiled_attention_36_b200 import binding as fb
 from exact_tiled_attention_36_b200 import inputs
-from tests.gpu_util import ATOL_L, ATOL_O, f64, guarded
+from tests.gpu_util import ATOL_L, f64, guarded, o_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -37,6 +37,7 @@ def run_fwd(fi, causal, scale=None, guard=True):
 
 
 def check(o, lse, o_ref, lse_ref, rows=None):
+    dtype = o.dtype
     o, lse = f64(o), f64(lse)
     if rows is not None:
         o, lse, o_ref, lse_ref = o[:, rows], lse[:, :, rows], o_ref[:, rows], lse_ref[:, :, rows]
@@ -44,9 +45,10 @@ def check(o, lse, o_ref, lse_ref, rows=None):
     assert np.isneginf(lse[empty]).all() and (o.transpose(0, 2, 1, 3)[empty] == 0).all()
     live = ~empty
     err_l = np.abs(lse[live] - lse_ref[live]).max() if live.any() else 0.0
-    err_o = np.abs(o - o_ref).max()
-    assert err_o <= ATOL_O and err_l <= ATOL_L, (err_o, err_l)
-    return err_o, err_l
+    err = np.abs(o - o_ref)
+    excess = (err - o_bound(o_ref, dtype)).max()
+    assert excess <= 0 and err_l <= ATOL_L, (err.max(), excess, err_l)
+    return err.max(), err_l
 
 
 SMALL = [
@@ -98,5 +100,7 @@ def test_fwd_full_size_sampled_rows(cfg):
     fi = inputs.make_fixed(cfg, with_do=False)
     o, lse = run_fwd(fi, cfg.causal, cfg.scale)
     rows = sample_rows(cfg.Nq, 24, cfg.seed)
+    if cfg.causal:  # the first rows see few keys: the largest |O| and the hardest rows for 16-bit P and O
+        rows = sorted(set(rows) | set(range(256)))
     o_ref, lse_ref = oracle.attn_fwd(fi.q, fi.k, fi.v, cfg.scale, cfg.causal, rows=rows)
     check(o, lse, o_ref, lse_ref, rows)
