@@ -15,6 +15,7 @@
 #include "fa.h"
 #include "fa_fwd.cuh"
 #include "fa_bwd.cuh"
+#include "fa_bwd_pp.cuh"
 
 namespace {
 
@@ -113,11 +114,13 @@ fa_status launch_fwd(int d, bool bf16, bool causal, bool varlen, const CUtensorM
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// d = 128 runs the two-sub-tile ping-pong kernel; d = 64 the single-tile one
+// (its dQ^T would need M = 64, so it keeps dQ = dS K with M = 128 queries).
 template <int D, bool BF16, bool CAUSAL>
 fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const fa::BwdArgs& a, dim3 grid, cudaStream_t stream) {
-    auto kern = fa::fa_bwd_kernel<D, BF16, CAUSAL>;
-    constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
+    auto kern = D == 128 ? fa::fa_bwd_pp_kernel<BF16, CAUSAL> : fa::fa_bwd_kernel<D, BF16, CAUSAL>;
+    constexpr int smem = D == 128 ? fa::BwdPPCfg::kSmemBytes : fa::BwdCfg<D>::kSmemBytes;
     static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
     if (!attr_ok) return FA_ERR_CUDA;
     kern<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, a);
