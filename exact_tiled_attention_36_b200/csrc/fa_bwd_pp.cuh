@@ -241,34 +241,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int qlim = key - (Nk - Nq);  // smallest query that sees this key
         const float sl2 = args.scale_log2;
         constexpr float kLog2eF = 1.4426950408889634074f;
+        // L (log2 units) and D of query qs + r, loaded one iteration ahead so the
+        // global-load latency overlaps the previous sub-tile's work.
+        auto load_ld = [&](int it_, float& l2, float& dd) {
+            l2 = INFINITY;
+            dd = 0.f;
+            if (r < 64 && it_ < n_it) {
+                const int q = (i0 + it_ % n_i) * 128 + t * 64 + r;
+                if (q < Nq) {
+                    const size_t row = (static_cast<size_t>(b) * args.Hq + hk * args.group + it_ / n_i) * Nq + q;
+                    const float L = __ldg(args.lse + row);
+                    l2 = (L == -INFINITY) ? INFINITY : L * kLog2eF;  // a row that saw no key has P = 0
+                    dd = __ldg(args.D + row);
+                }
+            }
+        };
+        float next_l2, next_dd;
+        load_ld(0, next_l2, next_dd);
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int h = hk * args.group + it / n_i;
             const int qs = (i0 + it % n_i) * 128 + t * 64;  // first query of this sub-tile
-            // L (log2 units) and D of the sub-tile's 64 queries. Buffer (t, it & 1)
-            // is rewritten at it + 2, when every thread of this warpgroup has
-            // arrived on ds_ready for it + 1.
+            // Buffer (t, it & 1) is rewritten at it + 2, when every thread of this
+            // warpgroup has arrived on ds_ready for it + 1.
             float* sL = sLD + (t * 2 + (it & 1)) * 128;
             float* sD = sL + 64;
             if (r < 64) {
-                const int q = qs + r;
-                float l2 = INFINITY, dd = 0.f;
-                if (q < Nq) {
-                    const size_t row = (static_cast<size_t>(b) * args.Hq + h) * Nq + q;
-                    const float L = args.lse[row];
-                    l2 = (L == -INFINITY) ? INFINITY : L * kLog2eF;  // a row that saw no key has P = 0
-                    dd = args.D[row];
-                }
-                sL[r] = l2;
-                sD[r] = dd;
+                sL[r] = next_l2;
+                sD[r] = next_dd;
                 mbar_arrive(&ld_full[t * 2 + (it & 1)]);
             }
+            load_ld(it + 1, next_l2, next_dd);
             ok = warp_all(mbar_wait(&ld_full[t * 2 + (it & 1)], (it >> 1) & 1, wc, 47));
             if (!ok) break;
             ok = warp_all(mbar_wait(&s_full[t], it & 1, wc, 48));
             if (!ok) break;
             tc_fence_after();
             uint8_t* ds_rows = sDS + t * C::kSlabBytes + (r >> 3) * 1024 + (r & 7) * 128;
+            // Masks matter only on the tile holding key Nk - 1 and, under the causal
+            // mask, on sub-tiles that reach below the diagonal (uniform per sub-tile).
+            const bool need_mask = (k0 + 128 > Nk) || (CAUSAL && qs < k0 + 127 - (Nk - Nq));
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 uint32_t sv[32], pv[32];
@@ -278,19 +290,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld_wait(pv);
                 uint32_t pk[16], dk16[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float p[2], ds[2];
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(sL + cc * 32 + e);
+                    const float4 d4 = *reinterpret_cast<const float4*>(sD + cc * 32 + e);
+                    const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dq[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float p[4], ds[4];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int qq = cc * 32 + e + u;
-                        bool vis = key_ok;
-                        if (CAUSAL) vis = vis && (qs + qq >= qlim);
-                        const float pe = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl2, -sL[qq]));
-                        p[u] = vis ? pe : 0.f;
-                        ds[u] = p[u] * (__uint_as_float(pv[e + u]) - sD[qq]);
+                    for (int u = 0; u < 4; ++u) {
+                        p[u] = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl2, -lq[u]));
+                        if (need_mask) {
+                            bool vis = key_ok;
+                            if (CAUSAL) vis = vis && (qs + cc * 32 + e + u >= qlim);
+                            p[u] = vis ? p[u] : 0.f;
+                        }
+                        ds[u] = p[u] * (__uint_as_float(pv[e + u]) - dq[u]);
                     }
                     pk[e >> 1] = pack2<BF16>(p[0], p[1]);
+                    pk[(e >> 1) + 1] = pack2<BF16>(p[2], p[3]);
                     dk16[e >> 1] = pack2<BF16>(ds[0], ds[1]);
+                    dk16[(e >> 1) + 1] = pack2<BF16>(ds[2], ds[3]);
                 }
                 // 16-bit pairs over columns this thread has already read (query 32 cc + e
                 // lands in column 16 cc + e / 2 of the sub-tile's region).
@@ -313,17 +332,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             ok = warp_all(mbar_wait(&dq_full[t], it & 1, wc, 49));
             if (!ok) break;
             tc_fence_after();
-            float* dst = args.dq_acc + (static_cast<size_t>(b) * Nq * args.Hq + h) * D + r;
             const size_t qstride = static_cast<size_t>(args.Hq) * D;
+            float* dst = args.dq_acc + (static_cast<size_t>(b) * Nq * args.Hq + h) * D + r +
+                         static_cast<size_t>(qs) * qstride;
+            const int q_end = Nq - qs;  // queries qs + c with c >= q_end do not exist
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 uint32_t v[32];
                 tmem_ld32(lane_base + C::kColS + t * 64 + cc * 32, v);
                 tmem_ld_wait(v);
+                if (q_end >= 64) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int q = qs + cc * 32 + c;
-                    if (q < Nq) red_add_f32(dst + static_cast<size_t>(q) * qstride, __uint_as_float(v[c]));
+                    for (int c = 0; c < 32; ++c) {
+                        red_add_f32(dst, __uint_as_float(v[c]));
+                        dst += qstride;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        if (cc * 32 + c < q_end) red_add_f32(dst, __uint_as_float(v[c]));
+                        dst += qstride;
+                    }
                 }
             }
             tc_fence_before();
