@@ -316,9 +316,18 @@ __global__ void __launch_bounds__(256, 1)
                 for (int c = 0; c < 128; ++c)
                     if (c >= lim) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
-            float mx = -INFINITY;
+            // Row max as 16 independent partial maxima (a single chain of 128
+            // dependent max operations would expose its whole latency).
+            float mxp[16];
 #pragma unroll
-            for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c >> 5][c & 31]));
+            for (int i = 0; i < 16; ++i) mxp[i] = __uint_as_float(s[i >> 5][i & 31]);
+#pragma unroll
+            for (int c = 16; c < 128; ++c) mxp[c & 15] = fmaxf(mxp[c & 15], __uint_as_float(s[c >> 5][c & 31]));
+#pragma unroll
+            for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+                for (int i = 0; i < w; ++i) mxp[i] = fmaxf(mxp[i], mxp[i + w]);
+            const float mx = mxp[0];
             const float m_new = fmaxf(m, mx * sl2);
             float alpha = 1.f;
             bool resc = false;
@@ -333,17 +342,19 @@ __global__ void __launch_bounds__(256, 1)
             // P is rounded to 16 bits for the P V product. l (exact fp32 sum)
             // gives L; lr, the sum of the ROUNDED values, normalises O, so the
             // weights applied to V sum to exactly one.
-            float rs = 0.f, rsr = 0.f;
+            float rsp[4] = {0.f, 0.f, 0.f, 0.f}, rsrp[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums
             uint32_t pk[2][32];
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
                 const float p0 = ex2_approx(fmaf(__uint_as_float(s[(2 * i) >> 5][(2 * i) & 31]), sl2, neg_m));
                 const float p1 = ex2_approx(fmaf(__uint_as_float(s[(2 * i + 1) >> 5][(2 * i + 1) & 31]), sl2, neg_m));
-                rs += p0 + p1;
+                rsp[i & 3] += p0 + p1;
                 const uint32_t u = pack2<BF16>(p0, p1);
-                rsr += unpack_lo<BF16>(u) + unpack_hi<BF16>(u);
+                rsrp[i & 3] += unpack_lo<BF16>(u) + unpack_hi<BF16>(u);
                 pk[i >> 5][i & 31] = u;
             }
+            const float rs = (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
+            const float rsr = (rsrp[0] + rsrp[1]) + (rsrp[2] + rsrp[3]);
             l = l * alpha + rs;
             lr = lr * alpha + rsr;
             if (j > 0 && __any_sync(0xffffffffu, resc)) {
