@@ -14,6 +14,7 @@
 
 #include "fa.h"
 #include "fa_fwd.cuh"
+#include "fa_fwd2.cuh"
 #include "fa_bwd.cuh"
 #include "fa_bwd_pp.cuh"
 
@@ -83,11 +84,19 @@ fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtyp
 template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                        dim3 grid, cudaStream_t stream) {
-    auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, VARLEN>;
-    constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
+    auto kern = fa::fa_fwd2_kernel<D, BF16, CAUSAL, VARLEN>;
+    constexpr int smem = fa::Fwd2Cfg<D>::kSmemBytes;
     static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
     if (!attr_ok) return FA_ERR_CUDA;
-    kern<<<grid, 256, smem, stream>>>(mq, mk, mv, a);
+    // The kernel moves registers between warpgroups with setmaxnreg; the split
+    // must fit the pool the CTA is launched with, or the increase would wait
+    // for registers that never come.
+    static int launch_regs = [&] {
+        cudaFuncAttributes fa_attr{};
+        return cudaFuncGetAttributes(&fa_attr, kern) == cudaSuccess ? fa_attr.numRegs : 0;
+    }();
+    if (launch_regs < fa::kFwd2MinLaunchRegs) return FA_ERR_UNSUPPORTED;
+    kern<<<grid, fa::kFwd2Threads, smem, stream>>>(mq, mk, mv, a);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -181,7 +190,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     a.Nk = Nk;
     a.scale_log2 = scale * kLog2e;
     a.err = err;
-    const unsigned nqt = static_cast<unsigned>((Nq + 127) / 128);
+    const unsigned nqt = static_cast<unsigned>((Nq + 255) / 256);  // 256-row units (two query tiles)
     if (nqt > 65535u) return FA_ERR_UNSUPPORTED;
     const dim3 grid = causal ? dim3(Hq, B, nqt) : dim3(nqt, Hq, B);
     return launch_fwd(d, bf16, causal != 0, false, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
@@ -224,7 +233,7 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
     a.Nk = max_seqlen_k;
     a.scale_log2 = scale * kLog2e;
     a.err = err;
-    const unsigned nqt = static_cast<unsigned>((max_seqlen_q + 127) / 128);
+    const unsigned nqt = static_cast<unsigned>((max_seqlen_q + 255) / 256);
     if (nqt > 65535u) return FA_ERR_UNSUPPORTED;
     const dim3 grid = causal ? dim3(Hq, num_seqs, nqt) : dim3(nqt, Hq, num_seqs);
     return launch_fwd(d, bf16, causal != 0, true, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));

@@ -80,7 +80,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s without progress
 // Wait for the phase with parity `parity` of `bar` to complete. Returns false
 // (and marks the CTA aborted) after kWaitLimitNs, or at once if another wait of
 // the CTA has already given up. `site` identifies the wait in the error word.
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, WaitCtx ctx, int site) {
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, WaitCtx ctx, int site) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -265,6 +265,17 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Register reallocation between warpgroups (all warps of a warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------------------
