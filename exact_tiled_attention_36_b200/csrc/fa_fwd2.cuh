@@ -327,17 +327,16 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                 for (int c = 0; c < 128; ++c)
                     if (c >= lim) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
-            // Row max as 16 independent partial maxima.
-            float mxp[16];
+            // Row max: 8 independent chains of three-input max.
+            float mxp[8];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) mxp[i] = __uint_as_float(sv[i >> 5][i & 31]);
+            for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
 #pragma unroll
-            for (int c = 16; c < 128; ++c) mxp[c & 15] = fmaxf(mxp[c & 15], __uint_as_float(sv[c >> 5][c & 31]));
-#pragma unroll
-            for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-                for (int i = 0; i < w; ++i) mxp[i] = fmaxf(mxp[i], mxp[i + w]);
-            const float m_new = fmaxf(m, mxp[0] * sl2);
+            for (int i = 0; i < 64; ++i)
+                mxp[i & 7] = fmax3(mxp[i & 7], __uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
+                                   __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
+            const float mx = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
+            const float m_new = fmaxf(m, mx * sl2);
             float alpha = 1.f;
             bool resc = false;
             if (m_new > m + kRescaleThreshold) {  // false while the row has seen no key
@@ -350,21 +349,27 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
             // P = 2^(S c - m) as 16-bit pairs (keys 2i, 2i + 1 in column i), partial sums
             // of the exact and of the rounded values.
-            float rsp[4] = {0.f, 0.f, 0.f, 0.f}, rsrp[4] = {0.f, 0.f, 0.f, 0.f};
+            // Pairs of keys go through the packed f32x2 FMA and adds.
+            const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(neg_m, neg_m);
+            uint64_t rs2[4] = {0, 0, 0, 0}, rsr2[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
             uint32_t pk[2][32];
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]), sl2, neg_m));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]), sl2, neg_m));
-                rsp[i & 3] += p0 + p1;
+                const uint64_t x = f2_pack(__uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
+                                           __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
+                float y0, y1;
+                f2_unpack(f2_fma(x, c2, m2), y0, y1);
+                const float p0 = ex2_approx(y0);
+                const float p1 = ex2_approx(y1);
+                rs2[i & 3] = f2_add(rs2[i & 3], f2_pack(p0, p1));
                 const uint32_t u = pack2<BF16>(p0, p1);
-                rsrp[i & 3] += unpack_lo<BF16>(u) + unpack_hi<BF16>(u);
+                rsr2[i & 3] = f2_add(rsr2[i & 3], f2_pack(unpack_lo<BF16>(u), unpack_hi<BF16>(u)));
                 pk[i >> 5][i & 31] = u;
             }
             tmem_st32(s_addr + 0, pk[0]);
             tmem_st32(s_addr + 32, pk[1]);
-            const float rs = (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
-            const float rsr = (rsrp[0] + rsrp[1]) + (rsrp[2] + rsrp[3]);
+            const float rs = f2_sum(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])));
+            const float rsr = f2_sum(f2_add(f2_add(rsr2[0], rsr2[1]), f2_add(rsr2[2], rsr2[3])));
             l = l * alpha + rs;
             lr = lr * alpha + rsr;
             // S_t was issued after the previous key tile's P_t V and MMAs of one thread
