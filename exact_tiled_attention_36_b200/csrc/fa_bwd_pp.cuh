@@ -34,7 +34,7 @@ struct BwdPPCfg {
     static constexpr int kDSOff = kDOOff + 2 * kTileBytes;  // 2 sub-tiles x [128 keys x 64 q] 16-bit
     static constexpr int kLDOff = kDSOff + 2 * kSlabBytes;  // [sub-tile][stage][L2 64 | D 64] fp32
     static constexpr int kBarOff = kLDOff + 2048;
-    static constexpr int kNumBars = 20;
+    static constexpr int kNumBars = 18;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16;
     static constexpr uint32_t kTmemCols = 512;
@@ -100,11 +100,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t* q_empty = bars + 3;    // [2 stages]
     uint64_t* s_full = bars + 5;     // [2 sub-tiles]
     uint64_t* ds_ready = bars + 7;   // [2]
-    uint64_t* dvdk = bars + 9;       // [2]
-    uint64_t* dq_full = bars + 11;   // [2]
-    uint64_t* dq_free = bars + 13;   // [2]
-    uint64_t* ld_full = bars + 15;   // [sub-tile * 2 + stage]
-    uint64_t* fin = bars + 19;
+    uint64_t* dq_full = bars + 9;    // [2]
+    uint64_t* dq_free = bars + 11;   // [2]
+    uint64_t* ld_full = bars + 13;   // [sub-tile * 2 + stage]
+    uint64_t* fin = bars + 17;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     int* abort_flag = reinterpret_cast<int*>(smem + C::kMiscOff + 4);
 
@@ -115,7 +114,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&q_empty[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&ds_ready[i], 128);
-            mbar_init(&dvdk[i], 1);
             mbar_init(&dq_full[i], 1);
             mbar_init(&dq_free[i], 128);
         }
@@ -200,9 +198,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tc_commit(&s_full[t]);
                 }
                 if (!ok) break;
-                // dV, dK from P^T_t / dS^T_t, then dQ^T_t once those reads are done
-                // (dQ^T_t overwrites P^T_t's columns; different accumulators are not
-                // ordered by the hardware, so wait for the commit).
+                // dV, dK from P^T_t / dS^T_t, then dQ^T_t into P^T_t's columns right
+                // behind them: tcgen05.mma operations of one thread execute in issue
+                // order, so dQ^T_t cannot overwrite P^T_t before dV has read it (the
+                // same holds for the next dP^T_t over dS^T_t).
                 for (int t = 0; ok && t < 2; ++t) {
                     if (!(ok = mbar_wait(&ds_ready[t], it & 1, wc, 45))) break;
                     tc_fence_after();
@@ -216,8 +215,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         mma_ts(tmem + C::kColDK, tmem + C::kColDP + t * 64 + kk * 8,
                                sdesc_sw128(q_addr + t * 8192 + kk * 2048, C::kSlabBytes, 1024), id_tm,
                                (it > 0 || t > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(&dvdk[t]);
-                    if (!(ok = mbar_wait(&dvdk[t], it & 1, wc, 46))) break;
                     const uint32_t ds_addr = smem_u32(sDS + t * C::kSlabBytes);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
@@ -243,16 +240,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         constexpr float kLog2eF = 1.4426950408889634074f;
         // L (log2 units) and D of query qs + r, loaded one iteration ahead so the
         // global-load latency overlaps the previous sub-tile's work.
+        // Stored negated: -L log2 e (so P = 2^(S c + that) is one FMA and an exp) and -D.
         auto load_ld = [&](int it_, float& l2, float& dd) {
-            l2 = INFINITY;
+            l2 = -INFINITY;
             dd = 0.f;
             if (r < 64 && it_ < n_it) {
                 const int q = (i0 + it_ % n_i) * 128 + t * 64 + r;
                 if (q < Nq) {
                     const size_t row = (static_cast<size_t>(b) * args.Hq + hk * args.group + it_ / n_i) * Nq + q;
                     const float L = __ldg(args.lse + row);
-                    l2 = (L == -INFINITY) ? INFINITY : L * kLog2eF;  // a row that saw no key has P = 0
-                    dd = __ldg(args.D + row);
+                    l2 = (L == -INFINITY) ? -INFINITY : -L * kLog2eF;  // a row that saw no key has P = 0
+                    dd = -__ldg(args.D + row);
                 }
             }
         };
@@ -281,6 +279,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // Masks matter only on the tile holding key Nk - 1 and, under the causal
             // mask, on sub-tiles that reach below the diagonal (uniform per sub-tile).
             const bool need_mask = (k0 + 128 > Nk) || (CAUSAL && qs < k0 + 127 - (Nk - Nq));
+            const uint64_t c2 = f2_pack(sl2, sl2);
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 uint32_t sv[32], pv[32];
@@ -291,20 +290,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 uint32_t pk[16], dk16[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4*>(sL + cc * 32 + e);
-                    const float4 d4 = *reinterpret_cast<const float4*>(sD + cc * 32 + e);
-                    const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dq[4] = {d4.x, d4.y, d4.z, d4.w};
+                    // pairs of queries through the packed f32x2 FMA, add and multiply
+                    const ulonglong2 nl = *reinterpret_cast<const ulonglong2*>(sL + cc * 32 + e);
+                    const ulonglong2 nd = *reinterpret_cast<const ulonglong2*>(sD + cc * 32 + e);
                     float p[4], ds[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        p[u] = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl2, -lq[u]));
-                        if (need_mask) {
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int u = e + 2 * h2;
+                        const uint64_t y = f2_fma(f2_pack(__uint_as_float(sv[u]), __uint_as_float(sv[u + 1])), c2,
+                                                  h2 ? nl.y : nl.x);
+                        float y0, y1;
+                        f2_unpack(y, y0, y1);
+                        p[2 * h2] = ex2_approx(y0);
+                        p[2 * h2 + 1] = ex2_approx(y1);
+                    }
+                    if (need_mask) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
                             bool vis = key_ok;
                             if (CAUSAL) vis = vis && (qs + cc * 32 + e + u >= qlim);
                             p[u] = vis ? p[u] : 0.f;
                         }
-                        ds[u] = p[u] * (__uint_as_float(pv[e + u]) - dq[u]);
+                    }
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int u = e + 2 * h2;
+                        const uint64_t dpm = f2_add(f2_pack(__uint_as_float(pv[u]), __uint_as_float(pv[u + 1])),
+                                                    h2 ? nd.y : nd.x);
+                        f2_unpack(f2_mul(f2_pack(p[2 * h2], p[2 * h2 + 1]), dpm), ds[2 * h2], ds[2 * h2 + 1]);
                     }
                     pk[e >> 1] = pack2<BF16>(p[0], p[1]);
                     pk[(e >> 1) + 1] = pack2<BF16>(p[2], p[3]);
