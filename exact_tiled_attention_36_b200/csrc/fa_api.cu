@@ -14,7 +14,6 @@
 
 #include "fa.h"
 #include "fa_fwd.cuh"
-#include "fa_fwd2.cuh"
 #include "fa_bwd.cuh"
 #include "fa_bwd_pp.cuh"
 
@@ -84,8 +83,8 @@ fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtyp
 template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                        dim3 grid, cudaStream_t stream) {
-    auto kern = fa::fa_fwd2_kernel<D, BF16, CAUSAL, VARLEN>;
-    constexpr int smem = fa::Fwd2Cfg<D>::kSmemBytes;
+    auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, VARLEN>;
+    constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
     static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
     if (!attr_ok) return FA_ERR_CUDA;
     // The kernel moves registers between warpgroups with setmaxnreg; the split
@@ -95,8 +94,8 @@ fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
         cudaFuncAttributes fa_attr{};
         return cudaFuncGetAttributes(&fa_attr, kern) == cudaSuccess ? fa_attr.numRegs : 0;
     }();
-    if (launch_regs < fa::kFwd2MinLaunchRegs) return FA_ERR_UNSUPPORTED;
-    kern<<<grid, fa::kFwd2Threads, smem, stream>>>(mq, mk, mv, a);
+    if (launch_regs < fa::kFwdMinLaunchRegs) return FA_ERR_UNSUPPORTED;
+    kern<<<grid, fa::kFwdThreads, smem, stream>>>(mq, mk, mv, a);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -1,31 +1,38 @@
-// fa_fwd.cuh: tiled exact attention forward for sm_100a.
+// fa_fwd.cuh: tiled exact attention forward for sm_100a, two query tiles per CTA.
 //
-// One CTA computes one 128-row query tile Q_i of one (batch, query head) and
-// walks the key/value tiles K_j, V_j of 128 rows with the online softmax
-// ("FlashAttention/zh", section "FlashAttention algorithm"): S_ij = Q_i K_j^T,
-// the running row max m and normaliser l, the rescale of the partial output by
-// exp(m_old - m_new), the final O_i / l_i and L_i = m_i + log l_i. The loop
-// order is query tile outside, key tile inside (the FlashAttention-2 work
-// split on the same page, section "variants").
+// One CTA computes two 128-row query tiles Q_0, Q_1 (rows q0 .. q0 + 255) of one
+// (batch, query head) and walks the key/value tiles K_j, V_j of 128 rows with
+// the online softmax ("FlashAttention/zh", section "FlashAttention algorithm":
+// S_ij = Q_i K_j^T, running row max m and normaliser l, rescale of the partial
+// output by exp(m_old - m_new), final O_i / l_i and L_i = m_i + log l_i), query
+// tiles outside and key tiles inside (the FlashAttention-2 split, section
+// "variants"). Every K/V tile loaded serves both query tiles, and the softmax of
+// one tile overlaps the tensor-core work of the other.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer: Q once, then K_j and V_j into NS-deep rings.
-//   warp 1      allocates TMEM and issues every tcgen05.mma from one thread:
-//               S_j = Q K_j^T into one of two TMEM score buffers (so S_{j+1}
-//               is computed while the softmax works on S_j), and
-//               O += P_j V_j with P_j read from TMEM; S_{j+2} is issued once
-//               P_j V_j has completed, since it reuses P_j's columns.
-//   warps 4-7   softmax: thread t owns query row t = TMEM lane t. It loads its
-//               row of S_j, masks, takes the row max, forms
-//               P = 2^(S * scale * log2 e - m) with the scale folded into one
-//               FFMA, writes P as 16-bit pairs over the first half of the same
-//               TMEM columns, keeps l (for L) and the sum of the rounded P
-//               (which normalises O), rescales its O row in TMEM when m has
-//               grown by more than 2^8 since the last rescale (exact: O and l
-//               share the stale reference max), and finally writes O / l and L.
-//   warps 2-3   idle.
+// Warp roles (384 threads):
+//   warp 0        TMA producer: Q_0, Q_1 once, then K_j, V_j into 2-stage (d = 128)
+//                 or 4-stage (d = 64) mbarrier rings.
+//   warp 1        TMEM allocation and the single MMA-issuing thread. Per key
+//                 tile j it issues O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T,
+//                 O_1 += P_1 V_j, S_1 = Q_1 K_{j+1}^T. S_t reuses the columns P_t
+//                 was read from with no wait in between: the tensor core executes
+//                 one thread's tcgen05.mma operations in issue order (the order
+//                 NVIDIA's own Blackwell attention example relies on; the GPU
+//                 parity tests check it).
+//   warps 4-7     softmax of tile 0; warps 8-11 softmax of tile 1. Thread r owns
+//                 query row r of its tile (TMEM lane r) and keeps the whole row of
+//                 S in registers: warps 0-3 hand registers over with setmaxnreg
+//                 (56 each) so that the softmax threads get 216. P =
+//                 2^(S scale log2 e - m) is formed with the scale folded into one
+//                 FFMA and written as 16-bit pairs over the first half of S's
+//                 columns. l (exact fp32) gives L; the sum of the rounded P
+//                 normalises O, so the weights applied to V sum to one. O is
+//                 rescaled in TMEM only when m has grown by more than 2^8 since
+//                 the last rescale (exact: O and l share the reference max).
+//   warps 2-3     idle.
 //
-// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,256+d) O.
+// TMEM columns: [0,128) S_0 / P_0, [128,256) S_1 / P_1, [256,256+d) O_0,
+// [256+d,256+2d) O_1.
 #pragma once
 
 #include "sm100.cuh"
@@ -47,55 +54,49 @@ struct FwdArgs {
     int* err;
 };
 
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O once m grew by > 2^8
+constexpr float kLn2 = 0.69314718055994530942f;
+
 template <int D>
 struct FwdCfg {
-    static constexpr int kSlabs = D / 64;        // 64-column slabs of 128 rows x 128 B
+    static constexpr int kSlabs = D / 64;
     static constexpr int kSlabBytes = 128 * 128;
-    static constexpr int kTileBytes = kSlabs * kSlabBytes;
-    static constexpr int kStages = (D == 128) ? 3 : 4;
-    static constexpr int kQOff = 0;
-    static constexpr int kKOff = kQOff + kTileBytes;
+    static constexpr int kTileBytes = kSlabs * kSlabBytes;  // 128 rows x d, 16-bit
+    static constexpr int kStages = (D == 128) ? 2 : 4;
+    static constexpr int kQOff = 0;                          // Q_0, Q_1
+    static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
     static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kSmemBytes = kMiscOff + 16;  // + slack for 1024-B alignment
+    static constexpr int kSmemBytes = kMiscOff + 16;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+    static constexpr uint32_t kColS = 0, kColO = 256;  // S_t at 128 t, O_t at 256 + d t
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O once m grew by > 2^8
-constexpr float kLn2 = 0.69314718055994530942f;
-
-__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
-
-// Time-bounded wait used only while draining at exit (ignores the abort flag).
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-    const uint32_t a = smem_u32(bar);
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(a, parity)) {
-        if (globaltimer_ns() - t0 > 200000000ull) break;
-    }
-}
+constexpr int kFwdThreads = 384;
+constexpr int kFwdRegsOther = 56;     // warps 0-3 after the split
+constexpr int kFwdRegsSoftmax = 216;  // warps 4-11 after the split
+// Registers at launch needed for the split to fit the CTA's pool.
+constexpr int kFwdMinLaunchRegs = (128 * kFwdRegsOther + 256 * kFwdRegsSoftmax + kFwdThreads - 1) / kFwdThreads;
 
 template <int D, bool BF16, bool CAUSAL, bool VARLEN>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
+                   const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
     using C = FwdCfg<D>;
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) uint8_t smem[];
-    if (!smem_base_ok(smem, args.err)) return;  // the 128-byte swizzle needs 1024-byte aligned tiles
+    if (!smem_base_ok(smem, args.err)) return;
 
-    // Non-causal grid (q tiles, Hq, batches): neighbouring CTAs share K/V in L2.
-    // Causal grid (Hq, batches, q tiles), the last query tile first: CTAs are
-    // dispatched heaviest first (longest-processing-time order), so the long
-    // tiles do not start in the last wave.
+    // Non-causal grid (256-row units, Hq, batches): neighbouring CTAs share K/V in
+    // L2. Causal grid (Hq, batches, units), last unit first: heaviest CTAs are
+    // dispatched first (longest-processing-time order).
     const int h = CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
     const int bidx = CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
-    const int q_tile = CAUSAL ? static_cast<int>(gridDim.z - 1 - blockIdx.z) : static_cast<int>(blockIdx.x);
-    const int q0 = q_tile * 128;
+    const int unit = CAUSAL ? static_cast<int>(gridDim.z - 1 - blockIdx.z) : static_cast<int>(blockIdx.x);
+    const int q0 = unit * 256;
 
     int q_len, k_len, q_row0, k_row0, tma_b;
     if constexpr (VARLEN) {
@@ -114,20 +115,23 @@ __global__ void __launch_bounds__(256, 1)
     if (q0 >= q_len) return;  // uniform over the CTA
 
     const int hk = h / args.group;
-    const int last_q = min(q0 + 127, q_len - 1);
-    const int kend = CAUSAL ? min(k_len, last_q + k_len - q_len + 1) : k_len;
-    const int n_kv = kend > 0 ? (kend + 127) / 128 : 0;
+    // Key tiles each query tile needs: tile t holds rows q0 + 128 t .. + 127.
+    auto tiles_needed = [&](int qt) -> int {
+        if (qt >= q_len) return 0;
+        const int last_q = min(qt + 127, q_len - 1);
+        const int kend = CAUSAL ? min(k_len, last_q + k_len - q_len + 1) : k_len;
+        return kend > 0 ? (kend + 127) / 128 : 0;
+    };
+    const int n_0 = tiles_needed(q0), n_1 = tiles_needed(q0 + 128);
+    const int n_kv = max(n_0, n_1);
 
-    // Query row q (0-based in this sequence) is written iff it exists and, for
-    // packed input, its token lies inside the caller's buffer.
+    using T16 = uint16_t;
+    T16* o_base = static_cast<T16*>(args.o);
     auto row_valid = [&](int q) -> bool {
         if (q >= q_len) return false;
         if constexpr (VARLEN) return q_row0 + q >= 0 && q_row0 + q < args.total_q;
         return true;
     };
-    // Output addressing of query row q (0-based within this sequence).
-    using T16 = uint16_t;
-    T16* o_base = static_cast<T16*>(args.o);
     auto o_row = [&](int q) -> T16* {
         const size_t tok = VARLEN ? static_cast<size_t>(q_row0 + q) : static_cast<size_t>(bidx) * args.Nq + q;
         return o_base + (tok * args.Hq + h) * D;
@@ -140,8 +144,8 @@ __global__ void __launch_bounds__(256, 1)
         }
     };
 
-    if (n_kv == 0) {  // no row of this tile sees any key: O = 0, L = -inf
-        if (threadIdx.x < 128) {
+    if (n_kv == 0) {  // no row of this unit sees any key: O = 0, L = -inf
+        if (threadIdx.x < 256) {
             const int q = q0 + static_cast<int>(threadIdx.x);
             if (row_valid(q)) {
                 uint4* dst = reinterpret_cast<uint4*>(o_row(q));
@@ -162,10 +166,10 @@ __global__ void __launch_bounds__(256, 1)
     uint64_t* k_empty = k_full + S;
     uint64_t* v_full = k_empty + S;
     uint64_t* v_empty = v_full + S;
-    uint64_t* s_full = v_empty + S;
-    uint64_t* p_full = s_full + 2;
-    uint64_t* o_done = p_full + 2;
-    uint64_t* mma_final = o_done + 1;
+    uint64_t* s_full = v_empty + S;  // [2 tiles]
+    uint64_t* p_full = s_full + 2;   // [2]
+    uint64_t* mma_final = p_full + 2;
+    uint64_t* sm_done = mma_final + 1;  // every softmax thread is past its last TMEM access
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     int* abort_flag = reinterpret_cast<int*>(smem + C::kMiscOff + 4);
 
@@ -184,8 +188,8 @@ __global__ void __launch_bounds__(256, 1)
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 128);
         }
-        mbar_init(o_done, 1);
         mbar_init(mma_final, 1);
+        mbar_init(sm_done, 256);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -203,26 +207,35 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
     const WaitCtx wc{abort_flag, args.err};
-
+    // Register split (warpgroup granularity): the producer/MMA warpgroup gives
+    // registers to the two softmax warpgroups, whose threads keep a whole row
+    // of S (128 values) in registers. 128 x kRegsOther + 256 x kRegsSoftmax
+    // must not exceed the 384 x (registers at launch) the CTA was given; the
+    // host checks the launch count before every launch.
+    if (warp < 4) {
+        setmaxnreg_dec<kFwdRegsOther>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, C::kTileBytes);
+            mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
 #pragma unroll
-            for (int s = 0; s < C::kSlabs; ++s)
-                tma_load_4d(sQ + s * C::kSlabBytes, &tm_q, q_full, s * 64, h, q_row0 + q0, tma_b);
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int s = 0; s < C::kSlabs; ++s)
+                    tma_load_4d(sQ + t * C::kTileBytes + s * C::kSlabBytes, &tm_q, q_full, s * 64, h,
+                                q_row0 + q0 + 128 * t, tma_b);
             int k_issued = 0, v_issued = 0;
             for (int j = 0; j < n_kv; ++j) {
                 const int st = j % S;
                 const uint32_t ph = (j / S) & 1;
-                if (!mbar_wait(&k_empty[st], ph ^ 1u, wc, 1)) break;
+                if (!mbar_wait(&k_empty[st], ph ^ 1u, wc, 61)) break;
                 mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
 #pragma unroll
                 for (int s = 0; s < C::kSlabs; ++s)
                     tma_load_4d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tm_k, &k_full[st], s * 64, hk,
                                 k_row0 + j * 128, tma_b);
                 ++k_issued;
-                if (!mbar_wait(&v_empty[st], ph ^ 1u, wc, 2)) break;
+                if (!mbar_wait(&v_empty[st], ph ^ 1u, wc, 62)) break;
                 mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
 #pragma unroll
                 for (int s = 0; s < C::kSlabs; ++s)
@@ -230,7 +243,6 @@ __global__ void __launch_bounds__(256, 1)
                                 k_row0 + j * 128, tma_b);
                 ++v_issued;
             }
-            // Drain: no TMA write may land after the CTA has exited.
             mbar_wait_drain(q_full, 0);
             for (int st = 0; st < S; ++st) {
                 if (k_issued > st) mbar_wait_drain(&k_full[st], ((st + S * ((k_issued - 1 - st) / S)) / S) & 1);
@@ -243,91 +255,105 @@ __global__ void __launch_bounds__(256, 1)
             constexpr uint32_t id_qk = idesc_f16(128, 128, BF16, false, false);
             constexpr uint32_t id_pv = idesc_f16(128, D, BF16, false, true);
             const uint32_t q_addr = smem_u32(sQ);
-            bool ok = mbar_wait(q_full, 0, wc, 3);
-            auto issue_s = [&](int j) -> bool {
-                const int st = j % S;
-                if (!mbar_wait(&k_full[st], (j / S) & 1, wc, 4)) return false;
-                tc_fence_after();
-                const uint32_t k_addr = smem_u32(sK + st * C::kTileBytes);
-                const uint32_t d_col = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
+            auto issue_s = [&](int t, int j) {
+                const uint32_t k_addr = smem_u32(sK + (j % S) * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
-                    mma_ss(d_col, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), id_qk,
-                           kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::kColS + 128 * t, sdesc_sw128(q_addr + t * C::kTileBytes + off, 16, 1024),
+                           sdesc_sw128(k_addr + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(&k_empty[st]);
-                tc_commit(&s_full[j & 1]);
-                return true;
+                tc_commit(&s_full[t]);
             };
-            if (ok) ok = issue_s(0);
-            if (ok && n_kv > 1) ok = issue_s(1);
+            bool ok = mbar_wait(q_full, 0, wc, 63);
+            if (ok) ok = mbar_wait(&k_full[0], 0, wc, 64);
+            if (ok) {
+                tc_fence_after();
+                if (n_0 > 0) issue_s(0, 0);
+                if (n_1 > 0) issue_s(1, 0);
+                tc_commit(&k_empty[0]);
+            }
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int st = j % S;
-                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, wc, 5)) break;
-                if (!mbar_wait(&v_full[st], (j / S) & 1, wc, 6)) break;
-                tc_fence_after();
+                const bool more = j + 1 < n_kv;
+                if (!(ok = mbar_wait(&v_full[st], (j / S) & 1, wc, 65))) break;
+                if (more && !(ok = mbar_wait(&k_full[(j + 1) % S], ((j + 1) / S) & 1, wc, 66))) break;
                 const uint32_t v_addr = smem_u32(sV + st * C::kTileBytes);
-                const uint32_t p_col = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
+                // For each tile: O_t += P_t V_j, then S_t of the next key tile into the
+                // same columns. tcgen05.mma operations of one thread execute in issue
+                // order, so the second cannot overwrite P_t before the first has read
+                // it, and S_t complete implies every earlier P_t V complete.
+                for (int t = 0; ok && t < 2; ++t) {
+                    const int ntt = t ? n_1 : n_0;
+                    if (j >= ntt) continue;
+                    if (!(ok = mbar_wait(&p_full[t], j & 1, wc, 67))) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_ts(tmem + C::kColO, p_col + kk * 8, sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024),
-                           id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
+                               sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    if (j + 1 < ntt) issue_s(t, j + 1);
                 }
                 tc_commit(&v_empty[st]);
-                tc_commit(o_done);
-                if (j + 2 < n_kv) {
-                    // S_{j+2} overwrites the columns P_j is read from: let P_j V_j finish first
-                    // (the ISA orders back-to-back MMAs only when they share the accumulator).
-                    ok = mbar_wait(o_done, j & 1, wc, 10);
-                    if (ok) ok = issue_s(j + 2);
-                }
+                if (more) tc_commit(&k_empty[(j + 1) % S]);
             }
             tc_commit(mma_final);
             mbar_wait_drain(mma_final, 0);
+            // TMEM is freed once the softmax warpgroups are done with it. Their waits
+            // are bounded, so the arrivals come (4 s bound here as a last resort).
+            const uint32_t a = smem_u32(sm_done);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < 4000000000ull) {
+            }
         }
-    } else if (warp >= 4) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+        return;  // warps 0-3 end here; no code is shared with the softmax warpgroups
+    } else {
+        setmaxnreg_inc<kFwdRegsSoftmax>();
         // ------------------------------------------------------------ softmax / correction / epilogue
+        const int t = (warp - 4) >> 2;  // query tile of this warpgroup
         const int w4 = warp & 3;
         const int r = w4 * 32 + lane;
-        const int q = q0 + r;
+        const int qt0 = q0 + 128 * t;
+        const int q = qt0 + r;
+        const int nt = t ? n_1 : n_0;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
+        const uint32_t s_addr = lane_base + C::kColS + 128 * t;
+        const uint32_t o_addr = lane_base + C::kColO + D * t;
         const int row_limit = CAUSAL ? min(k_len, q + k_len - q_len + 1) : k_len;
+        // Key tiles at or past this index need masking for some row of the tile.
+        const int min_limit = CAUSAL ? min(k_len, qt0 + k_len - q_len + 1) : k_len;
         const float sl2 = args.scale_log2;
         float m = -INFINITY, l = 0.f, lr = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            ok = warp_all(mbar_wait(&s_full[j & 1], (j >> 1) & 1, wc, 7));
+        for (int j = 0; j < nt; ++j) {
+            ok = warp_all(mbar_wait(&s_full[t], j & 1, wc, 69));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t s_addr = lane_base + ((j & 1) ? C::kColS1 : C::kColS0);
-            uint32_t s[4][32];
-            tmem_ld32(s_addr + 0, s[0]);
-            tmem_ld32(s_addr + 32, s[1]);
-            tmem_ld32(s_addr + 64, s[2]);
-            tmem_ld32(s_addr + 96, s[3]);
-            tmem_ld_wait(s[0]);
-            tmem_ld_wait(s[1]);
-            tmem_ld_wait(s[2]);
-            tmem_ld_wait(s[3]);
             const int lim = row_limit - j * 128;  // columns >= lim are masked
-            if (lim < 128) {
+            const bool need_mask = j * 128 + 128 > min_limit;
+            uint32_t sv[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
+            if (need_mask) {  // masked columns read as -inf: out of the max, P = 0
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (c >= lim) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                    if (c >= lim) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
-            // Row max as 16 independent partial maxima (a single chain of 128
-            // dependent max operations would expose its whole latency).
-            float mxp[16];
+            // Row max: 8 independent chains of three-input max.
+            float mxp[8];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) mxp[i] = __uint_as_float(s[i >> 5][i & 31]);
+            for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
 #pragma unroll
-            for (int c = 16; c < 128; ++c) mxp[c & 15] = fmaxf(mxp[c & 15], __uint_as_float(s[c >> 5][c & 31]));
-#pragma unroll
-            for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-                for (int i = 0; i < w; ++i) mxp[i] = fmaxf(mxp[i], mxp[i + w]);
-            const float mx = mxp[0];
+            for (int i = 0; i < 64; ++i)
+                mxp[i & 7] = fmax3(mxp[i & 7], __uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
+                                   __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
+            const float mx = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
             const float m_new = fmaxf(m, mx * sl2);
             float alpha = 1.f;
             bool resc = false;
@@ -339,48 +365,50 @@ __global__ void __launch_bounds__(256, 1)
                 m = m_new;
             }
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            // P is rounded to 16 bits for the P V product. l (exact fp32 sum)
-            // gives L; lr, the sum of the ROUNDED values, normalises O, so the
-            // weights applied to V sum to exactly one.
-            float rsp[4] = {0.f, 0.f, 0.f, 0.f}, rsrp[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums
+            // P = 2^(S c - m) as 16-bit pairs (keys 2i, 2i + 1 in column i), partial sums
+            // of the exact and of the rounded values.
+            // Pairs of keys go through the packed f32x2 FMA and adds.
+            const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(neg_m, neg_m);
+            uint64_t rs2[4] = {0, 0, 0, 0}, rsr2[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
             uint32_t pk[2][32];
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(s[(2 * i) >> 5][(2 * i) & 31]), sl2, neg_m));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(s[(2 * i + 1) >> 5][(2 * i + 1) & 31]), sl2, neg_m));
-                rsp[i & 3] += p0 + p1;
+                const uint64_t x = f2_pack(__uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
+                                           __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
+                float y0, y1;
+                f2_unpack(f2_fma(x, c2, m2), y0, y1);
+                const float p0 = ex2_approx(y0);
+                const float p1 = ex2_approx(y1);
+                rs2[i & 3] = f2_add(rs2[i & 3], f2_pack(p0, p1));
                 const uint32_t u = pack2<BF16>(p0, p1);
-                rsrp[i & 3] += unpack_lo<BF16>(u) + unpack_hi<BF16>(u);
+                rsr2[i & 3] = f2_add(rsr2[i & 3], f2_pack(unpack_lo<BF16>(u), unpack_hi<BF16>(u)));
                 pk[i >> 5][i & 31] = u;
-            }
-            const float rs = (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
-            const float rsr = (rsrp[0] + rsrp[1]) + (rsrp[2] + rsrp[3]);
-            l = l * alpha + rs;
-            lr = lr * alpha + rsr;
-            if (j > 0 && __any_sync(0xffffffffu, resc)) {
-                ok = warp_all(mbar_wait(o_done, (j - 1) & 1, wc, 8));
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t ov[32];
-                    tmem_ld32(lane_base + C::kColO + c0, ov);
-                    tmem_ld_wait(ov);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(lane_base + C::kColO + c0, ov);
-                }
-                tmem_st_wait();
             }
             tmem_st32(s_addr + 0, pk[0]);
             tmem_st32(s_addr + 32, pk[1]);
+            const float rs = f2_sum(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])));
+            const float rsr = f2_sum(f2_add(f2_add(rsr2[0], rsr2[1]), f2_add(rsr2[2], rsr2[3])));
+            l = l * alpha + rs;
+            lr = lr * alpha + rsr;
+            // S_t was issued after the previous key tile's P_t V and MMAs of one thread
+            // complete in order, so O_t is final for that tile here and can be
+            // rescaled in place.
+            if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t ov[32];
+                    tmem_ld32(o_addr + c0, ov);
+                    tmem_ld_wait(ov);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                    tmem_st32(o_addr + c0, ov);
+                }
+            }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&p_full[j & 1]);
+            mbar_arrive(&p_full[t]);
         }
-        // The last two P V products may both be in flight here, more than one
-        // phase of o_done apart, so the epilogue waits on the final commit.
-        if (ok) ok = warp_all(mbar_wait(mma_final, 0, wc, 9));
+        if (nt > 0 && ok) ok = warp_all(mbar_wait(mma_final, 0, wc, 70));
         if (ok) {
             tc_fence_after();
             const bool row_ok = row_valid(q);
@@ -388,13 +416,18 @@ __global__ void __launch_bounds__(256, 1)
             T16* dst = row_ok ? o_row(q) : nullptr;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t ov[32];
-                tmem_ld32(lane_base + C::kColO + c0, ov);
-                tmem_ld_wait(ov);
                 uint32_t pk[16];
+                if (nt > 0) {
+                    uint32_t ov[32];
+                    tmem_ld32(o_addr + c0, ov);
+                    tmem_ld_wait(ov);
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack2<BF16>(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack2<BF16>(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                }
                 if (row_ok) {
                     uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
@@ -402,24 +435,17 @@ __global__ void __launch_bounds__(256, 1)
                 }
             }
             if (row_ok) {
-                float L;
+                float L = -INFINITY;
                 if (l > 0.f) {
                     float lg;
                     asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l));
                     L = (m + lg) * kLn2;
-                } else {
-                    L = -INFINITY;
                 }
                 *lse_at(q) = L;
             }
         }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, C::kTmemCols);
+        tc_fence_before();
+        mbar_arrive(sm_done);
     }
 }
 

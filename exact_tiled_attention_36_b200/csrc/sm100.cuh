@@ -103,6 +103,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCt
 }
 
 
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+// Time-bounded wait used only while draining at exit (ignores the abort flag).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, parity)) {
+        if (globaltimer_ns() - t0 > 200000000ull) break;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
