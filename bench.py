@@ -406,6 +406,70 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- per-workload sweep
+def run_sweep(args):
+    """Forward (and the causal GQA backward) of every workload, one JSON line each.
+    Informational: the bench line of the contract is the default mode."""
+    import torch
+    from exact_tiled_attention_36_b200 import binding as fb
+    from exact_tiled_attention_36_b200 import inputs
+
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    stream = torch.cuda.current_stream()
+
+    def time_it(fn, iters):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if fb.fa_get_last_device_error(None) != fb.FA_OK:
+            raise RuntimeError("device error")
+        return e0.elapsed_time(e1) / iters
+
+    def emit(name, what, ms, flops, nbytes):
+        line = {"kind": "config_sweep", "workload": name, "pass": what, "ms": ms,
+                "tflops": flops / (ms / 1e3) / 1e12, "frac_of_bf16_burst": flops / (ms / 1e3) / 1e12 / peak,
+                "algorithmic_gbs": nbytes / (ms / 1e3) / 1e9, "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / hbm,
+                "peaks": peak_src}
+        print(json.dumps(line), flush=True)
+
+    for cfg in (inputs.TINY, inputs.VISION, inputs.VIT_RMSNORM, inputs.CAUSAL_GQA):
+        fi = inputs.make_fixed(cfg)
+        q, k, v = (t.cuda() for t in (fi.q, fi.k, fi.v))
+        B, N, Hq, d = q.shape
+        Hkv = k.shape[2]
+        o, lse = fb.attention_fwd(q, k, v, cfg.scale, cfg.causal)
+        flops = flops_fwd(B, N, Hq, d, cfg.causal)
+        nbytes = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
+        iters = 1000 if cfg is inputs.TINY else 30
+        ms = time_it(lambda: fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse), iters)
+        emit(cfg.name, "fwd", ms, flops, nbytes)
+        if cfg.backward:
+            do = fi.do.cuda()
+            ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, N, d), dtype=torch.uint8, device="cuda")
+            ms = time_it(lambda: fb.attention_bwd(q, k, v, o, lse, do, cfg.scale, cfg.causal, workspace=ws), 20)
+            emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+        del q, k, v, o, lse
+    for cfg in (inputs.VARLEN, inputs.VARLEN_KEYPAD):
+        vi = inputs.make_varlen(cfg)
+        q, k, v = (t.cuda() for t in (vi.q, vi.k, vi.v))
+        cu_q, cu_k = vi.cu_seqlens_q.cuda(), vi.cu_seqlens_k.cuda()
+        o, lse = fb.attention_varlen_fwd(q, k, v, cu_q, cu_k, vi.max_seqlen_q, vi.max_seqlen_k, cfg.scale, cfg.causal)
+        flops = sum(4.0 * lq * lk * cfg.d * cfg.Hq for lq, lk in zip(vi.seqlens_q, vi.seqlens_k))
+        nbytes = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
+        ms = time_it(lambda: fb.attention_varlen_fwd(q, k, v, cu_q, cu_k, vi.max_seqlen_q, vi.max_seqlen_k,
+                                                     cfg.scale, cfg.causal, out=o, lse=lse), 20)
+        emit(cfg.name, "fwd", ms, flops, nbytes)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,7 +479,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-small", action="store_true",
                     help="run only the warm-up steps on a smaller case (B=1, N=4096) for ncu captures")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="time the forward of every workload (and the causal GQA backward); one JSON line each")
     args = ap.parse_args()
+    if args.all_configs:
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

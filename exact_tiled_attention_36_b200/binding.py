@@ -40,6 +40,7 @@ _SIGS = {
     "fa_version": ([], ctypes.c_char_p),
     "fa_bwd_set_timing_events": ([_P, _P], None),
     "fa_bwd_noalloc": ([_P] * 9 + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_selftest_bounded_wait": ([_P], _I),
 }
 
 
@@ -104,6 +105,10 @@ def fa_get_last_device_error_site() -> int:
 
 def fa_bwd_set_timing_events(before, after) -> None:
     lib().fa_bwd_set_timing_events(before, after)
+
+
+def fa_selftest_bounded_wait(stream) -> int:
+    return lib().fa_selftest_bounded_wait(stream)
 
 
 def fa_version() -> str:

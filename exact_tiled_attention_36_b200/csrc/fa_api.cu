@@ -122,6 +122,22 @@ fa_status launch_fwd(int d, bool bf16, bool causal, bool varlen, const CUtensorM
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// One CTA waits, with the kernels' bounded wait, on an mbarrier that nothing
+// arrives on: the wait runs out, records the site and the kernel returns.
+constexpr int kSelftestSite = 99;
+__global__ void fa_selftest_wait_kernel(int* err) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        fa::mbar_init(&bar, 1);
+        abort_flag = 0;
+        fa::fence_mbar_init();
+    }
+    __syncthreads();
+    const fa::WaitCtx wc{&abort_flag, err};
+    fa::mbar_wait(&bar, 0, wc, kSelftestSite);
+}
+
 // d = 128 runs the two-sub-tile ping-pong kernel; d = 64 the single-tile one
 // (its dQ^T would need M = 64, so it keeps dQ = dS K with M = 128 queries).
 template <int D, bool BF16, bool CAUSAL>
@@ -327,6 +343,13 @@ fa_status fa_get_last_device_error(fa_stream_t stream) {
 }
 
 int fa_get_last_device_error_site(void) { return g_last_site; }
+
+fa_status fa_selftest_bounded_wait(fa_stream_t stream) {
+    int* err = error_word();
+    if (!err) return FA_ERR_CUDA;
+    fa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(err);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 void fa_bwd_set_timing_events(void* before, void* after) {
     g_bwd_ev_before = static_cast<cudaEvent_t>(before);

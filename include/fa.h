@@ -182,6 +182,16 @@ fa_status fa_get_last_device_error(fa_stream_t stream);
  * that was not 1024-byte aligned (the kernel then does nothing); 0 if none. */
 int fa_get_last_device_error_site(void);
 
+/*
+ * Self-test of the failure path (no counterpart in the pages): launches one
+ * CTA that waits, with the same bounded wait every kernel uses, on a barrier
+ * that nothing arrives on. About 2 s later the wait gives up and records its
+ * site (0x1000 + 99) in the device error word, and the kernel returns; the
+ * caller sees FA_ERR_TIMEOUT from fa_get_last_device_error and the context
+ * stays usable. Returns the launch status.
+ */
+fa_status fa_selftest_bounded_wait(fa_stream_t stream);
+
 /* Library version, "major.minor.patch". */
 const char* fa_version(void);
 
