@@ -15,7 +15,7 @@
 #include "fa.h"
 #include "fa_fwd.cuh"
 #include "fa_bwd.cuh"
-#include "fa_bwd_pp.cuh"
+#include "fa_bwd128.cuh"
 
 namespace {
 
@@ -138,16 +138,34 @@ __global__ void fa_selftest_wait_kernel(int* err) {
     fa::mbar_wait(&bar, 0, wc, kSelftestSite);
 }
 
-// d = 128 runs the two-sub-tile ping-pong kernel; d = 64 the single-tile one
-// (its dQ^T would need M = 64, so it keeps dQ = dS K with M = 128 queries).
+// d = 128 runs fa_bwd128_kernel (dQ^T = K^T dS^T with N = 128 queries); d = 64
+// the single-tile kernel (its dQ^T would need M = 64, so it keeps dQ = dS K with
+// M = 128 queries).
 template <int D, bool BF16, bool CAUSAL>
 fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const fa::BwdArgs& a, dim3 grid, cudaStream_t stream) {
-    auto kern = D == 128 ? fa::fa_bwd_pp_kernel<BF16, CAUSAL> : fa::fa_bwd_kernel<D, BF16, CAUSAL>;
-    constexpr int smem = D == 128 ? fa::BwdPPCfg::kSmemBytes : fa::BwdCfg<D>::kSmemBytes;
-    static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-    if (!attr_ok) return FA_ERR_CUDA;
-    kern<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, a);
+    if constexpr (D == 128) {
+        auto kern = fa::fa_bwd128_kernel<BF16, CAUSAL>;
+        constexpr int smem = fa::Bwd128Cfg::kSmemBytes;
+        static bool attr_ok =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+        if (!attr_ok) return FA_ERR_CUDA;
+        // The kernel moves registers between warpgroups with setmaxnreg; the split
+        // only fits if the launch holds enough registers per thread.
+        static int launch_regs = [&] {
+            cudaFuncAttributes fa_attr{};
+            return cudaFuncGetAttributes(&fa_attr, kern) == cudaSuccess ? fa_attr.numRegs : 0;
+        }();
+        if (launch_regs < fa::kBwd128MinLaunchRegs) return FA_ERR_UNSUPPORTED;
+        kern<<<grid, fa::kBwd128Threads, smem, stream>>>(mq, mk, mv, mdo, a);
+    } else {
+        auto kern = fa::fa_bwd_kernel<D, BF16, CAUSAL>;
+        constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
+        static bool attr_ok =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+        if (!attr_ok) return FA_ERR_CUDA;
+        kern<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, a);
+    }
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -254,10 +272,17 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
     return launch_fwd(d, bf16, causal != 0, true, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Floats in the dQ accumulator: [B, Nq, Hq, 64] for d = 64; for d = 128 the
+// queries of each (b, h) are padded to a multiple of four ([B, Hq, nq4, 128, 4]).
+static size_t acc_floats(int B, int Hq, int Nq, int d) {
+    if (d == 64) return static_cast<size_t>(B) * Hq * Nq * 64;
+    return static_cast<size_t>(B) * Hq * ((static_cast<size_t>(Nq) + 3) / 4) * 512;
+}
+
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {
     if (B < 1 || Hq < 1 || Nq < 0 || (d != 64 && d != 128)) return 0;
     const size_t rows = static_cast<size_t>(B) * Hq * Nq;
-    return round256(rows * sizeof(float)) + round256(rows * d * sizeof(float));
+    return round256(rows * sizeof(float)) + round256(acc_floats(B, Hq, Nq, d) * sizeof(float));
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
@@ -282,14 +307,15 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     if (rows > 0) {
         const size_t threads = rows * (d / 8);
         const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        const size_t acc_f4 = acc_floats(B, Hq, Nq, d) / 4;
         if (d == 64)
             fa::fa_bwd_preprocess<64><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
-                                                             static_cast<const uint16_t*>(dout), Dvec, dq_acc, B, Nq,
-                                                             Hq, bf16);
+                                                             static_cast<const uint16_t*>(dout), Dvec, dq_acc, acc_f4,
+                                                             B, Nq, Hq, bf16);
         else
             fa::fa_bwd_preprocess<128><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
-                                                              static_cast<const uint16_t*>(dout), Dvec, dq_acc, B,
-                                                              Nq, Hq, bf16);
+                                                              static_cast<const uint16_t*>(dout), Dvec, dq_acc,
+                                                              acc_f4, B, Nq, Hq, bf16);
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
     if (Nk > 0) {
@@ -302,6 +328,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
         a.lse = lse;
         a.D = Dvec;
         a.dq_acc = dq_acc;
+        a.nq4 = (Nq + 3) / 4;
         a.dk = dk;
         a.dv = dv;
         a.Hq = Hq;
@@ -323,9 +350,15 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
         if (timed && cudaEventRecord(g_bwd_ev_after, s) != cudaSuccess) return FA_ERR_CUDA;
     }
     if (rows > 0) {
-        const size_t n8 = rows * d / 8;
-        fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
-            dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16);
+        if (d == 64) {
+            const size_t n8 = rows * d / 8;
+            fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
+                dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16);
+        } else {
+            const size_t n = static_cast<size_t>(B) * Hq * ((Nq + 3) / 4) * 64;
+            fa::fa_bwd_dq_convert_g4<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+                dq_acc, static_cast<uint16_t*>(dq), B, Hq, Nq, (Nq + 3) / 4, scale, bf16);
+        }
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
     return FA_OK;

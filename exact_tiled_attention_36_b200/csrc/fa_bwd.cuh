@@ -22,6 +22,8 @@
 //                      and adds dQ_i into the fp32 accumulator with vector
 //                      reductions. dK, dV leave TMEM once, at the end.
 //   fa_bwd_dq_convert  dQ = dtype(scale * dQ_acc).
+//   (d = 128 runs fa_bwd128_kernel of fa_bwd128.cuh in place of fa_bwd_kernel
+//   and fa_bwd_dq_convert_g4 in place of fa_bwd_dq_convert.)
 //
 // Warp roles of fa_bwd_kernel (384 threads): warp 0 TMA producer, warp 1 TMEM
 // allocation and the single MMA-issuing thread, warps 2-3 idle, warps 4-11 two
@@ -42,7 +44,8 @@ namespace fa {
 struct BwdArgs {
     const float* lse;  // [B, Hq, Nq]
     const float* D;    // [B, Hq, Nq]
-    float* dq_acc;     // [B, Nq, Hq, d]
+    float* dq_acc;     // d = 64: [B, Nq, Hq, 64]; d = 128: [B, Hq, nq4, 128, 4] (see fa_bwd_dq_convert_g4)
+    int nq4;           // groups of four queries per (b, h) in the d = 128 layout: ceil(Nq / 4)
     void* dk;          // [B, Nk, Hkv, d]
     void* dv;
     int Hq, Hkv, group, Nq, Nk;
@@ -395,7 +398,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // A group of D/8 lanes handles one (b, q, h) row, 8 elements per lane.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float* Dvec,
-                                                          float* dq_acc, int B, int Nq, int Hq, bool bf16) {
+                                                          float* dq_acc, size_t acc_f4, int B, int Nq, int Hq,
+                                                          bool bf16) {
     constexpr int kLanes = D / 8;
     const size_t rows = static_cast<size_t>(B) * Nq * Hq;
     const size_t row = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / kLanes;
@@ -422,9 +426,13 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess(const uint16_t* o, cons
             acc = fmaf(a0, c0, acc);
             acc = fmaf(a1, c1, acc);
         }
-        float4* z = reinterpret_cast<float4*>(dq_acc + row * D) + sub * 2;
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // Zero the dQ accumulator (acc_f4 float4s; its layout depends on d).
+    {
+        const size_t nthreads = static_cast<size_t>(gridDim.x) * blockDim.x;
+        float4* z = reinterpret_cast<float4*>(dq_acc);
+        for (size_t g = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < acc_f4; g += nthreads)
+            z[g] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -454,6 +462,34 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert(const float* dq_acc, ui
                          pack2<false>(c.x * scale, c.y * scale), pack2<false>(c.z * scale, c.w * scale));
     }
     reinterpret_cast<uint4*>(dq)[i] = out;
+}
+
+// The d = 128 accumulator keeps four consecutive queries of one head-dimension
+// index together: element (b, h, q, c) sits at ((b Hq + h) nq4 + q / 4) 512 +
+// 4 c + q % 4, so a warp of the backward main kernel (lane = c) adds four
+// queries with one coalesced 512-byte vector reduction. One thread here turns
+// head-dimension indices 2p, 2p + 1 of a group of four queries into dQ[b, q, h, :].
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_g4(const float* dq_acc, uint16_t* dq, int B, int Hq,
+                                                             int Nq, int nq4, float scale, bool bf16) {
+    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // (b, h, g, p)
+    const size_t groups = static_cast<size_t>(B) * Hq * nq4;
+    if (i >= groups * 64) return;
+    const int p = static_cast<int>(i & 63);
+    const size_t bhg = i >> 6;
+    const int g = static_cast<int>(bhg % nq4);
+    const size_t bh = bhg / nq4;
+    const int h = static_cast<int>(bh % Hq);
+    const size_t b = bh / Hq;
+    const float4* src = reinterpret_cast<const float4*>(dq_acc) + bhg * 128 + 2 * p;
+    const float4 a = src[0], c = src[1];
+    const float lo[4] = {a.x, a.y, a.z, a.w}, hi[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int q = 4 * g + j;
+        if (q >= Nq) break;
+        const uint32_t v = bf16 ? pack2<true>(lo[j] * scale, hi[j] * scale) : pack2<false>(lo[j] * scale, hi[j] * scale);
+        reinterpret_cast<uint32_t*>(dq + ((b * Nq + q) * Hq + h) * 128)[p] = v;
+    }
 }
 
 }  // namespace fa

@@ -103,7 +103,9 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
 /*
  * Size in bytes of the caller-owned workspace fa_bwd needs: the per-row
  * D_i = sum_c dO_ic O_ic (float32 [B,Hq,Nq]) and the float32 dQ accumulator
- * ([B,Nq,Hq,d]), each rounded up to 256 bytes. Returns 0 for invalid sizes.
+ * (B*Hq*Nq*64 floats for d = 64; B*Hq*ceil(Nq/4)*4*128 floats for d = 128,
+ * whose layout groups four queries), each rounded up to 256 bytes. Returns 0
+ * for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
 

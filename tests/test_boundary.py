@@ -122,5 +122,7 @@ def test_workspace_size(lib):
     r256 = lambda x: (x + 255) // 256 * 256
     assert fb.fa_bwd_workspace_size(B, Hq, Nq, d) == r256(rows * 4) + r256(rows * d * 4)
     assert fb.fa_bwd_workspace_size(1, 1, 3, 64) == 256 + r256(3 * 64 * 4)
+    # d = 128 pads the queries of each (b, h) to a multiple of four
+    assert fb.fa_bwd_workspace_size(2, 3, 5, 128) == r256(2 * 3 * 5 * 4) + r256(2 * 3 * 8 * 128 * 4)
     assert fb.fa_bwd_workspace_size(0, 1, 1, 64) == 0
     assert fb.fa_bwd_workspace_size(1, 1, 1, 96) == 0

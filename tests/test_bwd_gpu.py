@@ -58,6 +58,8 @@ SMALL = [
     (2, 3, 1, 97, 250, 64, False, "fp16"),
     (1, 4, 4, 1, 5, 128, False, "bf16"),
     (1, 8, 2, 520, 520, 128, True, "bf16"),
+    (1, 4, 2, 300, 390, 128, False, "bf16"),
+    (2, 2, 1, 1000, 700, 128, False, "fp16"),
 ]
 
 
