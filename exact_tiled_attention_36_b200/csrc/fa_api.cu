@@ -70,6 +70,34 @@ int* error_word() {
     return ptr;
 }
 
+// Streaming multiprocessors of the current device (the persistent forward runs at
+// most one CTA per SM); cached per device.
+int sm_count() {
+    constexpr int kMaxDevices = 64;
+    static int counts[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    if (counts[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
+// Units of 256 query rows for every (batch, head) and the persistent grid over them.
+fa_status fwd_units(fa::FwdArgs& a, int nseq, int max_q, dim3& grid) {
+    const long long nu = (static_cast<long long>(max_q) + 255) / 256;
+    const long long n = nu * a.Hq * nseq;
+    if (n > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    const int sms = sm_count();
+    if (sms <= 0) return FA_ERR_CUDA;
+    a.nu = static_cast<int>(nu);
+    a.n_units = static_cast<int>(n);
+    grid = dim3(static_cast<unsigned>(n < sms ? n : sms));
+    return FA_OK;
+}
+
 fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype) {
     if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
@@ -223,9 +251,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     a.Nk = Nk;
     a.scale_log2 = scale * kLog2e;
     a.err = err;
-    const unsigned nqt = static_cast<unsigned>((Nq + 255) / 256);  // 256-row units (two query tiles)
-    if (nqt > 65535u) return FA_ERR_UNSUPPORTED;
-    const dim3 grid = causal ? dim3(Hq, B, nqt) : dim3(nqt, Hq, B);
+    dim3 grid;
+    if ((st = fwd_units(a, B, Nq, grid)) != FA_OK) return st;
     return launch_fwd(d, bf16, causal != 0, false, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -266,9 +293,8 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
     a.Nk = max_seqlen_k;
     a.scale_log2 = scale * kLog2e;
     a.err = err;
-    const unsigned nqt = static_cast<unsigned>((max_seqlen_q + 255) / 256);
-    if (nqt > 65535u) return FA_ERR_UNSUPPORTED;
-    const dim3 grid = causal ? dim3(Hq, num_seqs, nqt) : dim3(nqt, Hq, num_seqs);
+    dim3 grid;
+    if ((st = fwd_units(a, num_seqs, max_seqlen_q, grid)) != FA_OK) return st;
     return launch_fwd(d, bf16, causal != 0, true, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 

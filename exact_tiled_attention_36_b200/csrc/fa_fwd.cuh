@@ -1,17 +1,28 @@
-// fa_fwd.cuh: tiled exact attention forward for sm_100a, two query tiles per CTA.
+// fa_fwd.cuh: tiled exact attention forward for sm_100a, persistent CTAs with
+// two query tiles per work unit.
 //
-// One CTA computes two 128-row query tiles Q_0, Q_1 (rows q0 .. q0 + 255) of one
-// (batch, query head) and walks the key/value tiles K_j, V_j of 128 rows with
-// the online softmax ("FlashAttention/zh", section "FlashAttention algorithm":
-// S_ij = Q_i K_j^T, running row max m and normaliser l, rescale of the partial
-// output by exp(m_old - m_new), final O_i / l_i and L_i = m_i + log l_i), query
-// tiles outside and key tiles inside (the FlashAttention-2 split, section
-// "variants"). Every K/V tile loaded serves both query tiles, and the softmax of
-// one tile overlaps the tensor-core work of the other.
+// A work unit is two 128-row query tiles Q_0, Q_1 (rows q0 .. q0 + 255) of one
+// (batch, query head); the unit walks the key/value tiles K_j, V_j of 128 rows
+// with the online softmax ("FlashAttention/zh", section "FlashAttention
+// algorithm": S_ij = Q_i K_j^T, running row max m and normaliser l, rescale of
+// the partial output by exp(m_old - m_new), final O_i / l_i and L_i = m_i +
+// log l_i), query tiles outside and key tiles inside (the FlashAttention-2
+// split, section "variants"). Every K/V tile loaded serves both query tiles,
+// and the softmax of one tile overlaps the tensor-core work of the other.
+//
+// Persistent tile scheduler: the grid has at most one CTA per SM and CTA c
+// takes units c, 2G - 1 - c, 2G + c, ... of a fixed unit order (G CTAs; the
+// order alternates direction every round). Without the causal mask the order
+// keeps the units of one (batch, head) together so neighbouring CTAs share K/V
+// in the L2; under the causal mask it runs the heaviest units (the last query
+// rows) first. The CTA keeps its barriers, TMEM and K/V ring from unit to
+// unit: the producer loads the next unit's Q as soon as the current unit's
+// last S product has been issued, and the MMA thread issues the next unit's
+// first S products while the softmax warpgroups write the current unit's O.
 //
 // Warp roles (384 threads):
-//   warp 0        TMA producer: Q_0, Q_1 once, then K_j, V_j into 2-stage (d = 128)
-//                 or 4-stage (d = 64) mbarrier rings.
+//   warp 0        TMA producer: Q_0, Q_1 per unit, K_j, V_j into 2-stage (d = 128)
+//                 or 4-stage (d = 64) mbarrier rings that run across units.
 //   warp 1        TMEM allocation and the single MMA-issuing thread. Per key
 //                 tile j it issues O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T,
 //                 O_1 += P_1 V_j, S_1 = Q_1 K_{j+1}^T. S_t reuses the columns P_t
@@ -22,13 +33,15 @@
 //   warps 4-7     softmax of tile 0; warps 8-11 softmax of tile 1. Thread r owns
 //                 query row r of its tile (TMEM lane r) and keeps the whole row of
 //                 S in registers: warps 0-3 hand registers over with setmaxnreg
-//                 (56 each) so that the softmax threads get 216. P =
+//                 (80 each) so that the softmax threads get 208. P =
 //                 2^(S scale log2 e - m) is formed with the scale folded into one
 //                 FFMA and written as 16-bit pairs over the first half of S's
 //                 columns. l (exact fp32) gives L; the sum of the rounded P
 //                 normalises O, so the weights applied to V sum to one. O is
 //                 rescaled in TMEM only when m has grown by more than 2^8 since
 //                 the last rescale (exact: O and l share the reference max).
+//                 After the unit's last product each warpgroup writes its O_t
+//                 and L and releases O_t's columns for the next unit.
 //   warps 2-3     idle.
 //
 // TMEM columns: [0,128) S_0 / P_0, [128,256) S_1 / P_1, [256,256+d) O_0,
@@ -50,6 +63,8 @@ struct FwdArgs {
     int group;        // Hq / Hkv
     int Nq;           // fixed: sequence lengths; varlen: max_seqlen bounds
     int Nk;
+    int nu;           // units (256 query rows) per sequence: ceil(Nq / 256)
+    int n_units;      // nu * Hq * num_batches
     float scale_log2;  // scale * log2(e)
     int* err;
 };
@@ -67,7 +82,7 @@ struct FwdCfg {
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 1;
+    static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 1 + 1 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16;
     static constexpr uint32_t kTmemCols = 512;
@@ -76,10 +91,64 @@ struct FwdCfg {
 };
 
 constexpr int kFwdThreads = 384;
-constexpr int kFwdRegsOther = 56;     // warps 0-3 after the split
-constexpr int kFwdRegsSoftmax = 216;  // warps 4-11 after the split
+constexpr int kFwdRegsOther = 80;     // warps 0-3 after the split
+constexpr int kFwdRegsSoftmax = 208;  // warps 4-11 after the split
 // Registers at launch needed for the split to fit the CTA's pool.
 constexpr int kFwdMinLaunchRegs = (128 * kFwdRegsOther + 256 * kFwdRegsSoftmax + kFwdThreads - 1) / kFwdThreads;
+
+// Everything one role needs to know about a work unit; every role decodes the
+// same units in the same order.
+struct FwdUnit {
+    int h, bidx, q0;
+    int q_len, k_len, q_row0, k_row0, tma_b;
+    int n_0, n_1, n_kv;  // key tiles of query tile 0, of query tile 1, and their maximum
+    bool rows;           // the unit holds at least one query row
+};
+
+template <bool CAUSAL, bool VARLEN>
+__device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdArgs& a) {
+    FwdUnit w;
+    const int hb = a.Hq * a.num_batches;
+    int unit, r;
+    if (CAUSAL) {  // heaviest units (last query rows) first
+        unit = a.nu - 1 - u / hb;
+        r = u % hb;
+    } else {  // the units of one (batch, head) together
+        unit = u % a.nu;
+        r = u / a.nu;
+    }
+    w.h = r % a.Hq;
+    w.bidx = r / a.Hq;
+    w.q0 = unit * 256;
+    if constexpr (VARLEN) {
+        w.q_row0 = a.cu_q[w.bidx];
+        w.k_row0 = a.cu_k[w.bidx];
+        w.q_len = min(a.cu_q[w.bidx + 1] - w.q_row0, a.Nq);
+        w.k_len = min(a.cu_k[w.bidx + 1] - w.k_row0, a.Nk);
+        w.tma_b = 0;
+    } else {
+        w.q_row0 = 0;
+        w.k_row0 = 0;
+        w.q_len = a.Nq;
+        w.k_len = a.Nk;
+        w.tma_b = w.bidx;
+    }
+    w.rows = w.q0 < w.q_len;
+    // Key tiles query tile qt .. qt + 127 needs.
+    auto tiles_needed = [&](int qt) -> int {
+        if (qt >= w.q_len) return 0;
+        const int last_q = min(qt + 127, w.q_len - 1);
+        const int kend = CAUSAL ? min(w.k_len, last_q + w.k_len - w.q_len + 1) : w.k_len;
+        return kend > 0 ? (kend + 127) / 128 : 0;
+    };
+    w.n_0 = tiles_needed(w.q0);
+    w.n_1 = tiles_needed(w.q0 + 128);
+    w.n_kv = max(w.n_0, w.n_1);
+    return w;
+}
+
+// Unit of round k for CTA c of G: the direction alternates every round.
+__device__ __forceinline__ int fwd_unit_index(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
 
 template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -89,87 +158,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) uint8_t smem[];
     if (!smem_base_ok(smem, args.err)) return;
-
-    // Non-causal grid (256-row units, Hq, batches): neighbouring CTAs share K/V in
-    // L2. Causal grid (Hq, batches, units), last unit first: heaviest CTAs are
-    // dispatched first (longest-processing-time order).
-    const int h = CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
-    const int bidx = CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
-    const int unit = CAUSAL ? static_cast<int>(gridDim.z - 1 - blockIdx.z) : static_cast<int>(blockIdx.x);
-    const int q0 = unit * 256;
-
-    int q_len, k_len, q_row0, k_row0, tma_b;
-    if constexpr (VARLEN) {
-        q_row0 = args.cu_q[bidx];
-        k_row0 = args.cu_k[bidx];
-        q_len = min(args.cu_q[bidx + 1] - q_row0, args.Nq);
-        k_len = min(args.cu_k[bidx + 1] - k_row0, args.Nk);
-        tma_b = 0;
-    } else {
-        q_row0 = 0;
-        k_row0 = 0;
-        q_len = args.Nq;
-        k_len = args.Nk;
-        tma_b = bidx;
-    }
-    if (q0 >= q_len) return;  // uniform over the CTA
-
-    const int hk = h / args.group;
-    // Key tiles each query tile needs: tile t holds rows q0 + 128 t .. + 127.
-    auto tiles_needed = [&](int qt) -> int {
-        if (qt >= q_len) return 0;
-        const int last_q = min(qt + 127, q_len - 1);
-        const int kend = CAUSAL ? min(k_len, last_q + k_len - q_len + 1) : k_len;
-        return kend > 0 ? (kend + 127) / 128 : 0;
-    };
-    const int n_0 = tiles_needed(q0), n_1 = tiles_needed(q0 + 128);
-    const int n_kv = max(n_0, n_1);
+    const int G = static_cast<int>(gridDim.x);
+    const int cta = static_cast<int>(blockIdx.x);
 
     using T16 = uint16_t;
     T16* o_base = static_cast<T16*>(args.o);
-    auto row_valid = [&](int q) -> bool {
-        if (q >= q_len) return false;
-        if constexpr (VARLEN) return q_row0 + q >= 0 && q_row0 + q < args.total_q;
-        return true;
-    };
-    auto o_row = [&](int q) -> T16* {
-        const size_t tok = VARLEN ? static_cast<size_t>(q_row0 + q) : static_cast<size_t>(bidx) * args.Nq + q;
-        return o_base + (tok * args.Hq + h) * D;
-    };
-    auto lse_at = [&](int q) -> float* {
-        if constexpr (VARLEN) {
-            return args.lse + static_cast<size_t>(h) * args.total_q + q_row0 + q;
-        } else {
-            return args.lse + (static_cast<size_t>(bidx) * args.Hq + h) * args.Nq + q;
-        }
-    };
-
-    if (n_kv == 0) {  // no row of this unit sees any key: O = 0, L = -inf
-        if (threadIdx.x < 256) {
-            const int q = q0 + static_cast<int>(threadIdx.x);
-            if (row_valid(q)) {
-                uint4* dst = reinterpret_cast<uint4*>(o_row(q));
-#pragma unroll
-                for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-                *lse_at(q) = -INFINITY;
-            }
-        }
-        return;
-    }
-
     uint8_t* sQ = smem + C::kQOff;
     uint8_t* sK = smem + C::kKOff;
     uint8_t* sV = smem + C::kVOff;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;
+    uint64_t* q_empty = bars + 1;  // the unit's last S product has read Q
+    uint64_t* k_full = bars + 2;
     uint64_t* k_empty = k_full + S;
     uint64_t* v_full = k_empty + S;
     uint64_t* v_empty = v_full + S;
     uint64_t* s_full = v_empty + S;  // [2 tiles]
     uint64_t* p_full = s_full + 2;   // [2]
-    uint64_t* mma_final = p_full + 2;
-    uint64_t* sm_done = mma_final + 1;  // every softmax thread is past its last TMEM access
+    uint64_t* o_free = p_full + 2;   // [2] the epilogue has read O_t
+    uint64_t* o_ready = o_free + 2;  // every product of the unit is complete
+    uint64_t* sm_done = o_ready + 1;  // every softmax thread is past its last TMEM access
+    uint64_t* mma_done = sm_done + 1;  // every product this CTA issued is complete
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     int* abort_flag = reinterpret_cast<int*>(smem + C::kMiscOff + 4);
 
@@ -178,6 +187,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int i = 0; i < S; ++i) {
             mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], 1);
@@ -187,9 +197,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 128);
+            mbar_init(&o_free[i], 128);
         }
-        mbar_init(mma_final, 1);
+        mbar_init(o_ready, 1);
         mbar_init(sm_done, 256);
+        mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -217,33 +229,45 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
+            int k_issued = 0, v_issued = 0, nq = 0;  // K/V tiles and Q pairs issued so far
+            bool ok = true;
+            for (int rnd = 0; ok; ++rnd) {
+                const int u = fwd_unit_index(rnd, cta, G);
+                if (u >= args.n_units) break;
+                const FwdUnit w = fwd_unit<CAUSAL, VARLEN>(u, args);
+                if (!w.rows || w.n_kv == 0) continue;
+                // Q of this unit once the previous unit's last S product has read Q.
+                if (!(ok = mbar_wait(q_empty, (nq & 1) ^ 1u, wc, 60))) break;
+                mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+                for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int s = 0; s < C::kSlabs; ++s)
-                    tma_load_4d(sQ + t * C::kTileBytes + s * C::kSlabBytes, &tm_q, q_full, s * 64, h,
-                                q_row0 + q0 + 128 * t, tma_b);
-            int k_issued = 0, v_issued = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % S;
-                const uint32_t ph = (j / S) & 1;
-                if (!mbar_wait(&k_empty[st], ph ^ 1u, wc, 61)) break;
-                mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
+                    for (int s = 0; s < C::kSlabs; ++s)
+                        tma_load_4d(sQ + t * C::kTileBytes + s * C::kSlabBytes, &tm_q, q_full, s * 64, w.h,
+                                    w.q_row0 + w.q0 + 128 * t, w.tma_b);
+                ++nq;
+                const int hk = w.h / args.group;
+                for (int j = 0; j < w.n_kv; ++j) {
+                    const int g = k_issued, st = g % S;
+                    const uint32_t ph = (g / S) & 1;
+                    if (!(ok = mbar_wait(&k_empty[st], ph ^ 1u, wc, 61))) break;
+                    mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
 #pragma unroll
-                for (int s = 0; s < C::kSlabs; ++s)
-                    tma_load_4d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tm_k, &k_full[st], s * 64, hk,
-                                k_row0 + j * 128, tma_b);
-                ++k_issued;
-                if (!mbar_wait(&v_empty[st], ph ^ 1u, wc, 62)) break;
-                mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
+                    for (int s = 0; s < C::kSlabs; ++s)
+                        tma_load_4d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tm_k, &k_full[st], s * 64, hk,
+                                    w.k_row0 + j * 128, w.tma_b);
+                    ++k_issued;
+                    if (!(ok = mbar_wait(&v_empty[st], ph ^ 1u, wc, 62))) break;
+                    mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
 #pragma unroll
-                for (int s = 0; s < C::kSlabs; ++s)
-                    tma_load_4d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tm_v, &v_full[st], s * 64, hk,
-                                k_row0 + j * 128, tma_b);
-                ++v_issued;
+                    for (int s = 0; s < C::kSlabs; ++s)
+                        tma_load_4d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tm_v, &v_full[st], s * 64, hk,
+                                    w.k_row0 + j * 128, w.tma_b);
+                    ++v_issued;
+                }
             }
-            mbar_wait_drain(q_full, 0);
+            // Leave no load in flight: wait for the last one issued into every buffer.
+            if (nq > 0) mbar_wait_drain(q_full, (nq - 1) & 1);
             for (int st = 0; st < S; ++st) {
                 if (k_issued > st) mbar_wait_drain(&k_full[st], ((st + S * ((k_issued - 1 - st) / S)) / S) & 1);
                 if (v_issued > st) mbar_wait_drain(&v_full[st], ((st + S * ((v_issued - 1 - st) / S)) / S) & 1);
@@ -255,8 +279,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             constexpr uint32_t id_qk = idesc_f16(128, 128, BF16, false, false);
             constexpr uint32_t id_pv = idesc_f16(128, D, BF16, false, true);
             const uint32_t q_addr = smem_u32(sQ);
-            auto issue_s = [&](int t, int j) {
-                const uint32_t k_addr = smem_u32(sK + (j % S) * C::kTileBytes);
+            // S_t = Q_t K^T with the K tile of global ring index g.
+            auto issue_s = [&](int t, int g) {
+                const uint32_t k_addr = smem_u32(sK + (g % S) * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
@@ -265,40 +290,60 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 tc_commit(&s_full[t]);
             };
-            bool ok = mbar_wait(q_full, 0, wc, 63);
-            if (ok) ok = mbar_wait(&k_full[0], 0, wc, 64);
-            if (ok) {
+            int gk = 0, nq = 0;
+            int ps[2] = {0, 0};  // p_full phases consumed per tile
+            bool ok = true;
+            for (int rnd = 0; ok; ++rnd) {
+                const int u = fwd_unit_index(rnd, cta, G);
+                if (u >= args.n_units) break;
+                const FwdUnit w = fwd_unit<CAUSAL, VARLEN>(u, args);
+                if (!w.rows || w.n_kv == 0) continue;
+                if (!(ok = mbar_wait(q_full, nq & 1, wc, 63))) break;
+                if (!(ok = mbar_wait(&k_full[gk % S], (gk / S) & 1, wc, 64))) break;
                 tc_fence_after();
-                if (n_0 > 0) issue_s(0, 0);
-                if (n_1 > 0) issue_s(1, 0);
-                tc_commit(&k_empty[0]);
-            }
-            for (int j = 0; ok && j < n_kv; ++j) {
-                const int st = j % S;
-                const bool more = j + 1 < n_kv;
-                if (!(ok = mbar_wait(&v_full[st], (j / S) & 1, wc, 65))) break;
-                if (more && !(ok = mbar_wait(&k_full[(j + 1) % S], ((j + 1) / S) & 1, wc, 66))) break;
-                const uint32_t v_addr = smem_u32(sV + st * C::kTileBytes);
-                // For each tile: O_t += P_t V_j, then S_t of the next key tile into the
-                // same columns. tcgen05.mma operations of one thread execute in issue
-                // order, so the second cannot overwrite P_t before the first has read
-                // it, and S_t complete implies every earlier P_t V complete.
-                for (int t = 0; ok && t < 2; ++t) {
-                    const int ntt = t ? n_1 : n_0;
-                    if (j >= ntt) continue;
-                    if (!(ok = mbar_wait(&p_full[t], j & 1, wc, 67))) break;
-                    tc_fence_after();
+                // The first S products of this unit run while the softmax warpgroups
+                // still write the previous unit's O (they touch only the S columns).
+                if (w.n_0 > 0) issue_s(0, gk);
+                if (w.n_1 > 0) issue_s(1, gk);
+                if (w.n_kv == 1) tc_commit(q_empty);
+                tc_commit(&k_empty[gk % S]);
+                for (int j = 0; ok && j < w.n_kv; ++j) {
+                    const int g = gk + j, st = g % S;
+                    const bool more = j + 1 < w.n_kv;
+                    if (!(ok = mbar_wait(&v_full[st], (g / S) & 1, wc, 65))) break;
+                    if (more && !(ok = mbar_wait(&k_full[(g + 1) % S], ((g + 1) / S) & 1, wc, 66))) break;
+                    const uint32_t v_addr = smem_u32(sV + st * C::kTileBytes);
+                    // For each tile: O_t += P_t V_j, then S_t of the next key tile into the
+                    // same columns. tcgen05.mma operations of one thread execute in issue
+                    // order, so the second cannot overwrite P_t before the first has read
+                    // it, and S_t complete implies every earlier P_t V complete.
+                    for (int t = 0; ok && t < 2; ++t) {
+                        // O_t is overwritten by the unit's first P_t V: the previous
+                        // unit's epilogue must have read it (waited for every tile, so
+                        // the phases of o_free stay in step with the units).
+                        if (j == 0 && nq > 0 && !(ok = mbar_wait(&o_free[t], (nq - 1) & 1, wc, 67))) break;
+                        const int ntt = t ? w.n_1 : w.n_0;
+                        if (j >= ntt) continue;
+                        if (!(ok = mbar_wait(&p_full[t], ps[t] & 1, wc, 68))) break;
+                        ++ps[t];
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
-                               sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    if (j + 1 < ntt) issue_s(t, j + 1);
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
+                                   sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024), id_pv,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                        if (j + 1 < ntt) issue_s(t, g + 1);
+                    }
+                    if (j + 2 == w.n_kv) tc_commit(q_empty);  // the unit's last S products are issued
+                    tc_commit(&v_empty[st]);
+                    if (more) tc_commit(&k_empty[(g + 1) % S]);
                 }
-                tc_commit(&v_empty[st]);
-                if (more) tc_commit(&k_empty[(j + 1) % S]);
+                tc_commit(o_ready);
+                gk += w.n_kv;
+                ++nq;
             }
-            tc_commit(mma_final);
-            mbar_wait_drain(mma_final, 0);
+            tc_commit(mma_done);
+            mbar_wait_drain(mma_done, 0);
             // TMEM is freed once the softmax warpgroups are done with it. Their waits
             // are bounded, so the arrivals come (4 s bound here as a last resort).
             const uint32_t a = smem_u32(sm_done);
@@ -317,103 +362,136 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int t = (warp - 4) >> 2;  // query tile of this warpgroup
         const int w4 = warp & 3;
         const int r = w4 * 32 + lane;
-        const int qt0 = q0 + 128 * t;
-        const int q = qt0 + r;
-        const int nt = t ? n_1 : n_0;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
         const uint32_t s_addr = lane_base + C::kColS + 128 * t;
         const uint32_t o_addr = lane_base + C::kColO + D * t;
-        const int row_limit = CAUSAL ? min(k_len, q + k_len - q_len + 1) : k_len;
-        // Key tiles at or past this index need masking for some row of the tile.
-        const int min_limit = CAUSAL ? min(k_len, qt0 + k_len - q_len + 1) : k_len;
         const float sl2 = args.scale_log2;
-        float m = -INFINITY, l = 0.f, lr = 0.f;
+        int ss = 0, nq = 0;  // s_full phases consumed; units with work done
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
-            ok = warp_all(mbar_wait(&s_full[t], j & 1, wc, 69));
+        for (int rnd = 0; ok; ++rnd) {
+            const int u = fwd_unit_index(rnd, cta, G);
+            if (u >= args.n_units) break;
+            const FwdUnit w = fwd_unit<CAUSAL, VARLEN>(u, args);
+            if (!w.rows) continue;
+            const int qt0 = w.q0 + 128 * t;
+            const int q = qt0 + r;
+            const int nt = t ? w.n_1 : w.n_0;
+            // This thread's output row (computed where it is used, to keep registers
+            // free during the key loop).
+            auto row_ok = [&]() -> bool {
+                if constexpr (VARLEN) return q < w.q_len && w.q_row0 + q >= 0 && w.q_row0 + q < args.total_q;
+                return q < w.q_len;
+            };
+            auto out_row = [&]() -> T16* {
+                const size_t tok =
+                    VARLEN ? static_cast<size_t>(w.q_row0 + q) : static_cast<size_t>(w.bidx) * args.Nq + q;
+                return o_base + (tok * args.Hq + w.h) * D;
+            };
+            auto lse_row = [&]() -> float* {
+                return VARLEN ? args.lse + static_cast<size_t>(w.h) * args.total_q + w.q_row0 + q
+                              : args.lse + (static_cast<size_t>(w.bidx) * args.Hq + w.h) * args.Nq + q;
+            };
+            if (w.n_kv == 0) {  // no row of this unit sees any key: O = 0, L = -inf
+                if (row_ok()) {
+                    uint4* d4 = reinterpret_cast<uint4*>(out_row());
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c) d4[c] = make_uint4(0, 0, 0, 0);
+                    *lse_row() = -INFINITY;
+                }
+                continue;
+            }
+            const int row_limit = CAUSAL ? min(w.k_len, q + w.k_len - w.q_len + 1) : w.k_len;
+            // Key tiles at or past this index need masking for some row of the tile.
+            const int min_limit = CAUSAL ? min(w.k_len, qt0 + w.k_len - w.q_len + 1) : w.k_len;
+            float m = -INFINITY, l = 0.f, lr = 0.f;
+            for (int j = 0; j < nt; ++j) {
+                ok = warp_all(mbar_wait(&s_full[t], ss & 1, wc, 69));
+                if (!ok) break;
+                ++ss;
+                tc_fence_after();
+                const int lim = row_limit - j * 128;  // columns >= lim are masked
+                const bool need_mask = j * 128 + 128 > min_limit;
+                uint32_t sv[4][32];
+    #pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
+    #pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
+                if (need_mask) {  // masked columns read as -inf: out of the max, P = 0
+    #pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c >= lim) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                }
+                // Row max: 8 independent chains of three-input max.
+                float mxp[8];
+    #pragma unroll
+                for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
+    #pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    mxp[i & 7] = fmax3(mxp[i & 7], __uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
+                                       __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
+                const float mx = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
+                const float m_new = fmaxf(m, mx * sl2);
+                float alpha = 1.f;
+                bool resc = false;
+                if (m_new > m + kRescaleThreshold) {  // false while the row has seen no key
+                    if (m != -INFINITY) {
+                        alpha = ex2_approx(m - m_new);
+                        resc = true;
+                    }
+                    m = m_new;
+                }
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                // P = 2^(S c - m) as 16-bit pairs (keys 2i, 2i + 1 in column i), partial sums
+                // of the exact and of the rounded values.
+                // Pairs of keys go through the packed f32x2 FMA and adds.
+                const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(neg_m, neg_m);
+                uint64_t rs2[4] = {0, 0, 0, 0}, rsr2[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
+                uint32_t pk[2][32];
+    #pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const uint64_t x = f2_pack(__uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
+                                               __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
+                    float y0, y1;
+                    f2_unpack(f2_fma(x, c2, m2), y0, y1);
+                    const float p0 = ex2_approx(y0);
+                    const float p1 = ex2_approx(y1);
+                    rs2[i & 3] = f2_add(rs2[i & 3], f2_pack(p0, p1));
+                    const uint32_t u = pack2<BF16>(p0, p1);
+                    rsr2[i & 3] = f2_add(rsr2[i & 3], f2_pack(unpack_lo<BF16>(u), unpack_hi<BF16>(u)));
+                    pk[i >> 5][i & 31] = u;
+                }
+                tmem_st32(s_addr + 0, pk[0]);
+                tmem_st32(s_addr + 32, pk[1]);
+                const float rs = f2_sum(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])));
+                const float rsr = f2_sum(f2_add(f2_add(rsr2[0], rsr2[1]), f2_add(rsr2[2], rsr2[3])));
+                l = l * alpha + rs;
+                lr = lr * alpha + rsr;
+                // S_t was issued after the previous key tile's P_t V and MMAs of one thread
+                // complete in order, so O_t is final for that tile here and can be
+                // rescaled in place.
+                if (j > 0 && __any_sync(0xffffffffu, resc)) {
+    #pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t ov[32];
+                        tmem_ld32(o_addr + c0, ov);
+                        tmem_ld_wait(ov);
+    #pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                        tmem_st32(o_addr + c0, ov);
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&p_full[t]);
+            }
             if (!ok) break;
+            ok = warp_all(mbar_wait(o_ready, nq & 1, wc, 70));
+            if (!ok) break;
+            ++nq;
             tc_fence_after();
-            const int lim = row_limit - j * 128;  // columns >= lim are masked
-            const bool need_mask = j * 128 + 128 > min_limit;
-            uint32_t sv[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
-            if (need_mask) {  // masked columns read as -inf: out of the max, P = 0
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= lim) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-            }
-            // Row max: 8 independent chains of three-input max.
-            float mxp[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-                mxp[i & 7] = fmax3(mxp[i & 7], __uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
-                                   __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
-            const float mx = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
-            const float m_new = fmaxf(m, mx * sl2);
-            float alpha = 1.f;
-            bool resc = false;
-            if (m_new > m + kRescaleThreshold) {  // false while the row has seen no key
-                if (m != -INFINITY) {
-                    alpha = ex2_approx(m - m_new);
-                    resc = true;
-                }
-                m = m_new;
-            }
-            const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            // P = 2^(S c - m) as 16-bit pairs (keys 2i, 2i + 1 in column i), partial sums
-            // of the exact and of the rounded values.
-            // Pairs of keys go through the packed f32x2 FMA and adds.
-            const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(neg_m, neg_m);
-            uint64_t rs2[4] = {0, 0, 0, 0}, rsr2[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
-            uint32_t pk[2][32];
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const uint64_t x = f2_pack(__uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
-                                           __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
-                float y0, y1;
-                f2_unpack(f2_fma(x, c2, m2), y0, y1);
-                const float p0 = ex2_approx(y0);
-                const float p1 = ex2_approx(y1);
-                rs2[i & 3] = f2_add(rs2[i & 3], f2_pack(p0, p1));
-                const uint32_t u = pack2<BF16>(p0, p1);
-                rsr2[i & 3] = f2_add(rsr2[i & 3], f2_pack(unpack_lo<BF16>(u), unpack_hi<BF16>(u)));
-                pk[i >> 5][i & 31] = u;
-            }
-            tmem_st32(s_addr + 0, pk[0]);
-            tmem_st32(s_addr + 32, pk[1]);
-            const float rs = f2_sum(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])));
-            const float rsr = f2_sum(f2_add(f2_add(rsr2[0], rsr2[1]), f2_add(rsr2[2], rsr2[3])));
-            l = l * alpha + rs;
-            lr = lr * alpha + rsr;
-            // S_t was issued after the previous key tile's P_t V and MMAs of one thread
-            // complete in order, so O_t is final for that tile here and can be
-            // rescaled in place.
-            if (j > 0 && __any_sync(0xffffffffu, resc)) {
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t ov[32];
-                    tmem_ld32(o_addr + c0, ov);
-                    tmem_ld_wait(ov);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(o_addr + c0, ov);
-                }
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&p_full[t]);
-        }
-        if (nt > 0 && ok) ok = warp_all(mbar_wait(mma_final, 0, wc, 70));
-        if (ok) {
-            tc_fence_after();
-            const bool row_ok = row_valid(q);
             const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
-            T16* dst = row_ok ? o_row(q) : nullptr;
+            const bool out_ok = row_ok();
+            T16* dst = out_ok ? out_row() : nullptr;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t pk[16];
@@ -428,20 +506,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pk[i] = 0u;
                 }
-                if (row_ok) {
+                if (out_ok) {
                     uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                 }
             }
-            if (row_ok) {
+            // O_t's columns are free for the next unit's first P_t V.
+            tc_fence_before();
+            mbar_arrive(&o_free[t]);
+            if (out_ok) {
                 float L = -INFINITY;
                 if (l > 0.f) {
                     float lg;
                     asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l));
                     L = (m + lg) * kLn2;
                 }
-                *lse_at(q) = L;
+                *lse_row() = L;
             }
         }
         tc_fence_before();
