@@ -467,6 +467,27 @@ def run_sweep(args):
         ms = time_it(lambda: fb.attention_varlen_fwd(q, k, v, cu_q, cu_k, vi.max_seqlen_q, vi.max_seqlen_k,
                                                      cfg.scale, cfg.causal, out=o, lse=lse), 20)
         emit(cfg.name, "fwd", ms, flops, nbytes)
+        if cfg is inputs.VARLEN:
+            # the varlen backward on the same packed batch (dO drawn after Q, K, V)
+            do = inputs.make_varlen(cfg, with_do=True).do.cuda()
+            n, Tq, Tk = len(vi.seqlens_q), q.shape[0], k.shape[0]
+            ws = torch.empty(fb.fa_varlen_bwd_workspace_size(n, Tq, vi.max_seqlen_q, cfg.Hq, cfg.d),
+                             dtype=torch.uint8, device="cuda")
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            dt = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
+
+            def vbwd():
+                st = fb.fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                      do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                                      cu_q.data_ptr(), cu_k.data_ptr(), n, Tq, Tk, vi.max_seqlen_q,
+                                      vi.max_seqlen_k, cfg.Hq, cfg.Hkv, cfg.d, cfg.scale, int(cfg.causal), dt,
+                                      stream.cuda_stream)
+                if st != fb.FA_OK:
+                    raise RuntimeError(fb.fa_status_string(st))
+
+            ms = time_it(vbwd, 10)
+            emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+            del do, ws, dq, dk, dv
     return 0
 
 

@@ -1,6 +1,6 @@
 """Thin ctypes binding of libfa.so.
 
-The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_bwd_workspace_size``,
+The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
 ``fa_bwd``, ``fa_status_string`` and ``fa_get_last_device_error`` have the
 names, argument order and meaning of the C ABI in ``include/fa.h``: pointers
 are passed as integers (device addresses), streams as integers (0 = default
@@ -40,6 +40,8 @@ _SIGS = {
     "fa_version": ([], ctypes.c_char_p),
     "fa_bwd_set_timing_events": ([_P, _P], None),
     "fa_bwd_noalloc": ([_P] * 9 + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_varlen_bwd_workspace_size": ([_I] * 5, ctypes.c_size_t),
+    "fa_varlen_bwd": ([_P] * 12 + [_I] * 8 + [_F, _I, _I, _P], _I),
     "fa_selftest_bounded_wait": ([_P], _I),
 }
 
@@ -83,6 +85,17 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, 
            stream) -> int:
     return lib().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal,
                         dtype, stream)
+
+
+def fa_varlen_bwd_workspace_size(num_seqs, total_q, max_seqlen_q, Hq, d) -> int:
+    return int(lib().fa_varlen_bwd_workspace_size(num_seqs, total_q, max_seqlen_q, Hq, d))
+
+
+def fa_varlen_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q,
+                  total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream) -> int:
+    return lib().fa_varlen_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs,
+                               total_q, total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype,
+                               stream)
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
@@ -193,4 +206,27 @@ def attention_bwd(q, k, v, o, lse, dout, scale: float | None = None, causal: boo
     _check(fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
                   dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
                   int(bool(causal)), _dtype_code(q), _stream(stream)), "fa_bwd")
+    return dq, dk, dv
+
+
+def attention_varlen_bwd(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                         scale: float | None = None, causal: bool = False, workspace=None, stream=None):
+    """dQ, dK, dV of the packed varlen forward (same layouts as q, k, v; d = 128)."""
+    import torch
+    q, k, v, o, dout = _dev(q), _dev(k), _dev(v), _dev(o), _dev(dout)
+    lse = _dev(lse)
+    cu_q = _dev(cu_seqlens_q).to(torch.int32)
+    cu_k = _dev(cu_seqlens_k).to(torch.int32)
+    Tq, Hq, d = q.shape
+    Tk, Hkv, _ = k.shape
+    n = cu_q.numel() - 1
+    if scale is None:
+        scale = d ** -0.5
+    ws_bytes = fa_varlen_bwd_workspace_size(n, Tq, int(max_seqlen_q), Hq, d)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq, dk, dv = torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)
+    _check(fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), cu_q.data_ptr(), cu_k.data_ptr(),
+                         n, Tq, Tk, int(max_seqlen_q), int(max_seqlen_k), Hq, Hkv, d, float(scale),
+                         int(bool(causal)), _dtype_code(q), _stream(stream)), "fa_varlen_bwd")
     return dq, dk, dv

@@ -168,12 +168,12 @@ __global__ void fa_selftest_wait_kernel(int* err) {
 
 // d = 128 runs fa_bwd128_kernel (dQ^T = K^T dS^T with N = 128 queries); d = 64
 // the single-tile kernel (its dQ^T would need M = 64, so it keeps dQ = dS K with
-// M = 128 queries).
-template <int D, bool BF16, bool CAUSAL>
+// M = 128 queries; fixed length only).
+template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const fa::BwdArgs& a, dim3 grid, cudaStream_t stream) {
     if constexpr (D == 128) {
-        auto kern = fa::fa_bwd128_kernel<BF16, CAUSAL>;
+        auto kern = fa::fa_bwd128_kernel<BF16, CAUSAL, VARLEN>;
         constexpr int smem = fa::Bwd128Cfg::kSmemBytes;
         static bool attr_ok =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
@@ -187,6 +187,7 @@ fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
         if (launch_regs < fa::kBwd128MinLaunchRegs) return FA_ERR_UNSUPPORTED;
         kern<<<grid, fa::kBwd128Threads, smem, stream>>>(mq, mk, mv, mdo, a);
     } else {
+        static_assert(!VARLEN, "the d = 64 backward is fixed length only");
         auto kern = fa::fa_bwd_kernel<D, BF16, CAUSAL>;
         constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
         static bool attr_ok =
@@ -197,13 +198,107 @@ fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D>
+template <int D, bool VARLEN>
 fa_status launch_bwd_d(bool bf16, bool causal, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mdo, const fa::BwdArgs& a, dim3 grid, cudaStream_t s) {
-    if (bf16) return causal ? launch_bwd_t<D, true, true>(mq, mk, mv, mdo, a, grid, s)
-                            : launch_bwd_t<D, true, false>(mq, mk, mv, mdo, a, grid, s);
-    return causal ? launch_bwd_t<D, false, true>(mq, mk, mv, mdo, a, grid, s)
-                  : launch_bwd_t<D, false, false>(mq, mk, mv, mdo, a, grid, s);
+    if (bf16) return causal ? launch_bwd_t<D, true, true, VARLEN>(mq, mk, mv, mdo, a, grid, s)
+                            : launch_bwd_t<D, true, false, VARLEN>(mq, mk, mv, mdo, a, grid, s);
+    return causal ? launch_bwd_t<D, false, true, VARLEN>(mq, mk, mv, mdo, a, grid, s)
+                  : launch_bwd_t<D, false, false, VARLEN>(mq, mk, mv, mdo, a, grid, s);
+}
+
+// Floats in the dQ accumulator: [B, Nq, Hq, 64] for d = 64; for d = 128 the
+// queries of each (sequence, head) are padded to a multiple of four
+// ([B, Hq, nq4, 128, 4]); varlen uses the same layout with B = num_seqs and
+// Nq = max_seqlen_q.
+size_t acc_floats(int B, int Hq, int Nq, int d) {
+    if (d == 64) return static_cast<size_t>(B) * Hq * Nq * 64;
+    return static_cast<size_t>(B) * Hq * ((static_cast<size_t>(Nq) + 3) / 4) * 512;
+}
+
+// The backward of fa_bwd and fa_varlen_bwd. Fixed length: nseq = B, rows = B * Nq,
+// cu_q = cu_k = nullptr. Varlen: nseq = num_seqs, Nq / Nk the max_seqlen bounds,
+// rows = total_q, and the maps span the packed buffers (total_q / total_k rows).
+fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, void* workspace, int nseq, const int* cu_q,
+                     const int* cu_k, int total_q, int total_k, int Hq, int Hkv, int Nq, int Nk, int d,
+                     float scale, bool causal, bool bf16, cudaStream_t s) {
+    const bool varlen = cu_q != nullptr;
+    int* err = error_word();
+    if (!err) return FA_ERR_CUDA;
+    fa_status st;
+    const size_t rows = static_cast<size_t>(varlen ? total_q : nseq * static_cast<size_t>(Nq)) * Hq;
+    float* Dvec = static_cast<float*>(workspace);
+    float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256(rows * sizeof(float)));
+    const size_t acc_f4 = acc_floats(nseq, Hq, Nq, d) / 4;
+    if (rows > 0) {
+        const size_t threads = rows * (d / 8);
+        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        // D = rowsum(dO o O) over [rows, d] viewed as one batch of rows / Hq tokens:
+        // D lands in [Hq, tokens] = L's layout for varlen, [B, Hq, Nq] for fixed length.
+        const int pb = varlen ? 1 : nseq, pn = varlen ? total_q : Nq;
+        if (d == 64)
+            fa::fa_bwd_preprocess<64><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
+                                                             static_cast<const uint16_t*>(dout), Dvec, dq_acc, acc_f4,
+                                                             pb, pn, Hq, bf16);
+        else
+            fa::fa_bwd_preprocess<128><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
+                                                              static_cast<const uint16_t*>(dout), Dvec, dq_acc,
+                                                              acc_f4, pb, pn, Hq, bf16);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    const int kb = varlen ? 1 : nseq;
+    const int kq_rows = varlen ? total_q : Nq, kk_rows = varlen ? total_k : Nk;
+    if (kk_rows > 0 && Nk > 0) {
+        CUtensorMap mq{}, mdo{}, mk, mv;
+        if (kq_rows > 0 && (st = make_map(&mq, q, d, Hq, kq_rows, kb, bf16)) != FA_OK) return st;
+        if (kq_rows > 0 && (st = make_map(&mdo, dout, d, Hq, kq_rows, kb, bf16)) != FA_OK) return st;
+        if ((st = make_map(&mk, k, d, Hkv, kk_rows, kb, bf16)) != FA_OK) return st;
+        if ((st = make_map(&mv, v, d, Hkv, kk_rows, kb, bf16)) != FA_OK) return st;
+        fa::BwdArgs a{};
+        a.lse = lse;
+        a.D = Dvec;
+        a.dq_acc = dq_acc;
+        a.nq4 = (Nq + 3) / 4;
+        a.dk = dk;
+        a.dv = dv;
+        a.Hq = Hq;
+        a.Hkv = Hkv;
+        a.group = Hq / Hkv;
+        a.Nq = Nq;
+        a.Nk = Nk;
+        a.cu_q = cu_q;
+        a.cu_k = cu_k;
+        a.total_q = total_q;
+        a.scale = scale;
+        a.scale_log2 = scale * kLog2e;
+        a.err = err;
+        const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
+        if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
+        const dim3 grid = causal ? dim3(Hkv, nseq, nkt) : dim3(nkt, Hkv, nseq);
+        const bool timed = g_bwd_ev_before && g_bwd_ev_after;
+        if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;
+        if (varlen)
+            st = launch_bwd_d<128, true>(bf16, causal, mq, mk, mv, mdo, a, grid, s);
+        else
+            st = d == 64 ? launch_bwd_d<64, false>(bf16, causal, mq, mk, mv, mdo, a, grid, s)
+                         : launch_bwd_d<128, false>(bf16, causal, mq, mk, mv, mdo, a, grid, s);
+        if (st != FA_OK) return st;
+        if (timed && cudaEventRecord(g_bwd_ev_after, s) != cudaSuccess) return FA_ERR_CUDA;
+    }
+    if (rows > 0) {
+        if (d == 64) {
+            const size_t n8 = rows * d / 8;
+            fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
+                dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16);
+        } else {
+            const size_t n = static_cast<size_t>(nseq) * Hq * ((Nq + 3) / 4) * 64;
+            fa::fa_bwd_dq_convert_g4<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+                dq_acc, static_cast<uint16_t*>(dq), cu_q, nseq, Hq, Nq, (Nq + 3) / 4, scale, bf16);
+        }
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return FA_OK;
 }
 
 }  // namespace
@@ -298,13 +393,6 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
     return launch_fwd(d, bf16, causal != 0, true, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
-// Floats in the dQ accumulator: [B, Nq, Hq, 64] for d = 64; for d = 128 the
-// queries of each (b, h) are padded to a multiple of four ([B, Hq, nq4, 128, 4]).
-static size_t acc_floats(int B, int Hq, int Nq, int d) {
-    if (d == 64) return static_cast<size_t>(B) * Hq * Nq * 64;
-    return static_cast<size_t>(B) * Hq * ((static_cast<size_t>(Nq) + 3) / 4) * 512;
-}
-
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {
     if (B < 1 || Hq < 1 || Nq < 0 || (d != 64 && d != 128)) return 0;
     const size_t rows = static_cast<size_t>(B) * Hq * Nq;
@@ -323,71 +411,37 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
         return FA_ERR_MISALIGNED;
     if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
-    int* err = error_word();
-    if (!err) return FA_ERR_CUDA;
-    const bool bf16 = dtype == FA_BF16;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const size_t rows = static_cast<size_t>(B) * Nq * Hq;
-    float* Dvec = static_cast<float*>(workspace);
-    float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256(rows * sizeof(float)));
-    if (rows > 0) {
-        const size_t threads = rows * (d / 8);
-        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
-        const size_t acc_f4 = acc_floats(B, Hq, Nq, d) / 4;
-        if (d == 64)
-            fa::fa_bwd_preprocess<64><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
-                                                             static_cast<const uint16_t*>(dout), Dvec, dq_acc, acc_f4,
-                                                             B, Nq, Hq, bf16);
-        else
-            fa::fa_bwd_preprocess<128><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
-                                                              static_cast<const uint16_t*>(dout), Dvec, dq_acc,
-                                                              acc_f4, B, Nq, Hq, bf16);
-        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    }
-    if (Nk > 0) {
-        CUtensorMap mq{}, mdo{}, mk, mv;
-        if (Nq > 0 && (st = make_map(&mq, q, d, Hq, Nq, B, bf16)) != FA_OK) return st;
-        if (Nq > 0 && (st = make_map(&mdo, dout, d, Hq, Nq, B, bf16)) != FA_OK) return st;
-        if ((st = make_map(&mk, k, d, Hkv, Nk, B, bf16)) != FA_OK) return st;
-        if ((st = make_map(&mv, v, d, Hkv, Nk, B, bf16)) != FA_OK) return st;
-        fa::BwdArgs a{};
-        a.lse = lse;
-        a.D = Dvec;
-        a.dq_acc = dq_acc;
-        a.nq4 = (Nq + 3) / 4;
-        a.dk = dk;
-        a.dv = dv;
-        a.Hq = Hq;
-        a.Hkv = Hkv;
-        a.group = Hq / Hkv;
-        a.Nq = Nq;
-        a.Nk = Nk;
-        a.scale = scale;
-        a.scale_log2 = scale * kLog2e;
-        a.err = err;
-        const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
-        if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
-        const dim3 grid = causal ? dim3(Hkv, B, nkt) : dim3(nkt, Hkv, B);
-        const bool timed = g_bwd_ev_before && g_bwd_ev_after;
-        if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;
-        st = d == 64 ? launch_bwd_d<64>(bf16, causal != 0, mq, mk, mv, mdo, a, grid, s)
-                     : launch_bwd_d<128>(bf16, causal != 0, mq, mk, mv, mdo, a, grid, s);
-        if (st != FA_OK) return st;
-        if (timed && cudaEventRecord(g_bwd_ev_after, s) != cudaSuccess) return FA_ERR_CUDA;
-    }
-    if (rows > 0) {
-        if (d == 64) {
-            const size_t n8 = rows * d / 8;
-            fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
-                dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16);
-        } else {
-            const size_t n = static_cast<size_t>(B) * Hq * ((Nq + 3) / 4) * 64;
-            fa::fa_bwd_dq_convert_g4<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
-                dq_acc, static_cast<uint16_t*>(dq), B, Hq, Nq, (Nq + 3) / 4, scale, bf16);
-        }
-        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    }
-    return FA_OK;
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
+                      scale, causal != 0, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q, int Hq, int d) {
+    if (num_seqs < 1 || total_q < 0 || max_seqlen_q < 0 || Hq < 1 || d != 128) return 0;
+    const size_t rows = static_cast<size_t>(total_q) * Hq;
+    return round256(rows * sizeof(float)) + round256(acc_floats(num_seqs, Hq, max_seqlen_q, d) * sizeof(float));
+}
+
+fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* workspace, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
+                        int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
+                        fa_stream_t stream) {
+    if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+        return FA_ERR_INVALID_ARG;
+    if (!cu_seqlens_q || !cu_seqlens_k || !workspace || (total_q > 0 && (!q || !o || !lse || !dout || !dq)) ||
+        (total_k > 0 && (!k || !v || !dk || !dv)))
+        return FA_ERR_INVALID_ARG;
+    fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
+    if (st != FA_OK) return st;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+        return FA_ERR_MISALIGNED;
+    if (num_seqs > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, num_seqs, cu_seqlens_q, cu_seqlens_k, total_q,
+                      total_k, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal != 0, dtype == FA_BF16,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_get_last_device_error(fa_stream_t stream) {

@@ -48,7 +48,10 @@ struct BwdArgs {
     int nq4;           // groups of four queries per (b, h) in the d = 128 layout: ceil(Nq / 4)
     void* dk;          // [B, Nk, Hkv, d]
     void* dv;
-    int Hq, Hkv, group, Nq, Nk;
+    int Hq, Hkv, group, Nq, Nk;  // varlen: Nq, Nk are the max_seqlen bounds
+    const int* cu_q;             // varlen: [num_seqs + 1] row offsets of the packed buffers
+    const int* cu_k;
+    int total_q;                 // varlen: rows of q / o / dO (L and D are [Hq, total_q])
     float scale;
     float scale_log2;
     int* err;
@@ -468,9 +471,11 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert(const float* dq_acc, ui
 // index together: element (b, h, q, c) sits at ((b Hq + h) nq4 + q / 4) 512 +
 // 4 c + q % 4, so a warp of the backward main kernel (lane = c) adds four
 // queries with one coalesced 512-byte vector reduction. One thread here turns
-// head-dimension indices 2p, 2p + 1 of a group of four queries into dQ[b, q, h, :].
-__global__ void __launch_bounds__(256) fa_bwd_dq_convert_g4(const float* dq_acc, uint16_t* dq, int B, int Hq,
-                                                             int Nq, int nq4, float scale, bool bf16) {
+// head-dimension indices 2p, 2p + 1 of a group of four queries into dQ[token, h, :]:
+// token b Nq + q for fixed length, cu_q[b] + q for varlen (cu_q non-null; b is the
+// sequence, Nq the max_seqlen bound).
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_g4(const float* dq_acc, uint16_t* dq, const int* cu_q,
+                                                             int B, int Hq, int Nq, int nq4, float scale, bool bf16) {
     const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // (b, h, g, p)
     const size_t groups = static_cast<size_t>(B) * Hq * nq4;
     if (i >= groups * 64) return;
@@ -479,16 +484,22 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_g4(const float* dq_acc,
     const int g = static_cast<int>(bhg % nq4);
     const size_t bh = bhg / nq4;
     const int h = static_cast<int>(bh % Hq);
-    const size_t b = bh / Hq;
+    const int b = static_cast<int>(bh / Hq);
+    int q_len = Nq;
+    size_t row0 = static_cast<size_t>(b) * Nq;
+    if (cu_q) {
+        row0 = static_cast<size_t>(cu_q[b]);
+        q_len = min(cu_q[b + 1] - cu_q[b], Nq);
+    }
     const float4* src = reinterpret_cast<const float4*>(dq_acc) + bhg * 128 + 2 * p;
     const float4 a = src[0], c = src[1];
     const float lo[4] = {a.x, a.y, a.z, a.w}, hi[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int q = 4 * g + j;
-        if (q >= Nq) break;
+        if (q >= q_len) break;
         const uint32_t v = bf16 ? pack2<true>(lo[j] * scale, hi[j] * scale) : pack2<false>(lo[j] * scale, hi[j] * scale);
-        reinterpret_cast<uint32_t*>(dq + ((b * Nq + q) * Hq + h) * 128)[p] = v;
+        reinterpret_cast<uint32_t*>(dq + ((row0 + q) * Hq + h) * 128)[p] = v;
     }
 }
 

@@ -65,7 +65,7 @@ __device__ __forceinline__ uint32_t pair_col(int kk) {
     return static_cast<uint32_t>(kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
 }
 
-template <bool BF16, bool CAUSAL>
+template <bool BF16, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(kBwd128Threads, 1)
     fa_bwd128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -79,7 +79,28 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
     const int hk = CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
     const int b = CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
     const int k0 = kt * 128;
-    const int Nq = args.Nq, Nk = args.Nk;
+    // Rows of this sequence: fixed length, or varlen (b is the sequence; its rows
+    // start at q_row0 / k_row0 of the packed buffers).
+    int q_len, k_len, q_row0, k_row0, tma_b;
+    if constexpr (VARLEN) {
+        q_row0 = args.cu_q[b];
+        k_row0 = args.cu_k[b];
+        q_len = min(args.cu_q[b + 1] - q_row0, args.Nq);
+        k_len = min(args.cu_k[b + 1] - k_row0, args.Nk);
+        tma_b = 0;
+        if (k0 >= k_len) return;  // the tile lies past this sequence's keys
+    } else {
+        q_row0 = 0;
+        k_row0 = 0;
+        q_len = args.Nq;
+        k_len = args.Nk;
+        tma_b = b;
+    }
+    const int Nq = q_len, Nk = k_len;
+    // Token index of key `key` of this sequence in the dK / dV buffers.
+    auto key_tok = [&](int key) -> size_t {
+        return VARLEN ? static_cast<size_t>(k_row0 + key) : static_cast<size_t>(b) * Nk + key;
+    };
     const int n_qt = (Nq + 127) / 128;
     int i0 = 0;
     if (CAUSAL) {
@@ -97,7 +118,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         if (threadIdx.x < 128) {
             const int key = k0 + static_cast<int>(threadIdx.x);
             if (key < Nk) {
-                const size_t off = ((static_cast<size_t>(b) * Nk + key) * args.Hkv + hk) * D;
+                const size_t off = (key_tok(key) * args.Hkv + hk) * D;
                 uint4* a = reinterpret_cast<uint4*>(static_cast<T16*>(args.dk) + off);
                 uint4* c = reinterpret_cast<uint4*>(static_cast<T16*>(args.dv) + off);
 #pragma unroll
@@ -177,8 +198,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
-                tma_load_4d(sK + s * C::kSlabBytes, &tm_k, kv_full, s * 64, hk, k0, b);
-                tma_load_4d(sV + s * C::kSlabBytes, &tm_v, kv_full, s * 64, hk, k0, b);
+                tma_load_4d(sK + s * C::kSlabBytes, &tm_k, kv_full, s * 64, hk, k_row0 + k0, tma_b);
+                tma_load_4d(sV + s * C::kSlabBytes, &tm_v, kv_full, s * 64, hk, k_row0 + k0, tma_b);
             }
             int issued = 0;
             for (int it = 0; it < n_it; ++it) {
@@ -189,8 +210,10 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
                 mbar_arrive_expect_tx(&q_full[st], 2 * C::kTileBytes);
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    tma_load_4d(sQ + st * C::kTileBytes + s * C::kSlabBytes, &tm_q, &q_full[st], s * 64, h, q0, b);
-                    tma_load_4d(sDO + st * C::kTileBytes + s * C::kSlabBytes, &tm_do, &q_full[st], s * 64, h, q0, b);
+                    tma_load_4d(sQ + st * C::kTileBytes + s * C::kSlabBytes, &tm_q, &q_full[st], s * 64, h,
+                                q_row0 + q0, tma_b);
+                    tma_load_4d(sDO + st * C::kTileBytes + s * C::kSlabBytes, &tm_do, &q_full[st], s * 64, h,
+                                q_row0 + q0, tma_b);
                 }
                 ++issued;
                 // Warm the L2 with the tiles two iterations ahead.
@@ -199,8 +222,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
                     const int q2 = qtile(it + 2) * 128;
 #pragma unroll
                     for (int s = 0; s < 2; ++s) {
-                        tma_prefetch_l2_4d(&tm_q, s * 64, h2, q2, b);
-                        tma_prefetch_l2_4d(&tm_do, s * 64, h2, q2, b);
+                        tma_prefetch_l2_4d(&tm_q, s * 64, h2, q_row0 + q2, tma_b);
+                        tma_prefetch_l2_4d(&tm_do, s * 64, h2, q_row0 + q2, tma_b);
                     }
                 }
             }
@@ -301,7 +324,9 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             if (r < 64 && it_ < n_it) {
                 const int q = qtile(it_) * 128 + w * 64 + r;
                 if (q < Nq) {
-                    const size_t row = (static_cast<size_t>(b) * args.Hq + hk * args.group + it_ / n_i) * Nq + q;
+                    const int hq = hk * args.group + it_ / n_i;
+                    const size_t row = VARLEN ? static_cast<size_t>(hq) * args.total_q + q_row0 + q
+                                              : (static_cast<size_t>(b) * args.Hq + hq) * Nq + q;
                     const float L = __ldg(args.lse + row);
                     l2 = (L == -INFINITY) ? -INFINITY : -L * kLog2eF;  // a row that saw no key has P = 0
                     dd = -__ldg(args.D + row);
@@ -420,8 +445,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             // Warpgroup 0 writes dV, warpgroup 1 writes dK = scale * (dS^T Q).
             const uint32_t col = w == 0 ? C::kColDV : C::kColDK;
             const float mul = w == 0 ? 1.f : args.scale;
-            T16* dst = static_cast<T16*>(w == 0 ? args.dv : args.dk) +
-                       ((static_cast<size_t>(b) * Nk + key) * args.Hkv + hk) * D;
+            T16* dst = static_cast<T16*>(w == 0 ? args.dv : args.dk) + (key_tok(key) * args.Hkv + hk) * D;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t v[32];

@@ -153,6 +153,7 @@ class VarlenInputs:
     v: torch.Tensor  # [total_k, Hkv, d]
     k_padded: torch.Tensor = field(repr=False, default=None)  # [total_q, Hkv, d] before unpad
     v_padded: torch.Tensor = field(repr=False, default=None)
+    do: torch.Tensor | None = None  # [total_q, Hq, d] when drawn (with_do=True)
 
 
 def _cumsum(lengths: list[int]) -> torch.Tensor:
@@ -162,7 +163,8 @@ def _cumsum(lengths: list[int]) -> torch.Tensor:
     return torch.tensor(cu, dtype=torch.int32)
 
 
-def make_varlen(cfg: VarlenConfig, lengths: list[int] | None = None, **override) -> VarlenInputs:
+def make_varlen(cfg: VarlenConfig, lengths: list[int] | None = None, with_do: bool = False,
+                **override) -> VarlenInputs:
     """Draw a packed variable-length batch.
 
     Lengths are i.i.d. uniform integers in [min_len, max_len] from their own
@@ -170,6 +172,8 @@ def make_varlen(cfg: VarlenConfig, lengths: list[int] | None = None, **override)
     ``key_pad_frac`` > 0 the last floor(frac * L) keys of each sequence are
     padding: the full packed K/V is drawn, then the padding rows are removed
     (the unpad step), and ``cu_seqlens_k`` addresses the unpadded buffer.
+    With ``with_do`` the output gradient dO is drawn last, after V, so Q, K
+    and V are the same with or without it.
     """
     if override:
         cfg = VarlenConfig(**{**cfg.__dict__, **override})
@@ -183,6 +187,7 @@ def make_varlen(cfg: VarlenConfig, lengths: list[int] | None = None, **override)
     q = _normal(g, (total, cfg.Hq, cfg.d)).to(dt)
     kf = _normal(g, (total, cfg.Hkv, cfg.d)).to(dt)
     vf = _normal(g, (total, cfg.Hkv, cfg.d)).to(dt)
+    do = _normal(g, (total, cfg.Hq, cfg.d)).to(dt) if with_do else None
     lk = [n - int(cfg.key_pad_frac * n) for n in lengths]
     cu_q = _cumsum(lengths)
     if cfg.key_pad_frac > 0:
@@ -193,5 +198,5 @@ def make_varlen(cfg: VarlenConfig, lengths: list[int] | None = None, **override)
     else:
         k, v = kf, vf
     return VarlenInputs(cfg, lengths, lk, cu_q, _cumsum(lk), max(lengths, default=0),
-                        max(lk, default=0), q, k, v, kf, vf)
+                        max(lk, default=0), q, k, v, kf, vf, do)
 

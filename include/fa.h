@@ -129,6 +129,38 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  float scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * Size in bytes of the caller-owned workspace fa_varlen_bwd needs: D
+ * (float32 [Hq,total_q]) and the float32 dQ accumulator
+ * (num_seqs*Hq*ceil(max_seqlen_q/4)*4*128 floats, each sequence padded to
+ * max_seqlen_q), each rounded up to 256 bytes. d must be 128; returns 0 for
+ * invalid sizes.
+ */
+size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q, int Hq, int d);
+
+/*
+ * Backward, packed variable length: the gradients of fa_varlen_fwd, with
+ * the mathematics of fa_bwd applied to every sequence on its own ("FlashAttention/zh",
+ * section "backward pass and recomputation"; the varlen layout of the
+ * InternViT FlashAttention wrapper).
+ *   q, k, v, o, lse, cu_seqlens_q/k, num_seqs, total_q/k, max_seqlen_q/k:
+ *       exactly as given to / returned by fa_varlen_fwd.
+ *   dout [total_q, Hq, d] (input, dtype).
+ *   dq [total_q, Hq, d], dk and dv [total_k, Hkv, d] (outputs, dtype): rows
+ *       that belong to a sequence are overwritten; rows outside every
+ *       sequence are left as they were.
+ *   workspace: device buffer of fa_varlen_bwd_workspace_size(...) bytes,
+ *       16-byte aligned, owned by the caller.
+ *   d must be 128 (FA_ERR_UNSUPPORTED otherwise). Causal alignment is
+ *   bottom-right within each sequence.
+ */
+fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                        int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                        int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
+                        fa_stream_t stream);
+
+/*
  * Backward without a caller-provided workspace. This entry point has no
  * counterpart in the pages; it exists for callers that cannot allocate
  * device memory themselves (a host framework that owns every allocation,

@@ -126,3 +126,34 @@ def test_workspace_size(lib):
     assert fb.fa_bwd_workspace_size(2, 3, 5, 128) == r256(2 * 3 * 5 * 4) + r256(2 * 3 * 8 * 128 * 4)
     assert fb.fa_bwd_workspace_size(0, 1, 1, 64) == 0
     assert fb.fa_bwd_workspace_size(1, 1, 1, 96) == 0
+
+
+def varlen_bwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, ws=FAKE, cu_q=FAKE,
+             cu_k=FAKE, num_seqs=2, total_q=10, total_k=10, max_q=5, max_k=5, Hq=4, Hkv=2, d=128, scale=0.1,
+             causal=1, dtype=fb.FA_BF16, stream=None)
+    a.update(kw)
+    return fb.fa_varlen_bwd(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), fb.FA_ERR_INVALID_ARG),
+    (dict(cu_k=None), fb.FA_ERR_INVALID_ARG),
+    (dict(dk=None), fb.FA_ERR_INVALID_ARG),
+    (dict(num_seqs=0), fb.FA_ERR_INVALID_ARG),
+    (dict(max_k=-1), fb.FA_ERR_INVALID_ARG),
+    (dict(Hq=3), fb.FA_ERR_INVALID_ARG),
+    (dict(d=64), fb.FA_ERR_UNSUPPORTED),  # the varlen backward is d = 128 only
+    (dict(cu_q=FAKE + 2), fb.FA_ERR_MISALIGNED),
+    (dict(do=FAKE + 8), fb.FA_ERR_MISALIGNED),
+])
+def test_varlen_bwd_rejects_before_launch(lib, kw, code):
+    assert varlen_bwd(**kw) == code
+
+
+def test_varlen_workspace_size(lib):
+    r256 = lambda x: (x + 255) // 256 * 256
+    # D [Hq, total_q] and a dQ accumulator padded per sequence to max_seqlen_q (groups of four)
+    assert fb.fa_varlen_bwd_workspace_size(3, 100, 41, 2, 128) == r256(100 * 2 * 4) + r256(3 * 2 * 11 * 512 * 4)
+    assert fb.fa_varlen_bwd_workspace_size(3, 100, 41, 2, 64) == 0
+    assert fb.fa_varlen_bwd_workspace_size(0, 100, 41, 2, 128) == 0
