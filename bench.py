@@ -457,6 +457,27 @@ def run_sweep(args):
             ms = time_it(lambda: fb.attention_bwd(q, k, v, o, lse, do, cfg.scale, cfg.causal, workspace=ws), 20)
             emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
         del q, k, v, o, lse
+    # the ViT workload through the packed-QKV layout (B, S, 3, H, d), O written as (B, H, S, d)
+    cfg = inputs.VIT_RMSNORM
+    fi = inputs.make_fixed(cfg)
+    qkv = torch.stack([fi.q, fi.k, fi.v], dim=2).cuda()
+    q, k, v = qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2]
+    B, N, Hq, d = q.shape
+    o = torch.empty((B, Hq, N, d), dtype=q.dtype, device="cuda").permute(0, 2, 1, 3)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    st3 = lambda t: tuple(t.stride()[:3])
+
+    def packed():
+        r = fb.fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), st3(q),
+                              st3(k), st3(v), st3(o), B, Hq, Hq, N, N, d, cfg.scale, int(cfg.causal), fb.FA_BF16,
+                              stream.cuda_stream)
+        if r != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(r))
+
+    ms = time_it(packed, 30)
+    emit(cfg.name + "_packed_qkv", "fwd", ms, flops_fwd(B, N, Hq, d, cfg.causal),
+         2 * (q.numel() + k.numel() + v.numel() + q.numel()) + 4 * lse.numel())
+    del qkv, q, k, v, o, lse
     for cfg in (inputs.VARLEN, inputs.VARLEN_KEYPAD):
         vi = inputs.make_varlen(cfg)
         q, k, v = (t.cuda() for t in (vi.q, vi.k, vi.v))

@@ -1,6 +1,7 @@
 """Thin ctypes binding of libfa.so.
 
-The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
+The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_fwd_strided``, ``fa_varlen_fwd_strided``,
+``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
 ``fa_bwd``, ``fa_status_string`` and ``fa_get_last_device_error`` have the
 names, argument order and meaning of the C ABI in ``include/fa.h``: pointers
 are passed as integers (device addresses), streams as integers (0 = default
@@ -41,6 +42,8 @@ _SIGS = {
     "fa_bwd_set_timing_events": ([_P, _P], None),
     "fa_bwd_noalloc": ([_P] * 9 + [_I] * 6 + [_F, _I, _I, _P], _I),
     "fa_varlen_bwd_workspace_size": ([_I] * 5, ctypes.c_size_t),
+    "fa_fwd_strided": ([_P] * 9 + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_varlen_fwd_strided": ([_P] * 11 + [_I] * 8 + [_F, _I, _I, _P], _I),
     "fa_varlen_bwd": ([_P] * 12 + [_I] * 8 + [_F, _I, _I, _P], _I),
     "fa_selftest_bounded_wait": ([_P], _I),
 }
@@ -85,6 +88,29 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, 
            stream) -> int:
     return lib().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal,
                         dtype, stream)
+
+
+def _strides(st):
+    """A host int64 array of element strides (kept alive by the caller's reference)."""
+    return (ctypes.c_longlong * len(st))(*[int(x) for x in st]) if st is not None else None
+
+
+def fa_fwd_strided(q, k, v, o, lse, q_strides, k_strides, v_strides, o_strides, B, Hq, Hkv, Nq, Nk, d, scale,
+                   causal, dtype, stream) -> int:
+    """Strides are sequences of ints ({batch, token, head} in elements)."""
+    arrs = [_strides(x) for x in (q_strides, k_strides, v_strides, o_strides)]
+    return lib().fa_fwd_strided(q, k, v, o, lse, *[ctypes.cast(a, _P) if a is not None else None for a in arrs], B,
+                                Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream)
+
+
+def fa_varlen_fwd_strided(q, k, v, o, lse, q_strides, k_strides, v_strides, o_strides, cu_seqlens_q, cu_seqlens_k,
+                          num_seqs, total_q, total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype,
+                          stream) -> int:
+    """Strides are sequences of ints ({token, head} in elements)."""
+    arrs = [_strides(x) for x in (q_strides, k_strides, v_strides, o_strides)]
+    return lib().fa_varlen_fwd_strided(q, k, v, o, lse, *[ctypes.cast(a, _P) if a is not None else None for a in arrs],
+                                       cu_seqlens_q, cu_seqlens_k, num_seqs, total_q, total_k, max_seqlen_q,
+                                       max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream)
 
 
 def fa_varlen_bwd_workspace_size(num_seqs, total_q, max_seqlen_q, Hq, d) -> int:

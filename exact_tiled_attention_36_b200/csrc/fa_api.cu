@@ -40,15 +40,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 
 // Tensor map of a [batches, rows, H, d] 16-bit tensor, box = 128 rows x 64
 // columns of one head, 128-byte swizzle. Rows past `rows` read as zero.
-fa_status make_map(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16) {
+// 4-D map (d, H, rows, batches) over a tensor whose head, token and batch strides
+// are sh, ss, sb elements (d contiguous); each stride must be a multiple of 16 bytes.
+fa_status make_map_strided(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16,
+                           int64_t sh, int64_t ss, int64_t sb) {
     auto enc = encode_tiled();
     if (!enc) return FA_ERR_CUDA;
     if (rows < 1) rows = 1;
     if (batches < 1) batches = 1;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batches)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
-                                   static_cast<cuuint64_t>(rows) * H * d * 2};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sh) * 2, static_cast<cuuint64_t>(ss) * 2,
+                                   static_cast<cuuint64_t>(sb) * 2};
     const cuuint32_t box[4] = {64, 1, 128, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
@@ -56,6 +59,12 @@ fa_status make_map(CUtensorMap* m, const void* base, int d, int H, int64_t rows,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Contiguous [batches, rows, H, d].
+fa_status make_map(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16) {
+    return make_map_strided(m, base, d, H, rows, batches, bf16, d, static_cast<int64_t>(H) * d,
+                            (rows < 1 ? 1 : rows) * H * static_cast<int64_t>(d));
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -312,33 +321,55 @@ const char* fa_status_string(fa_status s) {
         case FA_OK: return "FA_OK";
         case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
         case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dim, dtype or size";
-        case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: tensor pointer not 16-byte aligned";
+        case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: tensor pointer or stride not 16-byte aligned";
         case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call failed";
         case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a bounded device wait ran out";
     }
     return "unknown fa_status";
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                 int Nq, int Nk, int d, float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
+}  // extern "C" (reopened below)
+
+namespace {
+
+// Element strides of one 16-bit tensor: batch, token, head (d is contiguous).
+struct Strides {
+    long long b, s, h;
+};
+
+// Strides must be positive and multiples of 8 elements (16 bytes, the TMA rule).
+fa_status check_strides(const Strides& t, bool with_batch) {
+    if (t.s <= 0 || t.h <= 0 || (with_batch && t.b <= 0)) return FA_ERR_INVALID_ARG;
+    if (t.s % 8 || t.h % 8 || (with_batch && t.b % 8)) return FA_ERR_MISALIGNED;
+    return FA_OK;
+}
+
+fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
+                    Strides sv, Strides so, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                    fa_dtype dtype, fa_stream_t stream) {
     if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if ((Nq > 0 && (!q || !o || !lse)) || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
     fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
     if (st != FA_OK) return st;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FA_ERR_MISALIGNED;
+    for (const Strides* t : {&sq, &sk, &sv, &so})
+        if ((st = check_strides(*t, true)) != FA_OK) return st;
     if (B > 65535) return FA_ERR_UNSUPPORTED;
     if (Nq == 0) return FA_OK;
     int* err = error_word();
     if (!err) return FA_ERR_CUDA;
     const bool bf16 = dtype == FA_BF16;
     CUtensorMap mq, mk{}, mv{};  // K/V maps stay unused (zero) when there is no key
-    if ((st = make_map(&mq, q, d, Hq, Nq, B, bf16)) != FA_OK) return st;
-    if (Nk > 0 && (st = make_map(&mk, k, d, Hkv, Nk, B, bf16)) != FA_OK) return st;
-    if (Nk > 0 && (st = make_map(&mv, v, d, Hkv, Nk, B, bf16)) != FA_OK) return st;
+    if ((st = make_map_strided(&mq, q, d, Hq, Nq, B, bf16, sq.h, sq.s, sq.b)) != FA_OK) return st;
+    if (Nk > 0 && (st = make_map_strided(&mk, k, d, Hkv, Nk, B, bf16, sk.h, sk.s, sk.b)) != FA_OK) return st;
+    if (Nk > 0 && (st = make_map_strided(&mv, v, d, Hkv, Nk, B, bf16, sv.h, sv.s, sv.b)) != FA_OK) return st;
     fa::FwdArgs a{};
     a.o = o;
     a.lse = lse;
+    a.o_sb = so.b;
+    a.o_ss = so.s;
+    a.o_sh = so.h;
     a.num_batches = B;
     a.Hq = Hq;
     a.group = Hq / Hkv;
@@ -351,10 +382,10 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     return launch_fwd(d, bf16, causal != 0, false, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
-fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
-                        const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
-                        int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
-                        fa_stream_t stream) {
+fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
+                     Strides sv, Strides so, const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                     int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d,
+                     float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
     if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
         return FA_ERR_INVALID_ARG;
     if (!cu_seqlens_q || !cu_seqlens_k || (total_q > 0 && (!q || !o || !lse)) || (total_k > 0 && (!k || !v)))
@@ -364,6 +395,8 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
         (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
         return FA_ERR_MISALIGNED;
+    for (const Strides* t : {&sq, &sk, &sv, &so})
+        if ((st = check_strides(*t, false)) != FA_OK) return st;
     if (num_seqs > 65535) return FA_ERR_UNSUPPORTED;
     if (max_seqlen_q == 0 || total_q == 0) return FA_OK;
     int* err = error_word();
@@ -372,12 +405,19 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
     // The maps span exactly the caller's buffers: a tile that runs past the
     // last packed row reads zeros instead of memory beyond the allocation.
     CUtensorMap mq, mk{}, mv{};
-    if ((st = make_map(&mq, q, d, Hq, total_q, 1, bf16)) != FA_OK) return st;
-    if (total_k > 0 && (st = make_map(&mk, k, d, Hkv, total_k, 1, bf16)) != FA_OK) return st;
-    if (total_k > 0 && (st = make_map(&mv, v, d, Hkv, total_k, 1, bf16)) != FA_OK) return st;
+    if ((st = make_map_strided(&mq, q, d, Hq, total_q, 1, bf16, sq.h, sq.s, sq.s * total_q)) != FA_OK) return st;
+    if (total_k > 0 &&
+        (st = make_map_strided(&mk, k, d, Hkv, total_k, 1, bf16, sk.h, sk.s, sk.s * total_k)) != FA_OK)
+        return st;
+    if (total_k > 0 &&
+        (st = make_map_strided(&mv, v, d, Hkv, total_k, 1, bf16, sv.h, sv.s, sv.s * total_k)) != FA_OK)
+        return st;
     fa::FwdArgs a{};
     a.o = o;
     a.lse = lse;
+    a.o_sb = 0;
+    a.o_ss = so.s;
+    a.o_sh = so.h;
     a.cu_q = cu_seqlens_q;
     a.cu_k = cu_seqlens_k;
     a.num_batches = num_seqs;
@@ -391,6 +431,62 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
     dim3 grid;
     if ((st = fwd_units(a, num_seqs, max_seqlen_q, grid)) != FA_OK) return st;
     return launch_fwd(d, bf16, causal != 0, true, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+Strides contiguous(int rows, int H, int d) {
+    return {static_cast<long long>(rows > 0 ? rows : 1) * H * d, static_cast<long long>(H) * d, d};
+}
+
+fa_status read_strides(const long long* p, bool with_batch, Strides* out) {
+    if (!p) return FA_ERR_INVALID_ARG;
+    *out = with_batch ? Strides{p[0], p[1], p[2]} : Strides{0, p[0], p[1]};
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                 int Nq, int Nk, int d, float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
+    return fwd_fixed(q, k, v, o, lse, contiguous(Nq, Hq, d), contiguous(Nk, Hkv, d), contiguous(Nk, Hkv, d),
+                     contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream);
+}
+
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const long long* q_strides, const long long* k_strides, const long long* v_strides,
+                         const long long* o_strides, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                         int causal, fa_dtype dtype, fa_stream_t stream) {
+    Strides sq, sk, sv, so;
+    fa_status st;
+    if ((st = read_strides(q_strides, true, &sq)) != FA_OK || (st = read_strides(k_strides, true, &sk)) != FA_OK ||
+        (st = read_strides(v_strides, true, &sv)) != FA_OK || (st = read_strides(o_strides, true, &so)) != FA_OK)
+        return st;
+    return fwd_fixed(q, k, v, o, lse, sq, sk, sv, so, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream);
+}
+
+fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
+                        int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
+                        fa_stream_t stream) {
+    return fwd_varlen(q, k, v, o, lse, contiguous(total_q, Hq, d), contiguous(total_k, Hkv, d),
+                      contiguous(total_k, Hkv, d), contiguous(total_q, Hq, d), cu_seqlens_q, cu_seqlens_k, num_seqs,
+                      total_q, total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream);
+}
+
+fa_status fa_varlen_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const long long* q_strides, const long long* k_strides,
+                                const long long* v_strides, const long long* o_strides, const int* cu_seqlens_q,
+                                const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
+                                int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
+                                fa_stream_t stream) {
+    Strides sq, sk, sv, so;
+    fa_status st;
+    if ((st = read_strides(q_strides, false, &sq)) != FA_OK || (st = read_strides(k_strides, false, &sk)) != FA_OK ||
+        (st = read_strides(v_strides, false, &sv)) != FA_OK || (st = read_strides(o_strides, false, &so)) != FA_OK)
+        return st;
+    return fwd_varlen(q, k, v, o, lse, sq, sk, sv, so, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q, total_k,
+                      max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {

@@ -63,6 +63,7 @@ struct FwdArgs {
     int group;        // Hq / Hkv
     int Nq;           // fixed: sequence lengths; varlen: max_seqlen bounds
     int Nk;
+    long long o_sb, o_ss, o_sh;  // O strides in elements: batch, token, head (d is contiguous)
     int nu;           // units (256 query rows) per sequence: ceil(Nq / 256)
     int n_units;      // nu * Hq * num_batches
     float scale_log2;  // scale * log2(e)
@@ -383,9 +384,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 return q < w.q_len;
             };
             auto out_row = [&]() -> T16* {
-                const size_t tok =
-                    VARLEN ? static_cast<size_t>(w.q_row0 + q) : static_cast<size_t>(w.bidx) * args.Nq + q;
-                return o_base + (tok * args.Hq + w.h) * D;
+                const long long row = VARLEN ? static_cast<long long>(w.q_row0 + q) * args.o_ss
+                                             : w.bidx * args.o_sb + static_cast<long long>(q) * args.o_ss;
+                return o_base + row + w.h * args.o_sh;
             };
             auto lse_row = [&]() -> float* {
                 return VARLEN ? args.lse + static_cast<size_t>(w.h) * args.total_q + w.q_row0 + q

@@ -57,7 +57,7 @@ typedef enum {
     FA_OK = 0,
     FA_ERR_INVALID_ARG = 1, /* null pointer, bad size, Hq % Hkv != 0, bad scale */
     FA_ERR_UNSUPPORTED = 2, /* head dim other than 64 / 128, unknown dtype, too large */
-    FA_ERR_MISALIGNED = 3,  /* a tensor pointer not 16-byte aligned */
+    FA_ERR_MISALIGNED = 3,  /* a tensor pointer or stride not 16-byte aligned */
     FA_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed */
     FA_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see fa_get_last_device_error) */
 } fa_status;
@@ -99,6 +99,35 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
                         int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
                         int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
                         fa_stream_t stream);
+
+/*
+ * Forward on strided views: the same computation as fa_fwd / fa_varlen_fwd
+ * for q, k, v, o that are not contiguous, e.g. the packed QKV layout
+ * (B, S, 3, H, d) of the InternViT FlashAttention wrapper, where q, k and v
+ * are views into one buffer (q_strides = {S*3*H*d, 3*H*d, d}, k at +H*d,
+ * v at +2*H*d), or a (B, H, S, d) layout.
+ *   *_strides: HOST arrays of element strides, read before the call returns.
+ *       fa_fwd_strided: {batch, token, head}; fa_varlen_fwd_strided: {token,
+ *       head} (the packed buffers have no batch dimension). Every stride must
+ *       be > 0 (FA_ERR_INVALID_ARG) and a multiple of 8 elements, 16 bytes
+ *       (FA_ERR_MISALIGNED); the last dimension d is contiguous. o must not
+ *       overlap itself or the inputs.
+ *   lse keeps the contiguous layouts of fa_fwd / fa_varlen_fwd.
+ * Every other argument, result and error is that of fa_fwd / fa_varlen_fwd.
+ */
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const long long* q_strides, const long long* k_strides,
+                         const long long* v_strides, const long long* o_strides,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+fa_status fa_varlen_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const long long* q_strides, const long long* k_strides,
+                                const long long* v_strides, const long long* o_strides,
+                                const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                                int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                                int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
+                                fa_stream_t stream);
 
 /*
  * Size in bytes of the caller-owned workspace fa_bwd needs: the per-row

@@ -157,3 +157,33 @@ def test_varlen_workspace_size(lib):
     assert fb.fa_varlen_bwd_workspace_size(3, 100, 41, 2, 128) == r256(100 * 2 * 4) + r256(3 * 2 * 11 * 512 * 4)
     assert fb.fa_varlen_bwd_workspace_size(3, 100, 41, 2, 64) == 0
     assert fb.fa_varlen_bwd_workspace_size(0, 100, 41, 2, 128) == 0
+
+
+def fwd_strided(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, sq=(3 * 8 * 64 * 8, 3 * 8 * 64, 64), sk=(3 * 8 * 64 * 8, 3 * 8 * 64, 64),
+             sv=(3 * 8 * 64 * 8, 3 * 8 * 64, 64), so=(8 * 8 * 64, 8 * 64, 64), B=1, Hq=8, Hkv=8, Nq=8, Nk=8, d=64,
+             scale=0.125, causal=0, dtype=fb.FA_BF16, stream=None)
+    a.update(kw)
+    return fb.fa_fwd_strided(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(sq=None), fb.FA_ERR_INVALID_ARG),
+    (dict(so=(512, 0, 64)), fb.FA_ERR_INVALID_ARG),
+    (dict(sk=(-8, 64, 64)), fb.FA_ERR_INVALID_ARG),
+    (dict(sv=(4096, 1540, 64)), fb.FA_ERR_MISALIGNED),  # token stride not a multiple of 8 elements
+    (dict(sq=(4096, 512, 68)), fb.FA_ERR_MISALIGNED),
+    (dict(d=96), fb.FA_ERR_UNSUPPORTED),
+    (dict(Nq=0), fb.FA_OK),
+])
+def test_fwd_strided_rejects_before_launch(lib, kw, code):
+    assert fwd_strided(**kw) == code
+
+
+def test_varlen_fwd_strided_rejects_before_launch(lib):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, sq=(3 * 2 * 128, 128), sk=(3 * 2 * 128, 128),
+             sv=(3 * 2 * 128, 128), so=(2 * 128, 128), cu_q=FAKE, cu_k=FAKE, num_seqs=2, total_q=10, total_k=10,
+             max_q=5, max_k=5, Hq=2, Hkv=2, d=128, scale=0.1, causal=0, dtype=fb.FA_FP16, stream=None)
+    assert fb.fa_varlen_fwd_strided(*{**a, "so": None}.values()) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_varlen_fwd_strided(*{**a, "sk": (770, 128)}.values()) == fb.FA_ERR_MISALIGNED
+    assert fb.fa_varlen_fwd_strided(*{**a, "total_q": 0}.values()) == fb.FA_OK

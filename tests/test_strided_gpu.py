@@ -1,0 +1,92 @@
+"""Forward on strided views (packed QKV, BHSD output) through the C ABI: the same
+result, bit for bit, as the contiguous path on copies of the same values, and
+within the oracle's tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_tiled_attention_36_b200 import binding as fb
+from exact_tiled_attention_36_b200 import inputs
+from tests.gpu_util import ATOL_L, f64, o_bound
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    fb.lib()
+    yield
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+
+
+def el_strides(t, batch=True):
+    st = t.stride()
+    return (st[0], st[1], st[2]) if batch else (st[0], st[1])
+
+
+@pytest.mark.parametrize("B,N,H,d,causal,dt", [
+    (2, 300, 4, 64, False, "bf16"),
+    (1, 513, 2, 128, True, "fp16"),
+    (3, 129, 3, 128, False, "bf16"),
+])
+def test_packed_qkv_matches_contiguous(B, N, H, d, causal, dt):
+    fi = inputs.make_fixed(inputs.TINY, B=B, Nq=N, Nk=N, Hq=H, Hkv=H, d=d, dtype=dt, seed=53, with_do=False)
+    qkv = torch.stack([fi.q, fi.k, fi.v], dim=2).cuda()  # (B, S, 3, H, d)
+    q, k, v = qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2]
+    o_bhsd = torch.full((B, H, N, d), 7.0, dtype=q.dtype, device="cuda")
+    o = o_bhsd.permute(0, 2, 1, 3)  # a (B, S, H, d) view of a (B, H, S, d) buffer
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    code = fb.FA_BF16 if dt == "bf16" else fb.FA_FP16
+    st = fb.fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), el_strides(q),
+                           el_strides(k), el_strides(v), el_strides(o), B, H, H, N, N, d, d ** -0.5, int(causal),
+                           code, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    o_ref, l_ref = fb.attention_fwd(q.contiguous(), k.contiguous(), v.contiguous(), d ** -0.5, causal)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref)
+    assert torch.equal(lse, l_ref)
+    rows = [0, 1, N // 2, N - 1]
+    o_or, l_or = oracle.attn_fwd(fi.q, fi.k, fi.v, d ** -0.5, causal, rows=rows)
+    got = f64(o)[:, rows]
+    assert (np.abs(got - o_or[:, rows]) <= o_bound(o_or[:, rows], q.dtype)).all()
+    assert np.abs(f64(lse)[:, :, rows] - l_or[:, :, rows]).max() <= ATOL_L
+
+
+def test_packed_kv_with_grouped_heads():
+    """q contiguous, k and v views of a packed (B, S, 2, Hkv, d) buffer, Hq = 4 Hkv."""
+    B, N, Hq, Hkv, d = 2, 260, 8, 2, 128
+    fi = inputs.make_fixed(inputs.CAUSAL_GQA, B=B, Nq=N, Nk=N, Hq=Hq, Hkv=Hkv, d=d, seed=59, with_do=False)
+    q = fi.q.cuda()
+    kv = torch.stack([fi.k, fi.v], dim=2).cuda()
+    k, v = kv[:, :, 0], kv[:, :, 1]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    st = fb.fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), el_strides(q),
+                           el_strides(k), el_strides(v), el_strides(o), B, Hq, Hkv, N, N, d, d ** -0.5, 1,
+                           fb.FA_BF16, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    o_ref, l_ref = fb.attention_fwd(q, k.contiguous(), v.contiguous(), d ** -0.5, True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+
+
+def test_varlen_packed_qkv_matches_contiguous():
+    vi = inputs.make_varlen(inputs.VARLEN, lengths=[300, 0, 77, 513], Hq=4, Hkv=4, d=128, dtype="fp16", seed=61)
+    qkv = torch.stack([vi.q, vi.k, vi.v], dim=1).cuda()  # (total, 3, H, d)
+    q, k, v = qkv[:, 0], qkv[:, 1], qkv[:, 2]
+    cu = vi.cu_seqlens_q.cuda()
+    T, H, d = q.shape
+    o = torch.empty((T, H, d), dtype=q.dtype, device="cuda")
+    lse = torch.empty((H, T), dtype=torch.float32, device="cuda")
+    st = fb.fa_varlen_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  el_strides(q, False), el_strides(k, False), el_strides(v, False),
+                                  el_strides(o, False), cu.data_ptr(), cu.data_ptr(), 4, T, T, vi.max_seqlen_q,
+                                  vi.max_seqlen_k, H, H, d, d ** -0.5, 1, fb.FA_FP16, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    o_ref, l_ref = fb.attention_varlen_fwd(q.contiguous(), k.contiguous(), v.contiguous(), cu, cu, vi.max_seqlen_q,
+                                           vi.max_seqlen_k, d ** -0.5, True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
