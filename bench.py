@@ -478,6 +478,26 @@ def run_sweep(args):
     emit(cfg.name + "_packed_qkv", "fwd", ms, flops_fwd(B, N, Hq, d, cfg.causal),
          2 * (q.numel() + k.numel() + v.numel() + q.numel()) + 4 * lse.numel())
     del qkv, q, k, v, o, lse
+    # the ViT workload with raw Q and K, their RMS normalisation fused (fa_fwd_qk_rmsnorm)
+    cfg = inputs.VIT_RMSNORM
+    fi = inputs.make_fixed(cfg, rmsnorm=False)
+    q, k, v = (t.cuda() for t in (fi.q, fi.k, fi.v))
+    B, N, Hq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    ws = torch.empty(fb.fa_fwd_qk_rmsnorm_workspace_size(B, N, Hq, d), dtype=torch.uint8, device="cuda")
+
+    def fused():
+        r = fb.fa_fwd_qk_rmsnorm(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 ws.data_ptr(), B, Hq, Hq, N, N, d, cfg.scale, int(cfg.causal), inputs.RMSNORM_EPS,
+                                 fb.FA_BF16, stream.cuda_stream)
+        if r != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(r))
+
+    ms = time_it(fused, 30)
+    emit(cfg.name + "_fused_qk_rmsnorm", "fwd", ms, flops_fwd(B, N, Hq, d, cfg.causal),
+         2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel())
+    del q, k, v, o, lse, ws
     for cfg in (inputs.VARLEN, inputs.VARLEN_KEYPAD):
         vi = inputs.make_varlen(cfg)
         q, k, v = (t.cuda() for t in (vi.q, vi.k, vi.v))

@@ -117,10 +117,10 @@ fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtyp
     return FA_OK;
 }
 
-template <int D, bool BF16, bool CAUSAL, bool VARLEN>
+template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool QKNORM>
 fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                        dim3 grid, cudaStream_t stream) {
-    auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, VARLEN>;
+    auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, VARLEN, QKNORM>;
     constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
     static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
     if (!attr_ok) return FA_ERR_CUDA;
@@ -136,25 +136,35 @@ fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D>
+template <int D, bool QKNORM>
 fa_status launch_fwd_d(bool bf16, bool causal, bool varlen, const CUtensorMap& mq, const CUtensorMap& mk,
                        const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
-    if (bf16) {
-        if (causal) return varlen ? launch_fwd_t<D, true, true, true>(mq, mk, mv, a, grid, s)
-                                  : launch_fwd_t<D, true, true, false>(mq, mk, mv, a, grid, s);
-        return varlen ? launch_fwd_t<D, true, false, true>(mq, mk, mv, a, grid, s)
-                      : launch_fwd_t<D, true, false, false>(mq, mk, mv, a, grid, s);
+    if constexpr (QKNORM) {  // fixed length only
+        if (bf16) return causal ? launch_fwd_t<D, true, true, false, true>(mq, mk, mv, a, grid, s)
+                                : launch_fwd_t<D, true, false, false, true>(mq, mk, mv, a, grid, s);
+        return causal ? launch_fwd_t<D, false, true, false, true>(mq, mk, mv, a, grid, s)
+                      : launch_fwd_t<D, false, false, false, true>(mq, mk, mv, a, grid, s);
+    } else {
+        if (bf16) {
+            if (causal) return varlen ? launch_fwd_t<D, true, true, true, false>(mq, mk, mv, a, grid, s)
+                                      : launch_fwd_t<D, true, true, false, false>(mq, mk, mv, a, grid, s);
+            return varlen ? launch_fwd_t<D, true, false, true, false>(mq, mk, mv, a, grid, s)
+                          : launch_fwd_t<D, true, false, false, false>(mq, mk, mv, a, grid, s);
+        }
+        if (causal) return varlen ? launch_fwd_t<D, false, true, true, false>(mq, mk, mv, a, grid, s)
+                                  : launch_fwd_t<D, false, true, false, false>(mq, mk, mv, a, grid, s);
+        return varlen ? launch_fwd_t<D, false, false, true, false>(mq, mk, mv, a, grid, s)
+                      : launch_fwd_t<D, false, false, false, false>(mq, mk, mv, a, grid, s);
     }
-    if (causal) return varlen ? launch_fwd_t<D, false, true, true>(mq, mk, mv, a, grid, s)
-                              : launch_fwd_t<D, false, true, false>(mq, mk, mv, a, grid, s);
-    return varlen ? launch_fwd_t<D, false, false, true>(mq, mk, mv, a, grid, s)
-                  : launch_fwd_t<D, false, false, false>(mq, mk, mv, a, grid, s);
 }
 
-fa_status launch_fwd(int d, bool bf16, bool causal, bool varlen, const CUtensorMap& mq, const CUtensorMap& mk,
-                     const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
-    return d == 64 ? launch_fwd_d<64>(bf16, causal, varlen, mq, mk, mv, a, grid, s)
-                   : launch_fwd_d<128>(bf16, causal, varlen, mq, mk, mv, a, grid, s);
+fa_status launch_fwd(int d, bool bf16, bool causal, bool varlen, bool qknorm, const CUtensorMap& mq,
+                     const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
+    if (qknorm)
+        return d == 64 ? launch_fwd_d<64, true>(bf16, causal, varlen, mq, mk, mv, a, grid, s)
+                       : launch_fwd_d<128, true>(bf16, causal, varlen, mq, mk, mv, a, grid, s);
+    return d == 64 ? launch_fwd_d<64, false>(bf16, causal, varlen, mq, mk, mv, a, grid, s)
+                   : launch_fwd_d<128, false>(bf16, causal, varlen, mq, mk, mv, a, grid, s);
 }
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -346,7 +356,8 @@ fa_status check_strides(const Strides& t, bool with_batch) {
 
 fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
                     Strides sv, Strides so, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
-                    fa_dtype dtype, fa_stream_t stream) {
+                    fa_dtype dtype, fa_stream_t stream, bool qknorm = false, float eps = 0.f,
+                    bool validate_only = false) {
     if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if ((Nq > 0 && (!q || !o || !lse)) || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
     fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
@@ -356,7 +367,7 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
     for (const Strides* t : {&sq, &sk, &sv, &so})
         if ((st = check_strides(*t, true)) != FA_OK) return st;
     if (B > 65535) return FA_ERR_UNSUPPORTED;
-    if (Nq == 0) return FA_OK;
+    if (Nq == 0 || validate_only) return FA_OK;
     int* err = error_word();
     if (!err) return FA_ERR_CUDA;
     const bool bf16 = dtype == FA_BF16;
@@ -376,10 +387,12 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
     a.Nq = Nq;
     a.Nk = Nk;
     a.scale_log2 = scale * kLog2e;
+    a.norm_eps = eps;
     a.err = err;
     dim3 grid;
     if ((st = fwd_units(a, B, Nq, grid)) != FA_OK) return st;
-    return launch_fwd(d, bf16, causal != 0, false, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
+    return launch_fwd(d, bf16, causal != 0, false, qknorm, mq, mk, mv, a, grid,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
@@ -430,7 +443,8 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
     a.err = err;
     dim3 grid;
     if ((st = fwd_units(a, num_seqs, max_seqlen_q, grid)) != FA_OK) return st;
-    return launch_fwd(d, bf16, causal != 0, true, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
+    return launch_fwd(d, bf16, causal != 0, true, false, mq, mk, mv, a, grid,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 Strides contiguous(int rows, int H, int d) {
@@ -451,6 +465,43 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int Nq, int Nk, int d, float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
     return fwd_fixed(q, k, v, o, lse, contiguous(Nq, Hq, d), contiguous(Nk, Hkv, d), contiguous(Nk, Hkv, d),
                      contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream);
+}
+
+size_t fa_fwd_qk_rmsnorm_workspace_size(int B, int Nk, int Hkv, int d) {
+    if (B < 1 || Nk < 0 || Hkv < 1 || (d != 64 && d != 128)) return 0;
+    return round256(static_cast<size_t>(B) * Nk * Hkv * d * 2);
+}
+
+fa_status fa_fwd_qk_rmsnorm(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, float eps,
+                            fa_dtype dtype, fa_stream_t stream) {
+    if (!(std::isfinite(eps) && eps >= 0.f)) return FA_ERR_INVALID_ARG;
+    if (Nk > 0 && !workspace) return FA_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+    // Everything fa_fwd checks, before anything runs (on the real K: the normalised
+    // copy has its layout).
+    fa_status st = fwd_fixed(q, k, v, o, lse, contiguous(Nq, Hq, d), contiguous(Nk, Hkv, d),
+                             contiguous(Nk, Hkv, d), contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                             dtype, stream, true, eps, /*validate_only=*/true);
+    if (st != FA_OK || Nq == 0) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t rows = static_cast<size_t>(B) * Nk * Hkv;
+    if (rows > 0) {
+        const size_t threads = rows * (d / 8);
+        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        const uint16_t* kx = static_cast<const uint16_t*>(k);
+        uint16_t* ky = static_cast<uint16_t*>(workspace);
+        if (d == 64)
+            dtype == FA_BF16 ? fa::fa_rms_normalise_rows<64, true><<<blocks, 256, 0, s>>>(kx, ky, rows, eps)
+                             : fa::fa_rms_normalise_rows<64, false><<<blocks, 256, 0, s>>>(kx, ky, rows, eps);
+        else
+            dtype == FA_BF16 ? fa::fa_rms_normalise_rows<128, true><<<blocks, 256, 0, s>>>(kx, ky, rows, eps)
+                             : fa::fa_rms_normalise_rows<128, false><<<blocks, 256, 0, s>>>(kx, ky, rows, eps);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return fwd_fixed(q, Nk > 0 ? workspace : k, v, o, lse, contiguous(Nq, Hq, d), contiguous(Nk, Hkv, d),
+                     contiguous(Nk, Hkv, d), contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype,
+                     stream, true, eps);
 }
 
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,

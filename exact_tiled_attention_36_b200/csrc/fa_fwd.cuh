@@ -67,6 +67,7 @@ struct FwdArgs {
     int nu;           // units (256 query rows) per sequence: ceil(Nq / 256)
     int n_units;      // nu * Hq * num_batches
     float scale_log2;  // scale * log2(e)
+    float norm_eps;    // QK RMS normalisation (fa_fwd_qk_rmsnorm): epsilon
     int* err;
 };
 
@@ -83,7 +84,7 @@ struct FwdCfg {
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 1 + 1 + 1;
+    static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 1 + 1 + 1 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16;
     static constexpr uint32_t kTmemCols = 512;
@@ -151,7 +152,58 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdArgs& a) {
 // Unit of round k for CTA c of G: the direction alternates every round.
 __device__ __forceinline__ int fwd_unit_index(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
 
-template <int D, bool BF16, bool CAUSAL, bool VARLEN>
+// RMS normalisation, in place, of row r of a 128-row tile in shared memory (the
+// 128-byte-swizzled layout of the TMA loads: 64-column slabs of 128-byte rows,
+// 16-byte chunk c of row r at chunk c ^ (r % 8)): x <- x / sqrt(mean(x^2) + eps),
+// unit gain, fp32 arithmetic, rounded to the 16-bit type.
+template <int D, bool BF16>
+__device__ __forceinline__ void rms_normalise_row(uint8_t* tile, int r, float eps) {
+    constexpr int kSlabs = D / 64;
+    // Sum of squares: pairs of elements through the packed f32x2 FMA into four
+    // independent accumulators, one 64-column slab (8 chunks) loaded at a time.
+    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int s = 0; s < kSlabs; ++s) {
+        uint4 x[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            x[c] = *reinterpret_cast<const uint4*>(tile + s * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t w[4] = {x[c].x, x[c].y, x[c].z, x[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint64_t p = f2_pack(unpack_lo<BF16>(w[i]), unpack_hi<BF16>(w[i]));
+                acc[i] = f2_fma(p, p, acc[i]);
+            }
+        }
+    }
+    const float ss = f2_sum(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
+    const float inv = rsqrtf(ss * (1.f / D) + eps);
+    const uint64_t inv2 = f2_pack(inv, inv);
+#pragma unroll
+    for (int s = 0; s < kSlabs; ++s)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint4* ptr = reinterpret_cast<uint4*>(tile + s * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+            const uint4 x = *ptr;
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(unpack_lo<BF16>(w[i]), unpack_hi<BF16>(w[i])), inv2), lo, hi);
+                o[i] = pack2<BF16>(lo, hi);
+            }
+            *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+}
+
+// QKNORM: Q arrives raw and each softmax thread RMS-normalises its own row of Q in
+// shared memory (over d) at the start of a unit, before the tensor core reads it;
+// K arrives normalised (fa_fwd_qk_rmsnorm runs fa_rms_normalise_rows over K first:
+// every CTA would otherwise redo each K tile once per unit).
+template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool QKNORM>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -180,6 +232,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint64_t* o_ready = o_free + 2;  // every product of the unit is complete
     uint64_t* sm_done = o_ready + 1;  // every softmax thread is past its last TMEM access
     uint64_t* mma_done = sm_done + 1;  // every product this CTA issued is complete
+    uint64_t* q_norm = mma_done + 1;   // QKNORM: Q of the unit normalised
+    // The barrier the MMA thread waits on before reading Q.
+    uint64_t* q_ready = QKNORM ? q_norm : q_full;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     int* abort_flag = reinterpret_cast<int*>(smem + C::kMiscOff + 4);
 
@@ -203,6 +258,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_init(o_ready, 1);
         mbar_init(sm_done, 256);
         mbar_init(mma_done, 1);
+        mbar_init(q_norm, 256);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -299,7 +355,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (u >= args.n_units) break;
                 const FwdUnit w = fwd_unit<CAUSAL, VARLEN>(u, args);
                 if (!w.rows || w.n_kv == 0) continue;
-                if (!(ok = mbar_wait(q_full, nq & 1, wc, 63))) break;
+                if (!(ok = mbar_wait(q_ready, nq & 1, wc, 63))) break;
                 if (!(ok = mbar_wait(&k_full[gk % S], (gk / S) & 1, wc, 64))) break;
                 tc_fence_after();
                 // The first S products of this unit run while the softmax warpgroups
@@ -404,6 +460,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const int row_limit = CAUSAL ? min(w.k_len, q + w.k_len - w.q_len + 1) : w.k_len;
             // Key tiles at or past this index need masking for some row of the tile.
             const int min_limit = CAUSAL ? min(w.k_len, qt0 + w.k_len - w.q_len + 1) : w.k_len;
+            if constexpr (QKNORM) {  // this thread's row of Q, before the unit's first S product
+                ok = warp_all(mbar_wait(q_full, nq & 1, wc, 57));
+                if (!ok) break;
+                rms_normalise_row<D, BF16>(sQ + t * C::kTileBytes, r, args.norm_eps);
+                fence_proxy_async_smem();
+                mbar_arrive(q_norm);
+            }
             float m = -INFINITY, l = 0.f, lr = 0.f;
             for (int j = 0; j < nt; ++j) {
                 ok = warp_all(mbar_wait(&s_full[t], ss & 1, wc, 69));
@@ -529,6 +592,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_before();
         mbar_arrive(sm_done);
     }
+}
+
+// RMS normalisation of rows of d 16-bit values (unit gain, fp32 arithmetic, rounded
+// to the 16-bit type): d / 8 threads per row, 8 values each.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_rms_normalise_rows(const uint16_t* x, uint16_t* y, size_t rows, float eps) {
+    constexpr int kLanes = D / 8;
+    const size_t row = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / kLanes;
+    const int sub = threadIdx.x % kLanes;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (row < rows) v = reinterpret_cast<const uint4*>(x + row * D)[sub];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint64_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint64_t p = f2_pack(unpack_lo<BF16>(w[i]), unpack_hi<BF16>(w[i]));
+        acc = f2_fma(p, p, acc);
+    }
+    float ss = f2_sum(acc);
+#pragma unroll
+    for (int off = kLanes / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = rsqrtf(ss * (1.f / D) + eps);
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = pack2<BF16>(unpack_lo<BF16>(w[i]) * inv, unpack_hi<BF16>(w[i]) * inv);
+    if (row < rows) reinterpret_cast<uint4*>(y + row * D)[sub] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 }  // namespace fa

@@ -101,6 +101,26 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
                         fa_stream_t stream);
 
 /*
+ * Forward with the query/key RMS normalisation fused in front of attention
+ * (the InternViT attention applies an RMSNorm to Q and K, per head, just
+ * before its FlashAttention call): with
+ *     q_hat = q / sqrt(mean_c(q_c^2) + eps),  k_hat = k / sqrt(mean_c(k_c^2) + eps)
+ * per (token, head) row over the d values (unit gain), computed in fp32 and
+ * rounded to dtype, the result is fa_fwd(q_hat, k_hat, v). q is read raw and
+ * normalised in shared memory inside the attention kernel (no extra pass over
+ * HBM); k is normalised once, by a row kernel, into `workspace` (each K tile
+ * serves many query tiles, so normalising it there would repeat the work).
+ *   workspace: device buffer of fa_fwd_qk_rmsnorm_workspace_size(B,Nk,Hkv,d)
+ *       bytes, 16-byte aligned, owned by the caller; on exit it holds k_hat.
+ *   eps must be finite and >= 0 (FA_ERR_INVALID_ARG). Fixed length only.
+ * Every other argument, result and error is that of fa_fwd.
+ */
+size_t fa_fwd_qk_rmsnorm_workspace_size(int B, int Nk, int Hkv, int d);
+fa_status fa_fwd_qk_rmsnorm(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                            float scale, int causal, float eps, fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Forward on strided views: the same computation as fa_fwd / fa_varlen_fwd
  * for q, k, v, o that are not contiguous, e.g. the packed QKV layout
  * (B, S, 3, H, d) of the InternViT FlashAttention wrapper, where q, k and v

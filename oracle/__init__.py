@@ -120,6 +120,20 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, key_keep=None, rows=No
     return o, lse
 
 
+def rms_normalise(x, eps: float, out_dtype=None):
+    """Per-row RMS normalisation over the last axis, unit gain, in fp64:
+    x / sqrt(mean(x^2) + eps). This is the Q/K normalisation the InternViT
+    attention applies before FlashAttention. With ``out_dtype`` (a torch dtype)
+    the result is rounded once to that type, as the tensor core consumes it
+    (the reading this build takes for the fused normalisation)."""
+    xf = _f64(x)
+    y = xf / np.sqrt((xf * xf).mean(axis=-1, keepdims=True) + eps)
+    if out_dtype is None:
+        return y
+    import torch
+    return torch.from_numpy(y).to(out_dtype)
+
+
 def attn_probs(q, k, scale: float, b: int, h: int, causal: bool = False, key_keep=None):
     """The Nq x Nk probability matrix of one (batch, query head)."""
     q, k = _f64(q), _f64(k)

@@ -187,3 +187,17 @@ def test_varlen_fwd_strided_rejects_before_launch(lib):
     assert fb.fa_varlen_fwd_strided(*{**a, "so": None}.values()) == fb.FA_ERR_INVALID_ARG
     assert fb.fa_varlen_fwd_strided(*{**a, "sk": (770, 128)}.values()) == fb.FA_ERR_MISALIGNED
     assert fb.fa_varlen_fwd_strided(*{**a, "total_q": 0}.values()) == fb.FA_OK
+
+
+@pytest.mark.parametrize("eps,code", [(-1.0, fb.FA_ERR_INVALID_ARG), (float("nan"), fb.FA_ERR_INVALID_ARG),
+                                      (float("inf"), fb.FA_ERR_INVALID_ARG)])
+def test_qk_rmsnorm_rejects_bad_eps(lib, eps, code):
+    assert fb.fa_fwd_qk_rmsnorm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 8, 8, 64, 0.1, 0, eps, fb.FA_BF16,
+                                None) == code
+    assert fb.fa_fwd_qk_rmsnorm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 8, 8, 96, 0.1, 0, 1e-6, fb.FA_BF16,
+                                None) == fb.FA_ERR_UNSUPPORTED
+    assert fb.fa_fwd_qk_rmsnorm(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 1, 8, 8, 64, 0.1, 0, 1e-6, fb.FA_BF16,
+                                None) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_fwd_qk_rmsnorm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, 1, 1, 1, 8, 8, 64, 0.1, 0, 1e-6,
+                                fb.FA_BF16, None) == fb.FA_ERR_MISALIGNED
+    assert fb.fa_fwd_qk_rmsnorm_workspace_size(2, 100, 3, 128) == (2 * 100 * 3 * 128 * 2 + 255) // 256 * 256

@@ -306,3 +306,26 @@ def test_inputs_are_seeded_and_shaped():
     vi = inputs.make_varlen(inputs.VARLEN, Hq=1, Hkv=1, d=8)
     assert len(vi.seqlens_q) == 32 and min(vi.seqlens_q) >= 64 and max(vi.seqlens_q) <= 4096
     assert int(vi.cu_seqlens_q[-1]) == vi.q.shape[0]
+
+
+def test_rms_normalise_pins():
+    """oracle.rms_normalise against what the definition fixes: the mean square of
+    each output row is ms / (ms + eps); a constant row c gives c / sqrt(c^2 + eps);
+    eps = 0 makes it invariant to positive scaling and keeps signs; and one
+    rounding to bf16 is within half an ulp of the fp64 value."""
+    import torch
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((5, 3, 16)) * rng.uniform(0.1, 10, (5, 3, 1))
+    eps = 1e-3
+    y = oracle.rms_normalise(x, eps)
+    ms = (x * x).mean(-1)
+    np.testing.assert_allclose((y * y).mean(-1), ms / (ms + eps), rtol=1e-12)
+    c = np.full((2, 8), -0.25)
+    np.testing.assert_allclose(oracle.rms_normalise(c, eps), -0.25 / np.sqrt(0.0625 + eps), rtol=1e-14)
+    y0 = oracle.rms_normalise(x, 0.0)
+    np.testing.assert_allclose(oracle.rms_normalise(3.5 * x, 0.0), y0, rtol=1e-12)
+    assert (np.sign(y0) == np.sign(x)).all()
+    yb = oracle.rms_normalise(torch.from_numpy(x).to(torch.bfloat16), eps, torch.bfloat16)
+    exact = oracle.rms_normalise(torch.from_numpy(x).to(torch.bfloat16), eps)
+    assert yb.dtype == torch.bfloat16
+    assert (np.abs(yb.double().numpy() - exact) <= np.abs(exact) * 2.0 ** -8 + 1e-30).all()
