@@ -55,20 +55,32 @@ def _load():
         lib = ctypes.CDLL(build())
         lib.ora_attn_fwd.restype = ctypes.c_int
         lib.ora_attn_fwd.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
-                                                                            _up, _ip, ctypes.c_int, _dp, _dp]
+                                                                            ctypes.c_int, _up, _ip, ctypes.c_int,
+                                                                            _dp, _dp]
         lib.ora_attn_probs.restype = ctypes.c_int
         lib.ora_attn_probs.argtypes = [_dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
-                                                                         _up, ctypes.c_int, ctypes.c_int, _dp]
+                                                                         ctypes.c_int, _up, ctypes.c_int,
+                                                                         ctypes.c_int, _dp]
         lib.ora_attn_bwd.restype = ctypes.c_int
         lib.ora_attn_bwd.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
-                                                                                 _up, _dp, _dp, _dp]
+                                                                                 ctypes.c_int, _up, _dp, _dp, _dp]
         lib.ora_attn_bwd_sampled.restype = ctypes.c_int
         lib.ora_attn_bwd_sampled.argtypes = ([_dp, _dp, _dp, _dp] + [ctypes.c_int] * 6 +
-                                             [ctypes.c_double, ctypes.c_int, _up, ctypes.c_int, ctypes.c_int,
+                                             [ctypes.c_double, ctypes.c_int, ctypes.c_int, _up, ctypes.c_int,
+                                              ctypes.c_int,
                                               _ip, ctypes.c_int, _ip, ctypes.c_int, _dp, _dp, _dp])
         lib.ora_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
+
+
+def _window(causal, window):
+    """(wl, wr) of the C oracle: keys visible to query i are those within wl before
+    and wr after its bottom-right-aligned key; a negative side is unbounded."""
+    if window is not None:
+        wl, wr = (int(x) for x in window)
+        return (wl if wl >= 0 else -1), (wr if wr >= 0 else -1)
+    return (-1, 0) if causal else (-1, -1)
 
 
 def num_threads() -> int:
@@ -94,8 +106,10 @@ def _mask_ptr(key_keep, B, Nk):
     return kk, _ptr(kk, _up)
 
 
-def attn_fwd(q, k, v, scale: float, causal: bool = False, key_keep=None, rows=None):
+def attn_fwd(q, k, v, scale: float, causal: bool = False, key_keep=None, rows=None, window=None):
     """O [B,Nq,Hq,d] and L [B,Hq,Nq] in fp64 by the plain definition.
+
+    ``window`` = (wl, wr) replaces ``causal`` with a sliding window (see _window).
 
     ``rows`` (sequence of query indices) restricts the work to those rows;
     the other entries of the returned arrays are NaN.
@@ -114,7 +128,7 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, key_keep=None, rows=No
         r, rp, nr = None, None, 0
     if B * Hq * (nr if rows is not None else Nq) > 0:
         err = _load().ora_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, float(scale),
-                                   int(bool(causal)), kp, rp, nr, _ptr(o), _ptr(lse))
+                                   *_window(causal, window), kp, rp, nr, _ptr(o), _ptr(lse))
         if err:
             raise RuntimeError(f"ora_attn_fwd failed with code {err}")
     return o, lse
@@ -134,7 +148,7 @@ def rms_normalise(x, eps: float, out_dtype=None):
     return torch.from_numpy(y).to(out_dtype)
 
 
-def attn_probs(q, k, scale: float, b: int, h: int, causal: bool = False, key_keep=None):
+def attn_probs(q, k, scale: float, b: int, h: int, causal: bool = False, key_keep=None, window=None):
     """The Nq x Nk probability matrix of one (batch, query head)."""
     q, k = _f64(q), _f64(k)
     B, Nq, Hq, d = q.shape
@@ -142,13 +156,13 @@ def attn_probs(q, k, scale: float, b: int, h: int, causal: bool = False, key_kee
     P = np.zeros((Nq, Nk))
     kk, kp = _mask_ptr(key_keep, B, Nk)
     err = _load().ora_attn_probs(_ptr(q), _ptr(k), B, Hq, Hkv, Nq, Nk, d, float(scale),
-                                 int(bool(causal)), kp, b, h, _ptr(P))
+                                 *_window(causal, window), kp, b, h, _ptr(P))
     if err:
         raise RuntimeError(f"ora_attn_probs failed with code {err}")
     return P
 
 
-def attn_bwd(q, k, v, do, scale: float, causal: bool = False, key_keep=None):
+def attn_bwd(q, k, v, do, scale: float, causal: bool = False, key_keep=None, window=None):
     """dQ, dK, dV in fp64 by the exact gradient of the definition."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, Nq, Hq, d = q.shape
@@ -156,14 +170,14 @@ def attn_bwd(q, k, v, do, scale: float, causal: bool = False, key_keep=None):
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     kk, kp = _mask_ptr(key_keep, B, Nk)
     err = _load().ora_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, Hq, Hkv, Nq, Nk, d,
-                               float(scale), int(bool(causal)), kp, _ptr(dq), _ptr(dk), _ptr(dv))
+                               float(scale), *_window(causal, window), kp, _ptr(dq), _ptr(dk), _ptr(dv))
     if err:
         raise RuntimeError(f"ora_attn_bwd failed with code {err}")
     return dq, dk, dv
 
 
 def attn_bwd_sampled(q, k, v, do, scale: float, b: int, hk: int, qrows, krows,
-                     causal: bool = False, key_keep=None):
+                     causal: bool = False, key_keep=None, window=None):
     """Gradients of sampled rows of one (batch, KV head) group.
 
     Returns (dq_rows [len(qrows), group, d], dk_rows [len(krows), d],
@@ -180,7 +194,7 @@ def attn_bwd_sampled(q, k, v, do, scale: float, b: int, hk: int, qrows, krows,
     dv = np.zeros_like(v)
     kk, kp = _mask_ptr(key_keep, B, Nk)
     err = _load().ora_attn_bwd_sampled(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B, Hq, Hkv, Nq, Nk, d,
-                                       float(scale), int(bool(causal)), kp, b, hk, _ptr(qr, _ip),
+                                       float(scale), *_window(causal, window), kp, b, hk, _ptr(qr, _ip),
                                        int(qr.size), _ptr(kr, _ip), int(kr.size), _ptr(dq), _ptr(dk),
                                        _ptr(dv))
     if err:

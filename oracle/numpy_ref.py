@@ -13,18 +13,26 @@ from __future__ import annotations
 import numpy as np
 
 
-def _mask(Nq, Nk, causal, keep_row):
+def _mask(Nq, Nk, causal, keep_row, window=None):
+    """Allowed (query, key) pairs. A window (wl, wr) allows the keys from wl
+    before to wr after the bottom-right-aligned diagonal (a negative side is
+    unbounded); it replaces `causal`, which is the window (-1, 0)."""
     allowed = np.ones((Nq, Nk), dtype=bool)
-    if causal:
-        i = np.arange(Nq)[:, None]
-        j = np.arange(Nk)[None, :]
-        allowed &= j <= i + (Nk - Nq)
+    diag = np.arange(Nk)[None, :] - np.arange(Nq)[:, None] - (Nk - Nq)  # key offset from the aligned diagonal
+    if window is not None:
+        wl, wr = window
+        if wl >= 0:
+            allowed &= diag >= -wl
+        if wr >= 0:
+            allowed &= diag <= wr
+    elif causal:
+        allowed &= diag <= 0
     if keep_row is not None:
         allowed &= np.asarray(keep_row, dtype=bool)[None, :]
     return allowed
 
 
-def fwd(q, k, v, scale, causal=False, key_keep=None):
+def fwd(q, k, v, scale, causal=False, key_keep=None, window=None):
     q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
     B, Nq, Hq, d = q.shape
     Nk, Hkv = k.shape[1], k.shape[2]
@@ -32,7 +40,7 @@ def fwd(q, k, v, scale, causal=False, key_keep=None):
     o = np.zeros_like(q)
     lse = np.zeros((B, Hq, Nq))
     for b in range(B):
-        allowed = _mask(Nq, Nk, causal, None if key_keep is None else key_keep[b])
+        allowed = _mask(Nq, Nk, causal, None if key_keep is None else key_keep[b], window)
         for h in range(Hq):
             S = scale * q[b, :, h, :] @ k[b, :, h // g, :].T
             S = np.where(allowed, S, -np.inf)
@@ -47,14 +55,14 @@ def fwd(q, k, v, scale, causal=False, key_keep=None):
     return o, lse
 
 
-def bwd(q, k, v, do, scale, causal=False, key_keep=None):
+def bwd(q, k, v, do, scale, causal=False, key_keep=None, window=None):
     q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
     B, Nq, Hq, d = q.shape
     Nk, Hkv = k.shape[1], k.shape[2]
     g = Hq // Hkv
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     for b in range(B):
-        allowed = _mask(Nq, Nk, causal, None if key_keep is None else key_keep[b])
+        allowed = _mask(Nq, Nk, causal, None if key_keep is None else key_keep[b], window)
         for h in range(Hq):
             K = k[b, :, h // g, :]
             V = v[b, :, h // g, :]

@@ -329,3 +329,73 @@ def test_rms_normalise_pins():
     exact = oracle.rms_normalise(torch.from_numpy(x).to(torch.bfloat16), eps)
     assert yb.dtype == torch.bfloat16
     assert (np.abs(yb.double().numpy() - exact) <= np.abs(exact) * 2.0 ** -8 + 1e-30).all()
+
+
+WINDOWS = [(2, 1), (0, 3), (5, 0), (-1, 2), (3, -1), (0, 0)]
+
+
+@pytest.mark.parametrize("window", WINDOWS)
+@pytest.mark.parametrize("Nq,Nk,Hq,Hkv", [(9, 9, 2, 1), (6, 11, 2, 2), (12, 7, 4, 2)])
+def test_window_numpy_crosscheck(window, Nq, Nk, Hq, Hkv):
+    """The C oracle's sliding window (per-element visibility) against the numpy
+    version's (a mask matrix built from key offsets), forward and backward."""
+    rng = np.random.default_rng(17)
+    q, k, v, do = (_rand(rng, 2, Nq, Hq, 4), _rand(rng, 2, Nk, Hkv, 4), _rand(rng, 2, Nk, Hkv, 4),
+                   _rand(rng, 2, Nq, Hq, 4))
+    o, lse = oracle.attn_fwd(q, k, v, 0.7, window=window)
+    o2, lse2 = numpy_ref.fwd(q, k, v, 0.7, window=window)
+    np.testing.assert_allclose(o, o2, atol=1e-12)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(lse2))
+    fin = np.isfinite(lse)
+    np.testing.assert_allclose(lse[fin], lse2[fin], atol=1e-12)
+    g = oracle.attn_bwd(q, k, v, do, 0.7, window=window)
+    g2 = numpy_ref.bwd(q, k, v, do, 0.7, window=window)
+    for a, b in zip(g, g2):
+        np.testing.assert_allclose(a, b, atol=1e-11)
+
+
+def test_window_special_cases():
+    """(-1, 0) is the causal mask; a window covering every key is no mask; the
+    window (0, 0) leaves each query its aligned key only, so O_i = V_a and L_i = S_ia,
+    and a row whose aligned key lies outside the keys sees nothing."""
+    rng = np.random.default_rng(19)
+    Nq, Nk = 7, 5
+    q, k, v = _rand(rng, 1, Nq, 2, 3), _rand(rng, 1, Nk, 2, 3), _rand(rng, 1, Nk, 2, 3)
+    for a, b in zip(oracle.attn_fwd(q, k, v, 0.5, window=(-1, 0)), oracle.attn_fwd(q, k, v, 0.5, causal=True)):
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(oracle.attn_fwd(q, k, v, 0.5, window=(Nk + Nq, Nk + Nq)), oracle.attn_fwd(q, k, v, 0.5)):
+        np.testing.assert_array_equal(a, b)
+    o, lse = oracle.attn_fwd(q, k, v, 0.5, window=(0, 0))
+    for i in range(Nq):
+        a = i + Nk - Nq
+        for h in range(2):
+            if 0 <= a < Nk:
+                np.testing.assert_allclose(o[0, i, h], v[0, a, h], atol=1e-15)
+                assert abs(lse[0, h, i] - 0.5 * float(q[0, i, h] @ k[0, a, h])) <= 1e-14
+            else:
+                assert (o[0, i, h] == 0).all() and np.isneginf(lse[0, h, i])
+
+
+def test_window_backward_matches_finite_differences():
+    rng = np.random.default_rng(23)
+    q, k, v, do = _rand(rng, 1, 6, 2, 3), _rand(rng, 1, 8, 1, 3), _rand(rng, 1, 8, 1, 3), _rand(rng, 1, 6, 2, 3)
+    window, scale = (2, 1), 0.6
+    grads = oracle.attn_bwd(q, k, v, do, scale, window=window)
+
+    def phi(qq, kk, vv):
+        o, _ = oracle.attn_fwd(qq, kk, vv, scale, window=window)
+        return float((o * do).sum())
+
+    h = 1e-6
+    for which, g in zip(range(3), grads):
+        base = [q, k, v]
+        fd = np.zeros_like(base[which])
+        it = np.nditer(base[which], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            plus = [t.copy() for t in base]
+            minus = [t.copy() for t in base]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            fd[idx] = (phi(*plus) - phi(*minus)) / (2 * h)
+        assert np.linalg.norm(fd - g) / np.linalg.norm(g) <= 1e-6, which
