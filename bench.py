@@ -457,6 +457,38 @@ def run_sweep(args):
             ms = time_it(lambda: fb.attention_bwd(q, k, v, o, lse, do, cfg.scale, cfg.causal, workspace=ws), 20)
             emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
         del q, k, v, o, lse
+    # local attention: the causal GQA prefill shape with a causal sliding window of 1024 keys
+    cfg = inputs.CAUSAL_GQA
+    fi = inputs.make_fixed(cfg)
+    q, k, v, do = (t.cuda() for t in (fi.q, fi.k, fi.v, fi.do))
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    wl, wr = 1024, 0
+    pairs = sum(min(i + 1, wl + 1) for i in range(N))  # visible (query, key) pairs per (batch, head)
+    wflops = 4.0 * d * pairs * B * Hq
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, N, d), dtype=torch.uint8, device="cuda")
+
+    def wfwd():
+        r = fb.fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N,
+                             N, d, cfg.scale, wl, wr, fb.FA_BF16, stream.cuda_stream)
+        if r != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(r))
+
+    def wbwd():
+        r = fb.fa_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, N, N, d,
+                             cfg.scale, wl, wr, fb.FA_BF16, stream.cuda_stream)
+        if r != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(r))
+
+    nb = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
+    emit(cfg.name + "_window1024", "fwd", time_it(wfwd, 30), wflops, nb)
+    emit(cfg.name + "_window1024", "bwd", time_it(wbwd, 20), 2.5 * wflops,
+         nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+    del q, k, v, do, o, lse, dq, dk, dv, ws
     # the ViT workload through the packed-QKV layout (B, S, 3, H, d), O written as (B, H, S, d)
     cfg = inputs.VIT_RMSNORM
     fi = inputs.make_fixed(cfg)

@@ -1,6 +1,7 @@
 """Thin ctypes binding of libfa.so.
 
 The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_fwd_strided``, ``fa_varlen_fwd_strided``, ``fa_fwd_qk_rmsnorm``,
+``fa_fwd_window``, ``fa_bwd_window``,
 ``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
 ``fa_bwd``, ``fa_status_string`` and ``fa_get_last_device_error`` have the
 names, argument order and meaning of the C ABI in ``include/fa.h``: pointers
@@ -43,6 +44,8 @@ _SIGS = {
     "fa_bwd_noalloc": ([_P] * 9 + [_I] * 6 + [_F, _I, _I, _P], _I),
     "fa_varlen_bwd_workspace_size": ([_I] * 5, ctypes.c_size_t),
     "fa_fwd_strided": ([_P] * 9 + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_fwd_window": ([_P] * 5 + [_I] * 6 + [_F, _I, _I, _I, _P], _I),
+    "fa_bwd_window": ([_P] * 10 + [_I] * 6 + [_F, _I, _I, _I, _P], _I),
     "fa_fwd_qk_rmsnorm": ([_P] * 6 + [_I] * 6 + [_F, _I, _F, _I, _P], _I),
     "fa_fwd_qk_rmsnorm_workspace_size": ([_I] * 4, ctypes.c_size_t),
     "fa_varlen_fwd_strided": ([_P] * 11 + [_I] * 8 + [_F, _I, _I, _P], _I),
@@ -90,6 +93,17 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, 
            stream) -> int:
     return lib().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal,
                         dtype, stream)
+
+
+def fa_fwd_window(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, window_left, window_right, dtype, stream) -> int:
+    return lib().fa_fwd_window(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, window_left, window_right, dtype,
+                               stream)
+
+
+def fa_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, window_left,
+                  window_right, dtype, stream) -> int:
+    return lib().fa_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale,
+                               window_left, window_right, dtype, stream)
 
 
 def fa_fwd_qk_rmsnorm_workspace_size(B, Nk, Hkv, d) -> int:

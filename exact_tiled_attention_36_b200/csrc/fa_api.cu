@@ -238,10 +238,11 @@ size_t acc_floats(int B, int Hq, int Nq, int d) {
 // The backward of fa_bwd and fa_varlen_bwd. Fixed length: nseq = B, rows = B * Nq,
 // cu_q = cu_k = nullptr. Varlen: nseq = num_seqs, Nq / Nk the max_seqlen bounds,
 // rows = total_q, and the maps span the packed buffers (total_q / total_k rows).
+// `causal` selects the masked kernels; their window is (wl, wr) (causal: (-1, 0)).
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dout, void* dq, void* dk, void* dv, void* workspace, int nseq, const int* cu_q,
                      const int* cu_k, int total_q, int total_k, int Hq, int Hkv, int Nq, int Nk, int d,
-                     float scale, bool causal, bool bf16, cudaStream_t s) {
+                     float scale, bool causal, bool bf16, cudaStream_t s, int wl = -1, int wr = 0) {
     const bool varlen = cu_q != nullptr;
     int* err = error_word();
     if (!err) return FA_ERR_CUDA;
@@ -291,6 +292,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         a.total_q = total_q;
         a.scale = scale;
         a.scale_log2 = scale * kLog2e;
+        a.wl = wl;
+        a.wr = wr;
         a.err = err;
         const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
         if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
@@ -317,6 +320,22 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         }
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
+    return FA_OK;
+}
+
+// The argument checks of fa_bwd (nothing is launched when one fails).
+fa_status bwd_checks(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                     float scale, int causal, fa_dtype dtype) {
+    if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    if ((Nq > 0 && (!q || !o || !lse || !dout || !dq)) || (Nk > 0 && (!k || !v || !dk || !dv)) || !workspace)
+        return FA_ERR_INVALID_ARG;
+    const fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return FA_ERR_MISALIGNED;
+    if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
     return FA_OK;
 }
 
@@ -354,10 +373,11 @@ fa_status check_strides(const Strides& t, bool with_batch) {
     return FA_OK;
 }
 
+// `causal` selects the masked kernels; their window is (wl, wr) (causal: (-1, 0)).
 fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
                     Strides sv, Strides so, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                     fa_dtype dtype, fa_stream_t stream, bool qknorm = false, float eps = 0.f,
-                    bool validate_only = false) {
+                    bool validate_only = false, int wl = -1, int wr = 0) {
     if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if ((Nq > 0 && (!q || !o || !lse)) || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
     fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
@@ -381,6 +401,8 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
     a.o_sb = so.b;
     a.o_ss = so.s;
     a.o_sh = so.h;
+    a.wl = wl;
+    a.wr = wr;
     a.num_batches = B;
     a.Hq = Hq;
     a.group = Hq / Hkv;
@@ -431,6 +453,8 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
     a.o_sb = 0;
     a.o_ss = so.s;
     a.o_sh = so.h;
+    a.wl = -1;
+    a.wr = 0;
     a.cu_q = cu_seqlens_q;
     a.cu_k = cu_seqlens_k;
     a.num_batches = num_seqs;
@@ -504,6 +528,16 @@ fa_status fa_fwd_qk_rmsnorm(const void* q, const void* k, const void* v, void* o
                      stream, true, eps);
 }
 
+fa_status fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Nq, int Nk, int d, float scale, int window_left, int window_right, fa_dtype dtype,
+                        fa_stream_t stream) {
+    const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
+    const bool masked = wl >= 0 || wr >= 0;
+    return fwd_fixed(q, k, v, o, lse, contiguous(Nq, Hq, d), contiguous(Nk, Hkv, d), contiguous(Nk, Hkv, d),
+                     contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, masked ? 1 : 0, dtype, stream, false, 0.f,
+                     false, wl, wr);
+}
+
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
                          const long long* q_strides, const long long* k_strides, const long long* v_strides,
                          const long long* o_strides, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
@@ -549,17 +583,24 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                  void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
                  float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
-    if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
-    if ((Nq > 0 && (!q || !o || !lse || !dout || !dq)) || (Nk > 0 && (!k || !v || !dk || !dv)) || !workspace)
-        return FA_ERR_INVALID_ARG;
-    fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
+    const fa_status st = bwd_checks(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                    dtype);
     if (st != FA_OK) return st;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
-        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
-        return FA_ERR_MISALIGNED;
-    if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
     return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
                       scale, causal != 0, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
+                        int Nq, int Nk, int d, float scale, int window_left, int window_right, fa_dtype dtype,
+                        fa_stream_t stream) {
+    const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
+    const bool masked = wl >= 0 || wr >= 0;
+    const fa_status st = bwd_checks(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale,
+                                    masked ? 1 : 0, dtype);
+    if (st != FA_OK) return st;
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
+                      scale, masked, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream), wl, wr);
 }
 
 size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q, int Hq, int d) {

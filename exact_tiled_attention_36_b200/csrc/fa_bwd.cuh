@@ -54,8 +54,33 @@ struct BwdArgs {
     int total_q;                 // varlen: rows of q / o / dO (L and D are [Hq, total_q])
     float scale;
     float scale_log2;
+    int wl, wr;  // MASKED: keys from wl before to wr after the aligned diagonal (< 0: unbounded)
     int* err;
 };
+
+// Queries [qlo, qhi) that see key `key` (bottom-right alignment: query q's aligned
+// key is q + Nk - Nq; with MASKED the window (wl, wr) of BwdArgs, else every query).
+template <bool MASKED>
+__device__ __forceinline__ void query_range(const BwdArgs& a, int key, int Nq, int Nk, int& qlo, int& qhi) {
+    qlo = 0;
+    qhi = Nq;
+    if (MASKED) {
+        const int q_aligned = key - (Nk - Nq);
+        if (a.wr >= 0) qlo = max(0, q_aligned - a.wr);
+        if (a.wl >= 0) qhi = min(Nq, q_aligned + a.wl + 1);
+    }
+}
+
+// Query tiles [i0, i0 + n_i) that see some key of the key tile at k0.
+template <bool MASKED>
+__device__ __forceinline__ void query_tiles(const BwdArgs& a, int k0, int Nq, int Nk, int& i0, int& n_i) {
+    int qlo, qhi, qlo2, qhi2;
+    query_range<MASKED>(a, k0, Nq, Nk, qlo, qhi);
+    query_range<MASKED>(a, min(k0 + 127, Nk - 1), Nq, Nk, qlo2, qhi2);
+    i0 = qlo / 128;
+    const int i_end = qhi2 > qlo ? (qhi2 + 127) / 128 : i0;
+    n_i = i_end - i0;
+}
 
 template <int D>
 struct BwdCfg {
@@ -95,15 +120,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int b = CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
     const int k0 = kt * 128;
     const int Nq = args.Nq, Nk = args.Nk;
-    const int n_qt = (Nq + 127) / 128;
-    // Causal: query q sees key k iff k <= q + (Nk - Nq). The first query tile
-    // that sees any key of this tile:
-    int i0 = 0;
-    if (CAUSAL) {
-        const int qmin = k0 - (Nk - Nq);
-        i0 = qmin <= 0 ? 0 : qmin / 128;
-    }
-    const int n_i = n_qt > i0 ? n_qt - i0 : 0;
+    int i0, n_i;
+    query_tiles<CAUSAL>(args, k0, Nq, Nk, i0, n_i);
     const int n_it = args.group * n_i;
 
     using T16 = uint16_t;
@@ -296,8 +314,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             ok = warp_all(mbar_wait(s_full, it & 1, wc, 27));
             if (!ok) break;
             tc_fence_after();
-            // Query q sees this thread's key iff key <= q + (Nk - Nq) (and key < Nk).
-            const int qlim = key - (Nk - Nq);  // smallest query that sees the key
+            // Queries [qlim, qlim_hi) see this thread's key (and only if key < Nk).
+            int qlim, qlim_hi;
+            query_range<CAUSAL>(args, key, Nq, Nk, qlim, qlim_hi);
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int c = wg * 2 + cc;  // 32-column chunk of the 128 queries
@@ -314,7 +333,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     for (int e = 0; e < 2; ++e) {
                         const int qq = c * 32 + t + e;
                         bool vis = key_ok;
-                        if (CAUSAL) vis = vis && (q0 + qq >= qlim);
+                        if (CAUSAL) vis = vis && (q0 + qq >= qlim) && (q0 + qq < qlim_hi);
                         const float pe = ex2_approx(fmaf(__uint_as_float(sv[t + e]), sl2, -sL[qq]));
                         p[e] = vis ? pe : 0.f;
                         ds[e] = p[e] * (__uint_as_float(pv[t + e]) - sD[qq]);

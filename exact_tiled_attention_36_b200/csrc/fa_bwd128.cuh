@@ -101,13 +101,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
     auto key_tok = [&](int key) -> size_t {
         return VARLEN ? static_cast<size_t>(k_row0 + key) : static_cast<size_t>(b) * Nk + key;
     };
-    const int n_qt = (Nq + 127) / 128;
-    int i0 = 0;
-    if (CAUSAL) {
-        const int qmin = k0 - (Nk - Nq);  // smallest query that sees key k0
-        i0 = qmin <= 0 ? 0 : qmin / 128;
-    }
-    const int n_i = n_qt > i0 ? n_qt - i0 : 0;
+    int i0, n_i;  // the query tiles that see some key of this tile
+    query_tiles<CAUSAL>(args, k0, Nq, Nk, i0, n_i);
     const int n_it = args.group * n_i;
 
     using T16 = uint16_t;
@@ -313,7 +308,12 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
         const int key = k0 + r;
         const bool key_ok = key < Nk;
-        const int qlim = key - (Nk - Nq);  // smallest query that sees this key
+        int qlim, qlim_hi;  // queries [qlim, qlim_hi) see this key
+        query_range<CAUSAL>(args, key, Nq, Nk, qlim, qlim_hi);
+        // Every key of the tile sees queries [qall_lo, qall_hi): slices inside need no mask.
+        int qall_lo, qdummy, qdummy2, qall_hi;
+        query_range<CAUSAL>(args, min(k0 + 127, Nk - 1), Nq, Nk, qall_lo, qdummy);
+        query_range<CAUSAL>(args, k0, Nq, Nk, qdummy2, qall_hi);
         const float sl2 = args.scale_log2;
         constexpr float kLog2eF = 1.4426950408889634074f;
         // -L log2 e and -D of query 64 w + r of iteration it_, loaded one iteration
@@ -356,9 +356,10 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             ok = warp_all(mbar_wait(s_full, it & 1, wc, 69));
             if (!ok) break;
             tc_fence_after();
-            // Masks matter only on the tile holding key Nk - 1 and, under the causal
-            // mask, on query columns that reach below the diagonal (uniform per warpgroup).
-            const bool need_mask = (k0 + 128 > Nk) || (CAUSAL && qs < k0 + 127 - (Nk - Nq));
+            // Masks matter only on the tile holding key Nk - 1 and, under a window mask
+            // (causal included), on query columns outside some key's window (uniform per
+            // warpgroup).
+            const bool need_mask = (k0 + 128 > Nk) || (CAUSAL && (qs < qall_lo || qs + 64 > qall_hi));
             float pf[64];
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
@@ -384,7 +385,10 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             bool vis = key_ok;
-                            if (CAUSAL) vis = vis && (qs + cc * 32 + e + u >= qlim);
+                            if (CAUSAL) {
+                                const int qv = qs + cc * 32 + e + u;
+                                vis = vis && qv >= qlim && qv < qlim_hi;
+                            }
                             p[u] = vis ? p[u] : 0.f;
                         }
                     }

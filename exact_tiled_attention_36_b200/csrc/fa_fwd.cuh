@@ -64,6 +64,7 @@ struct FwdArgs {
     int Nq;           // fixed: sequence lengths; varlen: max_seqlen bounds
     int Nk;
     long long o_sb, o_ss, o_sh;  // O strides in elements: batch, token, head (d is contiguous)
+    int wl, wr;       // MASKED: keys from wl before to wr after the aligned diagonal (< 0: unbounded)
     int nu;           // units (256 query rows) per sequence: ceil(Nq / 256)
     int n_units;      // nu * Hq * num_batches
     float scale_log2;  // scale * log2(e)
@@ -103,9 +104,25 @@ constexpr int kFwdMinLaunchRegs = (128 * kFwdRegsOther + 256 * kFwdRegsSoftmax +
 struct FwdUnit {
     int h, bidx, q0;
     int q_len, k_len, q_row0, k_row0, tma_b;
-    int n_0, n_1, n_kv;  // key tiles of query tile 0, of query tile 1, and their maximum
+    int jlo, n_kv;       // the unit walks key tiles jlo .. jlo + n_kv - 1 (steps 0 .. n_kv - 1)
+    int a0, b0, a1, b1;  // query tile t is active on steps a_t .. b_t - 1 (none if a_t == b_t)
     bool rows;           // the unit holds at least one query row
+    __device__ __forceinline__ int a(int t) const { return t ? a1 : a0; }
+    __device__ __forceinline__ int b(int t) const { return t ? b1 : b0; }
 };
+
+// First visible key and one past the last for query q (bottom-right alignment; the
+// window (wl, wr) of FwdArgs, or every key without a mask).
+template <bool MASKED>
+__device__ __forceinline__ void key_range(const FwdArgs& a, int q, int q_len, int k_len, int& lo, int& hi) {
+    lo = 0;
+    hi = k_len;
+    if (MASKED) {
+        const int aligned = q + k_len - q_len;
+        if (a.wl >= 0) lo = max(0, aligned - a.wl);
+        if (a.wr >= 0) hi = min(k_len, aligned + a.wr + 1);
+    }
+}
 
 template <bool CAUSAL, bool VARLEN>
 __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdArgs& a) {
@@ -136,16 +153,30 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdArgs& a) {
         w.tma_b = w.bidx;
     }
     w.rows = w.q0 < w.q_len;
-    // Key tiles query tile qt .. qt + 127 needs.
-    auto tiles_needed = [&](int qt) -> int {
-        if (qt >= w.q_len) return 0;
-        const int last_q = min(qt + 127, w.q_len - 1);
-        const int kend = CAUSAL ? min(w.k_len, last_q + w.k_len - w.q_len + 1) : w.k_len;
-        return kend > 0 ? (kend + 127) / 128 : 0;
+    // Key tiles [jl[t], jh[t]) query tile t (rows q0 + 128 t ..) needs: the window of its
+    // first row starts lowest, that of its last row ends highest.
+    auto tiles = [&](int qt, int& jl, int& jh) {
+        jl = jh = 0;
+        if (qt >= w.q_len) return;
+        int lo, hi, lo2, hi2;
+        key_range<CAUSAL>(a, qt, w.q_len, w.k_len, lo, hi);
+        key_range<CAUSAL>(a, min(qt + 127, w.q_len - 1), w.q_len, w.k_len, lo2, hi2);
+        if (hi2 > lo) {
+            jl = lo / 128;
+            jh = (hi2 + 127) / 128;
+        }
     };
-    w.n_0 = tiles_needed(w.q0);
-    w.n_1 = tiles_needed(w.q0 + 128);
-    w.n_kv = max(w.n_0, w.n_1);
+    int jl0, jh0, jl1, jh1;
+    tiles(w.q0, jl0, jh0);
+    tiles(w.q0 + 128, jl1, jh1);
+    const bool e0 = jh0 == jl0, e1 = jh1 == jl1;
+    w.jlo = e0 ? jl1 : (e1 ? jl0 : min(jl0, jl1));
+    const int jhi = e0 ? jh1 : (e1 ? jh0 : max(jh0, jh1));
+    w.n_kv = jhi - w.jlo;
+    w.a0 = e0 ? 0 : jl0 - w.jlo;
+    w.b0 = e0 ? 0 : jh0 - w.jlo;
+    w.a1 = e1 ? 0 : jl1 - w.jlo;
+    w.b1 = e1 ? 0 : jh1 - w.jlo;
     return w;
 }
 
@@ -312,14 +343,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
                         tma_load_4d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tm_k, &k_full[st], s * 64, hk,
-                                    w.k_row0 + j * 128, w.tma_b);
+                                    w.k_row0 + (w.jlo + j) * 128, w.tma_b);
                     ++k_issued;
                     if (!(ok = mbar_wait(&v_empty[st], ph ^ 1u, wc, 62))) break;
                     mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
                         tma_load_4d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tm_v, &v_full[st], s * 64, hk,
-                                    w.k_row0 + j * 128, w.tma_b);
+                                    w.k_row0 + (w.jlo + j) * 128, w.tma_b);
                     ++v_issued;
                 }
             }
@@ -360,8 +391,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tc_fence_after();
                 // The first S products of this unit run while the softmax warpgroups
                 // still write the previous unit's O (they touch only the S columns).
-                if (w.n_0 > 0) issue_s(0, gk);
-                if (w.n_1 > 0) issue_s(1, gk);
+                for (int t = 0; t < 2; ++t)
+                    if (w.a(t) == 0 && w.b(t) > 0) issue_s(t, gk);
                 if (w.n_kv == 1) tc_commit(q_empty);
                 tc_commit(&k_empty[gk % S]);
                 for (int j = 0; ok && j < w.n_kv; ++j) {
@@ -379,8 +410,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         // unit's epilogue must have read it (waited for every tile, so
                         // the phases of o_free stay in step with the units).
                         if (j == 0 && nq > 0 && !(ok = mbar_wait(&o_free[t], (nq - 1) & 1, wc, 67))) break;
-                        const int ntt = t ? w.n_1 : w.n_0;
-                        if (j >= ntt) continue;
+                        if (j < w.a(t) || j >= w.b(t)) {
+                            // under a window a tile can start later than the unit's first key tile
+                            if (j + 1 == w.a(t)) issue_s(t, g + 1);
+                            continue;
+                        }
                         if (!(ok = mbar_wait(&p_full[t], ps[t] & 1, wc, 68))) break;
                         ++ps[t];
                         tc_fence_after();
@@ -388,8 +422,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         for (int kk = 0; kk < 8; ++kk)
                             mma_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
                                    sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024), id_pv,
-                                   (j > 0 || kk > 0) ? 1u : 0u);
-                        if (j + 1 < ntt) issue_s(t, g + 1);
+                                   (j > w.a(t) || kk > 0) ? 1u : 0u);
+                        if (j + 1 < w.b(t)) issue_s(t, g + 1);
                     }
                     if (j + 2 == w.n_kv) tc_commit(q_empty);  // the unit's last S products are issued
                     tc_commit(&v_empty[st]);
@@ -432,7 +466,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!w.rows) continue;
             const int qt0 = w.q0 + 128 * t;
             const int q = qt0 + r;
-            const int nt = t ? w.n_1 : w.n_0;
+            const int nt = w.b(t) - w.a(t);  // key tiles w.jlo + w.a(t) + jj, jj < nt
             // This thread's output row (computed where it is used, to keep registers
             // free during the key loop).
             auto row_ok = [&]() -> bool {
@@ -457,9 +491,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 continue;
             }
-            const int row_limit = CAUSAL ? min(w.k_len, q + w.k_len - w.q_len + 1) : w.k_len;
-            // Key tiles at or past this index need masking for some row of the tile.
-            const int min_limit = CAUSAL ? min(w.k_len, qt0 + w.k_len - w.q_len + 1) : w.k_len;
+            // This row's visible keys [row_lo, row_hi); a key tile needs masking when it
+            // reaches below the last row's first key or past the first row's last key.
+            int row_lo, row_hi, lo_last, hi_dummy, lo_dummy, hi_first;
+            key_range<CAUSAL>(args, q, w.q_len, w.k_len, row_lo, row_hi);
+            key_range<CAUSAL>(args, min(qt0 + 127, max(w.q_len - 1, qt0)), w.q_len, w.k_len, lo_last, hi_dummy);
+            key_range<CAUSAL>(args, qt0, w.q_len, w.k_len, lo_dummy, hi_first);
+            const int j0 = w.jlo + w.a(t);  // key tile of this warpgroup's first step
             if constexpr (QKNORM) {  // this thread's row of Q, before the unit's first S product
                 ok = warp_all(mbar_wait(q_full, nq & 1, wc, 57));
                 if (!ok) break;
@@ -473,8 +511,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (!ok) break;
                 ++ss;
                 tc_fence_after();
-                const int lim = row_limit - j * 128;  // columns >= lim are masked
-                const bool need_mask = j * 128 + 128 > min_limit;
+                const int k0 = (j0 + j) * 128;
+                const int lim = row_hi - k0;     // columns >= lim are masked
+                const int lim_lo = row_lo - k0;  // and columns < lim_lo
+                const bool need_mask = k0 + 128 > hi_first || k0 < lo_last;
                 uint32_t sv[4][32];
     #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
@@ -483,7 +523,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (need_mask) {  // masked columns read as -inf: out of the max, P = 0
     #pragma unroll
                     for (int c = 0; c < 128; ++c)
-                        if (c >= lim) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                        if (c >= lim || c < lim_lo) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
                 }
                 // Row max: 8 independent chains of three-input max.
                 float mxp[8];

@@ -101,6 +101,26 @@ fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, fl
                         fa_stream_t stream);
 
 /*
+ * Sliding-window (local) attention, forward and backward: key j is visible to
+ * query i iff a - window_left <= j <= a + window_right, where a = i + Nk - Nq
+ * is i's bottom-right-aligned key; a negative side is unbounded. (-1, 0) is
+ * the causal mask, (-1, -1) no mask. Whole key tiles outside every row's
+ * window are skipped (the block-skipping of local attention, "YOLOv12 ...",
+ * section 4.2, and the tile skipping of "FlashAttention/zh"); the tiles on a
+ * window's edges are masked per element. A row whose window holds no key has
+ * O = 0 and L = -inf.
+ * Every other argument, result and error is that of fa_fwd / fa_bwd (the
+ * backward takes the lse of fa_fwd_window with the same window).
+ */
+fa_status fa_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                        float scale, int window_left, int window_right, fa_dtype dtype, fa_stream_t stream);
+fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                        int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                        float scale, int window_left, int window_right, fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Forward with the query/key RMS normalisation fused in front of attention
  * (the InternViT attention applies an RMSNorm to Q and K, per head, just
  * before its FlashAttention call): with

@@ -1,0 +1,114 @@
+"""Sliding-window (local) attention: fa_fwd_window / fa_bwd_window through the C ABI
+against the fp64 oracle with the same window."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_tiled_attention_36_b200 import binding as fb
+from exact_tiled_attention_36_b200 import inputs
+from tests.gpu_util import ATOL_L, RTOL_GRAD, f64, guarded, o_bound
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    fb.lib()
+    yield
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+
+
+def rel_l2(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def run(fi, window, backward=True):
+    q, k, v = fi.q.cuda(), fi.k.cuda(), fi.v.cuda()
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    dt = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
+    o, o_ok = guarded((B, Nq, Hq, d), q.dtype)
+    lse, l_ok = guarded((B, Hq, Nq), torch.float32)
+    wl, wr = window
+    st = fb.fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, Nk,
+                          d, d ** -0.5, wl, wr, dt, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    grads = None
+    if backward:
+        do = fi.do.cuda()
+        ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, Nq, d), dtype=torch.uint8, device="cuda")
+        dq, dq_ok = guarded((B, Nq, Hq, d), q.dtype)
+        dk, dk_ok = guarded((B, Nk, Hkv, d), q.dtype)
+        dv, dv_ok = guarded((B, Nk, Hkv, d), q.dtype)
+        st = fb.fa_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                              d ** -0.5, wl, wr, dt, 0)
+        assert st == fb.FA_OK, fb.fa_status_string(st)
+    torch.cuda.synchronize()
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    assert o_ok() and l_ok(), "write outside O / L"
+    if backward:
+        assert dq_ok() and dk_ok() and dv_ok(), "write outside dQ / dK / dV"
+        grads = (f64(dq), f64(dk), f64(dv))
+    return f64(o), f64(lse), grads
+
+
+CASES = [
+    # B, Nq, Nk, Hq, Hkv, d, window, dtype
+    (1, 700, 700, 2, 1, 128, (128, 0), "bf16"),
+    (2, 513, 513, 4, 2, 128, (200, 300), "fp16"),
+    (1, 400, 650, 2, 2, 64, (64, 64), "bf16"),
+    (1, 640, 300, 2, 1, 128, (-1, 100), "bf16"),
+    (1, 333, 333, 2, 2, 64, (0, 0), "fp16"),
+    (2, 300, 300, 4, 4, 128, (1000, -1), "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"b{c[0]}-{c[1]}x{c[2]}-h{c[3]}-{c[4]}-d{c[5]}-w{c[6][0]}_{c[6][1]}-{c[7]}")
+def test_window_fwd_bwd(case):
+    B, Nq, Nk, Hq, Hkv, d, window, dt = case
+    fi = inputs.make_fixed(inputs.CAUSAL_GQA, B=B, Nq=Nq, Nk=Nk, Hq=Hq, Hkv=Hkv, d=d, dtype=dt, seed=73)
+    o, lse, (dq, dk, dv) = run(fi, window)
+    o_ref, l_ref = oracle.attn_fwd(fi.q, fi.k, fi.v, d ** -0.5, window=window)
+    empty = np.isneginf(l_ref)
+    assert np.isneginf(lse[empty]).all()
+    assert (o.transpose(0, 2, 1, 3)[empty] == 0).all()
+    live = ~empty
+    assert np.abs(lse[live] - l_ref[live]).max() <= ATOL_L
+    assert (np.abs(o - o_ref) <= o_bound(o_ref, fi.q.dtype)).all()
+    rq, rk, rv = oracle.attn_bwd(fi.q, fi.k, fi.v, fi.do, d ** -0.5, window=window)
+    errs = [rel_l2(g, r) for g, r in ((dq, rq), (dk, rk), (dv, rv))]
+    assert max(errs) <= RTOL_GRAD, errs
+
+
+def test_causal_window_is_the_causal_path():
+    """(-1, 0) through the window entry points gives fa_fwd / fa_bwd with causal = 1
+    bit for bit."""
+    B, N, Hq, Hkv, d = 1, 520, 4, 2, 128
+    fi = inputs.make_fixed(inputs.CAUSAL_GQA, B=B, Nq=N, Nk=N, Hq=Hq, Hkv=Hkv, d=d, seed=79)
+    o, lse, (dq, dk, dv) = run(fi, (-1, 0))
+    q, k, v, do = (t.cuda() for t in (fi.q, fi.k, fi.v, fi.do))
+    o2, l2 = fb.attention_fwd(q, k, v, d ** -0.5, True)
+    dq2, dk2, dv2 = fb.attention_bwd(q, k, v, o2, l2, do, d ** -0.5, True)
+    torch.cuda.synchronize()
+    assert np.array_equal(o, f64(o2)) and np.array_equal(lse, f64(l2))
+    assert np.array_equal(dk, f64(dk2)) and np.array_equal(dv, f64(dv2))
+    assert rel_l2(dq, f64(dq2)) <= 1e-2  # dQ differs only in the order of its fp32 reductions
+
+
+def test_window_long_sequence_sampled_rows():
+    """A causal sliding window of 1024 keys over 8192 tokens: sampled rows of O and L,
+    and the dV identity sum_j dV_j = sum_i dO_i (rows of P sum to 1)."""
+    B, N, Hq, Hkv, d, window = 1, 8192, 4, 1, 128, (1024, 0)
+    fi = inputs.make_fixed(inputs.CAUSAL_GQA, B=B, Nq=N, Nk=N, Hq=Hq, Hkv=Hkv, d=d, seed=83)
+    o, lse, (dq, dk, dv) = run(fi, window)
+    rows = [0, 1, 1023, 1024, 1025, 4000, 8191]
+    o_ref, l_ref = oracle.attn_fwd(fi.q, fi.k, fi.v, d ** -0.5, window=window, rows=rows)
+    assert (np.abs(o[:, rows] - o_ref[:, rows]) <= o_bound(o_ref[:, rows], fi.q.dtype)).all()
+    assert np.abs(lse[:, :, rows] - l_ref[:, :, rows]).max() <= ATOL_L
+    ref = f64(fi.do).sum((0, 1))  # (Hq, d) -> the single KV head sums all query heads
+    assert rel_l2(dv.sum((0, 1))[0], ref.sum(0)) <= RTOL_GRAD
