@@ -117,10 +117,10 @@ fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtyp
     return FA_OK;
 }
 
-template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool QKNORM>
+template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM>
 fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                        dim3 grid, cudaStream_t stream) {
-    auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, VARLEN, QKNORM>;
+    auto kern = fa::fa_fwd_kernel<D, BF16, MASK, VARLEN, QKNORM>;
     constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
     static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
     if (!attr_ok) return FA_ERR_CUDA;
@@ -136,35 +136,30 @@ fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool QKNORM>
-fa_status launch_fwd_d(bool bf16, bool causal, bool varlen, const CUtensorMap& mq, const CUtensorMap& mk,
+// The instantiations: mask none / causal for every path; the sliding window for
+// fixed-length plain inputs only.
+template <int D, bool BF16>
+fa_status launch_fwd_b(int mask, bool varlen, bool qknorm, const CUtensorMap& mq, const CUtensorMap& mk,
                        const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
-    if constexpr (QKNORM) {  // fixed length only
-        if (bf16) return causal ? launch_fwd_t<D, true, true, false, true>(mq, mk, mv, a, grid, s)
-                                : launch_fwd_t<D, true, false, false, true>(mq, mk, mv, a, grid, s);
-        return causal ? launch_fwd_t<D, false, true, false, true>(mq, mk, mv, a, grid, s)
-                      : launch_fwd_t<D, false, false, false, true>(mq, mk, mv, a, grid, s);
-    } else {
-        if (bf16) {
-            if (causal) return varlen ? launch_fwd_t<D, true, true, true, false>(mq, mk, mv, a, grid, s)
-                                      : launch_fwd_t<D, true, true, false, false>(mq, mk, mv, a, grid, s);
-            return varlen ? launch_fwd_t<D, true, false, true, false>(mq, mk, mv, a, grid, s)
-                          : launch_fwd_t<D, true, false, false, false>(mq, mk, mv, a, grid, s);
-        }
-        if (causal) return varlen ? launch_fwd_t<D, false, true, true, false>(mq, mk, mv, a, grid, s)
-                                  : launch_fwd_t<D, false, true, false, false>(mq, mk, mv, a, grid, s);
-        return varlen ? launch_fwd_t<D, false, false, true, false>(mq, mk, mv, a, grid, s)
-                      : launch_fwd_t<D, false, false, false, false>(mq, mk, mv, a, grid, s);
+    constexpr int N = fa::kMaskNone, C = fa::kMaskCausal, W = fa::kMaskWindow;
+    if (qknorm) {
+        if (varlen || mask == W) return FA_ERR_UNSUPPORTED;
+        return mask == C ? launch_fwd_t<D, BF16, C, false, true>(mq, mk, mv, a, grid, s)
+                         : launch_fwd_t<D, BF16, N, false, true>(mq, mk, mv, a, grid, s);
     }
+    if (mask == W) return varlen ? FA_ERR_UNSUPPORTED : launch_fwd_t<D, BF16, W, false, false>(mq, mk, mv, a, grid, s);
+    if (mask == C) return varlen ? launch_fwd_t<D, BF16, C, true, false>(mq, mk, mv, a, grid, s)
+                                 : launch_fwd_t<D, BF16, C, false, false>(mq, mk, mv, a, grid, s);
+    return varlen ? launch_fwd_t<D, BF16, N, true, false>(mq, mk, mv, a, grid, s)
+                  : launch_fwd_t<D, BF16, N, false, false>(mq, mk, mv, a, grid, s);
 }
 
-fa_status launch_fwd(int d, bool bf16, bool causal, bool varlen, bool qknorm, const CUtensorMap& mq,
+fa_status launch_fwd(int d, bool bf16, int mask, bool varlen, bool qknorm, const CUtensorMap& mq,
                      const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
-    if (qknorm)
-        return d == 64 ? launch_fwd_d<64, true>(bf16, causal, varlen, mq, mk, mv, a, grid, s)
-                       : launch_fwd_d<128, true>(bf16, causal, varlen, mq, mk, mv, a, grid, s);
-    return d == 64 ? launch_fwd_d<64, false>(bf16, causal, varlen, mq, mk, mv, a, grid, s)
-                   : launch_fwd_d<128, false>(bf16, causal, varlen, mq, mk, mv, a, grid, s);
+    if (d == 64) return bf16 ? launch_fwd_b<64, true>(mask, varlen, qknorm, mq, mk, mv, a, grid, s)
+                             : launch_fwd_b<64, false>(mask, varlen, qknorm, mq, mk, mv, a, grid, s);
+    return bf16 ? launch_fwd_b<128, true>(mask, varlen, qknorm, mq, mk, mv, a, grid, s)
+                : launch_fwd_b<128, false>(mask, varlen, qknorm, mq, mk, mv, a, grid, s);
 }
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -373,11 +368,12 @@ fa_status check_strides(const Strides& t, bool with_batch) {
     return FA_OK;
 }
 
-// `causal` selects the masked kernels; their window is (wl, wr) (causal: (-1, 0)).
+// `causal` (0 or 1) is the caller's flag; a sliding window (wl, wr) other than the
+// causal (-1, 0) or none (-1, -1) selects the window kernels instead.
 fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
                     Strides sv, Strides so, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                     fa_dtype dtype, fa_stream_t stream, bool qknorm = false, float eps = 0.f,
-                    bool validate_only = false, int wl = -1, int wr = 0) {
+                    bool validate_only = false, bool window = false, int wl = -1, int wr = 0) {
     if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if ((Nq > 0 && (!q || !o || !lse)) || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
     fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
@@ -413,8 +409,8 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
     a.err = err;
     dim3 grid;
     if ((st = fwd_units(a, B, Nq, grid)) != FA_OK) return st;
-    return launch_fwd(d, bf16, causal != 0, false, qknorm, mq, mk, mv, a, grid,
-                      reinterpret_cast<cudaStream_t>(stream));
+    const int mask = window ? fa::kMaskWindow : (causal ? fa::kMaskCausal : fa::kMaskNone);
+    return launch_fwd(d, bf16, mask, false, qknorm, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
@@ -467,7 +463,7 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
     a.err = err;
     dim3 grid;
     if ((st = fwd_units(a, num_seqs, max_seqlen_q, grid)) != FA_OK) return st;
-    return launch_fwd(d, bf16, causal != 0, true, false, mq, mk, mv, a, grid,
+    return launch_fwd(d, bf16, causal ? fa::kMaskCausal : fa::kMaskNone, true, false, mq, mk, mv, a, grid,
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -532,10 +528,10 @@ fa_status fa_fwd_window(const void* q, const void* k, const void* v, void* o, fl
                         int Nq, int Nk, int d, float scale, int window_left, int window_right, fa_dtype dtype,
                         fa_stream_t stream) {
     const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
-    const bool masked = wl >= 0 || wr >= 0;
+    const bool none = wl < 0 && wr < 0, causal = wl < 0 && wr == 0;
     return fwd_fixed(q, k, v, o, lse, contiguous(Nq, Hq, d), contiguous(Nk, Hkv, d), contiguous(Nk, Hkv, d),
-                     contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, masked ? 1 : 0, dtype, stream, false, 0.f,
-                     false, wl, wr);
+                     contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, dtype, stream, false, 0.f,
+                     false, !none && !causal, wl, wr);
 }
 
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,

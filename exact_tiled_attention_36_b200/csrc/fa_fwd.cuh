@@ -111,25 +111,29 @@ struct FwdUnit {
     __device__ __forceinline__ int b(int t) const { return t ? b1 : b0; }
 };
 
-// First visible key and one past the last for query q (bottom-right alignment; the
-// window (wl, wr) of FwdArgs, or every key without a mask).
-template <bool MASKED>
+// Mask kinds of the forward: none, causal (the window (-1, 0), fixed at compile
+// time), or the sliding window (wl, wr) of FwdArgs.
+enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2 };
+
+// First visible key and one past the last for query q (bottom-right alignment).
+template <int MASK>
 __device__ __forceinline__ void key_range(const FwdArgs& a, int q, int q_len, int k_len, int& lo, int& hi) {
     lo = 0;
     hi = k_len;
-    if (MASKED) {
-        const int aligned = q + k_len - q_len;
+    const int aligned = q + k_len - q_len;
+    if (MASK == kMaskCausal) hi = min(k_len, aligned + 1);
+    if (MASK == kMaskWindow) {
         if (a.wl >= 0) lo = max(0, aligned - a.wl);
         if (a.wr >= 0) hi = min(k_len, aligned + a.wr + 1);
     }
 }
 
-template <bool CAUSAL, bool VARLEN>
+template <int MASK, bool VARLEN>
 __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdArgs& a) {
     FwdUnit w;
     const int hb = a.Hq * a.num_batches;
     int unit, r;
-    if (CAUSAL) {  // heaviest units (last query rows) first
+    if (MASK == kMaskCausal) {  // heaviest units (last query rows) first
         unit = a.nu - 1 - u / hb;
         r = u % hb;
     } else {  // the units of one (batch, head) together
@@ -159,8 +163,8 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdArgs& a) {
         jl = jh = 0;
         if (qt >= w.q_len) return;
         int lo, hi, lo2, hi2;
-        key_range<CAUSAL>(a, qt, w.q_len, w.k_len, lo, hi);
-        key_range<CAUSAL>(a, min(qt + 127, w.q_len - 1), w.q_len, w.k_len, lo2, hi2);
+        key_range<MASK>(a, qt, w.q_len, w.k_len, lo, hi);
+        key_range<MASK>(a, min(qt + 127, w.q_len - 1), w.q_len, w.k_len, lo2, hi2);
         if (hi2 > lo) {
             jl = lo / 128;
             jh = (hi2 + 127) / 128;
@@ -230,11 +234,13 @@ __device__ __forceinline__ void rms_normalise_row(uint8_t* tile, int r, float ep
         }
 }
 
+// MASK: kMaskNone, kMaskCausal (bottom-right, folded at compile time) or kMaskWindow
+// (the sliding window (wl, wr) of FwdArgs; fixed length only).
 // QKNORM: Q arrives raw and each softmax thread RMS-normalises its own row of Q in
 // shared memory (over d) at the start of a unit, before the tensor core reads it;
 // K arrives normalised (fa_fwd_qk_rmsnorm runs fa_rms_normalise_rows over K first:
 // every CTA would otherwise redo each K tile once per unit).
-template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool QKNORM>
+template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -322,7 +328,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int rnd = 0; ok; ++rnd) {
                 const int u = fwd_unit_index(rnd, cta, G);
                 if (u >= args.n_units) break;
-                const FwdUnit w = fwd_unit<CAUSAL, VARLEN>(u, args);
+                const FwdUnit w = fwd_unit<MASK, VARLEN>(u, args);
                 if (!w.rows || w.n_kv == 0) continue;
                 // Q of this unit once the previous unit's last S product has read Q.
                 if (!(ok = mbar_wait(q_empty, (nq & 1) ^ 1u, wc, 60))) break;
@@ -384,7 +390,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int rnd = 0; ok; ++rnd) {
                 const int u = fwd_unit_index(rnd, cta, G);
                 if (u >= args.n_units) break;
-                const FwdUnit w = fwd_unit<CAUSAL, VARLEN>(u, args);
+                const FwdUnit w = fwd_unit<MASK, VARLEN>(u, args);
                 if (!w.rows || w.n_kv == 0) continue;
                 if (!(ok = mbar_wait(q_ready, nq & 1, wc, 63))) break;
                 if (!(ok = mbar_wait(&k_full[gk % S], (gk / S) & 1, wc, 64))) break;
@@ -462,42 +468,42 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int rnd = 0; ok; ++rnd) {
             const int u = fwd_unit_index(rnd, cta, G);
             if (u >= args.n_units) break;
-            const FwdUnit w = fwd_unit<CAUSAL, VARLEN>(u, args);
+            const FwdUnit w = fwd_unit<MASK, VARLEN>(u, args);
             if (!w.rows) continue;
             const int qt0 = w.q0 + 128 * t;
             const int q = qt0 + r;
             const int nt = w.b(t) - w.a(t);  // key tiles w.jlo + w.a(t) + jj, jj < nt
             // This thread's output row (computed where it is used, to keep registers
             // free during the key loop).
-            auto row_ok = [&]() -> bool {
-                if constexpr (VARLEN) return q < w.q_len && w.q_row0 + q >= 0 && w.q_row0 + q < args.total_q;
-                return q < w.q_len;
+            // (The unit is decoded again there: nothing of it stays live across the loop.)
+            auto row_ok = [&](const FwdUnit& x) -> bool {
+                if constexpr (VARLEN) return q < x.q_len && x.q_row0 + q >= 0 && x.q_row0 + q < args.total_q;
+                return q < x.q_len;
             };
-            auto out_row = [&]() -> T16* {
-                const long long row = VARLEN ? static_cast<long long>(w.q_row0 + q) * args.o_ss
-                                             : w.bidx * args.o_sb + static_cast<long long>(q) * args.o_ss;
-                return o_base + row + w.h * args.o_sh;
+            auto out_row = [&](const FwdUnit& x) -> T16* {
+                const long long row = VARLEN ? static_cast<long long>(x.q_row0 + q) * args.o_ss
+                                             : x.bidx * args.o_sb + static_cast<long long>(q) * args.o_ss;
+                return o_base + row + x.h * args.o_sh;
             };
-            auto lse_row = [&]() -> float* {
-                return VARLEN ? args.lse + static_cast<size_t>(w.h) * args.total_q + w.q_row0 + q
-                              : args.lse + (static_cast<size_t>(w.bidx) * args.Hq + w.h) * args.Nq + q;
+            auto lse_row = [&](const FwdUnit& x) -> float* {
+                return VARLEN ? args.lse + static_cast<size_t>(x.h) * args.total_q + x.q_row0 + q
+                              : args.lse + (static_cast<size_t>(x.bidx) * args.Hq + x.h) * args.Nq + q;
             };
             if (w.n_kv == 0) {  // no row of this unit sees any key: O = 0, L = -inf
-                if (row_ok()) {
-                    uint4* d4 = reinterpret_cast<uint4*>(out_row());
+                if (row_ok(w)) {
+                    uint4* d4 = reinterpret_cast<uint4*>(out_row(w));
 #pragma unroll
                     for (int c = 0; c < D / 8; ++c) d4[c] = make_uint4(0, 0, 0, 0);
-                    *lse_row() = -INFINITY;
+                    *lse_row(w) = -INFINITY;
                 }
                 continue;
             }
-            // This row's visible keys [row_lo, row_hi); a key tile needs masking when it
-            // reaches below the last row's first key or past the first row's last key.
-            int row_lo, row_hi, lo_last, hi_dummy, lo_dummy, hi_first;
-            key_range<CAUSAL>(args, q, w.q_len, w.k_len, row_lo, row_hi);
-            key_range<CAUSAL>(args, min(qt0 + 127, max(w.q_len - 1, qt0)), w.q_len, w.k_len, lo_last, hi_dummy);
-            key_range<CAUSAL>(args, qt0, w.q_len, w.k_len, lo_dummy, hi_first);
-            const int j0 = w.jlo + w.a(t);  // key tile of this warpgroup's first step
+            // This row's visible keys, relative to the first key of this warpgroup's
+            // first step: [rel_lo, rel_hi).
+            int rel_lo, rel_hi;
+            key_range<MASK>(args, q, w.q_len, w.k_len, rel_lo, rel_hi);
+            rel_lo -= (w.jlo + w.a(t)) * 128;
+            rel_hi -= (w.jlo + w.a(t)) * 128;
             if constexpr (QKNORM) {  // this thread's row of Q, before the unit's first S product
                 ok = warp_all(mbar_wait(q_full, nq & 1, wc, 57));
                 if (!ok) break;
@@ -511,10 +517,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (!ok) break;
                 ++ss;
                 tc_fence_after();
-                const int k0 = (j0 + j) * 128;
-                const int lim = row_hi - k0;     // columns >= lim are masked
-                const int lim_lo = row_lo - k0;  // and columns < lim_lo
-                const bool need_mask = k0 + 128 > hi_first || k0 < lo_last;
+                const int lim = rel_hi - j * 128;     // columns >= lim are masked
+                const int lim_lo = rel_lo - j * 128;  // and, under a window, columns < lim_lo
+                // (uniform per warp: only tiles on a window's edge pay for the mask)
+                const bool need_mask =
+                    __any_sync(0xffffffffu, lim < 128 || (MASK == kMaskWindow && lim_lo > 0));
                 uint32_t sv[4][32];
     #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
@@ -523,7 +530,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (need_mask) {  // masked columns read as -inf: out of the max, P = 0
     #pragma unroll
                     for (int c = 0; c < 128; ++c)
-                        if (c >= lim || c < lim_lo) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                        if (c >= lim || (MASK == kMaskWindow && c < lim_lo)) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
                 }
                 // Row max: 8 independent chains of three-input max.
                 float mxp[8];
@@ -594,8 +601,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             ++nq;
             tc_fence_after();
             const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
-            const bool out_ok = row_ok();
-            T16* dst = out_ok ? out_row() : nullptr;
+            const FwdUnit we = fwd_unit<MASK, VARLEN>(u, args);
+            const bool out_ok = row_ok(we);
+            T16* dst = out_ok ? out_row(we) : nullptr;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t pk[16];
@@ -626,7 +634,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(l));
                     L = (m + lg) * kLn2;
                 }
-                *lse_row() = L;
+                *lse_row(we) = L;
             }
         }
         tc_fence_before();
