@@ -226,6 +226,58 @@ def varlen_fwd(q, k, v, cu_q, cu_k, scale: float, causal: bool = False):
     return o, lse
 
 
+def lse_merge(o_parts, l_parts):
+    """Merge of partial results over disjoint key sets, in fp64.
+
+    ``o_parts[s]`` is the attention output over key set s alone (normalised by
+    its own sum) and ``l_parts[s]`` its log-sum-exp. Over the union,
+    L = log sum_s exp(L_s) and O = sum_s exp(L_s - L) O_s: the rescaling step of
+    the online softmax ("FlashAttention/zh", section "online softmax trick")
+    applied to whole partial results. Parts with L_s = -inf (no key) weigh 0; if
+    every part is empty, O = 0 and L = -inf. Shapes: o_parts [S, ..., d],
+    l_parts [S, ...]."""
+    o = np.asarray(o_parts, dtype=np.float64)
+    l = np.asarray(l_parts, dtype=np.float64)
+    lm = l.max(axis=0)
+    empty = ~np.isfinite(lm)
+    lm_safe = np.where(empty, 0.0, lm)
+    w = np.where(np.isfinite(l), np.exp(l - lm_safe[None]), 0.0)
+    ws = w.sum(axis=0)
+    O = (w[..., None] * np.where(np.isfinite(l)[..., None], o, 0.0)).sum(axis=0)
+    O = np.where(empty[..., None], 0.0, O / np.where(empty, 1.0, ws)[..., None])
+    L = np.where(empty, -np.inf, lm_safe + np.log(np.where(empty, 1.0, ws)))
+    return O, L
+
+
+def paged_gather(pool, table_row, length: int, page_size: int):
+    """Keys 0 .. length-1 of one sequence of a paged cache: key p is row
+    p % page_size of page table_row[p // page_size] of ``pool``
+    [num_pages, page_size, H, d]. Returns [length, H, d]."""
+    pos = np.arange(int(length))
+    tr = np.asarray(table_row, dtype=np.int64)
+    return np.asarray(pool)[tr[pos // page_size], pos % page_size]
+
+
+def attn_decode(q, k, v, scale: float, seqlens=None, causal: bool = False):
+    """Attention of the Nq newest query tokens of each sequence against its
+    cache: sequence b attends to its first seqlens[b] keys (all Nk when
+    ``seqlens`` is None), as an independent problem of the plain definition
+    (attn_fwd; causal is bottom-right aligned within the sequence's keys).
+    q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]; returns O [B,Nq,Hq,d], L [B,Hq,Nq]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Hq, d = q.shape
+    Nk = k.shape[1]
+    o = np.zeros((B, Nq, Hq, d))
+    lse = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        n = Nk if seqlens is None else min(max(int(seqlens[b]), 0), Nk)
+        if n == 0 or Nq == 0:
+            continue
+        ob, lb = attn_fwd(q[b:b + 1], k[b:b + 1, :n], v[b:b + 1, :n], scale, causal)
+        o[b], lse[b] = ob[0], lb[0]
+    return o, lse
+
+
 def timed(fn, *args, **kw):
     """(result, seconds) of one call."""
     t0 = time.perf_counter()

@@ -399,3 +399,90 @@ def test_window_backward_matches_finite_differences():
             minus[which][idx] -= h
             fd[idx] = (phi(*plus) - phi(*minus)) / (2 * h)
         assert np.linalg.norm(fd - g) / np.linalg.norm(g) <= 1e-6, which
+
+
+# ---------------------------------------------------------------- decode: merge, paged cache, cache lengths
+@pytest.mark.parametrize("causal", [False, True])
+def test_lse_merge_of_key_chunks_equals_whole(causal):
+    """Attention over disjoint key chunks, merged by the log-sum-exp rule, equals
+    attention over all keys (the whole-problem oracle, and the numpy version)."""
+    rng = np.random.default_rng(51)
+    B, Nq, Nk, Hq, Hkv, d = 2, 3, 23, 4, 2, 8
+    q, k, v = _rand(rng, B, Nq, Hq, d), _rand(rng, B, Nk, Hkv, d), _rand(rng, B, Nk, Hkv, d)
+    o_all, l_all = oracle.attn_fwd(q, k, v, 0.7, causal)
+    cuts = [0, 5, 5, 16, Nk]  # one empty chunk
+    parts_o, parts_l = [], []
+    for a, e in zip(cuts[:-1], cuts[1:]):
+        keep = np.zeros((B, Nk), dtype=np.uint8)
+        keep[:, a:e] = 1
+        o_s, l_s = oracle.attn_fwd(q, k, v, 0.7, causal, key_keep=keep)
+        parts_o.append(o_s)
+        parts_l.append(np.moveaxis(l_s, 1, 2))  # [B, Nq, Hq] like o's leading axes
+    O, L = oracle.lse_merge(parts_o, parts_l)
+    np.testing.assert_allclose(O, o_all, atol=1e-12)
+    np.testing.assert_allclose(np.moveaxis(L, 2, 1), l_all, atol=1e-12)
+    o_np, l_np = numpy_ref.fwd(q, k, v, 0.7, causal)
+    np.testing.assert_allclose(O, o_np, atol=1e-12)
+
+
+def test_lse_merge_special_cases():
+    rng = np.random.default_rng(52)
+    o1, l1 = _rand(rng, 4, 3), _rand(rng, 4)
+    O, L = oracle.lse_merge([o1], [l1])  # one part: unchanged
+    np.testing.assert_allclose(O, o1, atol=1e-15)
+    np.testing.assert_allclose(L, l1, atol=1e-15)
+    O, L = oracle.lse_merge([o1, np.full_like(o1, np.nan)], [l1, np.full_like(l1, -np.inf)])  # empty part ignored
+    np.testing.assert_allclose(O, o1, atol=1e-15)
+    np.testing.assert_allclose(L, l1, atol=1e-15)
+    O, L = oracle.lse_merge([o1, o1], [l1, l1])  # two equal halves: O unchanged, L + ln 2
+    np.testing.assert_allclose(O, o1, atol=1e-14)
+    np.testing.assert_allclose(L, l1 + math.log(2), atol=1e-14)
+    O, L = oracle.lse_merge([o1], [np.full_like(l1, -np.inf)])  # nothing: O = 0, L = -inf
+    assert (O == 0).all() and np.isneginf(L).all()
+
+
+def test_paged_gather_inverts_a_scatter():
+    rng = np.random.default_rng(53)
+    n, page, H, d = 150, 16, 2, 4
+    k = _rand(rng, n, H, d)
+    n_pages = (n + page - 1) // page
+    table = rng.permutation(20)[:n_pages]  # pages drawn from a pool of 20 in random order
+    pool = np.full((20, page, H, d), np.nan)
+    for p in range(n):
+        pool[table[p // page], p % page] = k[p]
+    np.testing.assert_array_equal(oracle.paged_gather(pool, table, n, page), k)
+    assert oracle.paged_gather(pool, table, 0, page).shape == (0, H, d)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attn_decode_pins(causal):
+    rng = np.random.default_rng(54)
+    B, Nq, Nk, Hq, Hkv, d = 4, 3, 40, 4, 2, 8
+    q, k, v = _rand(rng, B, Nq, Hq, d), _rand(rng, B, Nk, Hkv, d), _rand(rng, B, Nk, Hkv, d)
+    # every sequence full: the plain forward
+    o, l = oracle.attn_decode(q, k, v, 0.5, None, causal)
+    o2, l2 = oracle.attn_fwd(q, k, v, 0.5, causal)
+    np.testing.assert_allclose(o, o2, atol=1e-13)
+    np.testing.assert_allclose(l, l2, atol=1e-13)
+    # own lengths: keys past the length never matter (NaN there), and each sequence is
+    # the numpy whole-matrix version on its prefix; length 0 gives O = 0, L = -inf
+    lens = [40, 17, 0, 2]
+    kn, vn = k.copy(), v.copy()
+    for b, n in enumerate(lens):
+        kn[b, n:] = np.nan
+        vn[b, n:] = np.nan
+    o, l = oracle.attn_decode(q, kn, vn, 0.5, lens, causal)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert (o[b] == 0).all() and np.isneginf(l[b]).all()
+            continue
+        ob, lb = numpy_ref.fwd(q[b:b + 1], k[b:b + 1, :n], v[b:b + 1, :n], 0.5, causal)
+        np.testing.assert_allclose(o[b], ob[0], atol=1e-12)
+        np.testing.assert_allclose(l[b], lb[0], atol=1e-12)
+    if not causal:  # a tail key mask on the full cache is the same thing
+        keep = np.zeros((B, Nk), dtype=np.uint8)
+        for b, n in enumerate(lens):
+            keep[b, :n] = 1
+        o3, l3 = oracle.attn_fwd(q, k, v, 0.5, False, key_keep=keep)
+        np.testing.assert_allclose(o, o3, atol=1e-13)
+        np.testing.assert_allclose(l, l3, atol=1e-13)
