@@ -1,7 +1,7 @@
 """Thin ctypes binding of libfa.so.
 
 The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_fwd_strided``, ``fa_varlen_fwd_strided``, ``fa_fwd_qk_rmsnorm``,
-``fa_fwd_window``, ``fa_bwd_window``,
+``fa_fwd_window``, ``fa_bwd_window``, ``fa_decode``, ``fa_decode_paged``, ``fa_decode_workspace_size``,
 ``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
 ``fa_bwd``, ``fa_status_string`` and ``fa_get_last_device_error`` have the
 names, argument order and meaning of the C ABI in ``include/fa.h``: pointers
@@ -51,6 +51,9 @@ _SIGS = {
     "fa_varlen_fwd_strided": ([_P] * 11 + [_I] * 8 + [_F, _I, _I, _P], _I),
     "fa_varlen_bwd": ([_P] * 12 + [_I] * 8 + [_F, _I, _I, _P], _I),
     "fa_selftest_bounded_wait": ([_P], _I),
+    "fa_decode_workspace_size": ([_I] * 5, ctypes.c_size_t),
+    "fa_decode": ([_P] * 7 + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_decode_paged": ([_P] * 8 + [_I] * 8 + [_F, _I, _I, _P], _I),
 }
 
 
@@ -154,6 +157,21 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, sca
     """fa_bwd with the library's own fixed-size workspace (for callers that cannot allocate)."""
     return lib().fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype,
                                 stream)
+
+
+def fa_decode_workspace_size(B, Hq, Hkv, Nq, d) -> int:
+    return int(lib().fa_decode_workspace_size(B, Hq, Hkv, Nq, d))
+
+
+def fa_decode(q, k, v, o, lse, cache_seqlens, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    return lib().fa_decode(q, k, v, o, lse, cache_seqlens, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype,
+                           stream)
+
+
+def fa_decode_paged(q, k_pages, v_pages, o, lse, cache_seqlens, block_table, workspace, B, Hq, Hkv, Nq, num_pages,
+                    page_size, max_pages, d, scale, causal, dtype, stream) -> int:
+    return lib().fa_decode_paged(q, k_pages, v_pages, o, lse, cache_seqlens, block_table, workspace, B, Hq, Hkv, Nq,
+                                 num_pages, page_size, max_pages, d, scale, causal, dtype, stream)
 
 
 def fa_status_string(s: int) -> str:
@@ -282,3 +300,38 @@ def attention_varlen_bwd(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_
                          n, Tq, Tk, int(max_seqlen_q), int(max_seqlen_k), Hq, Hkv, d, float(scale),
                          int(bool(causal)), _dtype_code(q), _stream(stream)), "fa_varlen_bwd")
     return dq, dk, dv
+
+
+def attention_decode(q, k_cache, v_cache, cache_seqlens=None, scale: float | None = None, causal: bool = False,
+                     block_table=None, workspace=None, out=None, lse=None, stream=None):
+    """Split-KV decode: q [B,Nq,Hq,d] (the newest Nq tokens) against a cache.
+
+    Contiguous cache: k/v [B,Nk,Hkv,d], sequence b using its first cache_seqlens[b]
+    keys (all Nk when None). Paged cache (block_table int32 [B,max_pages]): k/v
+    [num_pages,page_size,Hkv,d] and cache_seqlens required. Returns O [B,Nq,Hq,d]
+    and L float32 [B,Hq,Nq]."""
+    import torch
+    q, k, v = _dev(q), _dev(k_cache), _dev(v_cache)
+    B, Nq, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = d ** -0.5
+    sl = None if cache_seqlens is None else _dev(cache_seqlens).to(torch.int32)
+    ws_bytes = fa_decode_workspace_size(B, Hq, Hkv, Nq, d)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    o = torch.empty_like(q) if out is None else out
+    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    if block_table is None:
+        st = fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                       0 if sl is None else sl.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, k.shape[1], d, float(scale),
+                       int(bool(causal)), _dtype_code(q), _stream(stream))
+        _check(st, "fa_decode")
+    else:
+        if sl is None:
+            raise ValueError("a paged cache needs cache_seqlens")
+        bt = _dev(block_table).to(torch.int32)
+        st = fa_decode_paged(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), sl.data_ptr(),
+                             bt.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, k.shape[0], k.shape[1], bt.shape[1], d,
+                             float(scale), int(bool(causal)), _dtype_code(q), _stream(stream))
+        _check(st, "fa_decode_paged")
+    return o, L

@@ -16,6 +16,7 @@
 #include "fa_fwd.cuh"
 #include "fa_bwd.cuh"
 #include "fa_bwd128.cuh"
+#include "fa_decode.cuh"
 
 namespace {
 
@@ -38,12 +39,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
     return fn;
 }
 
-// Tensor map of a [batches, rows, H, d] 16-bit tensor, box = 128 rows x 64
-// columns of one head, 128-byte swizzle. Rows past `rows` read as zero.
+// Tensor map of a [batches, rows, H, d] 16-bit tensor, box = box_rows rows x
+// box_h heads x 64 columns, 128-byte swizzle. Rows past `rows` read as zero.
 // 4-D map (d, H, rows, batches) over a tensor whose head, token and batch strides
 // are sh, ss, sb elements (d contiguous); each stride must be a multiple of 16 bytes.
-fa_status make_map_strided(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16,
-                           int64_t sh, int64_t ss, int64_t sb) {
+fa_status make_map_box(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16,
+                       int64_t sh, int64_t ss, int64_t sb, int box_h, int box_rows) {
     auto enc = encode_tiled();
     if (!enc) return FA_ERR_CUDA;
     if (rows < 1) rows = 1;
@@ -52,13 +53,19 @@ fa_status make_map_strided(CUtensorMap* m, const void* base, int d, int H, int64
                                 static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batches)};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sh) * 2, static_cast<cuuint64_t>(ss) * 2,
                                    static_cast<cuuint64_t>(sb) * 2};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_h), static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Box = 128 rows x 64 columns of one head (the attention kernels' K/V/Q tiles).
+fa_status make_map_strided(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16,
+                           int64_t sh, int64_t ss, int64_t sb) {
+    return make_map_box(m, base, d, H, rows, batches, bf16, sh, ss, sb, 1, 128);
 }
 
 // Contiguous [batches, rows, H, d].
@@ -477,6 +484,163 @@ fa_status read_strides(const long long* p, bool with_batch, Strides* out) {
     return FA_OK;
 }
 
+// ---------------------------------------------------------------- decode
+// Row layout of the decode tile: nb blocks of gh heads, one block per 32 TMEM
+// lanes, when the group splits so (the exponentials then spread over the four
+// softmax warps); else one block of all g heads in lanes 0 .. g Nq - 1.
+void dec_layout(int g, int Nq, int& nb, int& gh) {
+    for (int k : {4, 2})
+        if (g % k == 0 && (g / k) * Nq <= 32) {
+            nb = k;
+            gh = g / k;
+            return;
+        }
+    nb = 1;
+    gh = g;
+}
+
+constexpr int kDecMaxCtas = 1024;
+
+// CTAs the split kernel may use on the current device (0 without one).
+int dec_max_ctas() {
+    const int sms = sm_count();
+    return sms < kDecMaxCtas ? sms : kDecMaxCtas;
+}
+
+// Workspace of the decode: meta (T and each item's first tile, int64), then the
+// partial L (fp32 [slots, R]) and O (fp32 [slots, R, d]), each 256-byte aligned;
+// slots = CTAs + items (the slot of CTA c's segment of item i is c + i).
+struct DecWs {
+    size_t meta, lse, total;
+};
+
+bool dec_ws(int B, int Hq, int Hkv, int Nq, int d, DecWs& w) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Nq < 0 || (d != 64 && d != 128)) return false;
+    const long long R = static_cast<long long>(Hq / Hkv) * Nq;
+    if (R > 128) return false;
+    const int G = dec_max_ctas();
+    if (G <= 0) return false;
+    const size_t items = static_cast<size_t>(B) * Hkv;
+    const size_t slots = items + G;
+    w.meta = round256((1 + items) * sizeof(long long));
+    w.lse = round256(slots * R * sizeof(float));
+    w.total = w.meta + w.lse + round256(slots * R * d * sizeof(float));
+    return true;
+}
+
+template <int D, bool BF16, bool SEQLENS, bool PAGED>
+fa_status launch_dec_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecodeArgs& a,
+                       int causal, bool run_split, cudaStream_t s) {
+    if (run_split) {
+        auto kern = fa::fa_decode_kernel<D, BF16, SEQLENS, PAGED>;
+        constexpr int smem = fa::DecCfg<D>::kSmemBytes;
+        static bool attr_ok =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+        if (!attr_ok) return FA_ERR_CUDA;
+        kern<<<a.G, fa::kDecThreads, smem, s>>>(mq, mk, mv, a, causal);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    fa::fa_decode_combine<D, BF16, SEQLENS><<<static_cast<unsigned>(a.B) * a.Hkv, 128, 0, s>>>(a);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+fa_status launch_dec_b(bool seqlens, bool paged, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const fa::DecodeArgs& a, int causal, bool run_split, cudaStream_t s) {
+    if (paged) return launch_dec_t<D, BF16, true, true>(mq, mk, mv, a, causal, run_split, s);
+    if (seqlens) return launch_dec_t<D, BF16, true, false>(mq, mk, mv, a, causal, run_split, s);
+    return launch_dec_t<D, BF16, false, false>(mq, mk, mv, a, causal, run_split, s);
+}
+
+// fa_decode (paged = false: k, v [B, Nk, Hkv, d]) and fa_decode_paged (k, v page
+// pools [num_pages, page_size, Hkv, d] through block_table [B, max_pages]).
+fa_status decode_common(const void* q, const void* k, const void* v, void* o, float* lse, const int* seqlens,
+                        const int* block_table, void* workspace, int B, int Hq, int Hkv, int Nq, int Nk,
+                        bool paged, int num_pages, int page_size, int max_pages, int d, float scale, int causal,
+                        fa_dtype dtype, fa_stream_t stream) {
+    if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
+    if (st != FA_OK) return st;
+    if (paged) {
+        if (!seqlens || !block_table || num_pages < 1 || max_pages < 1 || page_size < 16) return FA_ERR_INVALID_ARG;
+        if (!(page_size == 16 || page_size == 32 || page_size % 64 == 0)) return FA_ERR_UNSUPPORTED;
+    }
+    const int cap = paged ? (static_cast<long long>(max_pages) * page_size > 0x7fffffffLL ? -1 : max_pages * page_size)
+                          : Nk;
+    if (cap < 0) return FA_ERR_UNSUPPORTED;
+    if (Nq > 0 && (!q || !o || !lse || !workspace)) return FA_ERR_INVALID_ARG;
+    if (cap > 0 && (!k || !v)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        !aligned16(workspace) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u))
+        return FA_ERR_MISALIGNED;
+    const int g = Hq / Hkv;
+    if (static_cast<long long>(g) * Nq > 128) return FA_ERR_UNSUPPORTED;  // one tile holds a group's queries
+    const long long items = static_cast<long long>(B) * Hkv;
+    const long long max_tiles = items * ((static_cast<long long>(cap) + 127) / 128);
+    if (items > 0x7fffffffLL || max_tiles > (1LL << 40) || B > 65535 || Nq > 65535) return FA_ERR_UNSUPPORTED;
+    if (Nq == 0) return FA_OK;
+    int* err = error_word();
+    if (!err) return FA_ERR_CUDA;
+    DecWs w;
+    if (!dec_ws(B, Hq, Hkv, Nq, d, w)) return FA_ERR_CUDA;
+    const bool bf16 = dtype == FA_BF16;
+    int nb, gh;
+    dec_layout(g, Nq, nb, gh);
+    CUtensorMap mq, mk{}, mv{};
+    const long long hd = static_cast<long long>(Hq) * d;
+    if ((st = make_map_box(&mq, q, d, Hq, Nq, B, bf16, d, hd, hd * Nq, gh, Nq)) != FA_OK) return st;
+    const int page_box = page_size < 64 ? page_size : 64;
+    if (cap > 0) {
+        const long long kd = static_cast<long long>(Hkv) * d;
+        if (paged) {
+            if ((st = make_map_box(&mk, k, d, Hkv, page_size, num_pages, bf16, d, kd, kd * page_size, 1, page_box)) !=
+                    FA_OK ||
+                (st = make_map_box(&mv, v, d, Hkv, page_size, num_pages, bf16, d, kd, kd * page_size, 1, page_box)) !=
+                    FA_OK)
+                return st;
+        } else if ((st = make_map(&mk, k, d, Hkv, Nk, B, bf16)) != FA_OK ||
+                   (st = make_map(&mv, v, d, Hkv, Nk, B, bf16)) != FA_OK) {
+            return st;
+        }
+    }
+    fa::DecodeArgs a{};
+    a.o = o;
+    a.lse = lse;
+    a.meta = static_cast<long long*>(workspace);
+    a.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + w.meta);
+    a.o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + w.meta + w.lse);
+    a.seqlens = seqlens;
+    a.block_table = block_table;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = g;
+    a.Nq = Nq;
+    a.Nk = paged ? cap : Nk;
+    a.R = g * Nq;
+    a.cap = cap;
+    a.page_size = page_size;
+    a.max_pages = max_pages;
+    a.page_box = page_box;
+    a.nb = nb;
+    a.gh = gh;
+    a.scale_log2 = scale * kLog2e;
+    a.err = err;
+    // Fixed lengths: exactly T tiles; with lengths, at most T tiles (each CTA finds
+    // its share of the true T itself).
+    const int sms = dec_max_ctas();
+    a.G = static_cast<int>(max_tiles < sms ? max_tiles : sms);
+    const bool run_split = max_tiles > 0;
+    if (a.G < 1) a.G = 1;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool sl = seqlens != nullptr;
+    if (d == 64) return bf16 ? launch_dec_b<64, true>(sl, paged, mq, mk, mv, a, causal, run_split, s)
+                             : launch_dec_b<64, false>(sl, paged, mq, mk, mv, a, causal, run_split, s);
+    return bf16 ? launch_dec_b<128, true>(sl, paged, mq, mk, mv, a, causal, run_split, s)
+                : launch_dec_b<128, false>(sl, paged, mq, mk, mv, a, causal, run_split, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -626,6 +790,26 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
     return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, num_seqs, cu_seqlens_q, cu_seqlens_k, total_q,
                       total_k, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal != 0, dtype == FA_BF16,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int d) {
+    DecWs w;
+    return dec_ws(B, Hq, Hkv, Nq, d, w) ? w.total : 0;
+}
+
+fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, const int* cache_seqlens,
+                    void* workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                    fa_dtype dtype, fa_stream_t stream) {
+    return decode_common(q, k, v, o, lse, cache_seqlens, nullptr, workspace, B, Hq, Hkv, Nq, Nk, false, 0, 0, 0, d,
+                         scale, causal, dtype, stream);
+}
+
+fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o, float* lse,
+                          const int* cache_seqlens, const int* block_table, void* workspace, int B, int Hq, int Hkv,
+                          int Nq, int num_pages, int page_size, int max_pages, int d, float scale, int causal,
+                          fa_dtype dtype, fa_stream_t stream) {
+    return decode_common(q, k_pages, v_pages, o, lse, cache_seqlens, block_table, workspace, B, Hq, Hkv, Nq, 0, true,
+                         num_pages, page_size, max_pages, d, scale, causal, dtype, stream);
 }
 
 fa_status fa_get_last_device_error(fa_stream_t stream) {

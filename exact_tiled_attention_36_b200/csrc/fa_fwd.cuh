@@ -72,8 +72,6 @@ struct FwdArgs {
     int* err;
 };
 
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O once m grew by > 2^8
-constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
 struct FwdCfg {

@@ -377,4 +377,10 @@ __device__ __forceinline__ float unpack_hi(uint32_t u) {
     }
 }
 
+// Online softmax: rescale the partial output only once the row max has grown by
+// more than 2^8 since the last rescale (log2 units; exact, since O and the
+// normaliser share the reference max).
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.69314718055994530942f;
+
 }  // namespace fa

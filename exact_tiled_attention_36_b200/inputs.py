@@ -19,7 +19,12 @@ image or weight is used):
   with the key-padding path realised as unpad -> varlen (same page, the
   three execution paths of its FlashAttention wrapper);
 * a causal LLM prefill with grouped KV heads and a backward pass
-  ("FlashAttention/zh", sections on the algorithm and on recomputation).
+  ("FlashAttention/zh", sections on the algorithm and on recomputation);
+* LLM decode: one new query token per sequence against a long key/value cache,
+  the step that dominates text generation (the Gemma-3-12b-it generation
+  measurements on "Gemma-3-12b-it GPU利用率提升实测", which give no attention
+  shape, so the LLM prefill shape's heads are kept), optionally through the
+  paged KV cache of PagedAttention ("FlashAttention/zh", section "variants").
 """
 from __future__ import annotations
 
@@ -87,6 +92,32 @@ VARLEN_KEYPAD = VarlenConfig("varlen_keypad25_32seq_64to4096_h32_d128_fp16", num
                              causal=False, len_seed=3, seed=4, key_pad_frac=0.25)
 CAUSAL_GQA = FixedConfig("causal_gqa_b2_n8192_hq32_hkv8_d128", B=2, Hq=32, Hkv=8, Nq=8192,
                          Nk=8192, d=128, dtype="bf16", causal=True, seed=5, backward=True)
+
+
+@dataclass(frozen=True)
+class DecodeConfig:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int      # new query tokens per sequence
+    Nk: int      # cache capacity (keys) per sequence
+    d: int
+    dtype: str
+    causal: bool
+    seed: int
+    len_seed: int = -1  # >= 0: sequence lengths uniform in [min_len, Nk] from this seed; else all Nk
+    min_len: int = 1
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(self.d) ** 0.5
+
+
+DECODE = DecodeConfig("decode_b32_nk8192_hq32_hkv8_d128", B=32, Hq=32, Hkv=8, Nq=1, Nk=8192, d=128,
+                      dtype="bf16", causal=False, seed=6)
+DECODE_RAGGED = DecodeConfig("decode_ragged_b32_nk8192_hq32_hkv8_d128", B=32, Hq=32, Hkv=8, Nq=1, Nk=8192,
+                             d=128, dtype="bf16", causal=False, seed=6, len_seed=7)
 
 ALL_FIXED = (TINY, VISION, VIT_RMSNORM, CAUSAL_GQA)
 ALL_VARLEN = (VARLEN, VARLEN_KEYPAD)
@@ -200,3 +231,65 @@ def make_varlen(cfg: VarlenConfig, lengths: list[int] | None = None, with_do: bo
     return VarlenInputs(cfg, lengths, lk, cu_q, _cumsum(lk), max(lengths, default=0),
                         max(lk, default=0), q, k, v, kf, vf, do)
 
+
+
+@dataclass
+class DecodeInputs:
+    cfg: DecodeConfig
+    q: torch.Tensor        # [B, Nq, Hq, d]
+    k: torch.Tensor        # [B, Nk, Hkv, d]  contiguous caches; rows past a sequence's length hold NaN
+    v: torch.Tensor
+    seqlens: list[int] | None  # None: every sequence fills the cache
+    page_size: int = 0
+    k_pages: torch.Tensor | None = None  # [num_pages, page_size, Hkv, d]; unused rows NaN
+    v_pages: torch.Tensor | None = None
+    block_table: torch.Tensor | None = None  # int32 [B, max_pages]; unused entries -1
+
+
+def make_decode(cfg: DecodeConfig, lengths: list[int] | None = None, page_size: int = 0, spare_pages: int = 3,
+                **override) -> DecodeInputs:
+    """Draw a decode batch: Q, then the K and V caches (all rows drawn, in that
+    order), then the rows past each sequence's length are overwritten with NaN
+    (a cache slot not yet written may hold anything). Lengths: ``lengths``, else
+    uniform in [min_len, Nk] from ``len_seed``, else all Nk (``seqlens`` None).
+
+    With ``page_size`` the same caches are also laid out as page pools: the
+    pages of every sequence, plus ``spare_pages`` unused ones, are placed in a
+    random order (generator seed + 1) in pools filled with NaN, and block_table
+    row b lists the pages of sequence b in key order (-1 past its last page)."""
+    if override:
+        cfg = DecodeConfig(**{**cfg.__dict__, **override})
+    dt = DTYPES[cfg.dtype]
+    g = torch.Generator().manual_seed(cfg.seed)
+    q = _normal(g, (cfg.B, cfg.Nq, cfg.Hq, cfg.d)).to(dt)
+    k = _normal(g, (cfg.B, cfg.Nk, cfg.Hkv, cfg.d)).to(dt)
+    v = _normal(g, (cfg.B, cfg.Nk, cfg.Hkv, cfg.d)).to(dt)
+    if lengths is None and cfg.len_seed >= 0:
+        gl = torch.Generator().manual_seed(cfg.len_seed)
+        lengths = torch.randint(cfg.min_len, cfg.Nk + 1, (cfg.B,), generator=gl).tolist()
+    seqlens = None if lengths is None else [int(n) for n in lengths]
+    if seqlens is not None:
+        for b, n in enumerate(seqlens):
+            k[b, n:] = float("nan")
+            v[b, n:] = float("nan")
+    out = DecodeInputs(cfg, q, k, v, seqlens)
+    if page_size:
+        lens = seqlens if seqlens is not None else [cfg.Nk] * cfg.B
+        counts = [(n + page_size - 1) // page_size for n in lens]
+        max_pages = max(1, (cfg.Nk + page_size - 1) // page_size)
+        n_pages = sum(counts) + spare_pages
+        order = torch.randperm(n_pages, generator=torch.Generator().manual_seed(cfg.seed + 1)).tolist()
+        kp = torch.full((n_pages, page_size, cfg.Hkv, cfg.d), float("nan"), dtype=dt)
+        vp = torch.full_like(kp, float("nan"))
+        table = torch.full((cfg.B, max_pages), -1, dtype=torch.int32)
+        nxt = 0
+        for b, (n, c) in enumerate(zip(lens, counts)):
+            for i in range(c):
+                page = order[nxt]
+                nxt += 1
+                table[b, i] = page
+                rows = min(page_size, n - i * page_size)
+                kp[page, :rows] = k[b, i * page_size:i * page_size + rows]
+                vp[page, :rows] = v[b, i * page_size:i * page_size + rows]
+        out.page_size, out.k_pages, out.v_pages, out.block_table = page_size, kp, vp, table
+    return out

@@ -230,6 +230,54 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
                         fa_stream_t stream);
 
 /*
+ * Decode: attention of the Nq newest query tokens of each sequence against a
+ * long key/value cache (Nq = 1 for one generated token, a few for speculative
+ * decoding), by the same tiled online softmax as the forward ("FlashAttention/zh",
+ * section "FlashAttention algorithm"), with the keys split across the GPU:
+ * the key tiles of all (sequence, KV head) pairs are laid end to end and every
+ * CTA takes an equal share; each share leaves a partial output and its
+ * log-sum-exp, and a second kernel merges the shares of each pair with
+ * L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s (the online-softmax
+ * rescale applied to whole partial results; exact up to rounding). The query
+ * heads that share a KV head are one tile, so each K/V row is read from HBM
+ * once. The paged cache is the block-tiled KV cache of PagedAttention (named
+ * on "FlashAttention/zh", section "variants").
+ *   q [B,Nq,Hq,d] (dtype); o [B,Nq,Hq,d] (dtype), lse [B,Hq,Nq] (float32):
+ *       the layouts of fa_fwd.
+ *   fa_decode: k, v [B,Nk,Hkv,d], the caches (Nk = their capacity).
+ *   fa_decode_paged: k_pages, v_pages [num_pages,page_size,Hkv,d] page pools;
+ *       block_table DEVICE int32 [B,max_pages]: key position p of sequence b is
+ *       row p % page_size of page block_table[b*max_pages + p/page_size]. Entries
+ *       for positions past the sequence's length are not read; a page index
+ *       outside [0, num_pages) reads zeros. page_size must be 16, 32 or a
+ *       multiple of 64 (FA_ERR_UNSUPPORTED otherwise).
+ *   cache_seqlens: DEVICE int32 [B] or NULL (fa_decode only): sequence b uses
+ *       keys 0 .. cache_seqlens[b]-1, clamped to [0, capacity] (capacity = Nk,
+ *       or max_pages*page_size); NULL = every sequence uses all Nk keys. Rows
+ *       of the cache past a sequence's length may hold anything, NaN included.
+ *       Required (non-NULL) for fa_decode_paged.
+ *   causal: query token t of a sequence with n keys sees keys 0 .. t + n - Nq
+ *       (bottom-right alignment, as fa_fwd). A row that sees no key (n = 0, or
+ *       t + n - Nq < 0) gets O = 0 and lse = -inf.
+ *   workspace: device buffer of fa_decode_workspace_size(B,Hq,Hkv,Nq,d) bytes,
+ *       16-byte aligned, owned by the caller, for the partial results. The size
+ *       depends on the SM count of the CURRENT device: query it with the device
+ *       the call will run on current (0 when no device is visible).
+ *   (Hq / Hkv) * Nq must be at most 128 (FA_ERR_UNSUPPORTED otherwise; use
+ *   fa_fwd for longer query blocks). Every other argument, result and error
+ *   is that of fa_fwd; cache_seqlens and block_table must be 4-byte aligned.
+ */
+size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int d);
+fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cache_seqlens, void* workspace,
+                    int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                    float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o, float* lse,
+                          const int* cache_seqlens, const int* block_table, void* workspace,
+                          int B, int Hq, int Hkv, int Nq, int num_pages, int page_size, int max_pages, int d,
+                          float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Backward without a caller-provided workspace. This entry point has no
  * counterpart in the pages; it exists for callers that cannot allocate
  * device memory themselves (a host framework that owns every allocation,

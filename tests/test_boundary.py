@@ -201,3 +201,52 @@ def test_qk_rmsnorm_rejects_bad_eps(lib, eps, code):
     assert fb.fa_fwd_qk_rmsnorm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, 1, 1, 1, 8, 8, 64, 0.1, 0, 1e-6,
                                 fb.FA_BF16, None) == fb.FA_ERR_MISALIGNED
     assert fb.fa_fwd_qk_rmsnorm_workspace_size(2, 100, 3, 128) == (2 * 100 * 3 * 128 * 2 + 255) // 256 * 256
+
+
+def dec(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, sl=None, ws=FAKE, B=2, Hq=8, Hkv=2, Nq=1, Nk=64, d=128,
+             scale=0.1, causal=0, dtype=fb.FA_BF16, stream=None)
+    a.update(kw)
+    return fb.fa_decode(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), fb.FA_ERR_INVALID_ARG),
+    (dict(Hq=5), fb.FA_ERR_INVALID_ARG),
+    (dict(causal=2), fb.FA_ERR_INVALID_ARG),
+    (dict(Nk=-1), fb.FA_ERR_INVALID_ARG),
+    (dict(d=96), fb.FA_ERR_UNSUPPORTED),
+    (dict(Nq=64), fb.FA_ERR_UNSUPPORTED),  # 4 heads x 64 tokens > one 128-row tile
+    (dict(o=FAKE + 8), fb.FA_ERR_MISALIGNED),
+    (dict(sl=FAKE + 2), fb.FA_ERR_MISALIGNED),
+    (dict(Nq=0), fb.FA_OK),
+])
+def test_decode_rejects_before_launch(lib, kw, code):
+    assert dec(**kw) == code
+
+
+def dec_paged(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, sl=FAKE, bt=FAKE, ws=FAKE, B=2, Hq=8, Hkv=2, Nq=1,
+             num_pages=10, page_size=64, max_pages=4, d=128, scale=0.1, causal=1, dtype=fb.FA_BF16, stream=None)
+    a.update(kw)
+    return fb.fa_decode_paged(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(sl=None), fb.FA_ERR_INVALID_ARG),
+    (dict(bt=None), fb.FA_ERR_INVALID_ARG),
+    (dict(num_pages=0), fb.FA_ERR_INVALID_ARG),
+    (dict(page_size=8), fb.FA_ERR_INVALID_ARG),
+    (dict(page_size=48), fb.FA_ERR_UNSUPPORTED),
+    (dict(bt=FAKE + 1), fb.FA_ERR_MISALIGNED),
+    (dict(Nq=0), fb.FA_OK),
+    (dict(Nq=0, page_size=16), fb.FA_OK),
+    (dict(Nq=0, page_size=192), fb.FA_OK),
+])
+def test_decode_paged_rejects_before_launch(lib, kw, code):
+    assert dec_paged(**kw) == code
+
+
+def test_decode_workspace_size_invalid(lib):
+    for args in ((2, 8, 2, 1, 96), (2, 5, 2, 1, 128), (2, 8, 2, 33, 128), (0, 8, 2, 1, 128)):
+        assert fb.fa_decode_workspace_size(*args) == 0
