@@ -43,8 +43,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 // box_h heads x 64 columns, 128-byte swizzle. Rows past `rows` read as zero.
 // 4-D map (d, H, rows, batches) over a tensor whose head, token and batch strides
 // are sh, ss, sb elements (d contiguous); each stride must be a multiple of 16 bytes.
+// `promote_256`: L2 promotion of each request to 256 bytes (else 128). A row of one
+// head is 2 d bytes: with d = 64 the wider promotion also fetches the next head's row.
 fa_status make_map_box(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16,
-                       int64_t sh, int64_t ss, int64_t sb, int box_h, int box_rows) {
+                       int64_t sh, int64_t ss, int64_t sb, int box_h, int box_rows, bool promote_256 = true) {
     auto enc = encode_tiled();
     if (!enc) return FA_ERR_CUDA;
     if (rows < 1) rows = 1;
@@ -57,7 +59,8 @@ fa_status make_map_box(CUtensorMap* m, const void* base, int d, int H, int64_t r
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_SWIZZLE_128B,
+                     promote_256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
@@ -522,34 +525,77 @@ bool dec_ws(int B, int Hq, int Hkv, int Nq, int d, DecWs& w) {
     if (G <= 0) return false;
     const size_t items = static_cast<size_t>(B) * Hkv;
     const size_t slots = items + G;
+    // d = 64 may pair KV heads: half the items with twice the rows (bounded by this).
+    const size_t rows = d == 64 ? 2 * R : R;
     w.meta = round256((1 + items) * sizeof(long long));
-    w.lse = round256(slots * R * sizeof(float));
-    w.total = w.meta + w.lse + round256(slots * R * d * sizeof(float));
+    w.lse = round256(slots * rows * sizeof(float));
+    w.total = w.meta + w.lse + round256(slots * rows * d * sizeof(float));
     return true;
 }
 
-template <int D, bool BF16, bool SEQLENS, bool PAGED>
+// RN = 0: the row-per-lane kernel (any R <= 128); RN = 16 or 32: the narrow kernel
+// with the products' operands swapped (R <= RN).
+// PAIR (d = 64, narrow only): the split kernel runs as d = 128 over pairs of KV heads;
+// the merge writes d = 64.
+template <int D, bool BF16, bool SEQLENS, bool PAGED, int RN, bool PAIR = false>
 fa_status launch_dec_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecodeArgs& a,
                        int causal, bool run_split, cudaStream_t s) {
+    static_assert(!PAIR || (D == 64 && RN != 0), "paired KV heads: d = 64, narrow kernel");
+    constexpr int DK = PAIR ? 128 : D;
     if (run_split) {
-        auto kern = fa::fa_decode_kernel<D, BF16, SEQLENS, PAGED>;
-        constexpr int smem = fa::DecCfg<D>::kSmemBytes;
-        static bool attr_ok =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-        if (!attr_ok) return FA_ERR_CUDA;
-        kern<<<a.G, fa::kDecThreads, smem, s>>>(mq, mk, mv, a, causal);
+        if constexpr (RN == 0) {
+            auto kern = fa::fa_decode_kernel<D, BF16, SEQLENS, PAGED>;
+            constexpr int smem = fa::DecCfg<D>::kSmemBytes;
+            static bool attr_ok =
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+            if (!attr_ok) return FA_ERR_CUDA;
+            kern<<<a.G, fa::kDecThreads, smem, s>>>(mq, mk, mv, a, causal);
+        } else {
+            auto kern = fa::fa_decode_narrow_kernel<DK, BF16, SEQLENS, PAGED, RN>;
+            constexpr int smem = fa::DecNarrowCfg<DK, RN>::kSmemBytes;
+            static bool attr_ok =
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+            if (!attr_ok) return FA_ERR_CUDA;
+            kern<<<a.G, fa::kDecThreads, smem, s>>>(mq, mk, mv, a, causal);
+        }
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
-    fa::fa_decode_combine<D, BF16, SEQLENS><<<static_cast<unsigned>(a.B) * a.Hkv, 128, 0, s>>>(a);
+    // The merge launches as a programmatic dependent of the split kernel, so its
+    // launch overlaps the split kernel's tail; it waits for the split kernel's
+    // results in the kernel (griddepcontrol.wait).
+    const long long rows = static_cast<long long>(a.B) * a.Hkv * a.R;  // one block per (item, row)
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(rows));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = run_split ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, fa::fa_decode_combine<D, BF16, SEQLENS>, a) != cudaSuccess) return FA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
-fa_status launch_dec_b(bool seqlens, bool paged, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+template <int D, bool BF16, int RN, bool PAIR>
+fa_status launch_dec_r(bool seqlens, bool paged, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const fa::DecodeArgs& a, int causal, bool run_split, cudaStream_t s) {
-    if (paged) return launch_dec_t<D, BF16, true, true>(mq, mk, mv, a, causal, run_split, s);
-    if (seqlens) return launch_dec_t<D, BF16, true, false>(mq, mk, mv, a, causal, run_split, s);
-    return launch_dec_t<D, BF16, false, false>(mq, mk, mv, a, causal, run_split, s);
+    if (paged) return launch_dec_t<D, BF16, true, true, RN, PAIR>(mq, mk, mv, a, causal, run_split, s);
+    if (seqlens) return launch_dec_t<D, BF16, true, false, RN, PAIR>(mq, mk, mv, a, causal, run_split, s);
+    return launch_dec_t<D, BF16, false, false, RN, PAIR>(mq, mk, mv, a, causal, run_split, s);
+}
+
+template <int D, bool BF16>
+fa_status launch_dec_b(int rn, bool pair, bool seqlens, bool paged, const CUtensorMap& mq, const CUtensorMap& mk,
+                       const CUtensorMap& mv, const fa::DecodeArgs& a, int causal, bool run_split, cudaStream_t s) {
+    if constexpr (D == 64) {
+        if (pair) return rn == 16 ? launch_dec_r<64, BF16, 16, true>(seqlens, paged, mq, mk, mv, a, causal, run_split, s)
+                                  : launch_dec_r<64, BF16, 32, true>(seqlens, paged, mq, mk, mv, a, causal, run_split, s);
+    }
+    if (rn == 16) return launch_dec_r<D, BF16, 16, false>(seqlens, paged, mq, mk, mv, a, causal, run_split, s);
+    if (rn == 32) return launch_dec_r<D, BF16, 32, false>(seqlens, paged, mq, mk, mv, a, causal, run_split, s);
+    return launch_dec_r<D, BF16, 0, false>(seqlens, paged, mq, mk, mv, a, causal, run_split, s);
 }
 
 // fa_decode (paged = false: k, v [B, Nk, Hkv, d]) and fa_decode_paged (k, v page
@@ -578,29 +624,43 @@ fa_status decode_common(const void* q, const void* k, const void* v, void* o, fl
     if (static_cast<long long>(g) * Nq > 128) return FA_ERR_UNSUPPORTED;  // one tile holds a group's queries
     const long long items = static_cast<long long>(B) * Hkv;
     const long long max_tiles = items * ((static_cast<long long>(cap) + 127) / 128);
-    if (items > 0x7fffffffLL || max_tiles > (1LL << 40) || B > 65535 || Nq > 65535) return FA_ERR_UNSUPPORTED;
+    if (items * g * Nq > 0x7fffffffLL || max_tiles > (1LL << 40) || B > 65535 || Nq > 65535)
+        return FA_ERR_UNSUPPORTED;
     if (Nq == 0) return FA_OK;
     int* err = error_word();
     if (!err) return FA_ERR_CUDA;
     DecWs w;
     if (!dec_ws(B, Hq, Hkv, Nq, d, w)) return FA_ERR_CUDA;
     const bool bf16 = dtype == FA_BF16;
-    int nb, gh;
-    dec_layout(g, Nq, nb, gh);
+    // Up to 32 rows: the narrow kernel (one box of all g heads x Nq tokens); more:
+    // the row-per-lane kernel with its lane layout.
+    const int R = g * Nq;
+    // d = 64, even Hkv, R <= 16: pairs of KV heads (256-byte K/V rows), 2 roundup8(R)
+    // tile rows.
+    const bool pair = d == 64 && Hkv % 2 == 0 && R <= 16;
+    const int r8 = (R + 7) / 8 * 8;
+    const int rows = pair ? 2 * r8 : R;
+    const int rn = rows <= 16 ? 16 : (rows <= 32 ? 32 : 0);
+    int nb = 1, gh = g;
+    if (rn == 0) dec_layout(g, Nq, nb, gh);
     CUtensorMap mq, mk{}, mv{};
     const long long hd = static_cast<long long>(Hq) * d;
     if ((st = make_map_box(&mq, q, d, Hq, Nq, B, bf16, d, hd, hd * Nq, gh, Nq)) != FA_OK) return st;
     const int page_box = page_size < 64 ? page_size : 64;
     if (cap > 0) {
         const long long kd = static_cast<long long>(Hkv) * d;
+        // Paired heads: the caches seen as Hkv / 2 heads of 128 values (the same memory).
+        const int md = pair ? 128 : d, mh = pair ? Hkv / 2 : Hkv;
+        // Each K/V row of a head is read once: the L2 request stays at one head's row.
+        const bool p256 = md == 128;
         if (paged) {
-            if ((st = make_map_box(&mk, k, d, Hkv, page_size, num_pages, bf16, d, kd, kd * page_size, 1, page_box)) !=
-                    FA_OK ||
-                (st = make_map_box(&mv, v, d, Hkv, page_size, num_pages, bf16, d, kd, kd * page_size, 1, page_box)) !=
-                    FA_OK)
+            if ((st = make_map_box(&mk, k, md, mh, page_size, num_pages, bf16, md, kd, kd * page_size, 1, page_box,
+                                   p256)) != FA_OK ||
+                (st = make_map_box(&mv, v, md, mh, page_size, num_pages, bf16, md, kd, kd * page_size, 1, page_box,
+                                   p256)) != FA_OK)
                 return st;
-        } else if ((st = make_map(&mk, k, d, Hkv, Nk, B, bf16)) != FA_OK ||
-                   (st = make_map(&mv, v, d, Hkv, Nk, B, bf16)) != FA_OK) {
+        } else if ((st = make_map_box(&mk, k, md, mh, Nk, B, bf16, md, kd, kd * Nk, 1, 128, p256)) != FA_OK ||
+                   (st = make_map_box(&mv, v, md, mh, Nk, B, bf16, md, kd, kd * Nk, 1, 128, p256)) != FA_OK) {
             return st;
         }
     }
@@ -614,11 +674,14 @@ fa_status decode_common(const void* q, const void* k, const void* v, void* o, fl
     a.block_table = block_table;
     a.B = B;
     a.Hq = Hq;
-    a.Hkv = Hkv;
+    a.Hkv = pair ? Hkv / 2 : Hkv;  // items per sequence
     a.group = g;
     a.Nq = Nq;
     a.Nk = paged ? cap : Nk;
-    a.R = g * Nq;
+    a.R = pair ? 2 * R : R;  // rows per item
+    a.pair = pair ? 1 : 0;
+    a.rg = R;
+    a.r8 = pair ? r8 : 0;
     a.cap = cap;
     a.page_size = page_size;
     a.max_pages = max_pages;
@@ -630,15 +693,16 @@ fa_status decode_common(const void* q, const void* k, const void* v, void* o, fl
     // Fixed lengths: exactly T tiles; with lengths, at most T tiles (each CTA finds
     // its share of the true T itself).
     const int sms = dec_max_ctas();
-    a.G = static_cast<int>(max_tiles < sms ? max_tiles : sms);
+    const long long item_tiles = pair ? max_tiles / 2 : max_tiles;  // paired items hold two heads' tiles
+    a.G = static_cast<int>(item_tiles < sms ? item_tiles : sms);
     const bool run_split = max_tiles > 0;
     if (a.G < 1) a.G = 1;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool sl = seqlens != nullptr;
-    if (d == 64) return bf16 ? launch_dec_b<64, true>(sl, paged, mq, mk, mv, a, causal, run_split, s)
-                             : launch_dec_b<64, false>(sl, paged, mq, mk, mv, a, causal, run_split, s);
-    return bf16 ? launch_dec_b<128, true>(sl, paged, mq, mk, mv, a, causal, run_split, s)
-                : launch_dec_b<128, false>(sl, paged, mq, mk, mv, a, causal, run_split, s);
+    if (d == 64) return bf16 ? launch_dec_b<64, true>(rn, pair, sl, paged, mq, mk, mv, a, causal, run_split, s)
+                             : launch_dec_b<64, false>(rn, pair, sl, paged, mq, mk, mv, a, causal, run_split, s);
+    return bf16 ? launch_dec_b<128, true>(rn, false, sl, paged, mq, mk, mv, a, causal, run_split, s)
+                : launch_dec_b<128, false>(rn, false, sl, paged, mq, mk, mv, a, causal, run_split, s);
 }
 
 }  // namespace

@@ -56,6 +56,8 @@ struct DecodeArgs {
     int cap;               // keys a sequence can hold (Nk, or max_pages * page_size)
     int page_size, max_pages, page_box;  // paged: rows per page, pages per sequence, rows per TMA box
     int nb, gh;            // row layout: head blocks and heads per block
+    int pair, rg, r8;      // narrow, d = 64: items are pairs of KV heads (see fa_decode_narrow_kernel);
+                           // rg rows per KV head, the second head's rows from tile row r8
     int G;                 // CTAs of the split kernel
     float scale_log2;
     int* err;
@@ -135,38 +137,30 @@ __device__ __forceinline__ int dec_cta_of(long long t, long long T, int G) {
 
 __device__ __forceinline__ long long dec_split(int c, long long T, int G) { return (static_cast<long long>(c) * T) / G; }
 
-// PAGED: k and v are page pools [num_pages, page_size, Hkv, d] addressed through
-// block_table (requires SEQLENS). SEQLENS: sequence b has seqlens[b] keys (clamped
-// to [0, cap]); else every sequence has Nk. causal (runtime): query t of a
-// sequence of n keys sees keys 0 .. t + n - Nq (bottom-right alignment).
-template <int D, bool BF16, bool SEQLENS, bool PAGED>
-__global__ void __launch_bounds__(kDecThreads, 1)
-    fa_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const DecodeArgs args, const int causal) {
-    static_assert(SEQLENS || !PAGED, "a paged cache needs the sequence lengths");
-    using C = DecCfg<D>;
-    constexpr int S = C::kStages;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    if (!smem_base_ok(smem, args.err)) return;
+
+// The CTA's tile range [s_lo, s_hi) of the T tiles and the item holding s_lo.
+struct DecRange {
+    long long T, s_lo, s_hi;
+    DecItem first;
+};
+
+// Called by every thread of the CTA (it synchronises the CTA when sequence lengths
+// are given: every CTA then sums the per-sequence tile counts itself, a block
+// reduction, and finds the sequence holding its first tile, a block scan). Returns
+// false, for every thread, when the CTA has no tile. Uses 112 bytes at `misc + 8`.
+template <bool SEQLENS>
+__device__ __forceinline__ bool dec_locate(const DecodeArgs& args, uint8_t* misc, DecRange& rg) {
     const int G = args.G;
     const int cta = static_cast<int>(blockIdx.x);
     const int tid = static_cast<int>(threadIdx.x);
     const int warp = warp_id();
     const int lane = lane_id();
-    uint8_t* misc = smem + C::kMiscOff;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc);
-    int* abort_flag = reinterpret_cast<int*>(misc + 4);
-
-    // ---------------------------------------------------------------- the CTA's tiles
-    // T and the item holding the CTA's first tile. With sequence lengths every CTA
-    // sums the per-sequence tile counts itself (a block reduction, then a block scan
-    // that stops at the sequence holding that tile).
+    constexpr int kWarps = kDecThreads / 32;
     long long T, s_lo, s_hi;
     int b0;
     long long P0;  // first tile of sequence b0 (its KV head 0)
     if constexpr (SEQLENS) {
         int* found = reinterpret_cast<int*>(misc + 8);
-        long long* sh_T = reinterpret_cast<long long*>(misc + 16);
         int* sh_b0 = reinterpret_cast<int*>(misc + 24);
         long long* sh_P0 = reinterpret_cast<long long*>(misc + 32);
         long long* ws = reinterpret_cast<long long*>(misc + 48);  // [8] per-warp sums
@@ -182,12 +176,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         __syncthreads();
         T = 0;
 #pragma unroll
-        for (int w = 0; w < kDecThreads / 32; ++w) T += ws[w];
+        for (int w = 0; w < kWarps; ++w) T += ws[w];
         if (cta == 0 && tid == 0) args.meta[0] = T;
         s_lo = dec_split(cta, T, G);
         s_hi = dec_split(cta + 1, T, G);
-        if (s_lo >= s_hi) return;  // no tile for this CTA (fewer tiles than CTAs)
-        __syncthreads();           // every thread has read ws
+        if (s_lo >= s_hi) return false;  // fewer tiles than CTAs (uniform)
+        __syncthreads();                 // every thread has read ws
         long long run = 0;
         for (int base = 0; base < args.B; base += kDecThreads) {
             const int b = base + tid;
@@ -202,13 +196,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             __syncthreads();
             long long before = 0, total = 0;
 #pragma unroll
-            for (int w = 0; w < kDecThreads / 32; ++w) {
+            for (int w = 0; w < kWarps; ++w) {
                 const long long y = ws[w];
                 if (w < warp) before += y;
                 total += y;
             }
             const long long excl = run + before + incl - x;
-            if (x > 0 && excl <= s_lo && s_lo < excl + x) {
+            if (x > 0 && excl <= s_lo && s_lo < excl + x) {  // one thread at most
                 *sh_b0 = b;
                 *sh_P0 = excl;
                 *found = 1;
@@ -217,25 +211,150 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             if (*found) break;
             run += total;
         }
-        if (!*found) return;  // cannot happen: s_lo < T
+        if (!*found) return false;  // cannot happen: s_lo < T
         b0 = *sh_b0;
         P0 = *sh_P0;
-        (void)sh_T;
     } else {
         const long long per_b = static_cast<long long>(args.Hkv) * ((args.Nk + 127) / 128);
         T = per_b * args.B;
         s_lo = dec_split(cta, T, G);
         s_hi = dec_split(cta + 1, T, G);
-        if (s_lo >= s_hi) return;
+        if (s_lo >= s_hi) return false;
         b0 = static_cast<int>(s_lo / per_b);
         P0 = b0 * per_b;
     }
-    // The item holding tile s_lo; every role walks the items from here.
-    const DecItem first = [&] {
-        const int ntk = (dec_len<SEQLENS>(args, b0) + 127) / 128;
-        const int hk = static_cast<int>((s_lo - P0) / ntk);
-        return dec_item<SEQLENS>(args, b0, hk, P0 + static_cast<long long>(hk) * ntk);
-    }();
+    const int ntk = (dec_len<SEQLENS>(args, b0) + 127) / 128;
+    const int hk = static_cast<int>((s_lo - P0) / ntk);
+    rg.T = T;
+    rg.s_lo = s_lo;
+    rg.s_hi = s_hi;
+    rg.first = dec_item<SEQLENS>(args, b0, hk, P0 + static_cast<long long>(hk) * ntk);
+    return true;
+}
+
+// The TMA producer (one thread): per segment the group's query rows (nb boxes of
+// gh heads x Nq tokens, box k at q_block_off * k within each 64-column slab of
+// q_slab_bytes), then every K and V tile of the segment through the S-stage rings.
+// K and V tiles are 128 keys x d (16-bit), 64-column slabs of 16 KB.
+template <int D, bool SEQLENS, bool PAGED, int S>
+__device__ __forceinline__ void dec_produce(const DecodeArgs& args, const DecRange& rg, const CUtensorMap* tm_q,
+                                            const CUtensorMap* tm_k, const CUtensorMap* tm_v, uint8_t* sQ,
+                                            int q_slab_bytes, int q_block_off, uint8_t* sK, uint8_t* sV,
+                                            uint64_t* q_full, uint64_t* q_empty, uint64_t* k_full, uint64_t* k_empty,
+                                            uint64_t* v_full, uint64_t* v_empty, const WaitCtx& wc) {
+    constexpr int kSlabs = D / 64;
+    constexpr int kSlabBytes = 128 * 128;
+    constexpr int kTileBytes = kSlabs * kSlabBytes;
+    const int g = args.group;
+    int gk = 0, nq = 0, k_issued = 0, v_issued = 0;
+    bool ok = true;
+    // Paged: the pages of one key tile (boxes of page_box rows; one page holds whole
+    // boxes), read from the block table once per tile for both K and V, all reads in
+    // flight together. Boxes past the sequence's end are not loaded (their rows are
+    // masked, and zeroed in V).
+    constexpr int kMaxBoxes = 8;  // 128 keys / 16-row pages
+    int pages[kMaxBoxes];
+    int boxes = 0;
+    auto read_pages = [&](const DecItem& it, int kt) {
+        if constexpr (PAGED) {
+            const int pb = args.page_box;
+            boxes = (min(128, it.len - kt * 128) + pb - 1) / pb;
+            const int* bt = args.block_table + static_cast<size_t>(it.b) * args.max_pages;
+#pragma unroll
+            for (int x = 0; x < kMaxBoxes; ++x)
+                pages[x] = x < boxes ? bt[(kt * 128 + x * pb) / args.page_size] : 0;
+        }
+    };
+    // One K or V tile (key tile kt of item `it`) into ring buffer `dst`.
+    auto load_kv = [&](uint8_t* dst, const CUtensorMap* m, uint64_t* bar, const DecItem& it, int kt) {
+        if constexpr (!PAGED) {
+            mbar_arrive_expect_tx(bar, kTileBytes);
+#pragma unroll
+            for (int s = 0; s < kSlabs; ++s) tma_load_4d(dst + s * kSlabBytes, m, bar, s * 64, it.hk, kt * 128, it.b);
+        } else {
+            const int pb = args.page_box;
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(boxes * pb * 128 * kSlabs));
+#pragma unroll
+            for (int x = 0; x < kMaxBoxes; ++x) {
+                if (x >= boxes) break;
+                const int key = kt * 128 + x * pb;
+#pragma unroll
+                for (int s = 0; s < kSlabs; ++s)
+                    tma_load_4d(dst + s * kSlabBytes + x * pb * 128, m, bar, s * 64, it.hk, key % args.page_size,
+                                pages[x]);
+            }
+        }
+    };
+    for (DecItem it = rg.first; ok && it.P < rg.s_hi; it = dec_next<SEQLENS>(args, it, rg.T)) {
+        const long long lo = max(rg.s_lo, it.P), hi = min(rg.s_hi, it.P + it.ntk);
+        if (lo >= hi) continue;
+        const int j0 = static_cast<int>(lo - it.P), n = static_cast<int>(hi - lo);
+        if (SEQLENS && lo == it.P) args.meta[1 + static_cast<size_t>(it.b) * args.Hkv + it.hk] = it.P;
+        // Q of the group once the previous segment's last S product has read Q.
+        if (!(ok = mbar_wait(q_empty, (nq & 1) ^ 1u, wc, 80))) break;
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(args.pair ? 2 * 128 * args.rg : kSlabs * 128 * args.R));
+        if (args.pair) {
+            // KV heads 2 hk and 2 hk + 1 (64 columns each): the first group's rows in
+            // columns 0..63 from row 0, the second's in columns 64..127 from row r8.
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                tma_load_4d(sQ + k * q_slab_bytes + k * args.r8 * 128, tm_q, q_full, 0, (2 * it.hk + k) * g, 0, it.b);
+        } else {
+            for (int k = 0; k < args.nb; ++k)
+#pragma unroll
+                for (int s = 0; s < kSlabs; ++s)
+                    tma_load_4d(sQ + s * q_slab_bytes + k * q_block_off, tm_q, q_full, s * 64, it.hk * g + k * args.gh,
+                                0, it.b);
+        }
+        ++nq;
+        for (int j = 0; j < n; ++j) {
+            const int gg = gk + j, st = gg % S;
+            const uint32_t ph = (gg / S) & 1;
+            read_pages(it, j0 + j);
+            if (!(ok = mbar_wait(&k_empty[st], ph ^ 1u, wc, 81))) break;
+            load_kv(sK + st * kTileBytes, tm_k, &k_full[st], it, j0 + j);
+            ++k_issued;
+            if (!(ok = mbar_wait(&v_empty[st], ph ^ 1u, wc, 82))) break;
+            load_kv(sV + st * kTileBytes, tm_v, &v_full[st], it, j0 + j);
+            ++v_issued;
+        }
+        gk += n;
+    }
+    // Leave no load in flight: wait for the last one issued into every buffer.
+    if (nq > 0) mbar_wait_drain(q_full, (nq - 1) & 1);
+    for (int st = 0; st < S; ++st) {
+        if (k_issued > st) mbar_wait_drain(&k_full[st], ((st + S * ((k_issued - 1 - st) / S)) / S) & 1);
+        if (v_issued > st) mbar_wait_drain(&v_full[st], ((st + S * ((v_issued - 1 - st) / S)) / S) & 1);
+    }
+}
+
+// PAGED: k and v are page pools [num_pages, page_size, Hkv, d] addressed through
+// block_table (requires SEQLENS). SEQLENS: sequence b has seqlens[b] keys (clamped
+// to [0, cap]); else every sequence has Nk. causal (runtime): query t of a
+// sequence of n keys sees keys 0 .. t + n - Nq (bottom-right alignment).
+template <int D, bool BF16, bool SEQLENS, bool PAGED>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    fa_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const DecodeArgs args, const int causal) {
+    static_assert(SEQLENS || !PAGED, "a paged cache needs the sequence lengths");
+    using C = DecCfg<D>;
+    constexpr int S = C::kStages;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (!smem_base_ok(smem, args.err)) return;
+    // The merge kernel may be scheduled now; it waits for this grid before reading.
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int cta = static_cast<int>(blockIdx.x);
+    const int tid = static_cast<int>(threadIdx.x);
+    const int warp = warp_id();
+    const int lane = lane_id();
+    uint8_t* misc = smem + C::kMiscOff;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc);
+    int* abort_flag = reinterpret_cast<int*>(misc + 4);
+
+    DecRange rg;
+    if (!dec_locate<SEQLENS>(args, misc, rg)) return;  // no tile for this CTA
+    const long long T = rg.T, s_lo = rg.s_lo, s_hi = rg.s_hi;
+    const DecItem first = rg.first;
 
     uint8_t* sQ = smem + C::kQOff;
     uint8_t* sK = smem + C::kKOff;
@@ -301,68 +420,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int g = args.group;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            constexpr uint32_t kQBytesPerRow = C::kSlabs * 128;
-            int gk = 0, nq = 0, k_issued = 0, v_issued = 0;
-            bool ok = true;
-            // One K or V tile (key tile kt of item `it`) into ring buffer `dst`.
-            auto load_kv = [&](uint8_t* dst, const CUtensorMap* m, uint64_t* bar, const DecItem& it, int kt) {
-                if constexpr (!PAGED) {
-                    mbar_arrive_expect_tx(bar, C::kTileBytes);
-#pragma unroll
-                    for (int s = 0; s < C::kSlabs; ++s)
-                        tma_load_4d(dst + s * C::kSlabBytes, m, bar, s * 64, it.hk, kt * 128, it.b);
-                } else {
-                    // Boxes of page_box rows (one page holds whole boxes); boxes past the
-                    // sequence's end are not loaded (their rows are masked and zeroed).
-                    const int pb = args.page_box;
-                    const int keys = min(128, it.len - kt * 128);
-                    const int boxes = (keys + pb - 1) / pb;
-                    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(boxes * pb * 128 * C::kSlabs));
-                    const int* bt = args.block_table + static_cast<size_t>(it.b) * args.max_pages;
-                    for (int x = 0; x < boxes; ++x) {
-                        const int key = kt * 128 + x * pb;
-                        const int page = bt[key / args.page_size];
-#pragma unroll
-                        for (int s = 0; s < C::kSlabs; ++s)
-                            tma_load_4d(dst + s * C::kSlabBytes + x * pb * 128, m, bar, s * 64, it.hk,
-                                        key % args.page_size, page);
-                    }
-                }
-            };
-            for (DecItem it = first; ok && it.P < s_hi; it = dec_next<SEQLENS>(args, it, T)) {
-                const long long lo = max(s_lo, it.P), hi = min(s_hi, it.P + it.ntk);
-                if (lo >= hi) continue;
-                const int j0 = static_cast<int>(lo - it.P), n = static_cast<int>(hi - lo);
-                if (SEQLENS && lo == it.P) args.meta[1 + static_cast<size_t>(it.b) * args.Hkv + it.hk] = it.P;
-                // Q of the group once the previous segment's last S product has read Q.
-                if (!(ok = mbar_wait(q_empty, (nq & 1) ^ 1u, wc, 80))) break;
-                mbar_arrive_expect_tx(q_full, kQBytesPerRow * args.R);
-                for (int k = 0; k < args.nb; ++k)
-#pragma unroll
-                    for (int s = 0; s < C::kSlabs; ++s)
-                        tma_load_4d(sQ + s * C::kSlabBytes + (args.nb > 1 ? k * 4096 : 0), &tm_q, q_full, s * 64,
-                                    it.hk * g + k * args.gh, 0, it.b);
-                ++nq;
-                for (int j = 0; j < n; ++j) {
-                    const int gg = gk + j, st = gg % S;
-                    const uint32_t ph = (gg / S) & 1;
-                    if (!(ok = mbar_wait(&k_empty[st], ph ^ 1u, wc, 81))) break;
-                    load_kv(sK + st * C::kTileBytes, &tm_k, &k_full[st], it, j0 + j);
-                    ++k_issued;
-                    if (!(ok = mbar_wait(&v_empty[st], ph ^ 1u, wc, 82))) break;
-                    load_kv(sV + st * C::kTileBytes, &tm_v, &v_full[st], it, j0 + j);
-                    ++v_issued;
-                }
-                gk += n;
-            }
-            if (nq > 0) mbar_wait_drain(q_full, (nq - 1) & 1);
-            for (int st = 0; st < S; ++st) {
-                if (k_issued > st) mbar_wait_drain(&k_full[st], ((st + S * ((k_issued - 1 - st) / S)) / S) & 1);
-                if (v_issued > st) mbar_wait_drain(&v_full[st], ((st + S * ((v_issued - 1 - st) / S)) / S) & 1);
-            }
-        }
+        if (lane == 0)
+            dec_produce<D, SEQLENS, PAGED, S>(args, rg, &tm_q, &tm_k, &tm_v, sQ, C::kSlabBytes,
+                                              args.nb > 1 ? 4096 : 0, sK, sV, q_full, q_empty, k_full, k_empty,
+                                              v_full, v_empty, wc);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -589,67 +650,536 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
 }
 
-// Merge of the segments of one item per CTA: for each of its R rows,
-// L = log sum_s exp(L_s) and O = sum_s exp(L_s - L) O_s over the CTAs whose tile
-// range meets the item, written to o [B, Nq, Hq, d] and lse [B, Hq, Nq]. An item
-// without keys, or a row that sees none, gets O = 0 and L = -inf.
+// ------------------------------------------------------------------------ narrow
+// The narrow kernel, for R = (Hq / Hkv) * Nq <= 32 rows (one generated token with
+// up to 32 query heads per KV head, or a few speculative tokens): the products are
+// taken with the operands swapped, so that keys, not query rows, run along the 128
+// TMEM lanes and the tensor core's M = 128:
+//     S^T = K Q^T       (M = 128 keys, N = RN >= R query rows, K = d)
+//     O^T += V^T P^T    (M = d, N = RN, K = 128 keys)
+// Thread l of the softmax warpgroup owns key l of the tile and takes R
+// exponentials per tile (not 128), so the kernel streams K and V at the memory's
+// pace. All threads use one reference max per row: a tile that raises some row's
+// max by more than 2^8 over the reference (or the segment's first tile) takes the
+// cross-warp reduction, sets the reference to the exact max and rescales the
+// normalisers and O^T; other tiles need one vote and one meeting of the four warps.
+// P goes through shared memory as the [RN x 128] (keys contiguous) B operand of the
+// second product.
+// d = 64 with an even number of KV heads and at most 16 rows per head (`pair`):
+// an item is two adjacent KV heads, whose K and V rows form one contiguous 256-byte
+// row (a 128-byte row per head would halve what HBM delivers), and the kernel runs
+// as d = 128 with a block-diagonal Q: the first head's query rows hold their 64
+// values in columns 0..63 (zeros in 64..127), the second head's rows, from tile
+// row r8, in columns 64..127. Then S^T holds each row's scores against its own
+// head, and O^T lanes 64 k .. 64 k + 63 hold head k's outputs. Other d = 64 cases
+// keep M = 128 in the second product: its A operand's second 64 rows read the next
+// 16 KB of shared memory (V stages come before K stages, so that stays inside the
+// buffer) and land in TMEM lanes 64..127, which nothing reads.
+// TMEM: S^T_b at [32 b, 32 b + RN) for the kNS buffers, then O^T (lane = d index).
+template <int D, int RN>
+struct DecNarrowCfg {
+    static constexpr int kSlabs = D / 64;
+    static constexpr int kKVSlab = 128 * 128;             // 128 keys x 64 columns
+    static constexpr int kTileBytes = kSlabs * kKVSlab;
+    // S^T buffers (and P buffers): the MMA thread issues S^T of tile j + kNS right
+    // after P V of tile j, so the softmax has kNS tiles of slack over the products'
+    // latency (which, not the exponentials, bounds a short tile).
+    static constexpr int kNS = (D == 128) ? 3 : 4;
+    static constexpr int kStages = (D == 128) ? 3 : (RN == 16 ? 6 : 5);
+    static constexpr int kQSlab = RN * 128;               // RN rows x 64 columns
+    static constexpr int kPSlab = RN * 128;               // RN rows x 64 keys
+    static constexpr int kPBytes = 2 * kPSlab;            // 128 keys
+    static constexpr int kQOff = 0;
+    static constexpr int kPOff = kQOff + kSlabs * kQSlab;  // kNS P buffers
+    static constexpr int kVOff = kPOff + kNS * kPBytes;
+    static constexpr int kKOff = kVOff + kStages * kTileBytes;
+    static constexpr int kBarOff = kKOff + kStages * kTileBytes;
+    static constexpr int kNumBars = 2 + 4 * kStages + 3 * kNS + 4 + 5;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kFlagOff = kMiscOff + 128;        // int [2][4]: a warp's rows need the exact max
+    static constexpr int kRedOff = kFlagOff + 32;          // float [2][4][RN]: per-warp maxima
+    static constexpr int kSumOff = kRedOff + 2 * 4 * RN * 4;  // float [4][RN][2]: per-warp sums
+    static constexpr int kSmemBytes = kSumOff + 4 * RN * 2 * 4;
+    static constexpr uint32_t kColO = 32 * kNS;
+    static constexpr uint32_t kTmemCols = kColO + 32 <= 128 ? 128 : 256;
+    static_assert(RN == 16 || RN == 32, "N of the swapped products");
+    static_assert(kStages >= kNS, "a V buffer is reused only after the P V that read it");
+    static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0 && kVOff % 1024 == 0 && kKOff % 1024 == 0, "alignment");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+// Byte offset of key `key` (0..127) of row r in a [RN x 128] 16-bit K-major tile
+// with the 128-byte swizzle (two 64-key slabs of RN rows).
+template <int RN>
+__device__ __forceinline__ uint32_t dec_p_offset(int r, int key) {
+    return static_cast<uint32_t>((key >> 6) * (RN * 128) + r * 128 + ((((key & 63) >> 3) ^ (r & 7)) << 4) +
+                                 (key & 7) * 2);
+}
+
+template <int D, bool BF16, bool SEQLENS, bool PAGED, int RN>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    fa_decode_narrow_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const DecodeArgs args, const int causal) {
+    static_assert(SEQLENS || !PAGED, "a paged cache needs the sequence lengths");
+    using C = DecNarrowCfg<D, RN>;
+    constexpr int S = C::kStages;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (!smem_base_ok(smem, args.err)) return;
+    // The merge kernel may be scheduled now; it waits for this grid before reading.
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int cta = static_cast<int>(blockIdx.x);
+    const int tid = static_cast<int>(threadIdx.x);
+    const int warp = warp_id();
+    const int lane = lane_id();
+    uint8_t* misc = smem + C::kMiscOff;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc);
+    int* abort_flag = reinterpret_cast<int*>(misc + 4);
+
+    DecRange rg;
+    if (!dec_locate<SEQLENS>(args, misc, rg)) return;  // no tile for this CTA
+
+    uint8_t* sQ = smem + C::kQOff;
+    uint8_t* sP = smem + C::kPOff;
+    uint8_t* sK = smem + C::kKOff;
+    uint8_t* sV = smem + C::kVOff;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* q_full = bars;
+    uint64_t* q_empty = bars + 1;
+    uint64_t* k_full = bars + 2;
+    uint64_t* k_empty = k_full + S;
+    uint64_t* v_full = k_empty + S;
+    uint64_t* v_empty = v_full + S;
+    constexpr int NS = C::kNS;
+    uint64_t* s_full = v_empty + S;   // [NS] S^T buffer b holds tile gg (gg % NS == b)
+    uint64_t* p_full = s_full + NS;   // [NS]
+    uint64_t* pv_done = p_full + NS;  // [NS] P V of the tile in P buffer b complete
+    uint64_t* o_ready = pv_done + NS;
+    uint64_t* o_free = o_ready + 1;
+    uint64_t* mma_done = o_free + 1;
+    uint64_t* sm_done = mma_done + 1;
+
+    // Rows of Q that no load writes are zeros: rows R .. RN-1, and with paired KV heads
+    // everything outside the two groups' blocks (rows 0..rg-1 of columns 0..63, rows
+    // r8..r8+rg-1 of columns 64..127), which makes Q block-diagonal.
+    for (int i = tid; i < C::kSlabs * C::kQSlab / 16; i += kDecThreads) {
+        const int row = (i % (C::kQSlab / 16)) / 8, slab = i / (C::kQSlab / 16);
+        const bool loaded = args.pair ? (row >= slab * args.r8 && row < slab * args.r8 + args.rg) : row < args.R;
+        if (!loaded) reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    if (tid == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+        }
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 128);
+            mbar_init(&pv_done[i], 1);
+        }
+        mbar_init(o_ready, 1);
+        mbar_init(o_free, 128);
+        mbar_init(mma_done, 1);
+        mbar_init(sm_done, 128);
+        for (int i = 0; i < 5; ++i) mbar_init(sm_done + 1 + i, 4);  // softmax warps meeting: one arrival per warp
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+    const WaitCtx wc{abort_flag, args.err};
+
+    if (warp == 0) {
+        if (lane == 0)
+            dec_produce<D, SEQLENS, PAGED, S>(args, rg, &tm_q, &tm_k, &tm_v, sQ, C::kQSlab, 0, sK, sV, q_full,
+                                              q_empty, k_full, k_empty, v_full, v_empty, wc);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_f16(128, RN, BF16, false, false);
+            constexpr uint32_t id_pv = idesc_f16(128, RN, BF16, true, false);
+            const uint32_t q_addr = smem_u32(sQ);
+            // S^T into columns 32 (gg % NS) from the K tile of ring index gg.
+            auto issue_s = [&](int gg) {
+                const uint32_t k_addr = smem_u32(sK + (gg % S) * C::kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ko = (kk >> 2) * C::kKVSlab + (kk & 3) * 32;
+                    const uint32_t qo = (kk >> 2) * C::kQSlab + (kk & 3) * 32;
+                    mma_ss(tmem + 32 * (gg % NS), sdesc_sw128(k_addr + ko, 16, 1024),
+                           sdesc_sw128(q_addr + qo, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&s_full[gg % NS]);
+                tc_commit(&k_empty[gg % S]);
+            };
+            int gk = 0, nq = 0;
+            bool ok = true;
+            for (DecItem it = rg.first; ok && it.P < rg.s_hi; it = dec_next<SEQLENS>(args, it, rg.T)) {
+                const long long lo = max(rg.s_lo, it.P), hi = min(rg.s_hi, it.P + it.ntk);
+                if (lo >= hi) continue;
+                const int n = static_cast<int>(hi - lo);
+                if (!(ok = mbar_wait(q_full, nq & 1, wc, 100))) break;
+                for (int j = 0; ok && j < min(n, NS); ++j) {
+                    const int gg = gk + j;
+                    if (!(ok = mbar_wait(&k_full[gg % S], (gg / S) & 1, wc, 101))) break;
+                    tc_fence_after();
+                    issue_s(gg);
+                }
+                if (!ok) break;
+                if (n <= NS) tc_commit(q_empty);
+                for (int j = 0; ok && j < n; ++j) {
+                    const int gg = gk + j, st = gg % S, b = gg % NS;
+                    if (!(ok = mbar_wait(&v_full[st], (gg / S) & 1, wc, 102))) break;
+                    if (j == 0 && nq > 0 && !(ok = mbar_wait(o_free, (nq - 1) & 1, wc, 103))) break;
+                    if (!(ok = mbar_wait(&p_full[b], (gg / NS) & 1, wc, 104))) break;
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(sV + st * C::kTileBytes);
+                    const uint32_t p_addr = smem_u32(sP + b * C::kPBytes);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(tmem + C::kColO, sdesc_sw128(v_addr + kk * 2048, C::kKVSlab, 1024),
+                               sdesc_sw128(p_addr + (kk >> 2) * C::kPSlab + (kk & 3) * 32, 16, 1024), id_pv,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&pv_done[b]);
+                    tc_commit(&v_empty[st]);
+                    // S^T of tile gg + NS into the columns of tile gg; P of that tile goes to
+                    // the P buffer just read. The tensor core runs one thread's products in
+                    // issue order.
+                    if (j + NS < n) {
+                        const int g2 = gg + NS;
+                        if (!(ok = mbar_wait(&k_full[g2 % S], (g2 / S) & 1, wc, 105))) break;
+                        tc_fence_after();
+                        issue_s(g2);
+                        if (j + NS + 1 == n) tc_commit(q_empty);
+                    }
+                }
+                tc_commit(o_ready);
+                gk += n;
+                ++nq;
+            }
+            tc_commit(mma_done);
+            mbar_wait_drain(mma_done, 0);
+            const uint32_t a = smem_u32(sm_done);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < 4000000000ull) {
+            }
+        }
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax / epilogue
+        // Thread l: key l of every tile (TMEM lane l of S^T) and d index l of O^T. The
+        // four warps meet on mbarriers with one arrival per warp (bounded waits, so a
+        // warp that gave up on a wait cannot leave the others stuck).
+        const int w4 = warp - 4;
+        const int l_idx = w4 * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
+        const uint32_t o_addr = lane_base + C::kColO;
+        volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kFlagOff);
+        volatile float* red = reinterpret_cast<volatile float*>(smem + C::kRedOff);
+        volatile float* sums = reinterpret_cast<volatile float*>(smem + C::kSumOff);
+        uint64_t* xb_flag = sm_done + 1;     // [2] per tile parity
+        uint64_t* xb_red = xb_flag + 2;      // [2] per tile parity, slow tiles only
+        uint64_t* xb_sum = xb_red + 2;       // one per segment
+        const float sl2 = args.scale_log2;
+        const int g = args.group, R = args.R;
+        // Meet the other three warps: this warp's shared-memory writes are visible to
+        // them once every warp's wait returns.
+        auto meet = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+            return warp_all(mbar_wait(bar, parity, wc, site));
+        };
+        int gk = 0, nq = 0;
+        int n_red0 = 0, n_red1 = 0;  // uses of xb_red[0], xb_red[1] so far
+        bool ok = true;
+        for (DecItem it = rg.first; ok && it.P < rg.s_hi; it = dec_next<SEQLENS>(args, it, rg.T)) {
+            const long long lo = max(rg.s_lo, it.P), hi = min(rg.s_hi, it.P + it.ntk);
+            if (lo >= hi) continue;
+            const int j0 = static_cast<int>(lo - it.P), n = static_cast<int>(hi - lo);
+            // Row r (token r / g) sees keys below min(len, r / g + len - Nq + 1) under the
+            // causal mask, below len otherwise.
+            const int causal_base = it.len - args.Nq + 1;
+            float m[RN], l[RN], lr[RN];
+#pragma unroll
+            for (int r = 0; r < RN; ++r) {
+                m[r] = -INFINITY;
+                l[r] = 0.f;
+                lr[r] = 0.f;
+            }
+            for (int j = 0; j < n; ++j) {
+                const int gg = gk + j, par = gg & 1, b = gg % NS;
+                ok = warp_all(mbar_wait(&s_full[b], (gg / NS) & 1, wc, 106));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t sv[32];
+                tmem_ld32(lane_base + 32 * b, sv);
+                tmem_ld_wait(sv);
+                const int key = (j0 + j) * 128 + l_idx;
+                float x[RN];
+                bool exceed = false;
+                int t = 0, hc = 0;
+#pragma unroll
+                for (int r = 0; r < RN; ++r) {
+                    if (args.pair && r == args.r8) {  // the second KV head's rows start again at token 0
+                        t = 0;
+                        hc = 0;
+                    }
+                    const int khi = causal ? min(it.len, t + causal_base) : it.len;
+                    x[r] = key < khi ? __uint_as_float(sv[r]) * sl2 : -INFINITY;
+                    exceed |= x[r] > m[r] + kRescaleThreshold;
+                    if (++hc == g) {
+                        hc = 0;
+                        ++t;
+                    }
+                }
+                // Does any row need a new reference max? (Always on a row's first keys.)
+                const bool wexc = __any_sync(0xffffffffu, exceed);
+                if (lane == 0) flags[par * 4 + w4] = wexc ? 1 : 0;
+                ok = meet(&xb_flag[par], (gg >> 1) & 1, 107);
+                if (!ok) break;
+                if (flags[par * 4] | flags[par * 4 + 1] | flags[par * 4 + 2] | flags[par * 4 + 3]) {
+                    // The exact tile max of every row, then the reference moves there.
+                    volatile float* rd = red + par * 4 * RN;
+#pragma unroll
+                    for (int r = 0; r < RN; ++r) {
+                        float v = x[r];
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                        if (lane == r) rd[w4 * RN + r] = v;
+                    }
+                    ok = meet(&xb_red[par], (par ? n_red1 : n_red0) & 1, 108);
+                    if (par) ++n_red1; else ++n_red0;
+                    if (!ok) break;
+                    // O^T holds the products up to the previous tile once its P V is
+                    // complete; it is rescaled with the normalisers (by 1 where a row's
+                    // reference stays).
+                    const bool with_o = j > 0;
+                    uint32_t ov[32];
+                    if (with_o) {  // P V of tile gg - 1: its buffer's use (gg - 1) / NS
+                        ok = warp_all(mbar_wait(&pv_done[(gg - 1) % NS], ((gg - 1) / NS) & 1, wc, 109));
+                        if (!ok) break;
+                        tc_fence_after();
+                        tmem_ld32(o_addr, ov);
+                        tmem_ld_wait(ov);
+                    }
+#pragma unroll
+                    for (int r = 0; r < RN; ++r) {
+                        const float mx = fmaxf(fmaxf(rd[r], rd[RN + r]), fmaxf(rd[2 * RN + r], rd[3 * RN + r]));
+                        float alpha = 1.f;
+                        if (mx > m[r]) {
+                            if (m[r] != -INFINITY) alpha = ex2_approx(m[r] - mx);
+                            m[r] = mx;
+                        }
+                        l[r] *= alpha;
+                        lr[r] *= alpha;
+                        if (with_o) ov[r] = __float_as_uint(__uint_as_float(ov[r]) * alpha);
+                    }
+                    if (with_o) {
+                        tmem_st32(o_addr, ov);
+                        tmem_st_wait();
+                    }
+                }
+                // P = 2^(x - m) rounded to 16 bits: row r, key l of P buffer b (free: S^T of
+                // this tile complete implies P V of tile gg - NS complete).
+                uint8_t* pb = sP + b * C::kPBytes;
+#pragma unroll
+                for (int r = 0; r < RN; r += 2) {
+                    const float p0 = ex2_approx(x[r] + (m[r] == -INFINITY ? 0.f : -m[r]));
+                    const float p1 = ex2_approx(x[r + 1] + (m[r + 1] == -INFINITY ? 0.f : -m[r + 1]));
+                    l[r] += p0;
+                    l[r + 1] += p1;
+                    const uint32_t u = pack2<BF16>(p0, p1);
+                    lr[r] += unpack_lo<BF16>(u);
+                    lr[r + 1] += unpack_hi<BF16>(u);
+                    *reinterpret_cast<uint16_t*>(pb + dec_p_offset<RN>(r, l_idx)) = static_cast<uint16_t>(u & 0xffffu);
+                    *reinterpret_cast<uint16_t*>(pb + dec_p_offset<RN>(r + 1, l_idx)) = static_cast<uint16_t>(u >> 16);
+                }
+                // The sequence's last tile: rows of V past its end may hold anything
+                // (0 x NaN would reach O); they are zeroed before P V reads them. V's
+                // previous use of this buffer (tile gg - S, S >= NS) is complete: S^T of
+                // this tile is, so P V of tile gg - NS is.
+                if (SEQLENS && j0 + j == it.ntk - 1 && (it.len & 127) != 0) {
+                    ok = warp_all(mbar_wait(&v_full[gg % S], (gg / S) & 1, wc, 110));
+                    if (!ok) break;
+                    const int v0 = it.len & 127;
+                    const int per_slab = (128 - v0) * 8;
+                    uint8_t* vt = sV + (gg % S) * C::kTileBytes;
+                    for (int xx = l_idx; xx < per_slab * C::kSlabs; xx += 128) {
+                        const int s = xx / per_slab, rem = xx % per_slab;
+                        *reinterpret_cast<uint4*>(vt + s * C::kKVSlab + (v0 + rem / 8) * 128 + (rem % 8) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&p_full[b]);
+            }
+            if (!ok) break;
+            // Row sums over the 128 keys' threads.
+#pragma unroll
+            for (int r = 0; r < RN; ++r) {
+                float a = l[r], b = lr[r];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    a += __shfl_xor_sync(0xffffffffu, a, off);
+                    b += __shfl_xor_sync(0xffffffffu, b, off);
+                }
+                if (lane == r) {
+                    sums[(w4 * RN + r) * 2] = a;
+                    sums[(w4 * RN + r) * 2 + 1] = b;
+                }
+            }
+            ok = meet(xb_sum, nq & 1, 111);
+            if (!ok) break;
+            ok = warp_all(mbar_wait(o_ready, nq & 1, wc, 112));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t ov[32];
+            tmem_ld32(o_addr, ov);
+            tmem_ld_wait(ov);
+            const size_t slot = static_cast<size_t>(cta) + static_cast<size_t>(it.b) * args.Hkv + it.hk;
+            // Partial row rp of tile row r; with paired KV heads the rows of head group k
+            // sit in O^T lanes 64 k .. 64 k + 63 and partials have d = 64.
+            const bool pair = args.pair != 0;
+#pragma unroll
+            for (int r = 0; r < RN; ++r) {
+                const int k = (pair && r >= args.r8) ? 1 : 0;
+                const int rl = r - k * args.r8;
+                const bool valid = pair ? rl < args.rg : r < R;
+                const int rp = pair ? k * args.rg + rl : r;
+                if (valid) {
+                    float lt = 0.f, lrt = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        lt += sums[(w * RN + r) * 2];
+                        lrt += sums[(w * RN + r) * 2 + 1];
+                    }
+                    const float o_val = __uint_as_float(ov[r]) * (lrt > 0.f ? 1.f / lrt : 0.f);
+                    if (pair) {
+                        if ((l_idx >> 6) == k) args.o_part[(slot * R + rp) * 64 + (l_idx & 63)] = o_val;
+                    } else if (l_idx < D) {
+                        args.o_part[(slot * R + rp) * D + l_idx] = o_val;
+                    }
+                    if (l_idx == r) {
+                        float L = -INFINITY;
+                        if (lt > 0.f) {
+                            float lg;
+                            asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(lt));
+                            L = (m[r] + lg) * kLn2;
+                        }
+                        args.lse_part[slot * R + rp] = L;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(o_free);
+            gk += n;
+            ++nq;
+        }
+        tc_fence_before();
+        mbar_arrive(sm_done);
+    }
+}
+
+// Merge of the segments of each item: one block of four warps per (item, row r) of
+// the R rows: L = log sum_s exp(L_s) and O = sum_s exp(L_s - L) O_s over the CTAs
+// whose tile range meets the item (warp w takes every fourth segment, lanes d in
+// chunks of four), written to o [B, Nq, Hq, d] and lse [B, Hq, Nq]. An item without
+// keys, or a row that sees none, gets O = 0 and L = -inf.
 template <int D, bool BF16, bool SEQLENS>
 __global__ void __launch_bounds__(128) fa_decode_combine(const DecodeArgs a) {
-    const int item = static_cast<int>(blockIdx.x);
+    // Launched as a programmatic dependent of the split kernel: everything below
+    // reads what that kernel wrote, so wait for it to complete (no-op otherwise).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float4 part[4][D / 4];
+    const int lane = lane_id(), warp = warp_id();
+    const int item = static_cast<int>(blockIdx.x / a.R), r = static_cast<int>(blockIdx.x % a.R);
     const int b = item / a.Hkv, hk = item % a.Hkv;
     const int len = dec_len<SEQLENS>(a, b);
     const int ntk = (len + 127) / 128;
-    long long T, P;
-    if constexpr (SEQLENS) {  // written by the split kernel (which runs whenever some item has keys)
-        T = ntk > 0 ? a.meta[0] : 0;
-        P = ntk > 0 ? a.meta[1 + item] : 0;
-    } else {
-        T = static_cast<long long>(a.B) * a.Hkv * ntk;
-        P = static_cast<long long>(item) * ntk;
+    long long T = 0, P = 0;
+    if (ntk > 0) {
+        if constexpr (SEQLENS) {  // written by the split kernel, which runs whenever some item has keys
+            T = a.meta[0];
+            P = a.meta[1 + item];
+        } else {
+            T = static_cast<long long>(a.B) * a.Hkv * ntk;
+            P = static_cast<long long>(item) * ntk;
+        }
     }
     int c0 = 0, c1 = -1;
     if (ntk > 0 && T > 0) {
         c0 = dec_cta_of(P, T, a.G);
         c1 = dec_cta_of(P + ntk - 1, T, a.G);
     }
-    uint16_t* o = static_cast<uint16_t*>(a.o);
-    for (int idx = static_cast<int>(threadIdx.x); idx < a.R * (D / 8); idx += static_cast<int>(blockDim.x)) {
-        const int r = idx / (D / 8), c8 = idx % (D / 8);
-        const int t = r / a.group, h = hk * a.group + r % a.group;
-        float Lm = -INFINITY;
-        for (int c = c0; c <= c1; ++c)
-            if (dec_split(c, T, a.G) < dec_split(c + 1, T, a.G))
-                Lm = fmaxf(Lm, a.lse_part[static_cast<size_t>(c + item) * a.R + r]);
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float wsum = 0.f;
-        if (Lm != -INFINITY) {
-            for (int c = c0; c <= c1; ++c) {
-                if (dec_split(c, T, a.G) >= dec_split(c + 1, T, a.G)) continue;
-                const size_t row = static_cast<size_t>(c + item) * a.R + r;
-                const float w = expf(a.lse_part[row] - Lm);
-                if (w == 0.f) continue;
-                wsum += w;
-                const float4* src = reinterpret_cast<const float4*>(a.o_part + row * D + c8 * 8);
-                const float4 x0 = src[0], x1 = src[1];
-                acc[0] += w * x0.x;
-                acc[1] += w * x0.y;
-                acc[2] += w * x0.z;
-                acc[3] += w * x0.w;
-                acc[4] += w * x1.x;
-                acc[5] += w * x1.y;
-                acc[6] += w * x1.z;
-                acc[7] += w * x1.w;
-            }
-        }
-        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-        uint32_t pk[4];
+    // CTA c's range is empty only when there are fewer tiles than CTAs.
+    const bool all_have = T >= a.G;
+    auto has = [&](int c) { return all_have || dec_split(c, T, a.G) < dec_split(c + 1, T, a.G); };
+    const float* lp = a.lse_part + static_cast<size_t>(item) * a.R + r;  // segment of CTA c: lp[c * R]
+    // Every warp finds the max and the sum of weights itself (lanes over segments).
+    float Lm = -INFINITY;
+    for (int c = c0 + lane; c <= c1; c += 32)
+        if (has(c)) Lm = fmaxf(Lm, lp[static_cast<size_t>(c) * a.R]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) pk[i] = pack2<BF16>(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-        const size_t orow = (static_cast<size_t>(b) * a.Nq + t) * a.Hq + h;
-        *reinterpret_cast<uint4*>(o + orow * D + c8 * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        if (c8 == 0)
-            a.lse[(static_cast<size_t>(b) * a.Hq + h) * a.Nq + t] = wsum > 0.f ? Lm + logf(wsum) : -INFINITY;
+    for (int off = 16; off > 0; off >>= 1) Lm = fmaxf(Lm, __shfl_xor_sync(0xffffffffu, Lm, off));
+    float wsum = 0.f;
+    if (Lm != -INFINITY)
+        for (int c = c0 + lane; c <= c1; c += 32)
+            if (has(c)) wsum += expf(lp[static_cast<size_t>(c) * a.R] - Lm);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (Lm != -INFINITY && lane < D / 4) {
+#pragma unroll 2
+        for (int c = c0 + warp; c <= c1; c += 4) {
+            if (!has(c)) continue;
+            const size_t row = (static_cast<size_t>(c) + item) * a.R + r;
+            const float w = expf(a.lse_part[row] - Lm);
+            const float4 x = reinterpret_cast<const float4*>(a.o_part + row * D)[lane];
+            acc.x += w * x.x;
+            acc.y += w * x.y;
+            acc.z += w * x.z;
+            acc.w += w * x.w;
+        }
     }
+    if (lane < D / 4) part[warp][lane] = acc;
+    __syncthreads();
+    if (warp != 0 || lane >= D / 4) return;
+#pragma unroll
+    for (int w = 1; w < 4; ++w) {
+        const float4 y = part[w][lane];
+        acc.x += y.x;
+        acc.y += y.y;
+        acc.z += y.z;
+        acc.w += y.w;
+    }
+    // Row r of the item: with paired KV heads rows 0..rg-1 belong to KV head 2 hk and
+    // rows rg..2 rg-1 to KV head 2 hk + 1.
+    const int kv = a.pair ? 2 * hk + r / a.rg : hk;
+    const int rl = a.pair ? r % a.rg : r;
+    const int t = rl / a.group, h = kv * a.group + rl % a.group;
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    uint16_t* o = static_cast<uint16_t*>(a.o) + ((static_cast<size_t>(b) * a.Nq + t) * a.Hq + h) * D + lane * 4;
+    *reinterpret_cast<uint2*>(o) = make_uint2(pack2<BF16>(acc.x * inv, acc.y * inv), pack2<BF16>(acc.z * inv, acc.w * inv));
+    if (lane == 0)
+        a.lse[(static_cast<size_t>(b) * a.Hq + h) * a.Nq + t] = wsum > 0.f ? Lm + logf(wsum) : -INFINITY;
 }
 
 }  // namespace fa

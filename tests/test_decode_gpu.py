@@ -75,6 +75,9 @@ CASES = [
     (small(Hq=6, Hkv=2, Nq=20, Nk=300), [300, 260, 17], True),   # 60 rows in lanes 0..59 (no head split)
     (small(Hq=16, Hkv=1, Nq=8, Nk=900, d=64), None, True),       # 128 rows, the whole tile
     (small(B=40, Hkv=8, Hq=32, Nk=700, len_seed=9, min_len=0), None, False),  # many short items
+    (small(Hq=8, Hkv=4, Nq=3, Nk=1000, d=64), [1000, 2, 513], True),   # d = 64, paired KV heads, 6 rows each
+    (small(Hq=16, Hkv=2, Nq=2, Nk=600, d=64, dtype="fp16"), None, True),  # paired heads, 16 rows each
+    (small(Hq=6, Hkv=3, Nq=1, Nk=900, d=64), [900, 1, 128], False),   # d = 64, odd Hkv: no pairing
 ]
 
 
