@@ -408,7 +408,8 @@ def run_ours(args):
 
 # ----------------------------------------------------------------------------- per-workload sweep
 def run_sweep(args):
-    """Forward (and the causal GQA backward) of every workload, one JSON line each.
+    """Forward (and the backward where the workload has one) of every workload, and the
+    decode workloads, one JSON line each.
     Informational: the bench line of the contract is the default mode."""
     import torch
     from exact_tiled_attention_36_b200 import binding as fb
@@ -561,6 +562,46 @@ def run_sweep(args):
             ms = time_it(vbwd, 10)
             emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
             del do, ws, dq, dk, dv
+    # decode against a key/value cache, split over the keys (split kernel + merge kernel)
+    for cfg, page in ((inputs.DECODE, 0), (inputs.DECODE_RAGGED, 0), (inputs.DECODE_RAGGED, 64),
+                      (inputs.DECODE_RAGGED, 16), (inputs.DECODE_D64, 0), (inputs.DECODE_SPEC4, 0)):
+        di = inputs.make_decode(cfg, page_size=page)
+        q = di.q.cuda()
+        B, Nq, Hq, d = q.shape
+        Hkv = di.k.shape[2]
+        lens = di.seqlens if di.seqlens is not None else [cfg.Nk] * B
+        sl = None if di.seqlens is None else torch.tensor(di.seqlens, dtype=torch.int32, device="cuda")
+        ws = torch.empty(fb.fa_decode_workspace_size(B, Hq, Hkv, Nq, d), dtype=torch.uint8, device="cuda")
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device="cuda")
+        dt = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
+        if page:
+            kp, vp, bt = di.k_pages.cuda(), di.v_pages.cuda(), di.block_table.cuda()
+
+            def dec():
+                st = fb.fa_decode_paged(q.data_ptr(), kp.data_ptr(), vp.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                        sl.data_ptr(), bt.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, kp.shape[0],
+                                        page, bt.shape[1], d, cfg.scale, int(cfg.causal), dt, stream.cuda_stream)
+                if st != fb.FA_OK:
+                    raise RuntimeError(fb.fa_status_string(st))
+        else:
+            kc, vc = di.k.cuda(), di.v.cuda()
+
+            def dec():
+                st = fb.fa_decode(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  0 if sl is None else sl.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, cfg.Nk, d,
+                                  cfg.scale, int(cfg.causal), dt, stream.cuda_stream)
+                if st != fb.FA_OK:
+                    raise RuntimeError(fb.fa_status_string(st))
+
+        keys = sum(lens)
+        # attention FLOPs (masked pairs of the causal tokens excluded) and the bytes the
+        # step must move: every cached K and V row once, Q, O and L
+        vis = sum(min(n, max(0, t + n - Nq + 1)) if cfg.causal else n for n in lens for t in range(Nq))
+        flops = 4.0 * d * Hq * vis
+        nbytes = 2 * (2 * keys * Hkv * d + 2 * q.numel()) + 4 * lse.numel()
+        emit(cfg.name + (f"_paged{page}" if page else ""), "decode", time_it(dec, 50), flops, nbytes)
+        del di, q, o, lse, ws
     return 0
 
 

@@ -118,6 +118,10 @@ DECODE = DecodeConfig("decode_b32_nk8192_hq32_hkv8_d128", B=32, Hq=32, Hkv=8, Nq
                       dtype="bf16", causal=False, seed=6)
 DECODE_RAGGED = DecodeConfig("decode_ragged_b32_nk8192_hq32_hkv8_d128", B=32, Hq=32, Hkv=8, Nq=1, Nk=8192,
                              d=128, dtype="bf16", causal=False, seed=6, len_seed=7)
+DECODE_D64 = DecodeConfig("decode_b32_nk8192_hq32_hkv8_d64", B=32, Hq=32, Hkv=8, Nq=1, Nk=8192, d=64,
+                          dtype="bf16", causal=False, seed=6)
+DECODE_SPEC4 = DecodeConfig("decode_spec4_b32_nk8192_hq32_hkv8_d128", B=32, Hq=32, Hkv=8, Nq=4, Nk=8192, d=128,
+                            dtype="bf16", causal=True, seed=6)  # 4 speculative tokens per sequence, causal
 
 ALL_FIXED = (TINY, VISION, VIT_RMSNORM, CAUSAL_GQA)
 ALL_VARLEN = (VARLEN, VARLEN_KEYPAD)
