@@ -278,6 +278,38 @@ def attn_decode(q, k, v, scale: float, seqlens=None, causal: bool = False):
     return o, lse
 
 
+def e4m3_decode(codes):
+    """Values of E4M3 bytes in fp64, from the format's definition: 1 sign bit, 4
+    exponent bits with bias 7, 3 mantissa bits; exponent field 0 is subnormal
+    (m / 8 * 2^-6); the all-ones pattern S.1111.111 is NaN; there is no infinity.
+    The largest finite value is 1.75 * 2^8 = 448."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7))
+    val = np.where((e == 0xF) & (m == 0x7), np.nan, val)
+    return sign * val
+
+
+def fp8_dequantise(codes, scales, block: int = 128):
+    """Real values of a block-scaled E4M3 tensor: codes [B, N, H, d], scales
+    [B, H, ceil(N / block)]; element (b, i, h, c) = scales[b, h, i // block] *
+    e4m3(codes[b, i, h, c])."""
+    x = e4m3_decode(codes)
+    sc = np.asarray(scales, dtype=np.float64)
+    N = x.shape[1]
+    blk = np.arange(N) // block
+    return x * np.transpose(sc[:, :, blk], (0, 2, 1))[..., None]
+
+
+def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, scale: float, causal: bool = False):
+    """The FP8 forward's exact result: the plain definition (attn_fwd) on the
+    dequantised block-scaled E4M3 inputs."""
+    return attn_fwd(fp8_dequantise(q8, q_scale), fp8_dequantise(k8, k_scale), fp8_dequantise(v8, v_scale),
+                    scale, causal)
+
+
 def timed(fn, *args, **kw):
     """(result, seconds) of one call."""
     t0 = time.perf_counter()

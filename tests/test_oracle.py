@@ -486,3 +486,39 @@ def test_attn_decode_pins(causal):
         o3, l3 = oracle.attn_fwd(q, k, v, 0.5, False, key_keep=keep)
         np.testing.assert_allclose(o, o3, atol=1e-13)
         np.testing.assert_allclose(l, l3, atol=1e-13)
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) inputs
+def test_e4m3_decode_matches_torch_and_closed_forms():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_decode(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.isnan(ours), np.isnan(lib))
+    ok = ~np.isnan(lib)
+    np.testing.assert_array_equal(ours[ok], lib[ok])
+    assert np.isnan(ours[0x7F]) and np.isnan(ours[0xFF]) and np.isnan(ours).sum() == 2
+    assert ours[0x38] == 1.0 and ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9 and ours[0x08] == 2.0 ** -6
+    assert ours[0xB8] == -1.0 and ours[0x00] == 0.0 and ours[0x80] == 0.0
+
+
+def test_fp8_dequantise_blocks_and_attention():
+    rng = np.random.default_rng(71)
+    B, N, H, d = 2, 300, 3, 4
+    codes = rng.integers(0, 256, size=(B, N, H, d), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38  # no NaN codes
+    scales = rng.uniform(0.5, 2.0, size=(B, H, 3))
+    x = oracle.fp8_dequantise(codes, scales)
+    for b, i, h in [(0, 0, 0), (1, 127, 2), (1, 128, 1), (0, 299, 2), (1, 256, 0)]:
+        np.testing.assert_array_equal(x[b, i, h], scales[b, h, i // 128] * oracle.e4m3_decode(codes[b, i, h]))
+    # with unit scales and codes of exactly representable values the FP8 forward is the plain forward
+    q = rng.standard_normal((1, 5, 2, 8))
+    k = rng.standard_normal((1, 7, 1, 8))
+    v = rng.standard_normal((1, 7, 1, 8))
+    import torch
+    enc = lambda t: torch.from_numpy(t).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    q8, k8, v8 = enc(q), enc(k), enc(v)
+    o, l = oracle.attn_fwd_fp8(q8, k8, v8, np.ones((1, 2, 1)), np.ones((1, 1, 1)), np.ones((1, 1, 1)), 0.3, True)
+    o2, l2 = numpy_ref.fwd(oracle.e4m3_decode(q8), oracle.e4m3_decode(k8), oracle.e4m3_decode(v8), 0.3, True)
+    np.testing.assert_allclose(o, o2, atol=1e-12)
+    np.testing.assert_allclose(l, l2, atol=1e-12)
