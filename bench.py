@@ -434,11 +434,13 @@ def run_sweep(args):
             raise RuntimeError("device error")
         return e0.elapsed_time(e1) / iters
 
-    def emit(name, what, ms, flops, nbytes):
+    def emit(name, what, ms, flops, nbytes, fp8=False):
         line = {"kind": "config_sweep", "workload": name, "pass": what, "ms": ms,
                 "tflops": flops / (ms / 1e3) / 1e12, "frac_of_bf16_burst": flops / (ms / 1e3) / 1e12 / peak,
                 "algorithmic_gbs": nbytes / (ms / 1e3) / 1e9, "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / hbm,
                 "peaks": peak_src}
+        if fp8:  # the E4M3 tensor peak: the measured bf16 burst peak x the nominal 2x ratio
+            line["frac_of_fp8_peak"] = flops / (ms / 1e3) / 1e12 / (2.0 * peak)
         print(json.dumps(line), flush=True)
 
     for cfg in (inputs.TINY, inputs.VISION, inputs.VIT_RMSNORM, inputs.CAUSAL_GQA):
@@ -458,6 +460,26 @@ def run_sweep(args):
             ms = time_it(lambda: fb.attention_bwd(q, k, v, o, lse, do, cfg.scale, cfg.causal, workspace=ws), 20)
             emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
         del q, k, v, o, lse
+    # the causal GQA prefill shape with block-scaled E4M3 inputs (fa_fwd_fp8)
+    cfg = inputs.CAUSAL_GQA_FP8
+    f8 = inputs.make_fp8(cfg)
+    q8, k8, v8 = f8.q.cuda(), f8.k.cuda(), f8.v.cuda()
+    qs, ks, vs = f8.q_scale.cuda(), f8.k_scale.cuda(), f8.v_scale.cuda()
+    B, N, Hq, d = q8.shape
+    Hkv = k8.shape[2]
+    o = torch.empty((B, N, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+
+    def ffp8():
+        r = fb.fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), qs.data_ptr(), ks.data_ptr(), vs.data_ptr(),
+                          o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d, cfg.scale, int(cfg.causal),
+                          stream.cuda_stream)
+        if r != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(r))
+
+    emit(cfg.name, "fwd", time_it(ffp8, 30), flops_fwd(B, N, Hq, d, cfg.causal),
+         q8.numel() + k8.numel() + v8.numel() + 2 * o.numel() + 4 * lse.numel(), fp8=True)
+    del q8, k8, v8, qs, ks, vs, o, lse
     # local attention: the causal GQA prefill shape with a causal sliding window of 1024 keys
     cfg = inputs.CAUSAL_GQA
     fi = inputs.make_fixed(cfg)

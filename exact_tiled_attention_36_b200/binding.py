@@ -1,7 +1,7 @@
 """Thin ctypes binding of libfa.so.
 
 The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_fwd_strided``, ``fa_varlen_fwd_strided``, ``fa_fwd_qk_rmsnorm``,
-``fa_fwd_window``, ``fa_bwd_window``, ``fa_decode``, ``fa_decode_paged``, ``fa_decode_workspace_size``,
+``fa_fwd_window``, ``fa_bwd_window``, ``fa_fwd_fp8``, ``fa_decode``, ``fa_decode_paged``, ``fa_decode_workspace_size``,
 ``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
 ``fa_bwd``, ``fa_status_string`` and ``fa_get_last_device_error`` have the
 names, argument order and meaning of the C ABI in ``include/fa.h``: pointers
@@ -52,6 +52,7 @@ _SIGS = {
     "fa_varlen_bwd": ([_P] * 12 + [_I] * 8 + [_F, _I, _I, _P], _I),
     "fa_selftest_bounded_wait": ([_P], _I),
     "fa_decode_workspace_size": ([_I] * 5, ctypes.c_size_t),
+    "fa_fwd_fp8": ([_P] * 8 + [_I] * 6 + [_F, _I, _P], _I),
     "fa_decode": ([_P] * 7 + [_I] * 6 + [_F, _I, _I, _P], _I),
     "fa_decode_paged": ([_P] * 8 + [_I] * 8 + [_F, _I, _I, _P], _I),
 }
@@ -157,6 +158,10 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, sca
     """fa_bwd with the library's own fixed-size workspace (for callers that cannot allocate)."""
     return lib().fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype,
                                 stream)
+
+
+def fa_fwd_fp8(q, k, v, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream) -> int:
+    return lib().fa_fwd_fp8(q, k, v, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream)
 
 
 def fa_decode_workspace_size(B, Hq, Hkv, Nq, d) -> int:
@@ -334,4 +339,23 @@ def attention_decode(q, k_cache, v_cache, cache_seqlens=None, scale: float | Non
                              bt.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, k.shape[0], k.shape[1], bt.shape[1], d,
                              float(scale), int(bool(causal)), _dtype_code(q), _stream(stream))
         _check(st, "fa_decode_paged")
+    return o, L
+
+
+def attention_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, scale: float | None = None, causal: bool = False,
+                      out=None, lse=None, stream=None):
+    """FP8 forward: q8 [B,Nq,Hq,d], k8/v8 [B,Nk,Hkv,d] uint8 E4M3 codes with float32 block
+    factors [B,H,ceil(N/128)]; returns O bf16 [B,Nq,Hq,d] and L float32 [B,Hq,Nq]."""
+    import torch
+    q8, k8, v8 = _dev(q8), _dev(k8), _dev(v8)
+    qs, ks, vs = (_dev(t).to(torch.float32) for t in (q_scale, k_scale, v_scale))
+    B, Nq, Hq, d = q8.shape
+    _, Nk, Hkv, _ = k8.shape
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=q8.device) if out is None else out
+    L = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device) if lse is None else lse
+    _check(fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), qs.data_ptr(), ks.data_ptr(), vs.data_ptr(),
+                      o.data_ptr(), L.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+                      _stream(stream)), "fa_fwd_fp8")
     return o, L

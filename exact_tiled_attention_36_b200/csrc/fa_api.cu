@@ -45,19 +45,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 // are sh, ss, sb elements (d contiguous); each stride must be a multiple of 16 bytes.
 // `promote_256`: L2 promotion of each request to 256 bytes (else 128). A row of one
 // head is 2 d bytes: with d = 64 the wider promotion also fetches the next head's row.
+// `elem_bytes` = 1: one-byte elements (E4M3), a box of 128 columns (still 128 bytes).
 fa_status make_map_box(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16,
-                       int64_t sh, int64_t ss, int64_t sb, int box_h, int box_rows, bool promote_256 = true) {
+                       int64_t sh, int64_t ss, int64_t sb, int box_h, int box_rows, bool promote_256 = true,
+                       int elem_bytes = 2) {
     auto enc = encode_tiled();
     if (!enc) return FA_ERR_CUDA;
     if (rows < 1) rows = 1;
     if (batches < 1) batches = 1;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batches)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sh) * 2, static_cast<cuuint64_t>(ss) * 2,
-                                   static_cast<cuuint64_t>(sb) * 2};
-    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_h), static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint64_t eb = static_cast<cuuint64_t>(elem_bytes);
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(sh) * eb, static_cast<cuuint64_t>(ss) * eb,
+                                   static_cast<cuuint64_t>(sb) * eb};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_h),
+                               static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+    const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : (bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    CUresult r = enc(m, dt, 4,
                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B,
                      promote_256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -127,11 +133,11 @@ fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtyp
     return FA_OK;
 }
 
-template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM>
+template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM, bool FP8 = false>
 fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                        dim3 grid, cudaStream_t stream) {
-    auto kern = fa::fa_fwd_kernel<D, BF16, MASK, VARLEN, QKNORM>;
-    constexpr int smem = fa::FwdCfg<D>::kSmemBytes;
+    auto kern = fa::fa_fwd_kernel<D, BF16, MASK, VARLEN, QKNORM, FP8>;
+    constexpr int smem = fa::FwdCfg<D, FP8>::kSmemBytes;
     static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
     if (!attr_ok) return FA_ERR_CUDA;
     // The kernel moves registers between warpgroups with setmaxnreg; the split
@@ -475,6 +481,57 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
     if ((st = fwd_units(a, num_seqs, max_seqlen_q, grid)) != FA_OK) return st;
     return launch_fwd(d, bf16, causal ? fa::kMaskCausal : fa::kMaskNone, true, false, mq, mk, mv, a, grid,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+// The FP8 forward (fixed length, d = 128): E4M3 q, k, v with per-block factors.
+fa_status fwd_fp8(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
+                  const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                  float scale, int causal, fa_stream_t stream) {
+    if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    if ((Nq > 0 && (!q || !o || !lse || !q_scale)) || (Nk > 0 && (!k || !v || !k_scale || !v_scale)))
+        return FA_ERR_INVALID_ARG;
+    fa_status st = common_checks(Hq, Hkv, d, scale, causal, FA_BF16);
+    if (st != FA_OK) return st;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(q_scale) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+        return FA_ERR_MISALIGNED;
+    if (B > 65535) return FA_ERR_UNSUPPORTED;
+    if (Nq == 0) return FA_OK;
+    int* err = error_word();
+    if (!err) return FA_ERR_CUDA;
+    CUtensorMap mq, mk{}, mv{};
+    const long long hq = static_cast<long long>(Hq) * d, hk = static_cast<long long>(Hkv) * d;
+    if ((st = make_map_box(&mq, q, d, Hq, Nq, B, true, d, hq, hq * Nq, 1, 128, true, 1)) != FA_OK) return st;
+    if (Nk > 0 && ((st = make_map_box(&mk, k, d, Hkv, Nk, B, true, d, hk, hk * Nk, 1, 128, true, 1)) != FA_OK ||
+                   (st = make_map_box(&mv, v, d, Hkv, Nk, B, true, d, hk, hk * Nk, 1, 128, true, 1)) != FA_OK))
+        return st;
+    fa::FwdArgs a{};
+    a.o = o;
+    a.lse = lse;
+    a.o_sb = static_cast<long long>(Nq) * Hq * d;
+    a.o_ss = static_cast<long long>(Hq) * d;
+    a.o_sh = d;
+    a.wl = -1;
+    a.wr = 0;
+    a.num_batches = B;
+    a.Hq = Hq;
+    a.group = Hq / Hkv;
+    a.Nq = Nq;
+    a.Nk = Nk;
+    a.scale_log2 = scale * kLog2e;
+    a.q_scale = q_scale;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.nqb = (Nq + 127) / 128;
+    a.nkb = (Nk + 127) / 128;
+    a.err = err;
+    dim3 grid;
+    if ((st = fwd_units(a, B, Nq, grid)) != FA_OK) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return causal ? launch_fwd_t<128, true, fa::kMaskCausal, false, false, true>(mq, mk, mv, a, grid, s)
+                  : launch_fwd_t<128, true, fa::kMaskNone, false, false, true>(mq, mk, mv, a, grid, s);
 }
 
 Strides contiguous(int rows, int H, int d) {
@@ -854,6 +911,12 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
     return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, num_seqs, cu_seqlens_q, cu_seqlens_k, total_q,
                       total_k, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal != 0, dtype == FA_BF16,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,
+                     const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                     float scale, int causal, fa_stream_t stream) {
+    return fwd_fp8(q, k, v, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream);
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int d) {

@@ -69,16 +69,26 @@ struct FwdArgs {
     int n_units;      // nu * Hq * num_batches
     float scale_log2;  // scale * log2(e)
     float norm_eps;    // QK RMS normalisation (fa_fwd_qk_rmsnorm): epsilon
+    // FP8 (E4M3 Q, K, V): dequantisation factors per 128-token block of one head,
+    // q_scale [B, Hq, nqb], k_scale and v_scale [B, Hkv, nkb].
+    const float* q_scale;
+    const float* k_scale;
+    const float* v_scale;
+    int nqb, nkb;
     int* err;
 };
 
 
-template <int D>
+// FP8: one-byte elements (a 128-row tile of d = 128 is a single 128-byte-wide slab).
+template <int D, bool FP8 = false>
 struct FwdCfg {
-    static constexpr int kSlabs = D / 64;
+    static constexpr int kElemBytes = FP8 ? 1 : 2;
+    static constexpr int kSlabElems = 128 / kElemBytes;  // columns per 128-byte slab
+    static constexpr int kSlabs = D * kElemBytes / 128;
     static constexpr int kSlabBytes = 128 * 128;
-    static constexpr int kTileBytes = kSlabs * kSlabBytes;  // 128 rows x d, 16-bit
-    static constexpr int kStages = (D == 128) ? 2 : 4;
+    static constexpr int kTileBytes = kSlabs * kSlabBytes;  // 128 rows x d
+    static constexpr int kKSteps = D * kElemBytes / 32;    // 32 bytes of K per MMA instruction
+    static constexpr int kStages = FP8 ? 4 : ((D == 128) ? 2 : 4);
     static constexpr int kQOff = 0;                          // Q_0, Q_1
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
@@ -238,11 +248,17 @@ __device__ __forceinline__ void rms_normalise_row(uint8_t* tile, int r, float ep
 // shared memory (over d) at the start of a unit, before the tensor core reads it;
 // K arrives normalised (fa_fwd_qk_rmsnorm runs fa_rms_normalise_rows over K first:
 // every CTA would otherwise redo each K tile once per unit).
-template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM>
+// FP8: Q, K, V are E4M3 with per-block dequantisation factors (fixed length, d = 128):
+// S and P V run as kind::f8f6f4 products; the Q and K block factors join the exp2
+// factor of each (query tile, key tile) pair, and V's block factor v_j enters P as
+// 2^(log2(v_j / v_max)) before P is rounded to E4M3 (P <= 2^8 under the lazy
+// rescale, inside E4M3's range), so O = v_max * sum(P' V) / l. O is bf16.
+template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM, bool FP8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
-    using C = FwdCfg<D>;
+    static_assert(!FP8 || (D == 128 && BF16 && !VARLEN && !QKNORM && MASK != kMaskWindow), "FP8 forward shape");
+    using C = FwdCfg<D, FP8>;
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) uint8_t smem[];
     if (!smem_base_ok(smem, args.err)) return;
@@ -335,7 +351,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int t = 0; t < 2; ++t)
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
-                        tma_load_4d(sQ + t * C::kTileBytes + s * C::kSlabBytes, &tm_q, q_full, s * 64, w.h,
+                        tma_load_4d(sQ + t * C::kTileBytes + s * C::kSlabBytes, &tm_q, q_full, s * C::kSlabElems, w.h,
                                     w.q_row0 + w.q0 + 128 * t, w.tma_b);
                 ++nq;
                 const int hk = w.h / args.group;
@@ -346,14 +362,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
-                        tma_load_4d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tm_k, &k_full[st], s * 64, hk,
+                        tma_load_4d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tm_k, &k_full[st], s * C::kSlabElems, hk,
                                     w.k_row0 + (w.jlo + j) * 128, w.tma_b);
                     ++k_issued;
                     if (!(ok = mbar_wait(&v_empty[st], ph ^ 1u, wc, 62))) break;
                     mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
-                        tma_load_4d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tm_v, &v_full[st], s * 64, hk,
+                        tma_load_4d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tm_v, &v_full[st], s * C::kSlabElems, hk,
                                     w.k_row0 + (w.jlo + j) * 128, w.tma_b);
                     ++v_issued;
                 }
@@ -368,17 +384,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t id_qk = idesc_f16(128, 128, BF16, false, false);
-            constexpr uint32_t id_pv = idesc_f16(128, D, BF16, false, true);
+            constexpr uint32_t id_qk = FP8 ? idesc_e4m3(128, 128, false, false) : idesc_f16(128, 128, BF16, false, false);
+            constexpr uint32_t id_pv = FP8 ? idesc_e4m3(128, D, false, true) : idesc_f16(128, D, BF16, false, true);
             const uint32_t q_addr = smem_u32(sQ);
             // S_t = Q_t K^T with the K tile of global ring index g.
             auto issue_s = [&](int t, int g) {
                 const uint32_t k_addr = smem_u32(sK + (g % S) * C::kTileBytes);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < C::kKSteps; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColS + 128 * t, sdesc_sw128(q_addr + t * C::kTileBytes + off, 16, 1024),
-                           sdesc_sw128(k_addr + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t qd = sdesc_sw128(q_addr + t * C::kTileBytes + off, 16, 1024);
+                    const uint64_t kd = sdesc_sw128(k_addr + off, 16, 1024);
+                    if constexpr (FP8)
+                        mma_ss_f8(tmem + C::kColS + 128 * t, qd, kd, id_qk, kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss(tmem + C::kColS + 128 * t, qd, kd, id_qk, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(&s_full[t]);
             };
@@ -422,11 +442,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         if (!(ok = mbar_wait(&p_full[t], ps[t] & 1, wc, 68))) break;
                         ++ps[t];
                         tc_fence_after();
+                        if constexpr (FP8) {
+                            // P: four E4M3 keys per column, 32 keys (8 columns, 32 rows of V)
+                            // per instruction; V's d = 128 one-byte values are one 128-byte slab.
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
-                                   sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024), id_pv,
-                                   (j > w.a(t) || kk > 0) ? 1u : 0u);
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_ts_f8(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
+                                          sdesc_sw128(v_addr + kk * 4096, C::kSlabBytes, 1024), id_pv,
+                                          (j > w.a(t) || kk > 0) ? 1u : 0u);
+                        } else {
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
+                                       sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024), id_pv,
+                                       (j > w.a(t) || kk > 0) ? 1u : 0u);
+                        }
                         if (j + 1 < w.b(t)) issue_s(t, g + 1);
                     }
                     if (j + 2 == w.n_kv) tc_commit(q_empty);  // the unit's last S products are issued
@@ -460,7 +490,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
         const uint32_t s_addr = lane_base + C::kColS + 128 * t;
         const uint32_t o_addr = lane_base + C::kColO + D * t;
-        const float sl2 = args.scale_log2;
+        const float sl2_base = args.scale_log2;
         int ss = 0, nq = 0;  // s_full phases consumed; units with work done
         bool ok = true;
         for (int rnd = 0; ok; ++rnd) {
@@ -509,8 +539,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 fence_proxy_async_smem();
                 mbar_arrive(q_norm);
             }
+            // FP8: the query tile's dequantisation factor, and V's largest block factor
+            // over the tiles this warpgroup visits (P carries v_j / v_max <= 1).
+            float fq = 1.f, v_max = 1.f;
+            const float* ksc = nullptr;
+            const float* vsc = nullptr;
+            if constexpr (FP8) {
+                const int hkv = w.h / args.group;
+                const size_t kv_row = (static_cast<size_t>(w.bidx) * (args.Hq / args.group) + hkv) * args.nkb;
+                fq = args.q_scale[(static_cast<size_t>(w.bidx) * args.Hq + w.h) * args.nqb +
+                                  min(qt0 >> 7, args.nqb - 1)];
+                ksc = args.k_scale + kv_row + w.jlo + w.a(t);
+                vsc = args.v_scale + kv_row + w.jlo + w.a(t);
+                v_max = 0.f;
+                for (int jj = 0; jj < nt; ++jj) v_max = fmaxf(v_max, vsc[jj]);
+            }
             float m = -INFINITY, l = 0.f, lr = 0.f;
             for (int j = 0; j < nt; ++j) {
+                // Exp2 factor of this (query tile, key tile) pair; with FP8 also P's factor
+                // v_j / v_max as a bias in the exponent, and v_max / v_j back for l.
+                float sl2 = sl2_base, bias = 0.f, vr = 1.f;
+                if constexpr (FP8) {
+                    sl2 = sl2_base * fq * ksc[j];
+                    const float vj = vsc[j];
+                    vr = v_max / vj;
+                    float lg;
+                    asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(vj / v_max));
+                    bias = lg;
+                }
                 ok = warp_all(mbar_wait(&s_full[t], ss & 1, wc, 69));
                 if (!ok) break;
                 ++ss;
@@ -553,27 +609,48 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 // P = 2^(S c - m) as 16-bit pairs (keys 2i, 2i + 1 in column i), partial sums
                 // of the exact and of the rounded values.
                 // Pairs of keys go through the packed f32x2 FMA and adds.
-                const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(neg_m, neg_m);
+                const uint64_t c2 = f2_pack(sl2, sl2), m2 = f2_pack(neg_m + bias, neg_m + bias);
                 uint64_t rs2[4] = {0, 0, 0, 0}, rsr2[4] = {0, 0, 0, 0};  // (0.f, 0.f) pairs
-                uint32_t pk[2][32];
+                if constexpr (FP8) {
+                    // Four E4M3 keys per column (4i .. 4i + 3 in column i, the lowest in the
+                    // low byte); O is normalised by the exact sum.
+                    uint32_t pk8[32];
     #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const uint64_t x = f2_pack(__uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
-                                               __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
-                    float y0, y1;
-                    f2_unpack(f2_fma(x, c2, m2), y0, y1);
-                    const float p0 = ex2_approx(y0);
-                    const float p1 = ex2_approx(y1);
-                    rs2[i & 3] = f2_add(rs2[i & 3], f2_pack(p0, p1));
-                    const uint32_t u = pack2<BF16>(p0, p1);
-                    rsr2[i & 3] = f2_add(rsr2[i & 3], f2_pack(unpack_lo<BF16>(u), unpack_hi<BF16>(u)));
-                    pk[i >> 5][i & 31] = u;
+                    for (int i = 0; i < 32; ++i) {
+                        const uint64_t xa = f2_pack(__uint_as_float(sv[(4 * i) >> 5][(4 * i) & 31]),
+                                                    __uint_as_float(sv[(4 * i + 1) >> 5][(4 * i + 1) & 31]));
+                        const uint64_t xb = f2_pack(__uint_as_float(sv[(4 * i + 2) >> 5][(4 * i + 2) & 31]),
+                                                    __uint_as_float(sv[(4 * i + 3) >> 5][(4 * i + 3) & 31]));
+                        float y0, y1, y2, y3;
+                        f2_unpack(f2_fma(xa, c2, m2), y0, y1);
+                        f2_unpack(f2_fma(xb, c2, m2), y2, y3);
+                        const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+                        const float p2 = ex2_approx(y2), p3 = ex2_approx(y3);
+                        rs2[i & 3] = f2_add(rs2[i & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+                        pk8[i] = pack4_e4m3(p0, p1, p2, p3);
+                    }
+                    tmem_st32(s_addr + 0, pk8);
+                } else {
+                    uint32_t pk[2][32];
+    #pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const uint64_t x = f2_pack(__uint_as_float(sv[(2 * i) >> 5][(2 * i) & 31]),
+                                                   __uint_as_float(sv[(2 * i + 1) >> 5][(2 * i + 1) & 31]));
+                        float y0, y1;
+                        f2_unpack(f2_fma(x, c2, m2), y0, y1);
+                        const float p0 = ex2_approx(y0);
+                        const float p1 = ex2_approx(y1);
+                        rs2[i & 3] = f2_add(rs2[i & 3], f2_pack(p0, p1));
+                        const uint32_t u = pack2<BF16>(p0, p1);
+                        rsr2[i & 3] = f2_add(rsr2[i & 3], f2_pack(unpack_lo<BF16>(u), unpack_hi<BF16>(u)));
+                        pk[i >> 5][i & 31] = u;
+                    }
+                    tmem_st32(s_addr + 0, pk[0]);
+                    tmem_st32(s_addr + 32, pk[1]);
                 }
-                tmem_st32(s_addr + 0, pk[0]);
-                tmem_st32(s_addr + 32, pk[1]);
                 const float rs = f2_sum(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])));
                 const float rsr = f2_sum(f2_add(f2_add(rsr2[0], rsr2[1]), f2_add(rsr2[2], rsr2[3])));
-                l = l * alpha + rs;
+                l = l * alpha + rs * vr;
                 lr = lr * alpha + rsr;
                 // S_t was issued after the previous key tile's P_t V and MMAs of one thread
                 // complete in order, so O_t is final for that tile here and can be
@@ -598,7 +675,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!ok) break;
             ++nq;
             tc_fence_after();
-            const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
+            const float inv_l = FP8 ? (l > 0.f ? v_max / l : 0.f) : ((lr > 0.f) ? 1.f / lr : 0.f);
             const FwdUnit we = fwd_unit<MASK, VARLEN>(u, args);
             const bool out_ok = row_ok(we);
             T16* dst = out_ok ? out_row(we) : nullptr;

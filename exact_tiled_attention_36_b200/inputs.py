@@ -297,3 +297,50 @@ def make_decode(cfg: DecodeConfig, lengths: list[int] | None = None, page_size: 
                 vp[page, :rows] = v[b, i * page_size:i * page_size + rows]
         out.page_size, out.k_pages, out.v_pages, out.block_table = page_size, kp, vp, table
     return out
+
+
+@dataclass
+class Fp8Inputs:
+    cfg: FixedConfig
+    q: torch.Tensor        # uint8 E4M3 codes [B, Nq, Hq, d]
+    k: torch.Tensor        # [B, Nk, Hkv, d]
+    v: torch.Tensor
+    q_scale: torch.Tensor  # float32 [B, Hq, ceil(Nq / 128)]: real = scale * e4m3(code)
+    k_scale: torch.Tensor  # float32 [B, Hkv, ceil(Nk / 128)]
+    v_scale: torch.Tensor
+
+
+def _quantise_e4m3(x: torch.Tensor, block: int = 128):
+    """Block-scaled E4M3 codes of x [B, N, H, d]: per head and block of 128 tokens the
+    factor amax / 448 (1 for an all-zero block), codes = round-to-nearest E4M3 of
+    x / factor (torch's float8 conversion)."""
+    B, N, H, d = x.shape
+    nb = (N + block - 1) // block
+    scales = torch.ones((B, H, nb), dtype=torch.float32)
+    codes = torch.zeros((B, N, H, d), dtype=torch.uint8)
+    for i in range(nb):
+        blk = x[:, i * block:(i + 1) * block]
+        amax = blk.abs().amax(dim=(1, 3))  # [B, H]
+        sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        scales[:, :, i] = sc
+        q = (blk / sc[:, None, :, None]).clamp(-448.0, 448.0)
+        codes[:, i * block:(i + 1) * block] = q.to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, scales
+
+
+def make_fp8(cfg: FixedConfig, **override) -> Fp8Inputs:
+    """The fixed-length recipe (Q, K, V drawn N(0, 1) in fp32 in that order), then each
+    tensor quantised to block-scaled E4M3 (per head, 128 tokens per block)."""
+    if override:
+        cfg = FixedConfig(**{**cfg.__dict__, **override})
+    g = torch.Generator().manual_seed(cfg.seed)
+    q = _normal(g, (cfg.B, cfg.Nq, cfg.Hq, cfg.d))
+    k = _normal(g, (cfg.B, cfg.Nk, cfg.Hkv, cfg.d))
+    v = _normal(g, (cfg.B, cfg.Nk, cfg.Hkv, cfg.d))
+    (q8, qs), (k8, ks), (v8, vs) = (_quantise_e4m3(t) for t in (q, k, v))
+    return Fp8Inputs(cfg, q8, k8, v8, qs, ks, vs)
+
+
+# The causal GQA prefill shape with E4M3 inputs (forward).
+CAUSAL_GQA_FP8 = FixedConfig("causal_gqa_fp8_b2_n8192_hq32_hkv8_d128", B=2, Hq=32, Hkv=8, Nq=8192, Nk=8192, d=128,
+                             dtype="bf16", causal=True, seed=5)

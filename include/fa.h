@@ -170,6 +170,31 @@ fa_status fa_varlen_fwd_strided(const void* q, const void* k, const void* v, voi
                                 fa_stream_t stream);
 
 /*
+ * FP8 forward: the forward of fa_fwd on E4M3 inputs with per-block scaling
+ * ("FlashAttention/zh", section "variants": FlashAttention-3's FP8 support; the
+ * algorithm is that of fa_fwd). The real inputs are
+ *     Q[b, i, h, :] = q_scale[b, h, i / 128] * e4m3(q[b, i, h, :])
+ * and likewise K, V with k_scale, v_scale [b, kv head, j / 128]: one float32
+ * dequantisation factor per 128 tokens of one head. Both products run on the
+ * tensor core's 8-bit path; the probabilities P are rounded to E4M3 before the
+ * P V product (times v_j / v_max, the block's share of the largest V factor the
+ * query tile meets, which keeps them in E4M3's range), so O carries that rounding
+ * (relative 2^-4 per weight, or 2^-10 absolute below E4M3's normal range); O is
+ * normalised by the exact sum of P, and lse is that of the exact scores.
+ *   q [B,Nq,Hq,d], k and v [B,Nk,Hkv,d]: E4M3 bytes (1 sign, 4 exponent bits
+ *       with bias 7, 3 mantissa bits; 0x7F / 0xFF are NaN), 16-byte aligned.
+ *   q_scale [B,Hq,ceil(Nq/128)], k_scale and v_scale [B,Hkv,ceil(Nk/128)]:
+ *       DEVICE float32, finite and > 0 (not checked: they live on the device).
+ *   o [B,Nq,Hq,d] bf16, lse [B,Hq,Nq] float32, as fa_fwd.
+ *   d must be 128 (FA_ERR_UNSUPPORTED). Every other argument, result and error is
+ *   that of fa_fwd.
+ */
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v,
+                     const float* q_scale, const float* k_scale, const float* v_scale,
+                     void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                     float scale, int causal, fa_stream_t stream);
+
+/*
  * Size in bytes of the caller-owned workspace fa_bwd needs: the per-row
  * D_i = sum_c dO_ic O_ic (float32 [B,Hq,Nq]) and the float32 dQ accumulator
  * (B*Hq*Nq*64 floats for d = 64; B*Hq*ceil(Nq/4)*4*128 floats for d = 128,

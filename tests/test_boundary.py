@@ -250,3 +250,23 @@ def test_decode_paged_rejects_before_launch(lib, kw, code):
 def test_decode_workspace_size_invalid(lib):
     for args in ((2, 8, 2, 1, 96), (2, 5, 2, 1, 128), (2, 8, 2, 33, 128), (0, 8, 2, 1, 128)):
         assert fb.fa_decode_workspace_size(*args) == 0
+
+
+def fp8(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, qs=FAKE, ks=FAKE, vs=FAKE, o=FAKE, lse=FAKE, B=1, Hq=4, Hkv=2, Nq=8, Nk=8,
+             d=128, scale=0.1, causal=1, stream=None)
+    a.update(kw)
+    return fb.fa_fwd_fp8(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(qs=None), fb.FA_ERR_INVALID_ARG),
+    (dict(vs=None), fb.FA_ERR_INVALID_ARG),
+    (dict(Hq=3), fb.FA_ERR_INVALID_ARG),
+    (dict(d=64), fb.FA_ERR_UNSUPPORTED),
+    (dict(ks=FAKE + 2), fb.FA_ERR_MISALIGNED),
+    (dict(q=FAKE + 8), fb.FA_ERR_MISALIGNED),
+    (dict(Nq=0), fb.FA_OK),
+])
+def test_fp8_rejects_before_launch(lib, kw, code):
+    assert fp8(**kw) == code
