@@ -152,8 +152,8 @@ fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// The instantiations: mask none / causal for every path; the sliding window for
-// fixed-length plain inputs only.
+// The instantiations: mask none / causal / sliding window for plain inputs, fixed
+// length and varlen; QK normalisation for fixed length without a window.
 template <int D, bool BF16>
 fa_status launch_fwd_b(int mask, bool varlen, bool qknorm, const CUtensorMap& mq, const CUtensorMap& mk,
                        const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
@@ -163,7 +163,8 @@ fa_status launch_fwd_b(int mask, bool varlen, bool qknorm, const CUtensorMap& mq
         return mask == C ? launch_fwd_t<D, BF16, C, false, true>(mq, mk, mv, a, grid, s)
                          : launch_fwd_t<D, BF16, N, false, true>(mq, mk, mv, a, grid, s);
     }
-    if (mask == W) return varlen ? FA_ERR_UNSUPPORTED : launch_fwd_t<D, BF16, W, false, false>(mq, mk, mv, a, grid, s);
+    if (mask == W) return varlen ? launch_fwd_t<D, BF16, W, true, false>(mq, mk, mv, a, grid, s)
+                                 : launch_fwd_t<D, BF16, W, false, false>(mq, mk, mv, a, grid, s);
     if (mask == C) return varlen ? launch_fwd_t<D, BF16, C, true, false>(mq, mk, mv, a, grid, s)
                                  : launch_fwd_t<D, BF16, C, false, false>(mq, mk, mv, a, grid, s);
     return varlen ? launch_fwd_t<D, BF16, N, true, false>(mq, mk, mv, a, grid, s)
@@ -432,7 +433,8 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
 fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
                      Strides sv, Strides so, const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
                      int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d,
-                     float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
+                     float scale, int causal, fa_dtype dtype, fa_stream_t stream, bool window = false, int wl = -1,
+                     int wr = 0) {
     if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
         return FA_ERR_INVALID_ARG;
     if (!cu_seqlens_q || !cu_seqlens_k || (total_q > 0 && (!q || !o || !lse)) || (total_k > 0 && (!k || !v)))
@@ -465,8 +467,8 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
     a.o_sb = 0;
     a.o_ss = so.s;
     a.o_sh = so.h;
-    a.wl = -1;
-    a.wr = 0;
+    a.wl = window ? wl : -1;
+    a.wr = window ? wr : 0;
     a.cu_q = cu_seqlens_q;
     a.cu_k = cu_seqlens_k;
     a.num_batches = num_seqs;
@@ -479,8 +481,8 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
     a.err = err;
     dim3 grid;
     if ((st = fwd_units(a, num_seqs, max_seqlen_q, grid)) != FA_OK) return st;
-    return launch_fwd(d, bf16, causal ? fa::kMaskCausal : fa::kMaskNone, true, false, mq, mk, mv, a, grid,
-                      reinterpret_cast<cudaStream_t>(stream));
+    return launch_fwd(d, bf16, window ? fa::kMaskWindow : (causal ? fa::kMaskCausal : fa::kMaskNone), true, false,
+                      mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // The FP8 forward (fixed length, d = 128): E4M3 q, k, v with per-block factors.
@@ -762,6 +764,31 @@ fa_status decode_common(const void* q, const void* k, const void* v, void* o, fl
                 : launch_dec_b<128, false>(rn, false, sl, paged, mq, mk, mv, a, causal, run_split, s);
 }
 
+// The backward of fa_varlen_bwd / fa_varlen_bwd_window; the masked kernels take the
+// window (wl, wr) (causal: (-1, 0)).
+fa_status varlen_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, void* workspace, const int* cu_seqlens_q,
+                     const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
+                     int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
+                     fa_stream_t stream, int wl = -1, int wr = 0) {
+    if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+        return FA_ERR_INVALID_ARG;
+    if (!cu_seqlens_q || !cu_seqlens_k || !workspace || (total_q > 0 && (!q || !o || !lse || !dout || !dq)) ||
+        (total_k > 0 && (!k || !v || !dk || !dv)))
+        return FA_ERR_INVALID_ARG;
+    fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
+    if (st != FA_OK) return st;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+        return FA_ERR_MISALIGNED;
+    if (num_seqs > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, num_seqs, cu_seqlens_q, cu_seqlens_k, total_q,
+                      total_k, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal != 0, dtype == FA_BF16,
+                      reinterpret_cast<cudaStream_t>(stream), wl, wr);
+}
+
 }  // namespace
 
 extern "C" {
@@ -895,22 +922,31 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
                         const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
                         int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
                         fa_stream_t stream) {
-    if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
-        return FA_ERR_INVALID_ARG;
-    if (!cu_seqlens_q || !cu_seqlens_k || !workspace || (total_q > 0 && (!q || !o || !lse || !dout || !dq)) ||
-        (total_k > 0 && (!k || !v || !dk || !dv)))
-        return FA_ERR_INVALID_ARG;
-    fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
-    if (st != FA_OK) return st;
-    if (d != 128) return FA_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
-        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
-        (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
-        return FA_ERR_MISALIGNED;
-    if (num_seqs > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
-    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, num_seqs, cu_seqlens_q, cu_seqlens_k, total_q,
-                      total_k, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal != 0, dtype == FA_BF16,
-                      reinterpret_cast<cudaStream_t>(stream));
+    return varlen_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q,
+                      total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream);
+}
+
+fa_status fa_varlen_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs, int total_q,
+                               int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, float scale,
+                               int window_left, int window_right, fa_dtype dtype, fa_stream_t stream) {
+    const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
+    const bool none = wl < 0 && wr < 0, causal = wl < 0 && wr == 0;
+    return fwd_varlen(q, k, v, o, lse, contiguous(total_q, Hq, d), contiguous(total_k, Hkv, d),
+                      contiguous(total_k, Hkv, d), contiguous(total_q, Hq, d), cu_seqlens_q, cu_seqlens_k, num_seqs,
+                      total_q, total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal ? 1 : 0, dtype, stream,
+                      !none && !causal, wl, wr);
+}
+
+fa_status fa_varlen_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                               const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs, int total_q,
+                               int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, float scale,
+                               int window_left, int window_right, fa_dtype dtype, fa_stream_t stream) {
+    const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
+    const bool masked = wl >= 0 || wr >= 0;
+    return varlen_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q,
+                      total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, masked ? 1 : 0, dtype, stream, wl, wr);
 }
 
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,

@@ -121,6 +121,26 @@ fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void*
                         float scale, int window_left, int window_right, fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * Sliding-window attention on packed variable-length batches: the window of
+ * fa_fwd_window / fa_bwd_window applied within every sequence (a = i + Nk_s - Nq_s
+ * with that sequence's own lengths), over the packed layout and cu_seqlens of
+ * fa_varlen_fwd / fa_varlen_bwd. Every other argument, result and error is that of
+ * fa_varlen_fwd / fa_varlen_bwd (the backward takes the lse of
+ * fa_varlen_fwd_window with the same window; d = 128 for the backward).
+ */
+fa_status fa_varlen_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                               int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                               int Hq, int Hkv, int d, float scale, int window_left, int window_right,
+                               fa_dtype dtype, fa_stream_t stream);
+fa_status fa_varlen_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                               const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                               int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                               int Hq, int Hkv, int d, float scale, int window_left, int window_right,
+                               fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Forward with the query/key RMS normalisation fused in front of attention
  * (the InternViT attention applies an RMSNorm to Q and K, per head, just
  * before its FlashAttention call): with

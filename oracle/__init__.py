@@ -202,12 +202,13 @@ def attn_bwd_sampled(q, k, v, do, scale: float, b: int, hk: int, qrows, krows,
     return (dq[b][qr][:, hk * group:(hk + 1) * group, :], dk[b, kr, hk, :], dv[b, kr, hk, :])
 
 
-def varlen_fwd(q, k, v, cu_q, cu_k, scale: float, causal: bool = False):
+def varlen_fwd(q, k, v, cu_q, cu_k, scale: float, causal: bool = False, window=None):
     """Packed variable-length forward: each sequence is an independent B=1 problem.
 
     q [total_q,Hq,d], k/v [total_k,Hkv,d]; returns O [total_q,Hq,d] and
     L [Hq,total_q]. This follows the cu_seqlens addressing of the packed path
-    on the InternViT page: sequence s owns rows cu[s] .. cu[s+1]-1.
+    on the InternViT page: sequence s owns rows cu[s] .. cu[s+1]-1. ``window``
+    applies attn_fwd's window within every sequence.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     cu_q = [int(x) for x in np.asarray(cu_q)]
@@ -220,7 +221,7 @@ def varlen_fwd(q, k, v, cu_q, cu_k, scale: float, causal: bool = False):
         ka, ke = cu_k[s], cu_k[s + 1]
         if e == a:
             continue
-        os_, ls = attn_fwd(q[None, a:e], k[None, ka:ke], v[None, ka:ke], scale, causal)
+        os_, ls = attn_fwd(q[None, a:e], k[None, ka:ke], v[None, ka:ke], scale, causal, window=window)
         o[a:e] = os_[0]
         lse[:, a:e] = ls[0]
     return o, lse

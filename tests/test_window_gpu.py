@@ -112,3 +112,61 @@ def test_window_long_sequence_sampled_rows():
     assert np.abs(lse[:, :, rows] - l_ref[:, :, rows]).max() <= ATOL_L
     ref = f64(fi.do).sum((0, 1))  # (Hq, d) -> the single KV head sums all query heads
     assert rel_l2(dv.sum((0, 1))[0], ref.sum(0)) <= RTOL_GRAD
+
+
+VARLEN_CASES = [
+    # lengths, Hq, Hkv, d, window, dtype, key_pad_frac
+    ([700, 1, 0, 300, 129], 4, 2, 128, (128, 0), "bf16", 0.0),
+    ([513, 64, 900], 2, 2, 128, (100, 50), "fp16", 0.25),
+    ([257, 1000, 5], 4, 1, 64, (-1, 40), "bf16", 0.0),
+]
+
+
+@pytest.mark.parametrize("case", VARLEN_CASES, ids=lambda c: f"{len(c[0])}seq-h{c[1]}-{c[2]}-d{c[3]}-w{c[4][0]}_{c[4][1]}")
+def test_varlen_window(case):
+    """fa_varlen_fwd_window (and, for d = 128, fa_varlen_bwd_window): every sequence
+    against the oracle with the window applied within that sequence."""
+    lengths, Hq, Hkv, d, window, dt, pad = case
+    vi = inputs.make_varlen(inputs.VARLEN, lengths=lengths, Hq=Hq, Hkv=Hkv, d=d, dtype=dt, key_pad_frac=pad,
+                            seed=87, with_do=True)
+    q, k, v, do = vi.q.cuda(), vi.k.cuda(), vi.v.cuda(), vi.do.cuda()
+    cu_q, cu_k = vi.cu_seqlens_q.cuda(), vi.cu_seqlens_k.cuda()
+    Tq, Tk, n = q.shape[0], k.shape[0], len(lengths)
+    code = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
+    o, o_ok = guarded((Tq, Hq, d), q.dtype)
+    lse, l_ok = guarded((Hq, Tq), torch.float32)
+    wl, wr = window
+    st = fb.fa_varlen_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 cu_q.data_ptr(), cu_k.data_ptr(), n, Tq, Tk, vi.max_seqlen_q, vi.max_seqlen_k, Hq,
+                                 Hkv, d, d ** -0.5, wl, wr, code, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    torch.cuda.synchronize()
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK and o_ok() and l_ok()
+    o_ref, l_ref = oracle.varlen_fwd(vi.q, vi.k, vi.v, vi.cu_seqlens_q, vi.cu_seqlens_k, d ** -0.5, window=window)
+    o64, l64 = f64(o), f64(lse)
+    empty = np.isneginf(l_ref)
+    assert np.isneginf(l64[empty]).all() and (o64.transpose(1, 0, 2)[empty] == 0).all()
+    live = ~empty
+    assert np.abs(l64[live] - l_ref[live]).max() <= ATOL_L
+    assert (np.abs(o64 - o_ref) <= o_bound(o_ref, q.dtype)).all()
+    if d != 128:
+        return
+    ws = torch.empty(fb.fa_varlen_bwd_workspace_size(n, Tq, vi.max_seqlen_q, Hq, d), dtype=torch.uint8, device="cuda")
+    dq, dk, dv = torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)
+    st = fb.fa_varlen_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                                 cu_q.data_ptr(), cu_k.data_ptr(), n, Tq, Tk, vi.max_seqlen_q, vi.max_seqlen_k, Hq,
+                                 Hkv, d, d ** -0.5, wl, wr, code, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    torch.cuda.synchronize()
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    refs = [np.zeros(tuple(t.shape)) for t in (vi.q, vi.k, vi.v)]
+    for s, (Lq, Lk) in enumerate(zip(vi.seqlens_q, vi.seqlens_k)):
+        a, ka = int(vi.cu_seqlens_q[s]), int(vi.cu_seqlens_k[s])
+        if Lq == 0 and Lk == 0:
+            continue
+        rq, rk, rv = oracle.attn_bwd(vi.q[None, a:a + Lq], vi.k[None, ka:ka + Lk], vi.v[None, ka:ka + Lk],
+                                     vi.do[None, a:a + Lq], d ** -0.5, window=window)
+        refs[0][a:a + Lq], refs[1][ka:ka + Lk], refs[2][ka:ka + Lk] = rq[0], rk[0], rv[0]
+    errs = [rel_l2(f64(g), r) for g, r in zip((dq, dk, dv), refs)]
+    assert max(errs) <= RTOL_GRAD, errs
