@@ -55,18 +55,20 @@ def _load():
         lib = ctypes.CDLL(build())
         lib.ora_attn_fwd.restype = ctypes.c_int
         lib.ora_attn_fwd.argtypes = [_dp, _dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
-                                                                            ctypes.c_int, _up, _ip, ctypes.c_int,
-                                                                            _dp, _dp]
+                                                                            ctypes.c_int, ctypes.c_int, _up, _ip,
+                                                                            ctypes.c_int, _dp, _dp]
         lib.ora_attn_probs.restype = ctypes.c_int
         lib.ora_attn_probs.argtypes = [_dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
-                                                                         ctypes.c_int, _up, ctypes.c_int,
-                                                                         ctypes.c_int, _dp]
+                                                                         ctypes.c_int, ctypes.c_int, _up,
+                                                                         ctypes.c_int, ctypes.c_int, _dp]
         lib.ora_attn_bwd.restype = ctypes.c_int
         lib.ora_attn_bwd.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
-                                                                                 ctypes.c_int, _up, _dp, _dp, _dp]
+                                                                                 ctypes.c_int, ctypes.c_int, _up,
+                                                                                 _dp, _dp, _dp]
         lib.ora_attn_bwd_sampled.restype = ctypes.c_int
         lib.ora_attn_bwd_sampled.argtypes = ([_dp, _dp, _dp, _dp] + [ctypes.c_int] * 6 +
-                                             [ctypes.c_double, ctypes.c_int, ctypes.c_int, _up, ctypes.c_int,
+                                             [ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, _up,
+                                              ctypes.c_int,
                                               ctypes.c_int,
                                               _ip, ctypes.c_int, _ip, ctypes.c_int, _dp, _dp, _dp])
         lib.ora_num_threads.restype = ctypes.c_int
@@ -75,12 +77,16 @@ def _load():
 
 
 def _window(causal, window):
-    """(wl, wr) of the C oracle: keys visible to query i are those within wl before
-    and wr after its bottom-right-aligned key; a negative side is unbounded."""
+    """(wl, wr, na) of the C oracle: keys visible to query i are those within wl
+    before and wr after its bottom-right-aligned key (a negative side is
+    unbounded), and below the window also the global anchor keys 0 .. na - 1
+    (``window`` = (wl, wr) or (wl, wr, n_anchor))."""
     if window is not None:
-        wl, wr = (int(x) for x in window)
-        return (wl if wl >= 0 else -1), (wr if wr >= 0 else -1)
-    return (-1, 0) if causal else (-1, -1)
+        w = [int(x) for x in window]
+        wl, wr = w[0], w[1]
+        na = w[2] if len(w) > 2 else 0
+        return (wl if wl >= 0 else -1), (wr if wr >= 0 else -1), max(na, 0)
+    return (-1, 0, 0) if causal else (-1, -1, 0)
 
 
 def num_threads() -> int:

@@ -30,7 +30,7 @@
  * h / (Hq/Hkv). Masking: with a = i + (Nk - Nq) (bottom-right alignment),
  * key j is visible to query i iff
  *     key_keep == NULL or key_keep[b*Nk + j] != 0, and
- *     wl < 0 or j >= a - wl, and
+ *     wl < 0 or j >= a - wl or j < na (global anchor keys), and
  *     wr < 0 or j <= a + wr.
  * (wl, wr) is a sliding window of wl keys before and wr keys after the
  * aligned key; a negative side is unbounded. The causal mask is
@@ -45,10 +45,10 @@
 #include <omp.h>
 #endif
 
-static int visible(const unsigned char* key_keep, int b, int Nq, int Nk, int wl, int wr, int i, int j) {
+static int visible(const unsigned char* key_keep, int b, int Nq, int Nk, int wl, int wr, int na, int i, int j) {
     if (key_keep && !key_keep[(long)b * Nk + j]) return 0;
     const long a = (long)i + (long)(Nk - Nq);
-    if (wl >= 0 && (long)j < a - wl) return 0;
+    if (wl >= 0 && (long)j < a - wl && j >= na) return 0;
     if (wr >= 0 && (long)j > a + wr) return 0;
     return 1;
 }
@@ -62,11 +62,11 @@ static double dot(const double* a, const double* b, int d) {
 /* Probabilities of one query row: fills p[0..Nk) and returns m and l through
  * pointers. Returns 0 if the row has no visible key (p is all zero then). */
 static int softmax_row(const double* qi, const double* kbase, long kstride, int Nk, int d,
-                       double scale, const unsigned char* key_keep, int b, int Nq, int wl, int wr,
+                       double scale, const unsigned char* key_keep, int b, int Nq, int wl, int wr, int na,
                        int i, double* s, double* p, double* m_out, double* l_out) {
     double m = -INFINITY;
     for (int j = 0; j < Nk; ++j) {
-        if (visible(key_keep, b, Nq, Nk, wl, wr, i, j)) {
+        if (visible(key_keep, b, Nq, Nk, wl, wr, na, i, j)) {
             s[j] = scale * dot(qi, kbase + (long)j * kstride, d);
             if (s[j] > m) m = s[j];
         } else {
@@ -101,7 +101,7 @@ int ora_num_threads(void) {
 /* Forward. rows == NULL computes every query row; otherwise only the nrows
  * listed query indices (for every batch and head) are written to o and lse. */
 int ora_attn_fwd(const double* q, const double* k, const double* v, int B, int Hq, int Hkv,
-                 int Nq, int Nk, int d, double scale, int wl, int wr,
+                 int Nq, int Nk, int d, double scale, int wl, int wr, int na,
                  const unsigned char* key_keep, const int* rows, int nrows,
                  double* o, double* lse) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Nq < 0 || Nk < 0 || d <= 0) return 1;
@@ -131,7 +131,7 @@ int ora_attn_fwd(const double* q, const double* k, const double* v, int B, int H
             double m, l;
             double* oi = o + (((long)b * Nq + i) * Hq + h) * d;
             for (int c = 0; c < d; ++c) oi[c] = 0.0;
-            if (softmax_row(qi, kb, kvs, Nk, d, scale, key_keep, b, Nq, wl, wr, i, s, p, &m, &l)) {
+            if (softmax_row(qi, kb, kvs, Nk, d, scale, key_keep, b, Nq, wl, wr, na, i, s, p, &m, &l)) {
                 for (int j = 0; j < Nk; ++j) {
                     if (p[j] == 0.0) continue;
                     const double* vj = vb + (long)j * kvs;
@@ -150,7 +150,7 @@ int ora_attn_fwd(const double* q, const double* k, const double* v, int B, int H
 
 /* The probability matrix P of one (batch, query head), Nq x Nk, row-major. */
 int ora_attn_probs(const double* q, const double* k, int B, int Hq, int Hkv, int Nq, int Nk,
-                   int d, double scale, int wl, int wr, const unsigned char* key_keep, int b, int h,
+                   int d, double scale, int wl, int wr, int na, const unsigned char* key_keep, int b, int h,
                    double* P) {
     if (b < 0 || b >= B || h < 0 || h >= Hq || Hq % Hkv) return 1;
     const int hk = h / (Hq / Hkv);
@@ -159,7 +159,7 @@ int ora_attn_probs(const double* q, const double* k, int B, int Hq, int Hkv, int
     for (int i = 0; i < Nq; ++i) {
         double m, l;
         softmax_row(q + (((long)b * Nq + i) * Hq + h) * d, k + ((long)b * Nk * Hkv + hk) * d,
-                    (long)Hkv * d, Nk, d, scale, key_keep, b, Nq, wl, wr, i, s, P + (long)i * Nk,
+                    (long)Hkv * d, Nk, d, scale, key_keep, b, Nq, wl, wr, na, i, s, P + (long)i * Nk,
                     &m, &l);
     }
     free(s);
@@ -173,7 +173,7 @@ int ora_attn_probs(const double* q, const double* k, int B, int Hq, int Hkv, int
  * that can see none of the listed keys are skipped, which is exact because
  * they add nothing to those keys' gradients. */
 static int bwd_group(const double* q, const double* k, const double* v, const double* dout,
-                     int Nq, int Nk, int Hq, int Hkv, int d, double scale, int wl, int wr,
+                     int Nq, int Nk, int Hq, int Hkv, int d, double scale, int wl, int wr, int na,
                      const unsigned char* key_keep, int b, int hk, const int* qrows, int nq,
                      const int* krows, int nk, double* dq, double* dk, double* dv) {
     const int group = Hq / Hkv;
@@ -198,13 +198,13 @@ static int bwd_group(const double* q, const double* k, const double* v, const do
             if (krows) {
                 needed = want_q[i];
                 for (int t = 0; t < nk && !needed; ++t)
-                    needed = visible(key_keep, b, Nq, Nk, wl, wr, i, krows[t]);
+                    needed = visible(key_keep, b, Nq, Nk, wl, wr, na, i, krows[t]);
             }
             if (!needed) continue;
             const double* qi = q + ((long)b * Nq + i) * qs + (long)h * d;
             const double* doi = dout + ((long)b * Nq + i) * qs + (long)h * d;
             double m, l;
-            if (!softmax_row(qi, kb, kvs, Nk, d, scale, key_keep, b, Nq, wl, wr, i, s, p, &m, &l))
+            if (!softmax_row(qi, kb, kvs, Nk, d, scale, key_keep, b, Nq, wl, wr, na, i, s, p, &m, &l))
                 continue; /* no visible key: every gradient term of this row is 0 */
             double D = 0.0;
             for (int j = 0; j < Nk; ++j) {
@@ -241,7 +241,7 @@ static int bwd_group(const double* q, const double* k, const double* v, const do
 
 /* Full backward: dq [B,Nq,Hq,d], dk and dv [B,Nk,Hkv,d] (overwritten). */
 int ora_attn_bwd(const double* q, const double* k, const double* v, const double* dout, int B,
-                 int Hq, int Hkv, int Nq, int Nk, int d, double scale, int wl, int wr,
+                 int Hq, int Hkv, int Nq, int Nk, int d, double scale, int wl, int wr, int na,
                  const unsigned char* key_keep, double* dq, double* dk, double* dv) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Nq < 0 || Nk < 0 || d <= 0) return 1;
     memset(dq, 0, sizeof(double) * (size_t)B * Nq * Hq * d);
@@ -250,7 +250,7 @@ int ora_attn_bwd(const double* q, const double* k, const double* v, const double
     int err = 0;
 #pragma omp parallel for schedule(dynamic, 1)
     for (long t = 0; t < (long)B * Hkv; ++t) {
-        int e = bwd_group(q, k, v, dout, Nq, Nk, Hq, Hkv, d, scale, wl, wr, key_keep,
+        int e = bwd_group(q, k, v, dout, Nq, Nk, Hq, Hkv, d, scale, wl, wr, na, key_keep,
                           (int)(t / Hkv), (int)(t % Hkv), NULL, 0, NULL, 0, dq, dk, dv);
         if (e) {
 #pragma omp atomic write
@@ -266,7 +266,7 @@ int ora_attn_bwd(const double* q, const double* k, const double* v, const double
  * are written (dk/dv rows are overwritten, not accumulated). Parallel over
  * the sampled key rows is not needed: one call is one group. */
 int ora_attn_bwd_sampled(const double* q, const double* k, const double* v, const double* dout,
-                         int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, int wl, int wr,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, int wl, int wr, int na,
                          const unsigned char* key_keep, int b, int hk, const int* qrows, int nq,
                          const int* krows, int nk, double* dq, double* dk, double* dv) {
     if (b < 0 || b >= B || hk < 0 || hk >= Hkv || Hq % Hkv) return 1;
@@ -278,6 +278,6 @@ int ora_attn_bwd_sampled(const double* q, const double* k, const double* v, cons
     /* Split the group's query heads across threads would race on dk/dv; the
      * speed comes from the caller sampling few rows, so this runs serially
      * per group and callers may run several groups in parallel processes. */
-    return bwd_group(q, k, v, dout, Nq, Nk, Hq, Hkv, d, scale, wl, wr, key_keep, b, hk, qrows,
+    return bwd_group(q, k, v, dout, Nq, Nk, Hq, Hkv, d, scale, wl, wr, na, key_keep, b, hk, qrows,
                      nq, krows, nk ? nk : 0, dq, dk, dv);
 }

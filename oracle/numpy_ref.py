@@ -16,13 +16,15 @@ import numpy as np
 def _mask(Nq, Nk, causal, keep_row, window=None):
     """Allowed (query, key) pairs. A window (wl, wr) allows the keys from wl
     before to wr after the bottom-right-aligned diagonal (a negative side is
-    unbounded); it replaces `causal`, which is the window (-1, 0)."""
+    unbounded); it replaces `causal`, which is the window (-1, 0). A third entry
+    n_anchor also allows keys 0 .. n_anchor - 1 below the window (global anchors)."""
     allowed = np.ones((Nq, Nk), dtype=bool)
     diag = np.arange(Nk)[None, :] - np.arange(Nq)[:, None] - (Nk - Nq)  # key offset from the aligned diagonal
     if window is not None:
-        wl, wr = window
+        wl, wr = window[0], window[1]
+        anchor = np.arange(Nk)[None, :] < (window[2] if len(window) > 2 else 0)  # global anchor keys
         if wl >= 0:
-            allowed &= diag >= -wl
+            allowed &= (diag >= -wl) | anchor
         if wr >= 0:
             allowed &= diag <= wr
     elif causal:

@@ -331,7 +331,7 @@ def test_rms_normalise_pins():
     assert (np.abs(yb.double().numpy() - exact) <= np.abs(exact) * 2.0 ** -8 + 1e-30).all()
 
 
-WINDOWS = [(2, 1), (0, 3), (5, 0), (-1, 2), (3, -1), (0, 0)]
+WINDOWS = [(2, 1), (0, 3), (5, 0), (-1, 2), (3, -1), (0, 0), (1, 0, 2), (2, 1, 3), (0, -1, 1), (2, 0, 20)]
 
 
 @pytest.mark.parametrize("window", WINDOWS)
@@ -376,10 +376,11 @@ def test_window_special_cases():
                 assert (o[0, i, h] == 0).all() and np.isneginf(lse[0, h, i])
 
 
-def test_window_backward_matches_finite_differences():
+@pytest.mark.parametrize("window", [(2, 1), (1, 0, 3)])
+def test_window_backward_matches_finite_differences(window):
     rng = np.random.default_rng(23)
     q, k, v, do = _rand(rng, 1, 6, 2, 3), _rand(rng, 1, 8, 1, 3), _rand(rng, 1, 8, 1, 3), _rand(rng, 1, 6, 2, 3)
-    window, scale = (2, 1), 0.6
+    scale = 0.6
     grads = oracle.attn_bwd(q, k, v, do, scale, window=window)
 
     def phi(qq, kk, vv):
@@ -538,3 +539,28 @@ def test_varlen_window_equals_numpy_per_sequence():
             o2, l2 = numpy_ref.fwd(f(vi.q), f(vi.k), f(vi.v), 0.4, window=window)
             np.testing.assert_allclose(o[a:a + n], o2[0], atol=1e-12)
             np.testing.assert_allclose(lse[:, a:a + n], l2[0], atol=1e-12)
+
+
+def test_anchor_special_cases():
+    """Global anchors: n_anchor = 0 is the plain window; with an unbounded left side
+    anchors add nothing; anchors covering every key with an unbounded right side give
+    full attention; with the causal right bound (wr = 0) and a zero-width window, row i
+    sees exactly keys {0 .. n_anchor - 1} u {a} below its aligned key a, checked against
+    a direct softmax over those keys."""
+    rng = np.random.default_rng(29)
+    Nq, Nk = 9, 9
+    q, k, v = _rand(rng, 1, Nq, 2, 3), _rand(rng, 1, Nk, 1, 3), _rand(rng, 1, Nk, 1, 3)
+    for a, b in zip(oracle.attn_fwd(q, k, v, 0.5, window=(2, 1, 0)), oracle.attn_fwd(q, k, v, 0.5, window=(2, 1))):
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(oracle.attn_fwd(q, k, v, 0.5, window=(-1, 0, 4)), oracle.attn_fwd(q, k, v, 0.5, causal=True)):
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(oracle.attn_fwd(q, k, v, 0.5, window=(0, -1, Nk)), oracle.attn_fwd(q, k, v, 0.5)):
+        np.testing.assert_array_equal(a, b)
+    o, lse = oracle.attn_fwd(q, k, v, 0.5, window=(0, 0, 3))
+    for i in range(Nq):
+        keys = sorted(set(range(min(3, i + 1))) | {i})
+        for h in range(2):
+            s_ = np.array([0.5 * float(q[0, i, h] @ k[0, j, 0]) for j in keys])
+            w = np.exp(s_ - s_.max())
+            np.testing.assert_allclose(o[0, i, h], (w / w.sum()) @ v[0, keys, 0], atol=1e-14)
+            assert abs(lse[0, h, i] - (s_.max() + math.log(w.sum()))) <= 1e-13
