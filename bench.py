@@ -511,6 +511,27 @@ def run_sweep(args):
     emit(cfg.name + "_window1024", "fwd", time_it(wfwd, 30), wflops, nb)
     emit(cfg.name + "_window1024", "bwd", time_it(wbwd, 20), 2.5 * wflops,
          nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+    # the same window plus 4 global anchor keys (the first tokens, visible to every query)
+    na = 4
+    apairs = pairs + sum(max(0, min(na, i - wl)) for i in range(N))
+    aflops = 4.0 * d * apairs * B * Hq
+
+    def afwd():
+        r = fb.fa_fwd_window_anchor(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq,
+                                    Hkv, N, N, d, cfg.scale, wl, wr, na, fb.FA_BF16, stream.cuda_stream)
+        if r != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(r))
+
+    def abwd():
+        r = fb.fa_bwd_window_anchor(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                    do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq,
+                                    Hkv, N, N, d, cfg.scale, wl, wr, na, fb.FA_BF16, stream.cuda_stream)
+        if r != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(r))
+
+    emit(cfg.name + "_window1024_anchor4", "fwd", time_it(afwd, 30), aflops, nb)
+    emit(cfg.name + "_window1024_anchor4", "bwd", time_it(abwd, 20), 2.5 * aflops,
+         nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
     del q, k, v, do, o, lse, dq, dk, dv, ws
     # the ViT workload through the packed-QKV layout (B, S, 3, H, d), O written as (B, H, S, d)
     cfg = inputs.VIT_RMSNORM

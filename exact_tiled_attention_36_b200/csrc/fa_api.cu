@@ -153,11 +153,12 @@ fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 }
 
 // The instantiations: mask none / causal / sliding window for plain inputs, fixed
-// length and varlen; QK normalisation for fixed length without a window.
+// length and varlen; the window with global anchors for fixed length; QK
+// normalisation for fixed length without a window.
 template <int D, bool BF16>
 fa_status launch_fwd_b(int mask, bool varlen, bool qknorm, const CUtensorMap& mq, const CUtensorMap& mk,
                        const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
-    constexpr int N = fa::kMaskNone, C = fa::kMaskCausal, W = fa::kMaskWindow;
+    constexpr int N = fa::kMaskNone, C = fa::kMaskCausal, W = fa::kMaskWindow, A = fa::kMaskAnchor;
     if (qknorm) {
         if (varlen || mask == W) return FA_ERR_UNSUPPORTED;
         return mask == C ? launch_fwd_t<D, BF16, C, false, true>(mq, mk, mv, a, grid, s)
@@ -165,6 +166,7 @@ fa_status launch_fwd_b(int mask, bool varlen, bool qknorm, const CUtensorMap& mq
     }
     if (mask == W) return varlen ? launch_fwd_t<D, BF16, W, true, false>(mq, mk, mv, a, grid, s)
                                  : launch_fwd_t<D, BF16, W, false, false>(mq, mk, mv, a, grid, s);
+    if (mask == A) return varlen ? FA_ERR_UNSUPPORTED : launch_fwd_t<D, BF16, A, false, false>(mq, mk, mv, a, grid, s);
     if (mask == C) return varlen ? launch_fwd_t<D, BF16, C, true, false>(mq, mk, mv, a, grid, s)
                                  : launch_fwd_t<D, BF16, C, false, false>(mq, mk, mv, a, grid, s);
     return varlen ? launch_fwd_t<D, BF16, N, true, false>(mq, mk, mv, a, grid, s)
@@ -254,7 +256,8 @@ size_t acc_floats(int B, int Hq, int Nq, int d) {
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dout, void* dq, void* dk, void* dv, void* workspace, int nseq, const int* cu_q,
                      const int* cu_k, int total_q, int total_k, int Hq, int Hkv, int Nq, int Nk, int d,
-                     float scale, bool causal, bool bf16, cudaStream_t s, int wl = -1, int wr = 0) {
+                     float scale, bool causal, bool bf16, cudaStream_t s, int wl = -1, int wr = 0,
+                     int n_anchor = 0) {
     const bool varlen = cu_q != nullptr;
     int* err = error_word();
     if (!err) return FA_ERR_CUDA;
@@ -306,6 +309,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         a.scale_log2 = scale * kLog2e;
         a.wl = wl;
         a.wr = wr;
+        a.n_anchor = n_anchor;
         a.err = err;
         const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
         if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
@@ -390,7 +394,8 @@ fa_status check_strides(const Strides& t, bool with_batch) {
 fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, Strides sq, Strides sk,
                     Strides sv, Strides so, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                     fa_dtype dtype, fa_stream_t stream, bool qknorm = false, float eps = 0.f,
-                    bool validate_only = false, bool window = false, int wl = -1, int wr = 0) {
+                    bool validate_only = false, bool window = false, int wl = -1, int wr = 0,
+                    int n_anchor = 0) {
     if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if ((Nq > 0 && (!q || !o || !lse)) || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
     fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
@@ -416,6 +421,7 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
     a.o_sh = so.h;
     a.wl = wl;
     a.wr = wr;
+    a.n_anchor = n_anchor;
     a.num_batches = B;
     a.Hq = Hq;
     a.group = Hq / Hkv;
@@ -426,7 +432,8 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
     a.err = err;
     dim3 grid;
     if ((st = fwd_units(a, B, Nq, grid)) != FA_OK) return st;
-    const int mask = window ? fa::kMaskWindow : (causal ? fa::kMaskCausal : fa::kMaskNone);
+    const int mask = window ? (n_anchor > 0 ? fa::kMaskAnchor : fa::kMaskWindow)
+                            : (causal ? fa::kMaskCausal : fa::kMaskNone);
     return launch_fwd(d, bf16, mask, false, qknorm, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -846,6 +853,18 @@ fa_status fa_fwd_window(const void* q, const void* k, const void* v, void* o, fl
                      false, !none && !causal, wl, wr);
 }
 
+fa_status fa_fwd_window_anchor(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                               int Hkv, int Nq, int Nk, int d, float scale, int window_left, int window_right,
+                               int n_anchor, fa_dtype dtype, fa_stream_t stream) {
+    if (n_anchor < 0) return FA_ERR_INVALID_ARG;
+    const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
+    if (n_anchor == 0 || wl < 0)  // no anchors, or nothing below the window to add
+        return fa_fwd_window(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, wl, wr, dtype, stream);
+    return fwd_fixed(q, k, v, o, lse, contiguous(Nq, Hq, d), contiguous(Nk, Hkv, d), contiguous(Nk, Hkv, d),
+                     contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, 0, dtype, stream, false, 0.f, false, true,
+                     wl, wr, n_anchor);
+}
+
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
                          const long long* q_strides, const long long* k_strides, const long long* v_strides,
                          const long long* o_strides, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
@@ -909,6 +928,21 @@ fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void*
     if (st != FA_OK) return st;
     return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
                       scale, masked, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream), wl, wr);
+}
+
+fa_status fa_bwd_window_anchor(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int Hq,
+                               int Hkv, int Nq, int Nk, int d, float scale, int window_left, int window_right,
+                               int n_anchor, fa_dtype dtype, fa_stream_t stream) {
+    if (n_anchor < 0) return FA_ERR_INVALID_ARG;
+    const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
+    const bool masked = wl >= 0 || wr >= 0;
+    const fa_status st = bwd_checks(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale,
+                                    masked ? 1 : 0, dtype);
+    if (st != FA_OK) return st;
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
+                      scale, masked, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream), wl, wr,
+                      wl >= 0 ? n_anchor : 0);
 }
 
 size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q, int Hq, int d) {

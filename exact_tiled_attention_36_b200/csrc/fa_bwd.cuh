@@ -55,11 +55,13 @@ struct BwdArgs {
     float scale;
     float scale_log2;
     int wl, wr;  // MASKED: keys from wl before to wr after the aligned diagonal (< 0: unbounded)
+    int n_anchor;  // MASKED: keys 0 .. n_anchor - 1 are also visible below the window (global anchors)
     int* err;
 };
 
 // Queries [qlo, qhi) that see key `key` (bottom-right alignment: query q's aligned
 // key is q + Nk - Nq; with MASKED the window (wl, wr) of BwdArgs, else every query).
+// An anchor key (key < n_anchor) is seen by every query its right bound allows.
 template <bool MASKED>
 __device__ __forceinline__ void query_range(const BwdArgs& a, int key, int Nq, int Nk, int& qlo, int& qhi) {
     qlo = 0;
@@ -67,7 +69,7 @@ __device__ __forceinline__ void query_range(const BwdArgs& a, int key, int Nq, i
     if (MASKED) {
         const int q_aligned = key - (Nk - Nq);
         if (a.wr >= 0) qlo = max(0, q_aligned - a.wr);
-        if (a.wl >= 0) qhi = min(Nq, q_aligned + a.wl + 1);
+        if (a.wl >= 0 && key >= a.n_anchor) qhi = min(Nq, q_aligned + a.wl + 1);
     }
 }
 
@@ -77,6 +79,7 @@ __device__ __forceinline__ void query_tiles(const BwdArgs& a, int k0, int Nq, in
     int qlo, qhi, qlo2, qhi2;
     query_range<MASKED>(a, k0, Nq, Nk, qlo, qhi);
     query_range<MASKED>(a, min(k0 + 127, Nk - 1), Nq, Nk, qlo2, qhi2);
+    qhi2 = max(qhi, qhi2);  // an anchor first key sees further than the tile's last key
     i0 = qlo / 128;
     const int i_end = qhi2 > qlo ? (qhi2 + 127) / 128 : i0;
     n_i = i_end - i0;

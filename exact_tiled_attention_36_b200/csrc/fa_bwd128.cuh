@@ -311,9 +311,13 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         int qlim, qlim_hi;  // queries [qlim, qlim_hi) see this key
         query_range<CAUSAL>(args, key, Nq, Nk, qlim, qlim_hi);
         // Every key of the tile sees queries [qall_lo, qall_hi): slices inside need no mask.
+        // qlo grows with the key, so the last key's is the largest; qhi grows too except
+        // that anchor keys see every later query, so the smallest is that of the tile's
+        // first key that is not an anchor (its first key if none is).
         int qall_lo, qdummy, qdummy2, qall_hi;
-        query_range<CAUSAL>(args, min(k0 + 127, Nk - 1), Nq, Nk, qall_lo, qdummy);
-        query_range<CAUSAL>(args, k0, Nq, Nk, qdummy2, qall_hi);
+        const int k_last = min(k0 + 127, Nk - 1);
+        query_range<CAUSAL>(args, k_last, Nq, Nk, qall_lo, qdummy);
+        query_range<CAUSAL>(args, min(max(k0, args.n_anchor), k_last), Nq, Nk, qdummy2, qall_hi);
         const float sl2 = args.scale_log2;
         constexpr float kLog2eF = 1.4426950408889634074f;
         // -L log2 e and -D of query 64 w + r of iteration it_, loaded one iteration

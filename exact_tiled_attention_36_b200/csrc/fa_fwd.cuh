@@ -65,6 +65,7 @@ struct FwdArgs {
     int Nk;
     long long o_sb, o_ss, o_sh;  // O strides in elements: batch, token, head (d is contiguous)
     int wl, wr;       // MASKED: keys from wl before to wr after the aligned diagonal (< 0: unbounded)
+    int n_anchor;     // kMaskAnchor: keys 0 .. n_anchor - 1 are visible below the window too
     int nu;           // units (256 query rows) per sequence: ceil(Nq / 256)
     int n_units;      // nu * Hq * num_batches
     float scale_log2;  // scale * log2(e)
@@ -115,13 +116,22 @@ struct FwdUnit {
     int jlo, n_kv;       // the unit walks key tiles jlo .. jlo + n_kv - 1 (steps 0 .. n_kv - 1)
     int a0, b0, a1, b1;  // query tile t is active on steps a_t .. b_t - 1 (none if a_t == b_t)
     bool rows;           // the unit holds at least one query row
+    // kMaskAnchor: the walk is the anchor tiles 0 .. na - 1, then window tiles from jw
+    // (step s >= na is tile jw + s - na); query tile t sees anchor tiles 0 .. ta_t - 1
+    // and its window's tiles [jl_t, jh_t).
+    int na, jw, ta0, ta1, jl0, jh0, jl1, jh1;
     __device__ __forceinline__ int a(int t) const { return t ? a1 : a0; }
     __device__ __forceinline__ int b(int t) const { return t ? b1 : b0; }
+    __device__ __forceinline__ int ta(int t) const { return t ? ta1 : ta0; }
+    __device__ __forceinline__ int jl(int t) const { return t ? jl1 : jl0; }
+    __device__ __forceinline__ int jh(int t) const { return t ? jh1 : jh0; }
 };
 
 // Mask kinds of the forward: none, causal (the window (-1, 0), fixed at compile
-// time), or the sliding window (wl, wr) of FwdArgs.
-enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2 };
+// time), the sliding window (wl, wr) of FwdArgs, or that window plus the global
+// anchor keys 0 .. n_anchor - 1 (visible to a query whenever the window's right
+// bound allows them).
+enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2, kMaskAnchor = 3 };
 
 // First visible key and one past the last for query q (bottom-right alignment).
 template <int MASK>
@@ -130,7 +140,7 @@ __device__ __forceinline__ void key_range(const FwdArgs& a, int q, int q_len, in
     hi = k_len;
     const int aligned = q + k_len - q_len;
     if (MASK == kMaskCausal) hi = min(k_len, aligned + 1);
-    if (MASK == kMaskWindow) {
+    if (MASK == kMaskWindow || MASK == kMaskAnchor) {
         if (a.wl >= 0) lo = max(0, aligned - a.wl);
         if (a.wr >= 0) hi = min(k_len, aligned + a.wr + 1);
     }
@@ -181,6 +191,31 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdArgs& a) {
     int jl0, jh0, jl1, jh1;
     tiles(w.q0, jl0, jh0);
     tiles(w.q0 + 128, jl1, jh1);
+    if constexpr (MASK == kMaskAnchor) {
+        // Anchor tiles of query tile t: keys below n_anchor and below the largest
+        // right bound of its rows (its last row's).
+        auto anchors = [&](int qt) -> int {
+            if (qt >= w.q_len) return 0;
+            int lo, hi;
+            key_range<MASK>(a, min(qt + 127, w.q_len - 1), w.q_len, w.k_len, lo, hi);
+            return (min(a.n_anchor, hi) + 127) / 128;
+        };
+        w.ta0 = anchors(w.q0);
+        w.ta1 = anchors(w.q0 + 128);
+        w.jl0 = jl0;
+        w.jh0 = jh0;
+        w.jl1 = jl1;
+        w.jh1 = jh1;
+        w.na = max(w.ta0, w.ta1);
+        const bool f0 = jh0 == jl0, f1 = jh1 == jl1;
+        const int wlo = f0 ? jl1 : (f1 ? jl0 : min(jl0, jl1));
+        const int whi = f0 ? jh1 : (f1 ? jh0 : max(jh0, jh1));
+        w.jw = max(w.na, wlo);
+        w.jlo = 0;
+        w.n_kv = w.na + max(0, whi - w.jw);
+        w.a0 = w.b0 = w.a1 = w.b1 = 0;
+        return w;
+    }
     const bool e0 = jh0 == jl0, e1 = jh1 == jl1;
     w.jlo = e0 ? jl1 : (e1 ? jl0 : min(jl0, jl1));
     const int jhi = e0 ? jh1 : (e1 ? jh0 : max(jh0, jh1));
@@ -190,6 +225,36 @@ __device__ __forceinline__ FwdUnit fwd_unit(int u, const FwdArgs& a) {
     w.a1 = e1 ? 0 : jl1 - w.jlo;
     w.b1 = e1 ? 0 : jh1 - w.jlo;
     return w;
+}
+
+// Key tile of step s of the unit's walk.
+template <int MASK>
+__device__ __forceinline__ int fwd_tile(const FwdUnit& w, int s) {
+    if constexpr (MASK == kMaskAnchor) return s < w.na ? s : w.jw + s - w.na;
+    return w.jlo + s;
+}
+
+// Query tile t takes part in step s of the walk.
+template <int MASK>
+__device__ __forceinline__ bool fwd_active(const FwdUnit& w, int t, int s) {
+    if constexpr (MASK == kMaskAnchor) {
+        const int kt = fwd_tile<MASK>(w, s);
+        return kt < w.ta(t) || (kt >= w.jl(t) && kt < w.jh(t));
+    }
+    return s >= w.a(t) && s < w.b(t);
+}
+
+// Number of steps query tile t takes part in, and the key tile of its j-th (anchor
+// tiles first, then the window's tiles past them).
+template <int MASK>
+__device__ __forceinline__ int fwd_tile_steps(const FwdUnit& w, int t) {
+    if constexpr (MASK == kMaskAnchor) return w.ta(t) + max(0, w.jh(t) - max(w.jl(t), w.ta(t)));
+    return w.b(t) - w.a(t);
+}
+template <int MASK>
+__device__ __forceinline__ int fwd_tile_of(const FwdUnit& w, int t, int j) {
+    if constexpr (MASK == kMaskAnchor) return j < w.ta(t) ? j : max(w.jl(t), w.ta(t)) + j - w.ta(t);
+    return w.jlo + w.a(t) + j;
 }
 
 // Unit of round k for CTA c of G: the direction alternates every round.
@@ -257,7 +322,7 @@ template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM, bool FP8 = false
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
-    static_assert(!FP8 || (D == 128 && BF16 && !VARLEN && !QKNORM && MASK != kMaskWindow), "FP8 forward shape");
+    static_assert(!FP8 || (D == 128 && BF16 && !VARLEN && !QKNORM && MASK <= kMaskCausal), "FP8 forward shape");
     using C = FwdCfg<D, FP8>;
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -363,14 +428,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
                         tma_load_4d(sK + st * C::kTileBytes + s * C::kSlabBytes, &tm_k, &k_full[st], s * C::kSlabElems, hk,
-                                    w.k_row0 + (w.jlo + j) * 128, w.tma_b);
+                                    w.k_row0 + fwd_tile<MASK>(w, j) * 128, w.tma_b);
                     ++k_issued;
                     if (!(ok = mbar_wait(&v_empty[st], ph ^ 1u, wc, 62))) break;
                     mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
 #pragma unroll
                     for (int s = 0; s < C::kSlabs; ++s)
                         tma_load_4d(sV + st * C::kTileBytes + s * C::kSlabBytes, &tm_v, &v_full[st], s * C::kSlabElems, hk,
-                                    w.k_row0 + (w.jlo + j) * 128, w.tma_b);
+                                    w.k_row0 + fwd_tile<MASK>(w, j) * 128, w.tma_b);
                     ++v_issued;
                 }
             }
@@ -416,7 +481,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 // The first S products of this unit run while the softmax warpgroups
                 // still write the previous unit's O (they touch only the S columns).
                 for (int t = 0; t < 2; ++t)
-                    if (w.a(t) == 0 && w.b(t) > 0) issue_s(t, gk);
+                    if (MASK == kMaskAnchor ? fwd_active<MASK>(w, t, 0) : (w.a(t) == 0 && w.b(t) > 0)) issue_s(t, gk);
+                bool started0 = false, started1 = false;  // kMaskAnchor: tile t's first P V is issued
                 if (w.n_kv == 1) tc_commit(q_empty);
                 tc_commit(&k_empty[gk % S]);
                 for (int j = 0; ok && j < w.n_kv; ++j) {
@@ -434,14 +500,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         // unit's epilogue must have read it (waited for every tile, so
                         // the phases of o_free stay in step with the units).
                         if (j == 0 && nq > 0 && !(ok = mbar_wait(&o_free[t], (nq - 1) & 1, wc, 67))) break;
-                        if (j < w.a(t) || j >= w.b(t)) {
-                            // under a window a tile can start later than the unit's first key tile
-                            if (j + 1 == w.a(t)) issue_s(t, g + 1);
+                        if (!fwd_active<MASK>(w, t, j)) {
+                            // under a window a tile can start later than the unit's first key
+                            // tile (with anchors: again after the anchor tiles)
+                            if (MASK == kMaskAnchor ? (more && fwd_active<MASK>(w, t, j + 1)) : (j + 1 == w.a(t)))
+                                issue_s(t, g + 1);
                             continue;
                         }
                         if (!(ok = mbar_wait(&p_full[t], ps[t] & 1, wc, 68))) break;
                         ++ps[t];
                         tc_fence_after();
+                        // O_t accumulates from the tile's second P V on.
+                        const bool acc0 = MASK == kMaskAnchor ? (t ? started1 : started0) : (j > w.a(t));
+                        if (t) started1 = true; else started0 = true;
                         if constexpr (FP8) {
                             // P: four E4M3 keys per column, 32 keys (8 columns, 32 rows of V)
                             // per instruction; V's d = 128 one-byte values are one 128-byte slab.
@@ -449,15 +520,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                             for (int kk = 0; kk < 4; ++kk)
                                 mma_ts_f8(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
                                           sdesc_sw128(v_addr + kk * 4096, C::kSlabBytes, 1024), id_pv,
-                                          (j > w.a(t) || kk > 0) ? 1u : 0u);
+                                          (acc0 || kk > 0) ? 1u : 0u);
                         } else {
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
                                 mma_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
                                        sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024), id_pv,
-                                       (j > w.a(t) || kk > 0) ? 1u : 0u);
+                                       (acc0 || kk > 0) ? 1u : 0u);
                         }
-                        if (j + 1 < w.b(t)) issue_s(t, g + 1);
+                        if (MASK == kMaskAnchor ? (more && fwd_active<MASK>(w, t, j + 1)) : (j + 1 < w.b(t)))
+                            issue_s(t, g + 1);
                     }
                     if (j + 2 == w.n_kv) tc_commit(q_empty);  // the unit's last S products are issued
                     tc_commit(&v_empty[st]);
@@ -500,7 +572,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!w.rows) continue;
             const int qt0 = w.q0 + 128 * t;
             const int q = qt0 + r;
-            const int nt = w.b(t) - w.a(t);  // key tiles w.jlo + w.a(t) + jj, jj < nt
+            const int nt = fwd_tile_steps<MASK>(w, t);  // key tiles fwd_tile_of(w, t, jj), jj < nt
             // This thread's output row (computed where it is used, to keep registers
             // free during the key loop).
             // (The unit is decoded again there: nothing of it stays live across the loop.)
@@ -530,6 +602,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // first step: [rel_lo, rel_hi).
             int rel_lo, rel_hi;
             key_range<MASK>(args, q, w.q_len, w.k_len, rel_lo, rel_hi);
+            const int key_lo = rel_lo, key_hi = rel_hi;  // kMaskAnchor: absolute bounds
             rel_lo -= (w.jlo + w.a(t)) * 128;
             rel_hi -= (w.jlo + w.a(t)) * 128;
             if constexpr (QKNORM) {  // this thread's row of Q, before the unit's first S product
@@ -571,11 +644,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (!ok) break;
                 ++ss;
                 tc_fence_after();
-                const int lim = rel_hi - j * 128;     // columns >= lim are masked
-                const int lim_lo = rel_lo - j * 128;  // and, under a window, columns < lim_lo
+                // Columns >= lim are masked, and under a window columns < lim_lo (with
+                // anchors only those at or past anc, the first key that is not an anchor).
+                const int kb = MASK == kMaskAnchor ? fwd_tile_of<MASK>(w, t, j) * 128 : 0;
+                const int lim = MASK == kMaskAnchor ? key_hi - kb : rel_hi - j * 128;
+                const int lim_lo = MASK == kMaskAnchor ? key_lo - kb : rel_lo - j * 128;
+                const int anc = args.n_anchor - kb;
                 // (uniform per warp: only tiles on a window's edge pay for the mask)
                 const bool need_mask =
-                    __any_sync(0xffffffffu, lim < 128 || (MASK == kMaskWindow && lim_lo > 0));
+                    __any_sync(0xffffffffu, lim < 128 || (MASK == kMaskWindow && lim_lo > 0) ||
+                                                (MASK == kMaskAnchor && lim_lo > 0 && lim_lo > anc));
                 uint32_t sv[4][32];
     #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
@@ -584,7 +662,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (need_mask) {  // masked columns read as -inf: out of the max, P = 0
     #pragma unroll
                     for (int c = 0; c < 128; ++c)
-                        if (c >= lim || (MASK == kMaskWindow && c < lim_lo)) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                        if (c >= lim || (MASK == kMaskWindow && c < lim_lo) ||
+                            (MASK == kMaskAnchor && c < lim_lo && c >= anc))
+                            sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
                 }
                 // Row max: 8 independent chains of three-input max.
                 float mxp[8];

@@ -121,6 +121,27 @@ fa_status fa_bwd_window(const void* q, const void* k, const void* v, const void*
                         float scale, int window_left, int window_right, fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * Sliding window plus global anchor keys (the block-sparse local attention with
+ * globally visible keys of "YOLOv12 ...", section 4.2: key blocks outside the window
+ * are skipped, the anchor blocks are loaded for every query): key j is visible to
+ * query i iff j <= a + window_right (when window_right >= 0) and
+ * (j >= a - window_left or j < n_anchor), with a = i + Nk - Nq. Whole key tiles
+ * that are neither anchors nor inside some row's window are skipped. n_anchor >= 0
+ * (FA_ERR_INVALID_ARG otherwise); n_anchor = 0, or window_left < 0, is exactly
+ * fa_fwd_window / fa_bwd_window. Fixed length. Every other argument, result and
+ * error is that of fa_fwd_window / fa_bwd_window.
+ */
+fa_status fa_fwd_window_anchor(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                               int window_left, int window_right, int n_anchor,
+                               fa_dtype dtype, fa_stream_t stream);
+fa_status fa_bwd_window_anchor(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                               int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                               int window_left, int window_right, int n_anchor,
+                               fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Sliding-window attention on packed variable-length batches: the window of
  * fa_fwd_window / fa_bwd_window applied within every sequence (a = i + Nk_s - Nq_s
  * with that sequence's own lengths), over the packed layout and cu_seqlens of

@@ -170,3 +170,62 @@ def test_varlen_window(case):
         refs[0][a:a + Lq], refs[1][ka:ka + Lk], refs[2][ka:ka + Lk] = rq[0], rk[0], rv[0]
     errs = [rel_l2(f64(g), r) for g, r in zip((dq, dk, dv), refs)]
     assert max(errs) <= RTOL_GRAD, errs
+
+
+ANCHOR_CASES = [
+    # B, Nq, Nk, Hq, Hkv, d, (wl, wr, n_anchor), dtype
+    (1, 700, 700, 2, 1, 128, (128, 0, 4), "bf16"),      # causal window + 4 anchors (one partial tile)
+    (2, 1100, 1100, 4, 2, 128, (200, 0, 130), "fp16"),  # anchors past the first tile, gap before the windows
+    (1, 900, 900, 2, 2, 64, (64, 64, 300), "bf16"),     # two-sided window, anchors over 3 tiles
+    (1, 640, 1000, 2, 1, 128, (100, -1, 50), "bf16"),   # unbounded right side: anchors seen by every row
+    (1, 300, 300, 2, 1, 128, (0, 0, 1), "bf16"),        # each row: key 0 and its own key
+]
+
+
+@pytest.mark.parametrize("case", ANCHOR_CASES, ids=lambda c: f"b{c[0]}-{c[1]}x{c[2]}-d{c[5]}-w{c[6][0]}_{c[6][1]}_a{c[6][2]}")
+def test_window_anchor_fwd_bwd(case):
+    B, Nq, Nk, Hq, Hkv, d, window, dt = case
+    fi = inputs.make_fixed(inputs.CAUSAL_GQA, B=B, Nq=Nq, Nk=Nk, Hq=Hq, Hkv=Hkv, d=d, dtype=dt, seed=89)
+    q, k, v, do = (t.cuda() for t in (fi.q, fi.k, fi.v, fi.do))
+    code = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
+    wl, wr, na = window
+    o, o_ok = guarded((B, Nq, Hq, d), q.dtype)
+    lse, l_ok = guarded((B, Hq, Nq), torch.float32)
+    st = fb.fa_fwd_window_anchor(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+                                 Nq, Nk, d, d ** -0.5, wl, wr, na, code, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, Nq, d), dtype=torch.uint8, device="cuda")
+    dq, dq_ok = guarded((B, Nq, Hq, d), q.dtype)
+    dk, dk_ok = guarded((B, Nk, Hkv, d), q.dtype)
+    dv, dv_ok = guarded((B, Nk, Hkv, d), q.dtype)
+    st = fb.fa_bwd_window_anchor(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv,
+                                 Nq, Nk, d, d ** -0.5, wl, wr, na, code, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    torch.cuda.synchronize()
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    assert o_ok() and l_ok() and dq_ok() and dk_ok() and dv_ok(), "write outside an output"
+    o64, l64 = f64(o), f64(lse)
+    o_ref, l_ref = oracle.attn_fwd(fi.q, fi.k, fi.v, d ** -0.5, window=window)
+    empty = np.isneginf(l_ref)
+    assert np.isneginf(l64[empty]).all()
+    live = ~empty
+    assert np.abs(l64[live] - l_ref[live]).max() <= ATOL_L
+    assert (np.abs(o64 - o_ref) <= o_bound(o_ref, q.dtype)).all()
+    rq, rk, rv = oracle.attn_bwd(fi.q, fi.k, fi.v, fi.do, d ** -0.5, window=window)
+    errs = [rel_l2(f64(g), r) for g, r in ((dq, rq), (dk, rk), (dv, rv))]
+    assert max(errs) <= RTOL_GRAD, errs
+
+
+def test_window_anchor_zero_is_the_window_path():
+    B, N, Hq, Hkv, d = 1, 400, 2, 1, 128
+    fi = inputs.make_fixed(inputs.CAUSAL_GQA, B=B, Nq=N, Nk=N, Hq=Hq, Hkv=Hkv, d=d, seed=91)
+    o, lse, _ = run(fi, (64, 0), backward=False)
+    q, k, v = (t.cuda() for t in (fi.q, fi.k, fi.v))
+    o2 = torch.empty_like(q)
+    l2 = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    st = fb.fa_fwd_window_anchor(q.data_ptr(), k.data_ptr(), v.data_ptr(), o2.data_ptr(), l2.data_ptr(), B, Hq, Hkv,
+                                 N, N, d, d ** -0.5, 64, 0, 0, fb.FA_BF16, 0)
+    assert st == fb.FA_OK
+    torch.cuda.synchronize()
+    assert np.array_equal(o, f64(o2)) and np.array_equal(lse, f64(l2))
