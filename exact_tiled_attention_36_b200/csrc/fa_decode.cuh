@@ -234,14 +234,17 @@ __device__ __forceinline__ bool dec_locate(const DecodeArgs& args, uint8_t* misc
 
 // The TMA producer (one thread): per segment the group's query rows (nb boxes of
 // gh heads x Nq tokens, box k at q_block_off * k within each 64-column slab of
-// q_slab_bytes), then every K and V tile of the segment through the S-stage rings.
+// q_slab_bytes) into Q buffer nq % QB (q_tile_bytes apart), then every K and V tile
+// of the segment through the S-stage rings. With two Q buffers the next segment's Q
+// (and so its K and V) load while the current segment's products still read its Q.
 // K and V tiles are 128 keys x d (16-bit), 64-column slabs of 16 KB.
-template <int D, bool SEQLENS, bool PAGED, int S>
+template <int D, bool SEQLENS, bool PAGED, int S, int QB = 1>
 __device__ __forceinline__ void dec_produce(const DecodeArgs& args, const DecRange& rg, const CUtensorMap* tm_q,
                                             const CUtensorMap* tm_k, const CUtensorMap* tm_v, uint8_t* sQ,
                                             int q_slab_bytes, int q_block_off, uint8_t* sK, uint8_t* sV,
                                             uint64_t* q_full, uint64_t* q_empty, uint64_t* k_full, uint64_t* k_empty,
-                                            uint64_t* v_full, uint64_t* v_empty, const WaitCtx& wc) {
+                                            uint64_t* v_full, uint64_t* v_empty, const WaitCtx& wc,
+                                            int q_tile_bytes = 0) {
     constexpr int kSlabs = D / 64;
     constexpr int kSlabBytes = 128 * 128;
     constexpr int kTileBytes = kSlabs * kSlabBytes;
@@ -290,21 +293,26 @@ __device__ __forceinline__ void dec_produce(const DecodeArgs& args, const DecRan
         if (lo >= hi) continue;
         const int j0 = static_cast<int>(lo - it.P), n = static_cast<int>(hi - lo);
         if (SEQLENS && lo == it.P) args.meta[1 + static_cast<size_t>(it.b) * args.Hkv + it.hk] = it.P;
-        // Q of the group once the previous segment's last S product has read Q.
-        if (!(ok = mbar_wait(q_empty, (nq & 1) ^ 1u, wc, 80))) break;
-        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(args.pair ? 2 * 128 * args.rg : kSlabs * 128 * args.R));
+        // Q of the group once the last S product of the segment that used this buffer
+        // before has read it.
+        const int qb = nq % QB;
+        uint8_t* q_dst = sQ + qb * q_tile_bytes;
+        if (!(ok = mbar_wait(&q_empty[qb], ((nq / QB) & 1) ^ 1u, wc, 80))) break;
+        mbar_arrive_expect_tx(&q_full[qb],
+                              static_cast<uint32_t>(args.pair ? 2 * 128 * args.rg : kSlabs * 128 * args.R));
         if (args.pair) {
             // KV heads 2 hk and 2 hk + 1 (64 columns each): the first group's rows in
             // columns 0..63 from row 0, the second's in columns 64..127 from row r8.
 #pragma unroll
             for (int k = 0; k < 2; ++k)
-                tma_load_4d(sQ + k * q_slab_bytes + k * args.r8 * 128, tm_q, q_full, 0, (2 * it.hk + k) * g, 0, it.b);
+                tma_load_4d(q_dst + k * q_slab_bytes + k * args.r8 * 128, tm_q, &q_full[qb], 0, (2 * it.hk + k) * g,
+                            0, it.b);
         } else {
             for (int k = 0; k < args.nb; ++k)
 #pragma unroll
                 for (int s = 0; s < kSlabs; ++s)
-                    tma_load_4d(sQ + s * q_slab_bytes + k * q_block_off, tm_q, q_full, s * 64, it.hk * g + k * args.gh,
-                                0, it.b);
+                    tma_load_4d(q_dst + s * q_slab_bytes + k * q_block_off, tm_q, &q_full[qb], s * 64,
+                                it.hk * g + k * args.gh, 0, it.b);
         }
         ++nq;
         for (int j = 0; j < n; ++j) {
@@ -321,7 +329,10 @@ __device__ __forceinline__ void dec_produce(const DecodeArgs& args, const DecRan
         gk += n;
     }
     // Leave no load in flight: wait for the last one issued into every buffer.
-    if (nq > 0) mbar_wait_drain(q_full, (nq - 1) & 1);
+    for (int qb = 0; qb < QB; ++qb) {
+        const int uses = (nq + QB - 1 - qb) / QB;  // loads into Q buffer qb
+        if (uses > 0) mbar_wait_drain(&q_full[qb], (uses - 1) & 1);
+    }
     for (int st = 0; st < S; ++st) {
         if (k_issued > st) mbar_wait_drain(&k_full[st], ((st + S * ((k_issued - 1 - st) / S)) / S) & 1);
         if (v_issued > st) mbar_wait_drain(&v_full[st], ((st + S * ((v_issued - 1 - st) / S)) / S) & 1);
@@ -684,17 +695,18 @@ struct DecNarrowCfg {
     // S^T buffers (and P buffers): the MMA thread issues S^T of tile j + kNS right
     // after P V of tile j, so the softmax has kNS tiles of slack over the products'
     // latency (which, not the exponentials, bounds a short tile).
-    static constexpr int kNS = (D == 128) ? 3 : 4;
+    static constexpr int kNS = (D == 128) ? (RN == 16 ? 3 : 2) : 4;
     static constexpr int kStages = (D == 128) ? 3 : (RN == 16 ? 6 : 5);
     static constexpr int kQSlab = RN * 128;               // RN rows x 64 columns
+    static constexpr int kQBytes = kSlabs * kQSlab;       // one Q buffer (two: one per segment parity)
     static constexpr int kPSlab = RN * 128;               // RN rows x 64 keys
     static constexpr int kPBytes = 2 * kPSlab;            // 128 keys
     static constexpr int kQOff = 0;
-    static constexpr int kPOff = kQOff + kSlabs * kQSlab;  // kNS P buffers
+    static constexpr int kPOff = kQOff + 2 * kQBytes;      // kNS P buffers
     static constexpr int kVOff = kPOff + kNS * kPBytes;
     static constexpr int kKOff = kVOff + kStages * kTileBytes;
     static constexpr int kBarOff = kKOff + kStages * kTileBytes;
-    static constexpr int kNumBars = 2 + 4 * kStages + 3 * kNS + 4 + 5;
+    static constexpr int kNumBars = 4 + 4 * kStages + 3 * kNS + 4 + 5;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kFlagOff = kMiscOff + 128;        // int [2][4]: a warp's rows need the exact max
     static constexpr int kRedOff = kFlagOff + 32;          // float [2][4][RN]: per-warp maxima
@@ -743,9 +755,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     uint8_t* sK = smem + C::kKOff;
     uint8_t* sV = smem + C::kVOff;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-    uint64_t* q_full = bars;
-    uint64_t* q_empty = bars + 1;
-    uint64_t* k_full = bars + 2;
+    uint64_t* q_full = bars;       // [2] Q buffer of segment parity
+    uint64_t* q_empty = bars + 2;  // [2]
+    uint64_t* k_full = bars + 4;
     uint64_t* k_empty = k_full + S;
     uint64_t* v_full = k_empty + S;
     uint64_t* v_empty = v_full + S;
@@ -761,15 +773,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // Rows of Q that no load writes are zeros: rows R .. RN-1, and with paired KV heads
     // everything outside the two groups' blocks (rows 0..rg-1 of columns 0..63, rows
     // r8..r8+rg-1 of columns 64..127), which makes Q block-diagonal.
-    for (int i = tid; i < C::kSlabs * C::kQSlab / 16; i += kDecThreads) {
-        const int row = (i % (C::kQSlab / 16)) / 8, slab = i / (C::kQSlab / 16);
+    for (int i = tid; i < 2 * C::kQBytes / 16; i += kDecThreads) {
+        const int row = (i % (C::kQSlab / 16)) / 8, slab = (i / (C::kQSlab / 16)) % C::kSlabs;
         const bool loaded = args.pair ? (row >= slab * args.r8 && row < slab * args.r8 + args.rg) : row < args.R;
         if (!loaded) reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
     if (tid == 0) {
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1);
+        }
         for (int i = 0; i < S; ++i) {
             mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], 1);
@@ -806,14 +820,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     if (warp == 0) {
         if (lane == 0)
-            dec_produce<D, SEQLENS, PAGED, S>(args, rg, &tm_q, &tm_k, &tm_v, sQ, C::kQSlab, 0, sK, sV, q_full,
-                                              q_empty, k_full, k_empty, v_full, v_empty, wc);
+            dec_produce<D, SEQLENS, PAGED, S, 2>(args, rg, &tm_q, &tm_k, &tm_v, sQ, C::kQSlab, 0, sK, sV, q_full,
+                                                 q_empty, k_full, k_empty, v_full, v_empty, wc, C::kQBytes);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_f16(128, RN, BF16, false, false);
             constexpr uint32_t id_pv = idesc_f16(128, RN, BF16, true, false);
-            const uint32_t q_addr = smem_u32(sQ);
+            uint32_t q_addr = smem_u32(sQ);  // the current segment's Q buffer
             // S^T into columns 32 (gg % NS) from the K tile of ring index gg.
             auto issue_s = [&](int gg) {
                 const uint32_t k_addr = smem_u32(sK + (gg % S) * C::kTileBytes);
@@ -833,7 +847,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 const long long lo = max(rg.s_lo, it.P), hi = min(rg.s_hi, it.P + it.ntk);
                 if (lo >= hi) continue;
                 const int n = static_cast<int>(hi - lo);
-                if (!(ok = mbar_wait(q_full, nq & 1, wc, 100))) break;
+                const int qb = nq & 1;
+                q_addr = smem_u32(sQ + qb * C::kQBytes);
+                if (!(ok = mbar_wait(&q_full[qb], (nq >> 1) & 1, wc, 100))) break;
                 for (int j = 0; ok && j < min(n, NS); ++j) {
                     const int gg = gk + j;
                     if (!(ok = mbar_wait(&k_full[gg % S], (gg / S) & 1, wc, 101))) break;
@@ -841,7 +857,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     issue_s(gg);
                 }
                 if (!ok) break;
-                if (n <= NS) tc_commit(q_empty);
+                if (n <= NS) tc_commit(&q_empty[qb]);
                 for (int j = 0; ok && j < n; ++j) {
                     const int gg = gk + j, st = gg % S, b = gg % NS;
                     if (!(ok = mbar_wait(&v_full[st], (gg / S) & 1, wc, 102))) break;
@@ -865,7 +881,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                         if (!(ok = mbar_wait(&k_full[g2 % S], (g2 / S) & 1, wc, 105))) break;
                         tc_fence_after();
                         issue_s(g2);
-                        if (j + NS + 1 == n) tc_commit(q_empty);
+                        if (j + NS + 1 == n) tc_commit(&q_empty[qb]);
                     }
                 }
                 tc_commit(o_ready);
