@@ -60,10 +60,21 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
-def csrc_digest():
+# The device code each profiled kernel is compiled from (its header and what it
+# includes; the host file only encodes descriptors and launches).
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": ("sm100.cuh", "fa_fwd.cuh"),
+    "fa_bwd128_kernel": ("sm100.cuh", "fa_bwd.cuh", "fa_bwd128.cuh"),
+    "fa_decode_narrow_kernel": ("sm100.cuh", "fa_decode.cuh"),
+}
+
+
+def csrc_digest(kernel=None):
+    """sha256 (16 hex digits) of `kernel`'s source files (every csrc file if None)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "exact_tiled_attention_36_b200", "csrc")
-    for name in sorted(os.listdir(d)):
+    names = sorted(os.listdir(d)) if kernel is None else sorted(KERNEL_SOURCES[kernel])
+    for name in names:
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -79,7 +90,7 @@ def profiled_traffic(kernel):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-        if kv.get("csrc_sha256_16") == csrc_digest():
+        if kv.get("csrc_sha256_16") == csrc_digest(kernel):
             return float(kv["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
         pass
@@ -443,7 +454,12 @@ def run_sweep(args):
             line["frac_of_fp8_peak"] = flops / (ms / 1e3) / 1e12 / (2.0 * peak)
         print(json.dumps(line), flush=True)
 
+    def want(name):
+        return args.only is None or args.only in name
+
     for cfg in (inputs.TINY, inputs.VISION, inputs.VIT_RMSNORM, inputs.CAUSAL_GQA):
+        if not want(cfg.name):
+            continue
         fi = inputs.make_fixed(cfg)
         q, k, v = (t.cuda() for t in (fi.q, fi.k, fi.v))
         B, N, Hq, d = q.shape
@@ -462,6 +478,23 @@ def run_sweep(args):
         del q, k, v, o, lse
     # the causal GQA prefill shape with block-scaled E4M3 inputs (fa_fwd_fp8)
     cfg = inputs.CAUSAL_GQA_FP8
+    if want(cfg.name):
+        sweep_fp8(cfg, inputs, fb, torch, stream, time_it, emit)
+    if want(inputs.CAUSAL_GQA.name + "_window1024_anchor4"):
+        sweep_window(inputs, fb, torch, stream, time_it, emit)
+    if want(inputs.VIT_RMSNORM.name + "_packed_qkv_fused_qk_rmsnorm"):
+        sweep_vit_variants(inputs, fb, torch, stream, time_it, emit)
+    for cfg in (inputs.VARLEN, inputs.VARLEN_KEYPAD):
+        if want(cfg.name):
+            sweep_varlen(cfg, inputs, fb, torch, stream, time_it, emit)
+    for cfg, page in ((inputs.DECODE, 0), (inputs.DECODE_RAGGED, 0), (inputs.DECODE_RAGGED, 64),
+                      (inputs.DECODE_RAGGED, 16), (inputs.DECODE_D64, 0), (inputs.DECODE_SPEC4, 0)):
+        if want(cfg.name + (f"_paged{page}" if page else "")):
+            sweep_decode(cfg, page, inputs, fb, torch, stream, time_it, emit)
+    return 0
+
+
+def sweep_fp8(cfg, inputs, fb, torch, stream, time_it, emit):
     f8 = inputs.make_fp8(cfg)
     q8, k8, v8 = f8.q.cuda(), f8.k.cuda(), f8.v.cuda()
     qs, ks, vs = f8.q_scale.cuda(), f8.k_scale.cuda(), f8.v_scale.cuda()
@@ -479,8 +512,11 @@ def run_sweep(args):
 
     emit(cfg.name, "fwd", time_it(ffp8, 30), flops_fwd(B, N, Hq, d, cfg.causal),
          q8.numel() + k8.numel() + v8.numel() + 2 * o.numel() + 4 * lse.numel(), fp8=True)
-    del q8, k8, v8, qs, ks, vs, o, lse
-    # local attention: the causal GQA prefill shape with a causal sliding window of 1024 keys
+
+
+def sweep_window(inputs, fb, torch, stream, time_it, emit):
+    """Local attention: the causal GQA prefill shape with a causal sliding window of 1024
+    keys, alone and with 4 global anchor keys."""
     cfg = inputs.CAUSAL_GQA
     fi = inputs.make_fixed(cfg)
     q, k, v, do = (t.cuda() for t in (fi.q, fi.k, fi.v, fi.do))
@@ -532,8 +568,11 @@ def run_sweep(args):
     emit(cfg.name + "_window1024_anchor4", "fwd", time_it(afwd, 30), aflops, nb)
     emit(cfg.name + "_window1024_anchor4", "bwd", time_it(abwd, 20), 2.5 * aflops,
          nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
-    del q, k, v, do, o, lse, dq, dk, dv, ws
-    # the ViT workload through the packed-QKV layout (B, S, 3, H, d), O written as (B, H, S, d)
+
+
+def sweep_vit_variants(inputs, fb, torch, stream, time_it, emit):
+    """The ViT workload through the packed-QKV layout (B, S, 3, H, d), O written as
+    (B, H, S, d); and from raw Q and K with their RMS normalisation fused."""
     cfg = inputs.VIT_RMSNORM
     fi = inputs.make_fixed(cfg)
     qkv = torch.stack([fi.q, fi.k, fi.v], dim=2).cuda()
@@ -573,79 +612,79 @@ def run_sweep(args):
     ms = time_it(fused, 30)
     emit(cfg.name + "_fused_qk_rmsnorm", "fwd", ms, flops_fwd(B, N, Hq, d, cfg.causal),
          2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel())
-    del q, k, v, o, lse, ws
-    for cfg in (inputs.VARLEN, inputs.VARLEN_KEYPAD):
-        vi = inputs.make_varlen(cfg)
-        q, k, v = (t.cuda() for t in (vi.q, vi.k, vi.v))
-        cu_q, cu_k = vi.cu_seqlens_q.cuda(), vi.cu_seqlens_k.cuda()
-        o, lse = fb.attention_varlen_fwd(q, k, v, cu_q, cu_k, vi.max_seqlen_q, vi.max_seqlen_k, cfg.scale, cfg.causal)
-        flops = sum(4.0 * lq * lk * cfg.d * cfg.Hq for lq, lk in zip(vi.seqlens_q, vi.seqlens_k))
-        nbytes = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
-        ms = time_it(lambda: fb.attention_varlen_fwd(q, k, v, cu_q, cu_k, vi.max_seqlen_q, vi.max_seqlen_k,
-                                                     cfg.scale, cfg.causal, out=o, lse=lse), 20)
-        emit(cfg.name, "fwd", ms, flops, nbytes)
-        if cfg is inputs.VARLEN:
-            # the varlen backward on the same packed batch (dO drawn after Q, K, V)
-            do = inputs.make_varlen(cfg, with_do=True).do.cuda()
-            n, Tq, Tk = len(vi.seqlens_q), q.shape[0], k.shape[0]
-            ws = torch.empty(fb.fa_varlen_bwd_workspace_size(n, Tq, vi.max_seqlen_q, cfg.Hq, cfg.d),
-                             dtype=torch.uint8, device="cuda")
-            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-            dt = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
 
-            def vbwd():
-                st = fb.fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                      do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
-                                      cu_q.data_ptr(), cu_k.data_ptr(), n, Tq, Tk, vi.max_seqlen_q,
-                                      vi.max_seqlen_k, cfg.Hq, cfg.Hkv, cfg.d, cfg.scale, int(cfg.causal), dt,
-                                      stream.cuda_stream)
-                if st != fb.FA_OK:
-                    raise RuntimeError(fb.fa_status_string(st))
 
-            ms = time_it(vbwd, 10)
-            emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
-            del do, ws, dq, dk, dv
-    # decode against a key/value cache, split over the keys (split kernel + merge kernel)
-    for cfg, page in ((inputs.DECODE, 0), (inputs.DECODE_RAGGED, 0), (inputs.DECODE_RAGGED, 64),
-                      (inputs.DECODE_RAGGED, 16), (inputs.DECODE_D64, 0), (inputs.DECODE_SPEC4, 0)):
-        di = inputs.make_decode(cfg, page_size=page)
-        q = di.q.cuda()
-        B, Nq, Hq, d = q.shape
-        Hkv = di.k.shape[2]
-        lens = di.seqlens if di.seqlens is not None else [cfg.Nk] * B
-        sl = None if di.seqlens is None else torch.tensor(di.seqlens, dtype=torch.int32, device="cuda")
-        ws = torch.empty(fb.fa_decode_workspace_size(B, Hq, Hkv, Nq, d), dtype=torch.uint8, device="cuda")
-        o = torch.empty_like(q)
-        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device="cuda")
+
+def sweep_varlen(cfg, inputs, fb, torch, stream, time_it, emit):
+    vi = inputs.make_varlen(cfg)
+    q, k, v = (t.cuda() for t in (vi.q, vi.k, vi.v))
+    cu_q, cu_k = vi.cu_seqlens_q.cuda(), vi.cu_seqlens_k.cuda()
+    o, lse = fb.attention_varlen_fwd(q, k, v, cu_q, cu_k, vi.max_seqlen_q, vi.max_seqlen_k, cfg.scale, cfg.causal)
+    flops = sum(4.0 * lq * lk * cfg.d * cfg.Hq for lq, lk in zip(vi.seqlens_q, vi.seqlens_k))
+    nbytes = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
+    ms = time_it(lambda: fb.attention_varlen_fwd(q, k, v, cu_q, cu_k, vi.max_seqlen_q, vi.max_seqlen_k,
+                                                 cfg.scale, cfg.causal, out=o, lse=lse), 20)
+    emit(cfg.name, "fwd", ms, flops, nbytes)
+    if cfg is inputs.VARLEN:
+        # the varlen backward on the same packed batch (dO drawn after Q, K, V)
+        do = inputs.make_varlen(cfg, with_do=True).do.cuda()
+        n, Tq, Tk = len(vi.seqlens_q), q.shape[0], k.shape[0]
+        ws = torch.empty(fb.fa_varlen_bwd_workspace_size(n, Tq, vi.max_seqlen_q, cfg.Hq, cfg.d),
+                         dtype=torch.uint8, device="cuda")
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         dt = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
-        if page:
-            kp, vp, bt = di.k_pages.cuda(), di.v_pages.cuda(), di.block_table.cuda()
 
-            def dec():
-                st = fb.fa_decode_paged(q.data_ptr(), kp.data_ptr(), vp.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                        sl.data_ptr(), bt.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, kp.shape[0],
-                                        page, bt.shape[1], d, cfg.scale, int(cfg.causal), dt, stream.cuda_stream)
-                if st != fb.FA_OK:
-                    raise RuntimeError(fb.fa_status_string(st))
-        else:
-            kc, vc = di.k.cuda(), di.v.cuda()
+        def vbwd():
+            st = fb.fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                                  cu_q.data_ptr(), cu_k.data_ptr(), n, Tq, Tk, vi.max_seqlen_q,
+                                  vi.max_seqlen_k, cfg.Hq, cfg.Hkv, cfg.d, cfg.scale, int(cfg.causal), dt,
+                                  stream.cuda_stream)
+            if st != fb.FA_OK:
+                raise RuntimeError(fb.fa_status_string(st))
 
-            def dec():
-                st = fb.fa_decode(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                  0 if sl is None else sl.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, cfg.Nk, d,
-                                  cfg.scale, int(cfg.causal), dt, stream.cuda_stream)
-                if st != fb.FA_OK:
-                    raise RuntimeError(fb.fa_status_string(st))
+        ms = time_it(vbwd, 10)
+        emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
 
-        keys = sum(lens)
-        # attention FLOPs (masked pairs of the causal tokens excluded) and the bytes the
-        # step must move: every cached K and V row once, Q, O and L
-        vis = sum(min(n, max(0, t + n - Nq + 1)) if cfg.causal else n for n in lens for t in range(Nq))
-        flops = 4.0 * d * Hq * vis
-        nbytes = 2 * (2 * keys * Hkv * d + 2 * q.numel()) + 4 * lse.numel()
-        emit(cfg.name + (f"_paged{page}" if page else ""), "decode", time_it(dec, 50), flops, nbytes)
-        del di, q, o, lse, ws
-    return 0
+
+def sweep_decode(cfg, page, inputs, fb, torch, stream, time_it, emit):
+    """Decode against a key/value cache, split over the keys (split kernel + merge kernel)."""
+    di = inputs.make_decode(cfg, page_size=page)
+    q = di.q.cuda()
+    B, Nq, Hq, d = q.shape
+    Hkv = di.k.shape[2]
+    lens = di.seqlens if di.seqlens is not None else [cfg.Nk] * B
+    sl = None if di.seqlens is None else torch.tensor(di.seqlens, dtype=torch.int32, device="cuda")
+    ws = torch.empty(fb.fa_decode_workspace_size(B, Hq, Hkv, Nq, d), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device="cuda")
+    dt = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
+    if page:
+        kp, vp, bt = di.k_pages.cuda(), di.v_pages.cuda(), di.block_table.cuda()
+
+        def dec():
+            st = fb.fa_decode_paged(q.data_ptr(), kp.data_ptr(), vp.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                    sl.data_ptr(), bt.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, kp.shape[0],
+                                    page, bt.shape[1], d, cfg.scale, int(cfg.causal), dt, stream.cuda_stream)
+            if st != fb.FA_OK:
+                raise RuntimeError(fb.fa_status_string(st))
+    else:
+        kc, vc = di.k.cuda(), di.v.cuda()
+
+        def dec():
+            st = fb.fa_decode(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                              0 if sl is None else sl.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, cfg.Nk, d,
+                              cfg.scale, int(cfg.causal), dt, stream.cuda_stream)
+            if st != fb.FA_OK:
+                raise RuntimeError(fb.fa_status_string(st))
+
+    keys = sum(lens)
+    # attention FLOPs (masked pairs of the causal tokens excluded) and the bytes the
+    # step must move: every cached K and V row once, Q, O and L
+    vis = sum(min(n, max(0, t + n - Nq + 1)) if cfg.causal else n for n in lens for t in range(Nq))
+    flops = 4.0 * d * Hq * vis
+    nbytes = 2 * (2 * keys * Hkv * d + 2 * q.numel()) + 4 * lse.numel()
+    emit(cfg.name + (f"_paged{page}" if page else ""), "decode", time_it(dec, 50), flops, nbytes)
 
 
 def main():
@@ -659,6 +698,9 @@ def main():
                     help="run only the warm-up steps on a smaller case (B=1, N=4096) for ncu captures")
     ap.add_argument("--all-configs", action="store_true",
                     help="time the forward of every workload (and the causal GQA backward); one JSON line each")
+    ap.add_argument("--only", default=None,
+                    help="with --all-configs: only the workload groups whose name contains this text "
+                         "(e.g. decode, fp8, window, varlen)")
     args = ap.parse_args()
     if args.all_configs:
         return run_sweep(args)
