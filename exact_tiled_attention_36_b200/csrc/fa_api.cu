@@ -252,16 +252,29 @@ size_t acc_floats(int B, int Hq, int Nq, int d) {
 // The backward of fa_bwd and fa_varlen_bwd. Fixed length: nseq = B, rows = B * Nq,
 // cu_q = cu_k = nullptr. Varlen: nseq = num_seqs, Nq / Nk the max_seqlen bounds,
 // rows = total_q, and the maps span the packed buffers (total_q / total_k rows).
+// Element strides of every tensor the backward reads or writes (batch, token, head).
+struct BwdStrides {
+    fa::Strides3 q, k, v, o, dout, dq, dk, dv;
+};
+
 // `causal` selects the masked kernels; their window is (wl, wr) (causal: (-1, 0)).
+// `bs`: strided views (null: contiguous tensors).
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dout, void* dq, void* dk, void* dv, void* workspace, int nseq, const int* cu_q,
                      const int* cu_k, int total_q, int total_k, int Hq, int Hkv, int Nq, int Nk, int d,
                      float scale, bool causal, bool bf16, cudaStream_t s, int wl = -1, int wr = 0,
-                     int n_anchor = 0) {
+                     int n_anchor = 0, const BwdStrides* bs = nullptr) {
     const bool varlen = cu_q != nullptr;
     int* err = error_word();
     if (!err) return FA_ERR_CUDA;
     fa_status st;
+    auto cont = [&](int rows_, int H) {
+        return fa::Strides3{static_cast<long long>(rows_ > 0 ? rows_ : 1) * H * d, static_cast<long long>(H) * d, d};
+    };
+    BwdStrides def;
+    def.q = def.o = def.dout = def.dq = cont(varlen ? total_q : Nq, Hq);
+    def.k = def.v = def.dk = def.dv = cont(varlen ? total_k : Nk, Hkv);
+    const BwdStrides& S = bs ? *bs : def;
     const size_t rows = static_cast<size_t>(varlen ? total_q : nseq * static_cast<size_t>(Nq)) * Hq;
     float* Dvec = static_cast<float*>(workspace);
     float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256(rows * sizeof(float)));
@@ -275,21 +288,25 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         if (d == 64)
             fa::fa_bwd_preprocess<64><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
                                                              static_cast<const uint16_t*>(dout), Dvec, dq_acc, acc_f4,
-                                                             pb, pn, Hq, bf16);
+                                                             pb, pn, Hq, bf16, S.o, S.dout);
         else
             fa::fa_bwd_preprocess<128><<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(o),
                                                               static_cast<const uint16_t*>(dout), Dvec, dq_acc,
-                                                              acc_f4, pb, pn, Hq, bf16);
+                                                              acc_f4, pb, pn, Hq, bf16, S.o, S.dout);
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
     const int kb = varlen ? 1 : nseq;
     const int kq_rows = varlen ? total_q : Nq, kk_rows = varlen ? total_k : Nk;
     if (kk_rows > 0 && Nk > 0) {
         CUtensorMap mq{}, mdo{}, mk, mv;
-        if (kq_rows > 0 && (st = make_map(&mq, q, d, Hq, kq_rows, kb, bf16)) != FA_OK) return st;
-        if (kq_rows > 0 && (st = make_map(&mdo, dout, d, Hq, kq_rows, kb, bf16)) != FA_OK) return st;
-        if ((st = make_map(&mk, k, d, Hkv, kk_rows, kb, bf16)) != FA_OK) return st;
-        if ((st = make_map(&mv, v, d, Hkv, kk_rows, kb, bf16)) != FA_OK) return st;
+        if (kq_rows > 0 &&
+            (st = make_map_strided(&mq, q, d, Hq, kq_rows, kb, bf16, S.q.h, S.q.s, S.q.b)) != FA_OK)
+            return st;
+        if (kq_rows > 0 &&
+            (st = make_map_strided(&mdo, dout, d, Hq, kq_rows, kb, bf16, S.dout.h, S.dout.s, S.dout.b)) != FA_OK)
+            return st;
+        if ((st = make_map_strided(&mk, k, d, Hkv, kk_rows, kb, bf16, S.k.h, S.k.s, S.k.b)) != FA_OK) return st;
+        if ((st = make_map_strided(&mv, v, d, Hkv, kk_rows, kb, bf16, S.v.h, S.v.s, S.v.b)) != FA_OK) return st;
         fa::BwdArgs a{};
         a.lse = lse;
         a.D = Dvec;
@@ -297,6 +314,12 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         a.nq4 = (Nq + 3) / 4;
         a.dk = dk;
         a.dv = dv;
+        a.dk_sb = S.dk.b;
+        a.dk_ss = S.dk.s;
+        a.dk_sh = S.dk.h;
+        a.dv_sb = S.dv.b;
+        a.dv_ss = S.dv.s;
+        a.dv_sh = S.dv.h;
         a.Hq = Hq;
         a.Hkv = Hkv;
         a.group = Hq / Hkv;
@@ -328,11 +351,11 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         if (d == 64) {
             const size_t n8 = rows * d / 8;
             fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
-                dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16);
+                dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16, Nq, Hq, S.dq);
         } else {
             const size_t n = static_cast<size_t>(nseq) * Hq * ((Nq + 3) / 4) * 64;
             fa::fa_bwd_dq_convert_g4<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
-                dq_acc, static_cast<uint16_t*>(dq), cu_q, nseq, Hq, Nq, (Nq + 3) / 4, scale, bf16);
+                dq_acc, static_cast<uint16_t*>(dq), cu_q, nseq, Hq, Nq, (Nq + 3) / 4, scale, bf16, S.dq);
         }
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
@@ -943,6 +966,28 @@ fa_status fa_bwd_window_anchor(const void* q, const void* k, const void* v, cons
     return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
                       scale, masked, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream), wl, wr,
                       wl >= 0 ? n_anchor : 0);
+}
+
+fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                         const long long* q_strides, const long long* k_strides, const long long* v_strides,
+                         const long long* o_strides, const long long* do_strides, const long long* dq_strides,
+                         const long long* dk_strides, const long long* dv_strides, int B, int Hq, int Hkv, int Nq,
+                         int Nk, int d, float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
+    const long long* given[8] = {q_strides, k_strides, v_strides, o_strides, do_strides, dq_strides, dk_strides,
+                                 dv_strides};
+    Strides t[8];
+    fa_status st;
+    for (int i = 0; i < 8; ++i) {
+        if ((st = read_strides(given[i], true, &t[i])) != FA_OK) return st;
+        if ((st = check_strides(t[i], true)) != FA_OK) return st;
+    }
+    st = bwd_checks(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype);
+    if (st != FA_OK) return st;
+    auto s3 = [](const Strides& x) { return fa::Strides3{x.b, x.s, x.h}; };
+    const BwdStrides bs{s3(t[0]), s3(t[1]), s3(t[2]), s3(t[3]), s3(t[4]), s3(t[5]), s3(t[6]), s3(t[7])};
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
+                      scale, causal != 0, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream), -1, 0, 0, &bs);
 }
 
 size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q, int Hq, int d) {

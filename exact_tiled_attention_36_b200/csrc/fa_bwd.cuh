@@ -56,6 +56,9 @@ struct BwdArgs {
     float scale_log2;
     int wl, wr;  // MASKED: keys from wl before to wr after the aligned diagonal (< 0: unbounded)
     int n_anchor;  // MASKED: keys 0 .. n_anchor - 1 are also visible below the window (global anchors)
+    // dK and dV element strides: batch, token, head (d contiguous); varlen uses token
+    // (the packed row) and head only.
+    long long dk_sb, dk_ss, dk_sh, dv_sb, dv_ss, dv_sh;
     int* err;
 };
 
@@ -135,9 +138,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (threadIdx.x < 128) {
             const int key = k0 + static_cast<int>(threadIdx.x);
             if (key < Nk) {
-                const size_t off = ((static_cast<size_t>(b) * Nk + key) * args.Hkv + hk) * D;
-                uint4* a = reinterpret_cast<uint4*>(static_cast<T16*>(args.dk) + off);
-                uint4* c = reinterpret_cast<uint4*>(static_cast<T16*>(args.dv) + off);
+                uint4* a = reinterpret_cast<uint4*>(static_cast<T16*>(args.dk) + b * args.dk_sb +
+                                                    key * args.dk_ss + hk * args.dk_sh);
+                uint4* c = reinterpret_cast<uint4*>(static_cast<T16*>(args.dv) + b * args.dv_sb +
+                                                    key * args.dv_ss + hk * args.dv_sh);
 #pragma unroll
                 for (int i = 0; i < D / 8; ++i) a[i] = c[i] = make_uint4(0, 0, 0, 0);
             }
@@ -391,8 +395,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // Warpgroup 0 writes dV, warpgroup 1 writes dK = scale * (dS^T Q).
             const uint32_t col = wg == 0 ? C::kColDV : C::kColDK;
             const float mul = wg == 0 ? 1.f : args.scale;
-            T16* dst = static_cast<T16*>(wg == 0 ? args.dv : args.dk) +
-                       ((static_cast<size_t>(b) * Nk + key) * args.Hkv + hk) * D;
+            T16* dst = wg == 0 ? static_cast<T16*>(args.dv) + b * args.dv_sb + key * args.dv_ss + hk * args.dv_sh
+                               : static_cast<T16*>(args.dk) + b * args.dk_sb + key * args.dk_ss + hk * args.dk_sh;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t v[32];
@@ -419,20 +423,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
 }
 
+// Element strides (batch, token, head; d contiguous) of a 16-bit [B, N, H, d] tensor.
+struct Strides3 {
+    long long b, s, h;
+};
+
 // D[b,h,q] = sum_c dO[b,q,h,c] O[b,q,h,c] in fp32, and dQ_acc[b,q,h,:] = 0.
-// A group of D/8 lanes handles one (b, q, h) row, 8 elements per lane.
+// A group of D/8 lanes handles one (b, q, h) row, 8 elements per lane; o and dout
+// are addressed through their strides.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float* Dvec,
                                                           float* dq_acc, size_t acc_f4, int B, int Nq, int Hq,
-                                                          bool bf16) {
+                                                          bool bf16, Strides3 so, Strides3 sdo) {
     constexpr int kLanes = D / 8;
     const size_t rows = static_cast<size_t>(B) * Nq * Hq;
     const size_t row = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / kLanes;
     const int sub = threadIdx.x % kLanes;
     float acc = 0.f;
     if (row < rows) {
-        const uint4 a = reinterpret_cast<const uint4*>(o + row * D)[sub];
-        const uint4 c = reinterpret_cast<const uint4*>(dout + row * D)[sub];
+        const long long rh = static_cast<long long>(row % Hq), rbq = static_cast<long long>(row / Hq);
+        const long long rq = rbq % Nq, rb = rbq / Nq;
+        const uint4 a = reinterpret_cast<const uint4*>(o + rb * so.b + rq * so.s + rh * so.h)[sub];
+        const uint4 c = reinterpret_cast<const uint4*>(dout + rb * sdo.b + rq * sdo.s + rh * sdo.h)[sub];
         const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -471,11 +483,15 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess(const uint16_t* o, cons
     }
 }
 
-// dq[i] = dtype(scale * dq_acc[i]), 8 elements per thread.
+// dq = dtype(scale * dq_acc) for d = 64 (accumulator [B, Nq, Hq, 64]), 8 elements
+// per thread, dq addressed through its strides.
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert(const float* dq_acc, uint16_t* dq, size_t n8, float scale,
-                                                          bool bf16) {
+                                                          bool bf16, int Nq, int Hq, Strides3 sdq) {
     const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= n8) return;
+    const size_t row = i / 8;  // (b Nq + q) Hq + h; 8 threads per 64-value row
+    const long long h = static_cast<long long>(row % Hq), bq = static_cast<long long>(row / Hq);
+    uint16_t* dst = dq + (bq / Nq) * sdq.b + (bq % Nq) * sdq.s + h * sdq.h + (i % 8) * 8;
     const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * i];
     const float4 c = reinterpret_cast<const float4*>(dq_acc)[2 * i + 1];
     uint4 out;
@@ -486,7 +502,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert(const float* dq_acc, ui
         out = make_uint4(pack2<false>(a.x * scale, a.y * scale), pack2<false>(a.z * scale, a.w * scale),
                          pack2<false>(c.x * scale, c.y * scale), pack2<false>(c.z * scale, c.w * scale));
     }
-    reinterpret_cast<uint4*>(dq)[i] = out;
+    *reinterpret_cast<uint4*>(dst) = out;
 }
 
 // The d = 128 accumulator keeps four consecutive queries of one head-dimension
@@ -494,10 +510,12 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert(const float* dq_acc, ui
 // 4 c + q % 4, so a warp of the backward main kernel (lane = c) adds four
 // queries with one coalesced 512-byte vector reduction. One thread here turns
 // head-dimension indices 2p, 2p + 1 of a group of four queries into dQ[token, h, :]:
-// token b Nq + q for fixed length, cu_q[b] + q for varlen (cu_q non-null; b is the
-// sequence, Nq the max_seqlen bound).
+// token q of batch b for fixed length, packed row cu_q[b] + q for varlen (cu_q
+// non-null; b is the sequence, Nq the max_seqlen bound), addressed through dq's
+// strides (varlen: the token stride only).
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert_g4(const float* dq_acc, uint16_t* dq, const int* cu_q,
-                                                             int B, int Hq, int Nq, int nq4, float scale, bool bf16) {
+                                                             int B, int Hq, int Nq, int nq4, float scale, bool bf16,
+                                                             Strides3 sdq) {
     const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // (b, h, g, p)
     const size_t groups = static_cast<size_t>(B) * Hq * nq4;
     if (i >= groups * 64) return;
@@ -508,9 +526,9 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_g4(const float* dq_acc,
     const int h = static_cast<int>(bh % Hq);
     const int b = static_cast<int>(bh / Hq);
     int q_len = Nq;
-    size_t row0 = static_cast<size_t>(b) * Nq;
+    long long base = b * sdq.b;  // token 0 of this batch / sequence
     if (cu_q) {
-        row0 = static_cast<size_t>(cu_q[b]);
+        base = static_cast<long long>(cu_q[b]) * sdq.s;
         q_len = min(cu_q[b + 1] - cu_q[b], Nq);
     }
     const float4* src = reinterpret_cast<const float4*>(dq_acc) + bhg * 128 + 2 * p;
@@ -521,7 +539,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_g4(const float* dq_acc,
         const int q = 4 * g + j;
         if (q >= q_len) break;
         const uint32_t v = bf16 ? pack2<true>(lo[j] * scale, hi[j] * scale) : pack2<false>(lo[j] * scale, hi[j] * scale);
-        reinterpret_cast<uint32_t*>(dq + ((row0 + q) * Hq + h) * 128)[p] = v;
+        reinterpret_cast<uint32_t*>(dq + base + q * sdq.s + h * sdq.h)[p] = v;
     }
 }
 

@@ -97,9 +97,12 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         tma_b = b;
     }
     const int Nq = q_len, Nk = k_len;
-    // Token index of key `key` of this sequence in the dK / dV buffers.
-    auto key_tok = [&](int key) -> size_t {
-        return VARLEN ? static_cast<size_t>(k_row0 + key) : static_cast<size_t>(b) * Nk + key;
+    // Element offsets of key `key` of this sequence in the dK and dV buffers.
+    auto dk_off = [&](int key) -> long long {
+        return VARLEN ? (k_row0 + key) * args.dk_ss + hk * args.dk_sh : b * args.dk_sb + key * args.dk_ss + hk * args.dk_sh;
+    };
+    auto dv_off = [&](int key) -> long long {
+        return VARLEN ? (k_row0 + key) * args.dv_ss + hk * args.dv_sh : b * args.dv_sb + key * args.dv_ss + hk * args.dv_sh;
     };
     int i0, n_i;  // the query tiles that see some key of this tile
     query_tiles<CAUSAL>(args, k0, Nq, Nk, i0, n_i);
@@ -113,9 +116,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         if (threadIdx.x < 128) {
             const int key = k0 + static_cast<int>(threadIdx.x);
             if (key < Nk) {
-                const size_t off = (key_tok(key) * args.Hkv + hk) * D;
-                uint4* a = reinterpret_cast<uint4*>(static_cast<T16*>(args.dk) + off);
-                uint4* c = reinterpret_cast<uint4*>(static_cast<T16*>(args.dv) + off);
+                uint4* a = reinterpret_cast<uint4*>(static_cast<T16*>(args.dk) + dk_off(key));
+                uint4* c = reinterpret_cast<uint4*>(static_cast<T16*>(args.dv) + dv_off(key));
 #pragma unroll
                 for (int i = 0; i < D / 8; ++i) a[i] = c[i] = make_uint4(0, 0, 0, 0);
             }
@@ -453,7 +455,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             // Warpgroup 0 writes dV, warpgroup 1 writes dK = scale * (dS^T Q).
             const uint32_t col = w == 0 ? C::kColDV : C::kColDK;
             const float mul = w == 0 ? 1.f : args.scale;
-            T16* dst = static_cast<T16*>(w == 0 ? args.dv : args.dk) + (key_tok(key) * args.Hkv + hk) * D;
+            T16* dst = w == 0 ? static_cast<T16*>(args.dv) + dv_off(key) : static_cast<T16*>(args.dk) + dk_off(key);
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t v[32];

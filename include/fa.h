@@ -264,6 +264,23 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  float scale, int causal, fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * Backward on strided views: the gradients of fa_fwd / fa_fwd_strided for q, k, v,
+ * o, dout, dq, dk, dv that are not contiguous, e.g. the packed QKV layout
+ * (B, S, 3, H, d) with its gradient dqkv in the same layout (dq, dk, dv views at
+ * +0, +H*d, +2*H*d of one buffer). *_strides: HOST arrays {batch, token, head}
+ * of element strides with the rules of fa_fwd_strided; dq, dk and dv must not
+ * overlap each other or the inputs. lse and the workspace keep their layouts.
+ * Every other argument, result and error is that of fa_bwd.
+ */
+fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                         const long long* q_strides, const long long* k_strides, const long long* v_strides,
+                         const long long* o_strides, const long long* do_strides, const long long* dq_strides,
+                         const long long* dk_strides, const long long* dv_strides,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Size in bytes of the caller-owned workspace fa_varlen_bwd needs: D
  * (float32 [Hq,total_q]) and the float32 dQ accumulator
  * (num_seqs*Hq*ceil(max_seqlen_q/4)*4*128 floats, each sequence padded to

@@ -270,3 +270,14 @@ def fp8(**kw):
 ])
 def test_fp8_rejects_before_launch(lib, kw, code):
     assert fp8(**kw) == code
+
+
+def test_bwd_strided_rejects_before_launch(lib):
+    st = (3 * 8 * 64 * 8, 3 * 8 * 64, 64)
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, ws=FAKE, sq=st, sk=st,
+             sv=st, so=st, sdo=st, sdq=st, sdk=st, sdv=st, B=1, Hq=8, Hkv=8, Nq=8, Nk=8, d=64, scale=0.125, causal=0,
+             dtype=fb.FA_BF16, stream=None)
+    assert fb.fa_bwd_strided(*{**a, "sdq": None}.values()) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_bwd_strided(*{**a, "sdk": (4096, 1540, 64)}.values()) == fb.FA_ERR_MISALIGNED
+    assert fb.fa_bwd_strided(*{**a, "ws": None}.values()) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_bwd_strided(*{**a, "d": 96}.values()) == fb.FA_ERR_UNSUPPORTED

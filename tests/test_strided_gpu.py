@@ -90,3 +90,50 @@ def test_varlen_packed_qkv_matches_contiguous():
                                            vi.max_seqlen_k, d ** -0.5, True)
     torch.cuda.synchronize()
     assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+
+
+def rel_l2(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+@pytest.mark.parametrize("B,N,H,d,causal,dt", [
+    (2, 300, 4, 64, False, "bf16"),
+    (1, 513, 2, 128, True, "fp16"),
+    (2, 257, 4, 128, False, "bf16"),
+])
+def test_packed_qkv_backward(B, N, H, d, causal, dt):
+    """fa_bwd_strided on the packed layout: q, k, v views of qkv (B, S, 3, H, d), O in a
+    (B, H, S, d) buffer, dO a (B, H, S, d) view, and the gradients written into one
+    dqkv (B, S, 3, H, d) buffer. dK and dV equal the contiguous path's bit for bit,
+    dQ up to the order of its fp32 reductions, and all three the oracle's."""
+    fi = inputs.make_fixed(inputs.TINY, B=B, Nq=N, Nk=N, Hq=H, Hkv=H, d=d, dtype=dt, seed=57, with_do=True)
+    qkv = torch.stack([fi.q, fi.k, fi.v], dim=2).cuda()
+    q, k, v = qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2]
+    o_bhsd = torch.empty((B, H, N, d), dtype=q.dtype, device="cuda")
+    o = o_bhsd.permute(0, 2, 1, 3)
+    do = fi.do.cuda().permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)  # (B, S, H, d) view of BHSD
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    code = fb.FA_BF16 if dt == "bf16" else fb.FA_FP16
+    st = fb.fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), el_strides(q),
+                           el_strides(k), el_strides(v), el_strides(o), B, H, H, N, N, d, d ** -0.5, int(causal),
+                           code, 0)
+    assert st == fb.FA_OK
+    dqkv = torch.full_like(qkv, 3.0)
+    dq, dk, dv = dqkv[:, :, 0], dqkv[:, :, 1], dqkv[:, :, 2]
+    ws = torch.empty(fb.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    st = fb.fa_bwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), el_strides(q), el_strides(k),
+                           el_strides(v), el_strides(o), el_strides(do), el_strides(dq), el_strides(dk),
+                           el_strides(dv), B, H, H, N, N, d, d ** -0.5, int(causal), code, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    torch.cuda.synchronize()
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    dq_c, dk_c, dv_c = fb.attention_bwd(q.contiguous(), k.contiguous(), v.contiguous(), o.contiguous(), lse,
+                                        do.contiguous(), d ** -0.5, causal)
+    torch.cuda.synchronize()
+    assert torch.equal(dk, dk_c) and torch.equal(dv, dv_c)
+    assert rel_l2(f64(dq), f64(dq_c)) <= 1e-2
+    rq, rk, rv = oracle.attn_bwd(fi.q, fi.k, fi.v, fi.do, d ** -0.5, causal)
+    errs = [rel_l2(f64(g), r) for g, r in ((dq, rq), (dk, rk), (dv, rv))]
+    assert max(errs) <= 2e-2, errs
