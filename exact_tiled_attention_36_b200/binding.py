@@ -1,7 +1,8 @@
 """Thin ctypes binding of libfa.so.
 
 The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_fwd_strided``, ``fa_varlen_fwd_strided``, ``fa_fwd_qk_rmsnorm``,
-``fa_fwd_window``, ``fa_bwd_window``, ``fa_varlen_fwd_window``, ``fa_varlen_bwd_window``, ``fa_fwd_window_anchor``, ``fa_bwd_window_anchor``, ``fa_bwd_strided``, ``fa_fwd_fp8``, ``fa_decode``, ``fa_decode_paged``, ``fa_decode_workspace_size``,
+``fa_fwd_window``, ``fa_bwd_window``, ``fa_varlen_fwd_window``, ``fa_varlen_bwd_window``, ``fa_fwd_window_anchor``, ``fa_bwd_window_anchor``, ``fa_bwd_strided``, ``fa_pack_key_mask``,
+``fa_fwd_keymask``, ``fa_bwd_keymask``, ``fa_fwd_fp8``, ``fa_decode``, ``fa_decode_paged``, ``fa_decode_workspace_size``,
 ``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
 ``fa_bwd``, ``fa_status_string`` and ``fa_get_last_device_error`` have the
 names, argument order and meaning of the C ABI in ``include/fa.h``: pointers
@@ -53,6 +54,9 @@ _SIGS = {
     "fa_selftest_bounded_wait": ([_P], _I),
     "fa_decode_workspace_size": ([_I] * 5, ctypes.c_size_t),
     "fa_fwd_fp8": ([_P] * 8 + [_I] * 6 + [_F, _I, _P], _I),
+    "fa_pack_key_mask": ([_P, _P, _I, _I, _P], _I),
+    "fa_fwd_keymask": ([_P] * 6 + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_bwd_keymask": ([_P] * 11 + [_I] * 6 + [_F, _I, _I, _P], _I),
     "fa_bwd_strided": ([_P] * 18 + [_I] * 6 + [_F, _I, _I, _P], _I),
     "fa_fwd_window_anchor": ([_P] * 5 + [_I] * 6 + [_F, _I, _I, _I, _I, _P], _I),
     "fa_bwd_window_anchor": ([_P] * 10 + [_I] * 6 + [_F, _I, _I, _I, _I, _P], _I),
@@ -163,6 +167,20 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, sca
     """fa_bwd with the library's own fixed-size workspace (for callers that cannot allocate)."""
     return lib().fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype,
                                 stream)
+
+
+def fa_pack_key_mask(keep, key_bits, B, Nk, stream) -> int:
+    return lib().fa_pack_key_mask(keep, key_bits, B, Nk, stream)
+
+
+def fa_fwd_keymask(q, k, v, o, lse, key_bits, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    return lib().fa_fwd_keymask(q, k, v, o, lse, key_bits, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream)
+
+
+def fa_bwd_keymask(q, k, v, o, lse, dout, dq, dk, dv, workspace, key_bits, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                   dtype, stream) -> int:
+    return lib().fa_bwd_keymask(q, k, v, o, lse, dout, dq, dk, dv, workspace, key_bits, B, Hq, Hkv, Nq, Nk, d, scale,
+                                causal, dtype, stream)
 
 
 def fa_bwd_strided(q, k, v, o, lse, dout, dq, dk, dv, workspace, q_strides, k_strides, v_strides, o_strides,

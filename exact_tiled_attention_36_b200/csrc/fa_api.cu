@@ -133,10 +133,10 @@ fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtyp
     return FA_OK;
 }
 
-template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM, bool FP8 = false>
+template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM, bool FP8 = false, bool KEYMASK = false>
 fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                        dim3 grid, cudaStream_t stream) {
-    auto kern = fa::fa_fwd_kernel<D, BF16, MASK, VARLEN, QKNORM, FP8>;
+    auto kern = fa::fa_fwd_kernel<D, BF16, MASK, VARLEN, QKNORM, FP8, KEYMASK>;
     constexpr int smem = fa::FwdCfg<D, FP8>::kSmemBytes;
     static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
     if (!attr_ok) return FA_ERR_CUDA;
@@ -154,11 +154,17 @@ fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 
 // The instantiations: mask none / causal / sliding window for plain inputs, fixed
 // length and varlen; the window with global anchors for fixed length; QK
-// normalisation for fixed length without a window.
+// normalisation for fixed length without a window; key masks for fixed length
+// with mask none / causal.
 template <int D, bool BF16>
 fa_status launch_fwd_b(int mask, bool varlen, bool qknorm, const CUtensorMap& mq, const CUtensorMap& mk,
                        const CUtensorMap& mv, const fa::FwdArgs& a, dim3 grid, cudaStream_t s) {
     constexpr int N = fa::kMaskNone, C = fa::kMaskCausal, W = fa::kMaskWindow, A = fa::kMaskAnchor;
+    if (a.key_bits != nullptr) {  // key masks: fixed length, no window, no normalisation
+        if (qknorm || varlen || mask == W || mask == A) return FA_ERR_UNSUPPORTED;
+        return mask == C ? launch_fwd_t<D, BF16, C, false, false, false, true>(mq, mk, mv, a, grid, s)
+                         : launch_fwd_t<D, BF16, N, false, false, false, true>(mq, mk, mv, a, grid, s);
+    }
     if (qknorm) {
         if (varlen || mask == W) return FA_ERR_UNSUPPORTED;
         return mask == C ? launch_fwd_t<D, BF16, C, false, true>(mq, mk, mv, a, grid, s)
@@ -182,6 +188,21 @@ fa_status launch_fwd(int d, bool bf16, int mask, bool varlen, bool qknorm, const
 }
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// keep [B, Nk] bytes (non-zero = visible) -> bits [B, words]: bit i of word w is key
+// 32 w + i (zero past Nk).
+__global__ void fa_pack_key_mask_kernel(const uint8_t* keep, uint32_t* bits, int B, int Nk, int words) {
+    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<long long>(B) * words) return;
+    const long long b = idx / words;
+    const int w = static_cast<int>(idx % words);
+    uint32_t v = 0;
+    for (int i = 0; i < 32; ++i) {
+        const int key = 32 * w + i;
+        if (key < Nk && keep[b * Nk + key]) v |= 1u << i;
+    }
+    bits[idx] = v;
+}
 
 // One CTA waits, with the kernels' bounded wait, on an mbarrier that nothing
 // arrives on: the wait runs out, records the site and the kernel returns.
@@ -263,7 +284,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, void* dq, void* dk, void* dv, void* workspace, int nseq, const int* cu_q,
                      const int* cu_k, int total_q, int total_k, int Hq, int Hkv, int Nq, int Nk, int d,
                      float scale, bool causal, bool bf16, cudaStream_t s, int wl = -1, int wr = 0,
-                     int n_anchor = 0, const BwdStrides* bs = nullptr) {
+                     int n_anchor = 0, const BwdStrides* bs = nullptr, const uint32_t* key_bits = nullptr) {
     const bool varlen = cu_q != nullptr;
     int* err = error_word();
     if (!err) return FA_ERR_CUDA;
@@ -333,6 +354,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         a.wl = wl;
         a.wr = wr;
         a.n_anchor = n_anchor;
+        a.key_bits = key_bits;
+        a.kb_words = (Nk + 31) / 32;
         a.err = err;
         const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
         if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
@@ -418,7 +441,7 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
                     Strides sv, Strides so, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                     fa_dtype dtype, fa_stream_t stream, bool qknorm = false, float eps = 0.f,
                     bool validate_only = false, bool window = false, int wl = -1, int wr = 0,
-                    int n_anchor = 0) {
+                    int n_anchor = 0, const uint32_t* key_bits = nullptr) {
     if (B < 1 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if ((Nq > 0 && (!q || !o || !lse)) || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
     fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
@@ -445,6 +468,8 @@ fa_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float*
     a.wl = wl;
     a.wr = wr;
     a.n_anchor = n_anchor;
+    a.key_bits = key_bits;
+    a.kb_words = (Nk + 31) / 32;
     a.num_batches = B;
     a.Hq = Hq;
     a.group = Hq / Hkv;
@@ -888,6 +913,27 @@ fa_status fa_fwd_window_anchor(const void* q, const void* k, const void* v, void
                      wl, wr, n_anchor);
 }
 
+fa_status fa_pack_key_mask(const unsigned char* keep, unsigned int* key_bits, int B, int Nk, fa_stream_t stream) {
+    if (B < 1 || Nk < 0 || (Nk > 0 && (!keep || !key_bits))) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(key_bits) & 3u) return FA_ERR_MISALIGNED;
+    const int words = (Nk + 31) / 32;
+    const long long n = static_cast<long long>(B) * words;
+    if (n == 0) return FA_OK;
+    fa_pack_key_mask_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        keep, key_bits, B, Nk, words);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_keymask(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const unsigned int* key_bits, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                         int causal, fa_dtype dtype, fa_stream_t stream) {
+    if (Nk > 0 && !key_bits) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(key_bits) & 3u) return FA_ERR_MISALIGNED;
+    return fwd_fixed(q, k, v, o, lse, contiguous(Nq, Hq, d), contiguous(Nk, Hkv, d), contiguous(Nk, Hkv, d),
+                     contiguous(Nq, Hq, d), B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, stream, false, 0.f, false,
+                     false, -1, 0, 0, key_bits);
+}
+
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
                          const long long* q_strides, const long long* k_strides, const long long* v_strides,
                          const long long* o_strides, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
@@ -988,6 +1034,20 @@ fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void
     const BwdStrides bs{s3(t[0]), s3(t[1]), s3(t[2]), s3(t[3]), s3(t[4]), s3(t[5]), s3(t[6]), s3(t[7])};
     return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
                       scale, causal != 0, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream), -1, 0, 0, &bs);
+}
+
+fa_status fa_bwd_keymask(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                         const unsigned int* key_bits, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                         int causal, fa_dtype dtype, fa_stream_t stream) {
+    if (Nk > 0 && !key_bits) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(key_bits) & 3u) return FA_ERR_MISALIGNED;
+    const fa_status st = bwd_checks(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                    dtype);
+    if (st != FA_OK) return st;
+    return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, nullptr, nullptr, 0, 0, Hq, Hkv, Nq, Nk, d,
+                      scale, causal != 0, dtype == FA_BF16, reinterpret_cast<cudaStream_t>(stream), -1, 0, 0, nullptr,
+                      key_bits);
 }
 
 size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q, int Hq, int d) {

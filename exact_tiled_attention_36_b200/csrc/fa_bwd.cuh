@@ -59,8 +59,33 @@ struct BwdArgs {
     // dK and dV element strides: batch, token, head (d contiguous); varlen uses token
     // (the packed row) and head only.
     long long dk_sb, dk_ss, dk_sh, dv_sb, dv_ss, dv_sh;
+    // Key mask (null: none): bit j % 32 of word b * kb_words + j / 32 set = key j of batch b
+    // is visible (ANDed with the window).
+    const uint32_t* key_bits;
+    int kb_words;
     int* err;
 };
+
+// Key `key` of batch b is visible under the key mask of `a` (always without one).
+__device__ __forceinline__ bool key_kept(const BwdArgs& a, int b, int key) {
+    return a.key_bits == nullptr ||
+           ((a.key_bits[static_cast<size_t>(b) * a.kb_words + (key >> 5)] >> (key & 31)) & 1u) != 0u;
+}
+
+// Some key of the tile [k0, min(k0 + 128, Nk)) of batch b is masked out by the key mask.
+__device__ __forceinline__ bool tile_keys_masked(const BwdArgs& a, int b, int k0, int Nk) {
+    if (a.key_bits == nullptr) return false;
+    bool masked = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int kw = k0 + 32 * i;  // first key of word i
+        if (kw >= Nk) break;
+        const uint32_t valid = Nk - kw >= 32 ? ~0u : ((1u << (Nk - kw)) - 1u);
+        const uint32_t w = a.key_bits[static_cast<size_t>(b) * a.kb_words + (kw >> 5)];
+        masked = masked || ((w & valid) != valid);
+    }
+    return masked;
+}
 
 // Queries [qlo, qhi) that see key `key` (bottom-right alignment: query q's aligned
 // key is q + Nk - Nq; with MASKED the window (wl, wr) of BwdArgs, else every query).
@@ -290,7 +315,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int r = w4 * 32 + lane;  // TMEM lane: key row for S^T / dP^T / dV / dK, query row for dQ
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
         const int key = k0 + r;
-        const bool key_ok = key < Nk;
+        const bool key_in = key < Nk;                          // a row of dK / dV to write
+        const bool key_ok = key_in && key_kept(args, b, key);  // a key that takes part
         const float sl2 = args.scale_log2;
         constexpr float kLog2eF = 1.4426950408889634074f;
         bool ok = true;
@@ -406,7 +432,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack2<BF16>(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
-                if (key_ok) {
+                if (key_in) {
                     uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);

@@ -309,7 +309,9 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         const int r = w4 * 32 + lane;  // TMEM lane: key row
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
         const int key = k0 + r;
-        const bool key_ok = key < Nk;
+        const bool key_in = key < Nk;                          // a row of dK / dV to write
+        const bool key_ok = key_in && key_kept(args, b, key);  // a key that takes part
+        const bool keys_masked = tile_keys_masked(args, b, k0, Nk);  // uniform
         int qlim, qlim_hi;  // queries [qlim, qlim_hi) see this key
         query_range<CAUSAL>(args, key, Nq, Nk, qlim, qlim_hi);
         // Every key of the tile sees queries [qall_lo, qall_hi): slices inside need no mask.
@@ -365,7 +367,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             // Masks matter only on the tile holding key Nk - 1 and, under a window mask
             // (causal included), on query columns outside some key's window (uniform per
             // warpgroup).
-            const bool need_mask = (k0 + 128 > Nk) || (CAUSAL && (qs < qall_lo || qs + 64 > qall_hi));
+            const bool need_mask =
+                (k0 + 128 > Nk) || keys_masked || (CAUSAL && (qs < qall_lo || qs + 64 > qall_hi));
             float pf[64];
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
@@ -465,7 +468,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     pk[i] = pack2<BF16>(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
-                if (key_ok) {
+                if (key_in) {
                     uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);

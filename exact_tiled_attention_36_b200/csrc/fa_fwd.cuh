@@ -66,6 +66,10 @@ struct FwdArgs {
     long long o_sb, o_ss, o_sh;  // O strides in elements: batch, token, head (d is contiguous)
     int wl, wr;       // MASKED: keys from wl before to wr after the aligned diagonal (< 0: unbounded)
     int n_anchor;     // kMaskAnchor: keys 0 .. n_anchor - 1 are visible below the window too
+    // Key mask (null: none): bit j % 32 of word b * kb_words + j / 32 set = key j of batch b
+    // is visible (ANDed with the mask kind).
+    const uint32_t* key_bits;
+    int kb_words;
     int nu;           // units (256 query rows) per sequence: ceil(Nq / 256)
     int n_units;      // nu * Hq * num_batches
     float scale_log2;  // scale * log2(e)
@@ -318,7 +322,9 @@ __device__ __forceinline__ void rms_normalise_row(uint8_t* tile, int r, float ep
 // factor of each (query tile, key tile) pair, and V's block factor v_j enters P as
 // 2^(log2(v_j / v_max)) before P is rounded to E4M3 (P <= 2^8 under the lazy
 // rescale, inside E4M3's range), so O = v_max * sum(P' V) / l. O is bf16.
-template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM, bool FP8 = false>
+// KEYMASK: args.key_bits masks keys too (a compile-time switch, so that the other
+// instantiations carry none of its per-tile work).
+template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM, bool FP8 = false, bool KEYMASK = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -650,10 +656,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const int lim = MASK == kMaskAnchor ? key_hi - kb : rel_hi - j * 128;
                 const int lim_lo = MASK == kMaskAnchor ? key_lo - kb : rel_lo - j * 128;
                 const int anc = args.n_anchor - kb;
+                // Key mask: the keep bits of this key tile's 128 keys (all set: nothing to do).
+                uint32_t kw0 = ~0u, kw1 = ~0u, kw2 = ~0u, kw3 = ~0u;
+                if constexpr (KEYMASK) {
+                    const int ktile = fwd_tile_of<MASK>(w, t, j);
+                    const uint32_t* kbp = args.key_bits + static_cast<size_t>(w.bidx) * args.kb_words + ktile * 4;
+                    const int rem = args.kb_words - ktile * 4;
+                    kw0 = rem > 0 ? kbp[0] : 0u;
+                    kw1 = rem > 1 ? kbp[1] : 0u;
+                    kw2 = rem > 2 ? kbp[2] : 0u;
+                    kw3 = rem > 3 ? kbp[3] : 0u;
+                }
+                const bool keys_masked = KEYMASK && (kw0 & kw1 & kw2 & kw3) != ~0u;
                 // (uniform per warp: only tiles on a window's edge pay for the mask)
                 const bool need_mask =
                     __any_sync(0xffffffffu, lim < 128 || (MASK == kMaskWindow && lim_lo > 0) ||
-                                                (MASK == kMaskAnchor && lim_lo > 0 && lim_lo > anc));
+                                                (MASK == kMaskAnchor && lim_lo > 0 && lim_lo > anc) || keys_masked);
                 uint32_t sv[4][32];
     #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
@@ -661,10 +679,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
                 if (need_mask) {  // masked columns read as -inf: out of the max, P = 0
     #pragma unroll
-                    for (int c = 0; c < 128; ++c)
+                    for (int c = 0; c < 128; ++c) {
+                        const uint32_t kw = c < 32 ? kw0 : (c < 64 ? kw1 : (c < 96 ? kw2 : kw3));
                         if (c >= lim || (MASK == kMaskWindow && c < lim_lo) ||
-                            (MASK == kMaskAnchor && c < lim_lo && c >= anc))
+                            (MASK == kMaskAnchor && c < lim_lo && c >= anc) || (KEYMASK && !((kw >> (c & 31)) & 1u)))
                             sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                    }
                 }
                 // Row max: 8 independent chains of three-input max.
                 float mxp[8];

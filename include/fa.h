@@ -162,6 +162,28 @@ fa_status fa_varlen_bwd_window(const void* q, const void* k, const void* v, cons
                                fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * Key-padding masks of any shape (not only a tail of each sequence): key j of
+ * batch b takes part iff bit j % 32 of key_bits[b * ceil(Nk/32) + j / 32] is set,
+ * on top of the causal mask when causal = 1; a query row left with no key gets
+ * O = 0 and lse = -inf. This is the general boolean key mask the unpad -> varlen
+ * path of the InternViT FlashAttention wrapper can only express as a tail; key
+ * tiles with every bit set pay nothing for it.
+ *   key_bits: DEVICE uint32 [B, ceil(Nk/32)], 4-byte aligned (bits past Nk ignored).
+ *   fa_pack_key_mask builds it from a DEVICE byte mask keep [B, Nk] (non-zero =
+ *   keep), asynchronously on `stream`.
+ * Every other argument, result and error is that of fa_fwd / fa_bwd (the backward
+ * takes the lse of fa_fwd_keymask with the same mask).
+ */
+fa_status fa_pack_key_mask(const unsigned char* keep, unsigned int* key_bits, int B, int Nk, fa_stream_t stream);
+fa_status fa_fwd_keymask(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const unsigned int* key_bits, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+fa_status fa_bwd_keymask(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                         const unsigned int* key_bits, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Forward with the query/key RMS normalisation fused in front of attention
  * (the InternViT attention applies an RMSNorm to Q and K, per head, just
  * before its FlashAttention call): with

@@ -281,3 +281,15 @@ def test_bwd_strided_rejects_before_launch(lib):
     assert fb.fa_bwd_strided(*{**a, "sdk": (4096, 1540, 64)}.values()) == fb.FA_ERR_MISALIGNED
     assert fb.fa_bwd_strided(*{**a, "ws": None}.values()) == fb.FA_ERR_INVALID_ARG
     assert fb.fa_bwd_strided(*{**a, "d": 96}.values()) == fb.FA_ERR_UNSUPPORTED
+
+
+def test_keymask_rejects_before_launch(lib):
+    assert fb.fa_fwd_keymask(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 8, 8, 128, 0.1, 0, fb.FA_BF16,
+                             None) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_fwd_keymask(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, 1, 2, 2, 8, 8, 128, 0.1, 0, fb.FA_BF16,
+                             None) == fb.FA_ERR_MISALIGNED
+    assert fb.fa_bwd_keymask(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 8, 8, 128,
+                             0.1, 0, fb.FA_BF16, None) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_pack_key_mask(None, FAKE, 1, 8, None) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_pack_key_mask(FAKE, FAKE + 1, 1, 8, None) == fb.FA_ERR_MISALIGNED
+    assert fb.fa_pack_key_mask(FAKE, FAKE, 1, 0, None) == fb.FA_OK
