@@ -77,12 +77,6 @@ fa_status make_map_strided(CUtensorMap* m, const void* base, int d, int H, int64
     return make_map_box(m, base, d, H, rows, batches, bf16, sh, ss, sb, 1, 128);
 }
 
-// Contiguous [batches, rows, H, d].
-fa_status make_map(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16) {
-    return make_map_strided(m, base, d, H, rows, batches, bf16, d, static_cast<int64_t>(H) * d,
-                            (rows < 1 ? 1 : rows) * H * static_cast<int64_t>(d));
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int* error_word() {

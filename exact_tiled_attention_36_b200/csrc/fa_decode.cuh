@@ -96,9 +96,17 @@ __device__ __forceinline__ int dec_active_warps(const DecodeArgs& a) {
     return a.nb > 1 ? a.nb : (a.R + 31) / 32;
 }
 
-// One item (sequence b, KV head hk): its keys and its first tile in the sequence of T.
+// The split balances cost, not tiles: an item of ntk > 0 key tiles costs
+// ntk + kDecItemCost units, the first kDecItemCost standing for a segment's fixed
+// work (loading Q, the first products, the epilogue). Otherwise a CTA whose share
+// starts many short items would take longer than one with the same tiles of a
+// single item.
+constexpr int kDecItemCost = 2;
+
+// One item (sequence b, KV head hk): its keys, and the first unit of its cost in the
+// sequence of T units (its tiles are units P + kDecItemCost ..).
 struct DecItem {
-    int b, hk, len, ntk;
+    int b, hk, len, ntk, cost;
     long long P;
 };
 
@@ -116,17 +124,29 @@ __device__ __forceinline__ DecItem dec_item(const DecodeArgs& a, int b, int hk, 
     it.P = P;
     it.len = dec_len<SEQLENS>(a, b);
     it.ntk = (it.len + 127) / 128;
+    it.cost = it.ntk > 0 ? it.ntk + kDecItemCost : 0;
     return it;
+}
+
+// The key tiles [j0, j0 + n) of item `it` in the cost range [s_lo, s_hi) of a CTA
+// (false: none).
+__device__ __forceinline__ bool dec_segment(long long s_lo, long long s_hi, const DecItem& it, int& j0, int& n) {
+    const long long r0 = it.P + kDecItemCost;  // the unit of the item's first tile
+    const long long lo = max(s_lo, r0), hi = min(s_hi, it.P + it.cost);
+    if (lo >= hi) return false;
+    j0 = static_cast<int>(lo - r0);
+    n = static_cast<int>(hi - lo);
+    return true;
 }
 
 // The item after `it`; past the last one P = T (the walk ends there).
 template <bool SEQLENS>
 __device__ __forceinline__ DecItem dec_next(const DecodeArgs& a, const DecItem& it, long long T) {
-    if (it.hk + 1 < a.Hkv) return dec_item<SEQLENS>(a, it.b, it.hk + 1, it.P + it.ntk);
-    if (it.b + 1 < a.B) return dec_item<SEQLENS>(a, it.b + 1, 0, it.P + it.ntk);
+    if (it.hk + 1 < a.Hkv) return dec_item<SEQLENS>(a, it.b, it.hk + 1, it.P + it.cost);
+    if (it.b + 1 < a.B) return dec_item<SEQLENS>(a, it.b + 1, 0, it.P + it.cost);
     DecItem e = it;
     e.P = T;
-    e.ntk = 0;
+    e.ntk = e.cost = 0;
     return e;
 }
 
@@ -164,8 +184,10 @@ __device__ __forceinline__ bool dec_locate(const DecodeArgs& args, uint8_t* misc
         int* sh_b0 = reinterpret_cast<int*>(misc + 24);
         long long* sh_P0 = reinterpret_cast<long long*>(misc + 32);
         long long* ws = reinterpret_cast<long long*>(misc + 48);  // [8] per-warp sums
-        auto tiles_of = [&](int b) -> long long {
-            return b < args.B ? static_cast<long long>(args.Hkv) * ((dec_len<true>(args, b) + 127) / 128) : 0;
+        auto tiles_of = [&](int b) -> long long {  // cost units of sequence b (all its KV heads)
+            if (b >= args.B) return 0;
+            const int ntk = (dec_len<true>(args, b) + 127) / 128;
+            return ntk > 0 ? static_cast<long long>(args.Hkv) * (ntk + kDecItemCost) : 0;
         };
         long long v = 0;
         for (int b = tid; b < args.B; b += kDecThreads) v += tiles_of(b);
@@ -215,7 +237,8 @@ __device__ __forceinline__ bool dec_locate(const DecodeArgs& args, uint8_t* misc
         b0 = *sh_b0;
         P0 = *sh_P0;
     } else {
-        const long long per_b = static_cast<long long>(args.Hkv) * ((args.Nk + 127) / 128);
+        const int ntk = (args.Nk + 127) / 128;
+        const long long per_b = ntk > 0 ? static_cast<long long>(args.Hkv) * (ntk + kDecItemCost) : 0;
         T = per_b * args.B;
         s_lo = dec_split(cta, T, G);
         s_hi = dec_split(cta + 1, T, G);
@@ -223,12 +246,12 @@ __device__ __forceinline__ bool dec_locate(const DecodeArgs& args, uint8_t* misc
         b0 = static_cast<int>(s_lo / per_b);
         P0 = b0 * per_b;
     }
-    const int ntk = (dec_len<SEQLENS>(args, b0) + 127) / 128;
-    const int hk = static_cast<int>((s_lo - P0) / ntk);
+    const int cost = (dec_len<SEQLENS>(args, b0) + 127) / 128 + kDecItemCost;  // of each KV head of b0
+    const int hk = static_cast<int>((s_lo - P0) / cost);
     rg.T = T;
     rg.s_lo = s_lo;
     rg.s_hi = s_hi;
-    rg.first = dec_item<SEQLENS>(args, b0, hk, P0 + static_cast<long long>(hk) * ntk);
+    rg.first = dec_item<SEQLENS>(args, b0, hk, P0 + static_cast<long long>(hk) * cost);
     return true;
 }
 
@@ -289,10 +312,10 @@ __device__ __forceinline__ void dec_produce(const DecodeArgs& args, const DecRan
         }
     };
     for (DecItem it = rg.first; ok && it.P < rg.s_hi; it = dec_next<SEQLENS>(args, it, rg.T)) {
-        const long long lo = max(rg.s_lo, it.P), hi = min(rg.s_hi, it.P + it.ntk);
-        if (lo >= hi) continue;
-        const int j0 = static_cast<int>(lo - it.P), n = static_cast<int>(hi - lo);
-        if (SEQLENS && lo == it.P) args.meta[1 + static_cast<size_t>(it.b) * args.Hkv + it.hk] = it.P;
+        if (SEQLENS && it.cost > 0 && it.P >= rg.s_lo)  // the item starts in this CTA's range
+            args.meta[1 + static_cast<size_t>(it.b) * args.Hkv + it.hk] = it.P;
+        int j0, n;
+        if (!dec_segment(rg.s_lo, rg.s_hi, it, j0, n)) continue;
         // Q of the group once the last S product of the segment that used this buffer
         // before has read it.
         const int qb = nq % QB;
@@ -456,9 +479,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             int gk = 0, nq = 0;
             bool ok = true;
             for (DecItem it = first; ok && it.P < s_hi; it = dec_next<SEQLENS>(args, it, T)) {
-                const long long lo = max(s_lo, it.P), hi = min(s_hi, it.P + it.ntk);
-                if (lo >= hi) continue;
-                const int n = static_cast<int>(hi - lo);
+                int j0, n;
+                if (!dec_segment(s_lo, s_hi, it, j0, n)) continue;
                 if (!(ok = mbar_wait(q_full, nq & 1, wc, 83))) break;
                 for (int j = 0; ok && j < min(n, 2); ++j) {
                     const int gg = gk + j;
@@ -519,9 +541,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         int gk = 0, nq = 0;
         bool ok = true;
         for (DecItem it = first; ok && it.P < s_hi; it = dec_next<SEQLENS>(args, it, T)) {
-            const long long lo = max(s_lo, it.P), hi = min(s_hi, it.P + it.ntk);
-            if (lo >= hi) continue;
-            const int j0 = static_cast<int>(lo - it.P), n = static_cast<int>(hi - lo);
+            int j0, n;
+            if (!dec_segment(s_lo, s_hi, it, j0, n)) continue;
             // This row's keys [0, key_hi), relative to the segment's first key.
             int key_hi = it.len;
             if (causal) key_hi = min(it.len, t + it.len - args.Nq + 1);
@@ -844,9 +865,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             int gk = 0, nq = 0;
             bool ok = true;
             for (DecItem it = rg.first; ok && it.P < rg.s_hi; it = dec_next<SEQLENS>(args, it, rg.T)) {
-                const long long lo = max(rg.s_lo, it.P), hi = min(rg.s_hi, it.P + it.ntk);
-                if (lo >= hi) continue;
-                const int n = static_cast<int>(hi - lo);
+                int j0, n;
+                if (!dec_segment(rg.s_lo, rg.s_hi, it, j0, n)) continue;
                 const int qb = nq & 1;
                 q_addr = smem_u32(sQ + qb * C::kQBytes);
                 if (!(ok = mbar_wait(&q_full[qb], (nq >> 1) & 1, wc, 100))) break;
@@ -926,9 +946,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         int n_red0 = 0, n_red1 = 0;  // uses of xb_red[0], xb_red[1] so far
         bool ok = true;
         for (DecItem it = rg.first; ok && it.P < rg.s_hi; it = dec_next<SEQLENS>(args, it, rg.T)) {
-            const long long lo = max(rg.s_lo, it.P), hi = min(rg.s_hi, it.P + it.ntk);
-            if (lo >= hi) continue;
-            const int j0 = static_cast<int>(lo - it.P), n = static_cast<int>(hi - lo);
+            int j0, n;
+            if (!dec_segment(rg.s_lo, rg.s_hi, it, j0, n)) continue;
             // Row r (token r / g) sees keys below min(len, r / g + len - Nq + 1) under the
             // causal mask, below len otherwise.
             const int causal_base = it.len - args.Nq + 1;
@@ -1136,14 +1155,15 @@ __global__ void __launch_bounds__(128) fa_decode_combine(const DecodeArgs a) {
             T = a.meta[0];
             P = a.meta[1 + item];
         } else {
-            T = static_cast<long long>(a.B) * a.Hkv * ntk;
-            P = static_cast<long long>(item) * ntk;
+            T = static_cast<long long>(a.B) * a.Hkv * (ntk + kDecItemCost);
+            P = static_cast<long long>(item) * (ntk + kDecItemCost);
         }
     }
+    // The CTAs whose cost range holds one of the item's tiles (units P + kDecItemCost ..).
     int c0 = 0, c1 = -1;
     if (ntk > 0 && T > 0) {
-        c0 = dec_cta_of(P, T, a.G);
-        c1 = dec_cta_of(P + ntk - 1, T, a.G);
+        c0 = dec_cta_of(P + kDecItemCost, T, a.G);
+        c1 = dec_cta_of(P + kDecItemCost + ntk - 1, T, a.G);
     }
     // CTA c's range is empty only when there are fewer tiles than CTAs.
     const bool all_have = T >= a.G;
