@@ -337,6 +337,33 @@ def run_ours(args):
         raise RuntimeError("device error during the timed region")
     total_ms = max_over_ranks(total_ms, world, "cuda")
 
+    # The forward's own metric: forward calls back to back (no backward between them, so
+    # the GPU is not held at the power cap the step loop settles at); the tensors touched
+    # per call (~340 MB) are larger than the L2.
+    n_fwd = max(10, min(3 * K, 30))
+
+    def fwd_call():
+        st = fb.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d,
+                       scale, 1, dt, sh)
+        if st != fb.FA_OK:
+            raise RuntimeError(fb.fa_status_string(st))
+
+    torch.cuda.synchronize()
+    time.sleep(0.5)  # let the clocks recover from the step loop
+    for _ in range(3):
+        fwd_call()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(n_fwd):
+        fwd_call()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    fwd_alone_ms = max_over_ranks(f0.elapsed_time(f1), world, "cuda") / n_fwd
+
     # end to end through the C ABI with host buffers: H2D of q, k, v, dO from
     # pinned memory, fwd + bwd, D2H of dq, dk, dv, every step.
     hq, hk, hv, hdo = (t.pin_memory() for t in (fi.q, fi.k, fi.v, fi.do))
@@ -401,13 +428,16 @@ def run_ours(args):
         "bwd_frac_of_sustained": f_bwd / (bwd_avg / 1e3) / 1e12 / peak,
         "bwd_frac_of_burst": f_bwd / (bwd_avg / 1e3) / 1e12 / peak_burst,
         "fwd_ms": fwd_avg, "bwd_ms": bwd_avg, "bwd_main_kernel_ms": main_avg,
+        "fwd_alone": {"calls": n_fwd, "ms": fwd_alone_ms, "tflops": f_fwd / (fwd_alone_ms / 1e3) / 1e12,
+                      "frac_of_burst": f_fwd / (fwd_alone_ms / 1e3) / 1e12 / peak_burst,
+                      "how": "forward calls back to back after the step loop, CUDA events, max over ranks"},
         "roofline": {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "peak_kind": f"bf16_tflops_sustained ({peak_src})",
                      "peak_burst": peak_burst, "frac_of_burst": achieved / peak_burst,
                      "traffic": profiled_traffic(kname)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": K_e2e},
-        "gpu_launches": K * 4,
+        "gpu_launches": K * 4,  # per step: forward, preprocess, main backward, dQ convert
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
