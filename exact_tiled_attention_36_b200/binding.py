@@ -1,7 +1,9 @@
 """Thin ctypes binding of libfa.so.
 
 The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_fwd_strided``, ``fa_varlen_fwd_strided``, ``fa_fwd_qk_rmsnorm``,
-``fa_fwd_window``, ``fa_bwd_window``, ``fa_varlen_fwd_window``, ``fa_varlen_bwd_window``, ``fa_fwd_window_anchor``, ``fa_bwd_window_anchor``, ``fa_bwd_strided``, ``fa_pack_key_mask``,
+``fa_fwd_window``, ``fa_bwd_window``, ``fa_varlen_fwd_window``, ``fa_varlen_bwd_window``, ``fa_fwd_window_anchor``,
+``fa_bwd_window_anchor``, ``fa_varlen_fwd_window_anchor``, ``fa_varlen_bwd_window_anchor``, ``fa_bwd_strided``,
+``fa_pack_key_mask``,
 ``fa_fwd_keymask``, ``fa_bwd_keymask``, ``fa_fwd_fp8``, ``fa_decode``, ``fa_decode_paged``, ``fa_decode_workspace_size``,
 ``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
 ``fa_bwd``, ``fa_status_string`` and ``fa_get_last_device_error`` have the
@@ -62,6 +64,8 @@ _SIGS = {
     "fa_bwd_window_anchor": ([_P] * 10 + [_I] * 6 + [_F, _I, _I, _I, _I, _P], _I),
     "fa_varlen_fwd_window": ([_P] * 7 + [_I] * 8 + [_F, _I, _I, _I, _P], _I),
     "fa_varlen_bwd_window": ([_P] * 12 + [_I] * 8 + [_F, _I, _I, _I, _P], _I),
+    "fa_varlen_fwd_window_anchor": ([_P] * 7 + [_I] * 8 + [_F, _I, _I, _I, _I, _P], _I),
+    "fa_varlen_bwd_window_anchor": ([_P] * 12 + [_I] * 8 + [_F, _I, _I, _I, _I, _P], _I),
     "fa_decode": ([_P] * 7 + [_I] * 6 + [_F, _I, _I, _P], _I),
     "fa_decode_paged": ([_P] * 8 + [_I] * 8 + [_F, _I, _I, _P], _I),
 }
@@ -218,6 +222,22 @@ def fa_varlen_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlen
     return lib().fa_varlen_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k,
                                       num_seqs, total_q, total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale,
                                       window_left, window_right, dtype, stream)
+
+
+def fa_varlen_fwd_window_anchor(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q, total_k, max_seqlen_q,
+                                max_seqlen_k, Hq, Hkv, d, scale, window_left, window_right, n_anchor, dtype,
+                                stream) -> int:
+    return lib().fa_varlen_fwd_window_anchor(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q, total_k,
+                                             max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, window_left, window_right,
+                                             n_anchor, dtype, stream)
+
+
+def fa_varlen_bwd_window_anchor(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs,
+                                total_q, total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, window_left,
+                                window_right, n_anchor, dtype, stream) -> int:
+    return lib().fa_varlen_bwd_window_anchor(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q,
+                                             cu_seqlens_k, num_seqs, total_q, total_k, max_seqlen_q, max_seqlen_k, Hq,
+                                             Hkv, d, scale, window_left, window_right, n_anchor, dtype, stream)
 
 
 def fa_fwd_fp8(q, k, v, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream) -> int:

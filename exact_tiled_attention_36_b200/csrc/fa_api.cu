@@ -166,7 +166,8 @@ fa_status launch_fwd_b(int mask, bool varlen, bool qknorm, const CUtensorMap& mq
     }
     if (mask == W) return varlen ? launch_fwd_t<D, BF16, W, true, false>(mq, mk, mv, a, grid, s)
                                  : launch_fwd_t<D, BF16, W, false, false>(mq, mk, mv, a, grid, s);
-    if (mask == A) return varlen ? FA_ERR_UNSUPPORTED : launch_fwd_t<D, BF16, A, false, false>(mq, mk, mv, a, grid, s);
+    if (mask == A) return varlen ? launch_fwd_t<D, BF16, A, true, false>(mq, mk, mv, a, grid, s)
+                                 : launch_fwd_t<D, BF16, A, false, false>(mq, mk, mv, a, grid, s);
     if (mask == C) return varlen ? launch_fwd_t<D, BF16, C, true, false>(mq, mk, mv, a, grid, s)
                                  : launch_fwd_t<D, BF16, C, false, false>(mq, mk, mv, a, grid, s);
     return varlen ? launch_fwd_t<D, BF16, N, true, false>(mq, mk, mv, a, grid, s)
@@ -483,7 +484,7 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
                      Strides sv, Strides so, const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
                      int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d,
                      float scale, int causal, fa_dtype dtype, fa_stream_t stream, bool window = false, int wl = -1,
-                     int wr = 0) {
+                     int wr = 0, int n_anchor = 0) {
     if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
         return FA_ERR_INVALID_ARG;
     if (!cu_seqlens_q || !cu_seqlens_k || (total_q > 0 && (!q || !o || !lse)) || (total_k > 0 && (!k || !v)))
@@ -518,6 +519,7 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
     a.o_sh = so.h;
     a.wl = window ? wl : -1;
     a.wr = window ? wr : 0;
+    a.n_anchor = window ? n_anchor : 0;
     a.cu_q = cu_seqlens_q;
     a.cu_k = cu_seqlens_k;
     a.num_batches = num_seqs;
@@ -530,8 +532,9 @@ fa_status fwd_varlen(const void* q, const void* k, const void* v, void* o, float
     a.err = err;
     dim3 grid;
     if ((st = fwd_units(a, num_seqs, max_seqlen_q, grid)) != FA_OK) return st;
-    return launch_fwd(d, bf16, window ? fa::kMaskWindow : (causal ? fa::kMaskCausal : fa::kMaskNone), true, false,
-                      mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
+    const int mask = window ? (a.n_anchor > 0 ? fa::kMaskAnchor : fa::kMaskWindow)
+                            : (causal ? fa::kMaskCausal : fa::kMaskNone);
+    return launch_fwd(d, bf16, mask, true, false, mq, mk, mv, a, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // The FP8 forward (fixed length, d = 128): E4M3 q, k, v with per-block factors.
@@ -813,13 +816,13 @@ fa_status decode_common(const void* q, const void* k, const void* v, void* o, fl
                 : launch_dec_b<128, false>(rn, false, sl, paged, mq, mk, mv, a, causal, run_split, s);
 }
 
-// The backward of fa_varlen_bwd / fa_varlen_bwd_window; the masked kernels take the
-// window (wl, wr) (causal: (-1, 0)).
+// The backward of fa_varlen_bwd / fa_varlen_bwd_window(_anchor); the masked kernels
+// take the window (wl, wr) (causal: (-1, 0)) and the anchor keys of every sequence.
 fa_status varlen_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dout, void* dq, void* dk, void* dv, void* workspace, const int* cu_seqlens_q,
                      const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
                      int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
-                     fa_stream_t stream, int wl = -1, int wr = 0) {
+                     fa_stream_t stream, int wl = -1, int wr = 0, int n_anchor = 0) {
     if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
         return FA_ERR_INVALID_ARG;
     if (!cu_seqlens_q || !cu_seqlens_k || !workspace || (total_q > 0 && (!q || !o || !lse || !dout || !dq)) ||
@@ -835,7 +838,7 @@ fa_status varlen_bwd(const void* q, const void* k, const void* v, const void* o,
     if (num_seqs > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
     return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, num_seqs, cu_seqlens_q, cu_seqlens_k, total_q,
                       total_k, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal != 0, dtype == FA_BF16,
-                      reinterpret_cast<cudaStream_t>(stream), wl, wr);
+                      reinterpret_cast<cudaStream_t>(stream), wl, wr, n_anchor);
 }
 
 }  // namespace
@@ -1080,6 +1083,36 @@ fa_status fa_varlen_bwd_window(const void* q, const void* k, const void* v, cons
     const bool masked = wl >= 0 || wr >= 0;
     return varlen_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q,
                       total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, masked ? 1 : 0, dtype, stream, wl, wr);
+}
+
+fa_status fa_varlen_fwd_window_anchor(const void* q, const void* k, const void* v, void* o, float* lse,
+                                      const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs, int total_q,
+                                      int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d,
+                                      float scale, int window_left, int window_right, int n_anchor, fa_dtype dtype,
+                                      fa_stream_t stream) {
+    if (n_anchor < 0) return FA_ERR_INVALID_ARG;
+    const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
+    if (n_anchor == 0 || wl < 0)  // no anchors, or nothing below the window to add
+        return fa_varlen_fwd_window(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q, total_k,
+                                    max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, wl, wr, dtype, stream);
+    return fwd_varlen(q, k, v, o, lse, contiguous(total_q, Hq, d), contiguous(total_k, Hkv, d),
+                      contiguous(total_k, Hkv, d), contiguous(total_q, Hq, d), cu_seqlens_q, cu_seqlens_k, num_seqs,
+                      total_q, total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, 0, dtype, stream, true, wl, wr,
+                      n_anchor);
+}
+
+fa_status fa_varlen_bwd_window_anchor(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                      const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                                      const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs, int total_q,
+                                      int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d,
+                                      float scale, int window_left, int window_right, int n_anchor, fa_dtype dtype,
+                                      fa_stream_t stream) {
+    if (n_anchor < 0) return FA_ERR_INVALID_ARG;
+    const int wl = window_left < 0 ? -1 : window_left, wr = window_right < 0 ? -1 : window_right;
+    const bool masked = wl >= 0 || wr >= 0;
+    return varlen_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q,
+                      total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, masked ? 1 : 0, dtype, stream, wl, wr,
+                      wl >= 0 ? n_anchor : 0);
 }
 
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_scale, const float* k_scale,

@@ -162,6 +162,28 @@ fa_status fa_varlen_bwd_window(const void* q, const void* k, const void* v, cons
                                fa_dtype dtype, fa_stream_t stream);
 
 /*
+ * The window with global anchor keys (fa_fwd_window_anchor / fa_bwd_window_anchor) on
+ * packed variable-length batches: within every sequence its first n_anchor keys are
+ * the anchors (key j of sequence s, counted from cu_seqlens_k[s], is visible to its
+ * query i iff j <= a + window_right (when window_right >= 0) and (j >= a - window_left
+ * or j < n_anchor), a = i + Nk_s - Nq_s). n_anchor >= 0 (FA_ERR_INVALID_ARG
+ * otherwise); n_anchor = 0, or window_left < 0, is exactly fa_varlen_fwd_window /
+ * fa_varlen_bwd_window. Every other argument, result and error is that of those calls.
+ */
+fa_status fa_varlen_fwd_window_anchor(const void* q, const void* k, const void* v, void* o, float* lse,
+                                      const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                                      int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                                      int Hq, int Hkv, int d, float scale, int window_left, int window_right,
+                                      int n_anchor, fa_dtype dtype, fa_stream_t stream);
+fa_status fa_varlen_bwd_window_anchor(const void* q, const void* k, const void* v, const void* o,
+                                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                      void* workspace, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                      int num_seqs, int total_q, int total_k, int max_seqlen_q,
+                                      int max_seqlen_k, int Hq, int Hkv, int d, float scale,
+                                      int window_left, int window_right, int n_anchor,
+                                      fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Key-padding masks of any shape (not only a tail of each sequence): key j of
  * batch b takes part iff bit j % 32 of key_bits[b * ceil(Nk/32) + j / 32] is set,
  * on top of the causal mask when causal = 1; a query row left with no key gets

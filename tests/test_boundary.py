@@ -293,3 +293,15 @@ def test_keymask_rejects_before_launch(lib):
     assert fb.fa_pack_key_mask(None, FAKE, 1, 8, None) == fb.FA_ERR_INVALID_ARG
     assert fb.fa_pack_key_mask(FAKE, FAKE + 1, 1, 8, None) == fb.FA_ERR_MISALIGNED
     assert fb.fa_pack_key_mask(FAKE, FAKE, 1, 0, None) == fb.FA_OK
+
+
+def test_varlen_window_anchor_rejects_before_launch(lib):
+    base = [FAKE] * 5 + [FAKE, FAKE, 2, 256, 256, 128, 128, 4, 2, 128, 0.1, 64, 0]
+    assert fb.fa_varlen_fwd_window_anchor(*base, -1, fb.FA_BF16, None) == fb.FA_ERR_INVALID_ARG
+    no_cu = [FAKE] * 5 + [None, FAKE] + base[7:]
+    assert fb.fa_varlen_fwd_window_anchor(*no_cu, 4, fb.FA_BF16, None) == fb.FA_ERR_INVALID_ARG
+    bwd = [FAKE] * 12 + [2, 256, 256, 128, 128, 4, 2, 128, 0.1, 64, 0]
+    assert fb.fa_varlen_bwd_window_anchor(*bwd, -1, fb.FA_BF16, None) == fb.FA_ERR_INVALID_ARG
+    d64 = bwd[:19] + [64] + bwd[20:]
+    assert fb.fa_varlen_bwd_window_anchor(*d64, 4, fb.FA_BF16, None) == fb.FA_ERR_UNSUPPORTED
+    assert fb.fa_varlen_bwd_window_anchor(*bwd, 4, fb.FA_BF16 + 7, None) == fb.FA_ERR_UNSUPPORTED

@@ -119,13 +119,20 @@ VARLEN_CASES = [
     ([700, 1, 0, 300, 129], 4, 2, 128, (128, 0), "bf16", 0.0),
     ([513, 64, 900], 2, 2, 128, (100, 50), "fp16", 0.25),
     ([257, 1000, 5], 4, 1, 64, (-1, 40), "bf16", 0.0),
+    # with global anchors (wl, wr, n_anchor): the first n_anchor keys of every sequence
+    ([700, 1, 0, 300, 129], 4, 2, 128, (128, 0, 4), "bf16", 0.0),
+    ([513, 64, 900], 2, 2, 128, (100, 50, 130), "fp16", 0.25),
+    ([1100, 257, 640], 2, 1, 128, (200, -1, 300), "bf16", 0.0),
+    ([257, 1000, 5], 4, 1, 64, (60, 0, 200), "bf16", 0.0),
 ]
 
 
-@pytest.mark.parametrize("case", VARLEN_CASES, ids=lambda c: f"{len(c[0])}seq-h{c[1]}-{c[2]}-d{c[3]}-w{c[4][0]}_{c[4][1]}")
+@pytest.mark.parametrize("case", VARLEN_CASES,
+                         ids=lambda c: f"{len(c[0])}seq-h{c[1]}-{c[2]}-d{c[3]}-w" + "_".join(map(str, c[4])))
 def test_varlen_window(case):
-    """fa_varlen_fwd_window (and, for d = 128, fa_varlen_bwd_window): every sequence
-    against the oracle with the window applied within that sequence."""
+    """fa_varlen_fwd_window (and, for d = 128, fa_varlen_bwd_window), or with anchors
+    fa_varlen_fwd_window_anchor / fa_varlen_bwd_window_anchor: every sequence against
+    the oracle with the window (and anchors) applied within that sequence."""
     lengths, Hq, Hkv, d, window, dt, pad = case
     vi = inputs.make_varlen(inputs.VARLEN, lengths=lengths, Hq=Hq, Hkv=Hkv, d=d, dtype=dt, key_pad_frac=pad,
                             seed=87, with_do=True)
@@ -135,10 +142,12 @@ def test_varlen_window(case):
     code = fb.FA_BF16 if q.dtype == torch.bfloat16 else fb.FA_FP16
     o, o_ok = guarded((Tq, Hq, d), q.dtype)
     lse, l_ok = guarded((Hq, Tq), torch.float32)
-    wl, wr = window
-    st = fb.fa_varlen_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                 cu_q.data_ptr(), cu_k.data_ptr(), n, Tq, Tk, vi.max_seqlen_q, vi.max_seqlen_k, Hq,
-                                 Hkv, d, d ** -0.5, wl, wr, code, 0)
+    wl, wr = window[:2]
+    anchors = tuple(window[2:])  # (n_anchor,) or ()
+    fwd = fb.fa_varlen_fwd_window_anchor if anchors else fb.fa_varlen_fwd_window
+    st = fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), cu_q.data_ptr(),
+             cu_k.data_ptr(), n, Tq, Tk, vi.max_seqlen_q, vi.max_seqlen_k, Hq, Hkv, d, d ** -0.5, wl, wr, *anchors,
+             code, 0)
     assert st == fb.FA_OK, fb.fa_status_string(st)
     torch.cuda.synchronize()
     assert fb.fa_get_last_device_error(None) == fb.FA_OK and o_ok() and l_ok()
@@ -153,10 +162,10 @@ def test_varlen_window(case):
         return
     ws = torch.empty(fb.fa_varlen_bwd_workspace_size(n, Tq, vi.max_seqlen_q, Hq, d), dtype=torch.uint8, device="cuda")
     dq, dk, dv = torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)
-    st = fb.fa_varlen_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
-                                 cu_q.data_ptr(), cu_k.data_ptr(), n, Tq, Tk, vi.max_seqlen_q, vi.max_seqlen_k, Hq,
-                                 Hkv, d, d ** -0.5, wl, wr, code, 0)
+    bwd = fb.fa_varlen_bwd_window_anchor if anchors else fb.fa_varlen_bwd_window
+    st = bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(), dq.data_ptr(),
+             dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), cu_q.data_ptr(), cu_k.data_ptr(), n, Tq, Tk,
+             vi.max_seqlen_q, vi.max_seqlen_k, Hq, Hkv, d, d ** -0.5, wl, wr, *anchors, code, 0)
     assert st == fb.FA_OK, fb.fa_status_string(st)
     torch.cuda.synchronize()
     assert fb.fa_get_last_device_error(None) == fb.FA_OK
