@@ -3,6 +3,7 @@
 The functions ``fa_fwd``, ``fa_varlen_fwd``, ``fa_fwd_strided``, ``fa_varlen_fwd_strided``, ``fa_fwd_qk_rmsnorm``,
 ``fa_fwd_window``, ``fa_bwd_window``, ``fa_varlen_fwd_window``, ``fa_varlen_bwd_window``, ``fa_fwd_window_anchor``,
 ``fa_bwd_window_anchor``, ``fa_varlen_fwd_window_anchor``, ``fa_varlen_bwd_window_anchor``, ``fa_bwd_strided``,
+``fa_varlen_bwd_strided``,
 ``fa_pack_key_mask``,
 ``fa_fwd_keymask``, ``fa_bwd_keymask``, ``fa_fwd_fp8``, ``fa_decode``, ``fa_decode_paged``, ``fa_decode_workspace_size``,
 ``fa_bwd_workspace_size``, ``fa_varlen_bwd``,
@@ -60,6 +61,7 @@ _SIGS = {
     "fa_fwd_keymask": ([_P] * 6 + [_I] * 6 + [_F, _I, _I, _P], _I),
     "fa_bwd_keymask": ([_P] * 11 + [_I] * 6 + [_F, _I, _I, _P], _I),
     "fa_bwd_strided": ([_P] * 18 + [_I] * 6 + [_F, _I, _I, _P], _I),
+    "fa_varlen_bwd_strided": ([_P] * 20 + [_I] * 8 + [_F, _I, _I, _P], _I),
     "fa_fwd_window_anchor": ([_P] * 5 + [_I] * 6 + [_F, _I, _I, _I, _I, _P], _I),
     "fa_bwd_window_anchor": ([_P] * 10 + [_I] * 6 + [_F, _I, _I, _I, _I, _P], _I),
     "fa_varlen_fwd_window": ([_P] * 7 + [_I] * 8 + [_F, _I, _I, _I, _P], _I),
@@ -195,6 +197,18 @@ def fa_bwd_strided(q, k, v, o, lse, dout, dq, dk, dv, workspace, q_strides, k_st
                                 _strides(k_strides), _strides(v_strides), _strides(o_strides), _strides(do_strides),
                                 _strides(dq_strides), _strides(dk_strides), _strides(dv_strides), B, Hq, Hkv, Nq, Nk,
                                 d, scale, causal, dtype, stream)
+
+
+def fa_varlen_bwd_strided(q, k, v, o, lse, dout, dq, dk, dv, workspace, q_strides, k_strides, v_strides, o_strides,
+                          do_strides, dq_strides, dk_strides, dv_strides, cu_seqlens_q, cu_seqlens_k, num_seqs,
+                          total_q, total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype,
+                          stream) -> int:
+    """*_strides: (token, head) element strides (host), as fa_varlen_fwd_strided."""
+    return lib().fa_varlen_bwd_strided(q, k, v, o, lse, dout, dq, dk, dv, workspace, _strides(q_strides),
+                                       _strides(k_strides), _strides(v_strides), _strides(o_strides),
+                                       _strides(do_strides), _strides(dq_strides), _strides(dk_strides),
+                                       _strides(dv_strides), cu_seqlens_q, cu_seqlens_k, num_seqs, total_q, total_k,
+                                       max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream)
 
 
 def fa_fwd_window_anchor(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, window_left, window_right, n_anchor, dtype,

@@ -822,7 +822,8 @@ fa_status varlen_bwd(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, void* dq, void* dk, void* dv, void* workspace, const int* cu_seqlens_q,
                      const int* cu_seqlens_k, int num_seqs, int total_q, int total_k, int max_seqlen_q,
                      int max_seqlen_k, int Hq, int Hkv, int d, float scale, int causal, fa_dtype dtype,
-                     fa_stream_t stream, int wl = -1, int wr = 0, int n_anchor = 0) {
+                     fa_stream_t stream, int wl = -1, int wr = 0, int n_anchor = 0,
+                     const BwdStrides* bs = nullptr) {
     if (num_seqs < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
         return FA_ERR_INVALID_ARG;
     if (!cu_seqlens_q || !cu_seqlens_k || !workspace || (total_q > 0 && (!q || !o || !lse || !dout || !dq)) ||
@@ -838,7 +839,7 @@ fa_status varlen_bwd(const void* q, const void* k, const void* v, const void* o,
     if (num_seqs > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
     return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, workspace, num_seqs, cu_seqlens_q, cu_seqlens_k, total_q,
                       total_k, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal != 0, dtype == FA_BF16,
-                      reinterpret_cast<cudaStream_t>(stream), wl, wr, n_anchor);
+                      reinterpret_cast<cudaStream_t>(stream), wl, wr, n_anchor, bs);
 }
 
 }  // namespace
@@ -1060,6 +1061,32 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
                         fa_stream_t stream) {
     return varlen_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q,
                       total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream);
+}
+
+fa_status fa_varlen_bwd_strided(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                                const long long* q_strides, const long long* k_strides, const long long* v_strides,
+                                const long long* o_strides, const long long* do_strides,
+                                const long long* dq_strides, const long long* dk_strides,
+                                const long long* dv_strides, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                int num_seqs, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int Hq,
+                                int Hkv, int d, float scale, int causal, fa_dtype dtype, fa_stream_t stream) {
+    const long long* given[8] = {q_strides, k_strides, v_strides, o_strides, do_strides, dq_strides, dk_strides,
+                                 dv_strides};
+    Strides t[8];
+    fa_status st;
+    for (int i = 0; i < 8; ++i) {
+        if ((st = read_strides(given[i], false, &t[i])) != FA_OK) return st;
+        if ((st = check_strides(t[i], false)) != FA_OK) return st;
+    }
+    // One "batch" of all packed rows: its stride only sizes the TMA maps' last dimension.
+    auto s3 = [](const Strides& x, int rows) {
+        return fa::Strides3{x.s * static_cast<long long>(rows > 0 ? rows : 1), x.s, x.h};
+    };
+    const BwdStrides bs{s3(t[0], total_q), s3(t[1], total_k), s3(t[2], total_k), s3(t[3], total_q),
+                        s3(t[4], total_q), s3(t[5], total_q), s3(t[6], total_k), s3(t[7], total_k)};
+    return varlen_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, num_seqs, total_q,
+                      total_k, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, scale, causal, dtype, stream, -1, 0, 0, &bs);
 }
 
 fa_status fa_varlen_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -357,6 +357,26 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
                         fa_stream_t stream);
 
 /*
+ * Backward of packed variable-length batches on strided views: the gradients of
+ * fa_varlen_fwd / fa_varlen_fwd_strided for q, k, v, o, dout, dq, dk, dv that are not
+ * contiguous, e.g. a packed (total, 3, H, d) QKV buffer with its gradient dqkv in the
+ * same layout. *_strides: HOST arrays {token, head} of element strides with the rules
+ * of fa_varlen_fwd_strided; dq, dk and dv must not overlap each other or the inputs.
+ * lse and the workspace keep their layouts. Every other argument, result and error is
+ * that of fa_varlen_bwd (d = 128).
+ */
+fa_status fa_varlen_bwd_strided(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                void* workspace, const long long* q_strides,
+                                const long long* k_strides, const long long* v_strides,
+                                const long long* o_strides, const long long* do_strides,
+                                const long long* dq_strides, const long long* dk_strides,
+                                const long long* dv_strides, const int* cu_seqlens_q,
+                                const int* cu_seqlens_k, int num_seqs, int total_q, int total_k,
+                                int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d,
+                                float scale, int causal, fa_dtype dtype, fa_stream_t stream);
+
+/*
  * Decode: attention of the Nq newest query tokens of each sequence against a
  * long key/value cache (Nq = 1 for one generated token, a few for speculative
  * decoding), by the same tiled online softmax as the forward ("FlashAttention/zh",

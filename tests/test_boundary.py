@@ -305,3 +305,17 @@ def test_varlen_window_anchor_rejects_before_launch(lib):
     d64 = bwd[:19] + [64] + bwd[20:]
     assert fb.fa_varlen_bwd_window_anchor(*d64, 4, fb.FA_BF16, None) == fb.FA_ERR_UNSUPPORTED
     assert fb.fa_varlen_bwd_window_anchor(*bwd, 4, fb.FA_BF16 + 7, None) == fb.FA_ERR_UNSUPPORTED
+
+
+def test_varlen_bwd_strided_rejects_before_launch(lib):
+    st = (3 * 4 * 128, 128)
+    ptrs = [FAKE] * 10
+    strides = [st] * 8
+    tail = [FAKE, FAKE, 2, 256, 256, 128, 128, 4, 4, 128, 0.1, 0, fb.FA_BF16, None]
+    assert fb.fa_varlen_bwd_strided(*ptrs, *strides[:5], None, *strides[6:], *tail) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_varlen_bwd_strided(*ptrs, *strides[:6], (1540, 64), st, *tail) == fb.FA_ERR_MISALIGNED
+    assert fb.fa_varlen_bwd_strided(*ptrs, *strides[:7], (0, 128), *tail) == fb.FA_ERR_INVALID_ARG
+    d64 = tail[:9] + [64] + tail[10:]
+    assert fb.fa_varlen_bwd_strided(*ptrs, *strides, *d64) == fb.FA_ERR_UNSUPPORTED
+    no_ws = [FAKE] * 9 + [None]
+    assert fb.fa_varlen_bwd_strided(*no_ws, *strides, *tail) == fb.FA_ERR_INVALID_ARG

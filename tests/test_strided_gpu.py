@@ -137,3 +137,53 @@ def test_packed_qkv_backward(B, N, H, d, causal, dt):
     rq, rk, rv = oracle.attn_bwd(fi.q, fi.k, fi.v, fi.do, d ** -0.5, causal)
     errs = [rel_l2(f64(g), r) for g, r in ((dq, rq), (dk, rk), (dv, rv))]
     assert max(errs) <= 2e-2, errs
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_packed_qkv_backward(causal):
+    """fa_varlen_bwd_strided on a packed (total, 3, H, d) QKV buffer: O in an (H, total,
+    d) buffer, dO an (H, total, d) view, the gradients into one dqkv (total, 3, H, d).
+    dK and dV equal the contiguous varlen backward's bit for bit, dQ up to the order of
+    its fp32 reductions, and all three the oracle's, sequence by sequence."""
+    lengths = [300, 0, 77, 513, 129]
+    vi = inputs.make_varlen(inputs.VARLEN, lengths=lengths, Hq=4, Hkv=4, d=128, dtype="bf16", seed=63, with_do=True)
+    qkv = torch.stack([vi.q, vi.k, vi.v], dim=1).cuda()  # (total, 3, H, d)
+    q, k, v = qkv[:, 0], qkv[:, 1], qkv[:, 2]
+    cu = vi.cu_seqlens_q.cuda()
+    T, H, d = q.shape
+    n = len(lengths)
+    o = torch.empty((H, T, d), dtype=q.dtype, device="cuda").permute(1, 0, 2)
+    do = vi.do.cuda().permute(1, 0, 2).contiguous().permute(1, 0, 2)
+    lse = torch.empty((H, T), dtype=torch.float32, device="cuda")
+    st = fb.fa_varlen_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  el_strides(q, False), el_strides(k, False), el_strides(v, False),
+                                  el_strides(o, False), cu.data_ptr(), cu.data_ptr(), n, T, T, vi.max_seqlen_q,
+                                  vi.max_seqlen_k, H, H, d, d ** -0.5, int(causal), fb.FA_BF16, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    dqkv = torch.full_like(qkv, 3.0)
+    dq, dk, dv = dqkv[:, 0], dqkv[:, 1], dqkv[:, 2]
+    ws = torch.empty(fb.fa_varlen_bwd_workspace_size(n, T, vi.max_seqlen_q, H, d), dtype=torch.uint8, device="cuda")
+    st = fb.fa_varlen_bwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                                  *[el_strides(t, False) for t in (q, k, v, o, do, dq, dk, dv)], cu.data_ptr(),
+                                  cu.data_ptr(), n, T, T, vi.max_seqlen_q, vi.max_seqlen_k, H, H, d, d ** -0.5,
+                                  int(causal), fb.FA_BF16, 0)
+    assert st == fb.FA_OK, fb.fa_status_string(st)
+    torch.cuda.synchronize()
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    dq_c, dk_c, dv_c = fb.attention_varlen_bwd(q.contiguous(), k.contiguous(), v.contiguous(), o.contiguous(), lse,
+                                               do.contiguous(), cu, cu, vi.max_seqlen_q, vi.max_seqlen_k,
+                                               d ** -0.5, causal)
+    torch.cuda.synchronize()
+    assert torch.equal(dk, dk_c) and torch.equal(dv, dv_c)
+    assert rel_l2(f64(dq), f64(dq_c)) <= 1e-2
+    refs = [np.zeros(tuple(t.shape)) for t in (vi.q, vi.k, vi.v)]
+    for s, L in enumerate(lengths):
+        a = int(vi.cu_seqlens_q[s])
+        if L == 0:
+            continue
+        rq, rk, rv = oracle.attn_bwd(vi.q[None, a:a + L], vi.k[None, a:a + L], vi.v[None, a:a + L],
+                                     vi.do[None, a:a + L], d ** -0.5, causal)
+        refs[0][a:a + L], refs[1][a:a + L], refs[2][a:a + L] = rq[0], rk[0], rv[0]
+    errs = [rel_l2(f64(g), r) for g, r in zip((dq, dk, dv), refs)]
+    assert max(errs) <= 2e-2, errs
