@@ -533,6 +533,18 @@ def run_sweep(args):
         iters = 1000 if cfg is inputs.TINY else 30
         ms = time_it(lambda: fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse), iters)
         emit(cfg.name, "fwd", ms, flops, nbytes)
+        if cfg is inputs.TINY:
+            # Eager calls this small are bound by the host's per-call work (Python, the C ABI
+            # call, encoding the tensor maps); 100 calls captured in a CUDA graph and replayed
+            # give the device's time per call.
+            g = torch.cuda.CUDAGraph()
+            gs = torch.cuda.Stream()
+            with torch.cuda.graph(g, stream=gs):
+                for _ in range(100):
+                    fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse, stream=gs)
+            ms = time_it(g.replay, 10) / 100
+            emit(cfg.name, "fwd_graph_replay", ms, flops, nbytes)
+            del g
         if cfg.backward:
             do = fi.do.cuda()
             ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, N, d), dtype=torch.uint8, device="cuda")

@@ -217,7 +217,7 @@ __global__ void fa_selftest_wait_kernel(int* err) {
 
 // d = 128 runs fa_bwd128_kernel (dQ^T = K^T dS^T with N = 128 queries); d = 64
 // the single-tile kernel (its dQ^T would need M = 64, so it keeps dQ = dS K with
-// M = 128 queries; fixed length only).
+// M = 128 queries).
 template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const fa::BwdArgs& a, dim3 grid, cudaStream_t stream) {
@@ -236,8 +236,7 @@ fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
         if (launch_regs < fa::kBwd128MinLaunchRegs) return FA_ERR_UNSUPPORTED;
         kern<<<grid, fa::kBwd128Threads, smem, stream>>>(mq, mk, mv, mdo, a);
     } else {
-        static_assert(!VARLEN, "the d = 64 backward is fixed length only");
-        auto kern = fa::fa_bwd_kernel<D, BF16, CAUSAL>;
+        auto kern = fa::fa_bwd_kernel<D, BF16, CAUSAL, VARLEN>;
         constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
         static bool attr_ok =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
@@ -358,7 +357,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         const bool timed = g_bwd_ev_before && g_bwd_ev_after;
         if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;
         if (varlen)
-            st = launch_bwd_d<128, true>(bf16, causal, mq, mk, mv, mdo, a, grid, s);
+            st = d == 64 ? launch_bwd_d<64, true>(bf16, causal, mq, mk, mv, mdo, a, grid, s)
+                         : launch_bwd_d<128, true>(bf16, causal, mq, mk, mv, mdo, a, grid, s);
         else
             st = d == 64 ? launch_bwd_d<64, false>(bf16, causal, mq, mk, mv, mdo, a, grid, s)
                          : launch_bwd_d<128, false>(bf16, causal, mq, mk, mv, mdo, a, grid, s);
@@ -367,9 +367,10 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
     }
     if (rows > 0) {
         if (d == 64) {
-            const size_t n8 = rows * d / 8;
+            // the accumulator's rows: [sequences, Nq (varlen: max_seqlen_q), Hq]
+            const size_t n8 = static_cast<size_t>(nseq) * Nq * Hq * d / 8;
             fa::fa_bwd_dq_convert<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
-                dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16, Nq, Hq, S.dq);
+                dq_acc, static_cast<uint16_t*>(dq), n8, scale, bf16, Nq, Hq, S.dq, cu_q);
         } else {
             const size_t n = static_cast<size_t>(nseq) * Hq * ((Nq + 3) / 4) * 64;
             fa::fa_bwd_dq_convert_g4<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
@@ -831,7 +832,6 @@ fa_status varlen_bwd(const void* q, const void* k, const void* v, const void* o,
         return FA_ERR_INVALID_ARG;
     fa_status st = common_checks(Hq, Hkv, d, scale, causal, dtype);
     if (st != FA_OK) return st;
-    if (d != 128) return FA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
         (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
@@ -1049,7 +1049,7 @@ fa_status fa_bwd_keymask(const void* q, const void* k, const void* v, const void
 }
 
 size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q, int Hq, int d) {
-    if (num_seqs < 1 || total_q < 0 || max_seqlen_q < 0 || Hq < 1 || d != 128) return 0;
+    if (num_seqs < 1 || total_q < 0 || max_seqlen_q < 0 || Hq < 1 || (d != 64 && d != 128)) return 0;
     const size_t rows = static_cast<size_t>(total_q) * Hq;
     return round256(rows * sizeof(float)) + round256(acc_floats(num_seqs, Hq, max_seqlen_q, d) * sizeof(float));
 }

@@ -134,7 +134,7 @@ struct BwdCfg {
 
 constexpr int kBwdThreads = 384;
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool VARLEN = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -150,7 +150,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int hk = CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
     const int b = CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
     const int k0 = kt * 128;
-    const int Nq = args.Nq, Nk = args.Nk;
+    // Rows of this sequence: fixed length, or varlen (b is the sequence; its rows
+    // start at q_row0 / k_row0 of the packed buffers, and the rows of a tile past its
+    // lengths belong to the next sequence, so they are masked, not zero-filled).
+    int q_len, k_len, q_row0, k_row0, tma_b;
+    if constexpr (VARLEN) {
+        q_row0 = args.cu_q[b];
+        k_row0 = args.cu_k[b];
+        q_len = min(args.cu_q[b + 1] - q_row0, args.Nq);
+        k_len = min(args.cu_k[b + 1] - k_row0, args.Nk);
+        tma_b = 0;
+        if (k0 >= k_len) return;  // the tile lies past this sequence's keys
+    } else {
+        q_row0 = 0;
+        k_row0 = 0;
+        q_len = args.Nq;
+        k_len = args.Nk;
+        tma_b = b;
+    }
+    const int Nq = q_len, Nk = k_len;
+    // Element offsets of key `key` of this sequence in the dK and dV buffers.
+    auto dk_off = [&](int key) -> long long {
+        return VARLEN ? (k_row0 + key) * args.dk_ss + hk * args.dk_sh : b * args.dk_sb + key * args.dk_ss + hk * args.dk_sh;
+    };
+    auto dv_off = [&](int key) -> long long {
+        return VARLEN ? (k_row0 + key) * args.dv_ss + hk * args.dv_sh : b * args.dv_sb + key * args.dv_ss + hk * args.dv_sh;
+    };
     int i0, n_i;
     query_tiles<CAUSAL>(args, k0, Nq, Nk, i0, n_i);
     const int n_it = args.group * n_i;
@@ -163,10 +188,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (threadIdx.x < 128) {
             const int key = k0 + static_cast<int>(threadIdx.x);
             if (key < Nk) {
-                uint4* a = reinterpret_cast<uint4*>(static_cast<T16*>(args.dk) + b * args.dk_sb +
-                                                    key * args.dk_ss + hk * args.dk_sh);
-                uint4* c = reinterpret_cast<uint4*>(static_cast<T16*>(args.dv) + b * args.dv_sb +
-                                                    key * args.dv_ss + hk * args.dv_sh);
+                uint4* a = reinterpret_cast<uint4*>(static_cast<T16*>(args.dk) + dk_off(key));
+                uint4* c = reinterpret_cast<uint4*>(static_cast<T16*>(args.dv) + dv_off(key));
 #pragma unroll
                 for (int i = 0; i < D / 8; ++i) a[i] = c[i] = make_uint4(0, 0, 0, 0);
             }
@@ -233,8 +256,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
 #pragma unroll
             for (int s = 0; s < D / 64; ++s) {
-                tma_load_4d(sK + s * C::kSlabBytes, &tm_k, kv_full, s * 64, hk, k0, b);
-                tma_load_4d(sV + s * C::kSlabBytes, &tm_v, kv_full, s * 64, hk, k0, b);
+                tma_load_4d(sK + s * C::kSlabBytes, &tm_k, kv_full, s * 64, hk, k_row0 + k0, tma_b);
+                tma_load_4d(sV + s * C::kSlabBytes, &tm_v, kv_full, s * 64, hk, k_row0 + k0, tma_b);
             }
             int issued = 0;
             for (int it = 0; it < n_it; ++it) {
@@ -245,8 +268,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mbar_arrive_expect_tx(&q_full[st], 2 * C::kTileBytes);
 #pragma unroll
                 for (int s = 0; s < D / 64; ++s) {
-                    tma_load_4d(sQ + st * C::kTileBytes + s * C::kSlabBytes, &tm_q, &q_full[st], s * 64, h, q0, b);
-                    tma_load_4d(sDO + st * C::kTileBytes + s * C::kSlabBytes, &tm_do, &q_full[st], s * 64, h, q0, b);
+                    tma_load_4d(sQ + st * C::kTileBytes + s * C::kSlabBytes, &tm_q, &q_full[st], s * 64, h,
+                                q_row0 + q0, tma_b);
+                    tma_load_4d(sDO + st * C::kTileBytes + s * C::kSlabBytes, &tm_do, &q_full[st], s * 64, h,
+                                q_row0 + q0, tma_b);
                 }
                 ++issued;
             }
@@ -333,7 +358,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int q = q0 + r;
                 float l2 = INFINITY, dd = 0.f;
                 if (q < Nq) {
-                    const size_t row = (static_cast<size_t>(b) * args.Hq + h) * Nq + q;
+                    const size_t row = VARLEN ? static_cast<size_t>(h) * args.total_q + q_row0 + q
+                                              : (static_cast<size_t>(b) * args.Hq + h) * Nq + q;
                     const float L = args.lse[row];
                     l2 = (L == -INFINITY) ? INFINITY : L * kLog2eF;  // a row that saw no key has P = 0
                     dd = args.D[row];
@@ -399,7 +425,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const int q = q0 + r;
-            float* dst = args.dq_acc + ((static_cast<size_t>(b) * Nq + q) * args.Hq + h) * D;
+            // [sequences, max_seqlen_q, Hq, d] (fixed length: args.Nq = Nq)
+            float* dst = args.dq_acc + ((static_cast<size_t>(b) * args.Nq + q) * args.Hq + h) * D;
 #pragma unroll
             for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
                 uint32_t v[32];
@@ -421,8 +448,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // Warpgroup 0 writes dV, warpgroup 1 writes dK = scale * (dS^T Q).
             const uint32_t col = wg == 0 ? C::kColDV : C::kColDK;
             const float mul = wg == 0 ? 1.f : args.scale;
-            T16* dst = wg == 0 ? static_cast<T16*>(args.dv) + b * args.dv_sb + key * args.dv_ss + hk * args.dv_sh
-                               : static_cast<T16*>(args.dk) + b * args.dk_sb + key * args.dk_ss + hk * args.dk_sh;
+            T16* dst = wg == 0 ? static_cast<T16*>(args.dv) + dv_off(key) : static_cast<T16*>(args.dk) + dk_off(key);
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t v[32];
@@ -512,12 +538,20 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess(const uint16_t* o, cons
 // dq = dtype(scale * dq_acc) for d = 64 (accumulator [B, Nq, Hq, 64]), 8 elements
 // per thread, dq addressed through its strides.
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert(const float* dq_acc, uint16_t* dq, size_t n8, float scale,
-                                                          bool bf16, int Nq, int Hq, Strides3 sdq) {
+                                                          bool bf16, int Nq, int Hq, Strides3 sdq,
+                                                          const int* cu_q = nullptr) {
     const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= n8) return;
     const size_t row = i / 8;  // (b Nq + q) Hq + h; 8 threads per 64-value row
     const long long h = static_cast<long long>(row % Hq), bq = static_cast<long long>(row / Hq);
-    uint16_t* dst = dq + (bq / Nq) * sdq.b + (bq % Nq) * sdq.s + h * sdq.h + (i % 8) * 8;
+    const long long b = bq / Nq, q = bq % Nq;
+    uint16_t* dst;
+    if (cu_q) {  // varlen: Nq = max_seqlen_q; rows past the sequence's length are padding
+        if (q >= cu_q[b + 1] - cu_q[b]) return;
+        dst = dq + (cu_q[b] + q) * sdq.s + h * sdq.h + (i % 8) * 8;
+    } else {
+        dst = dq + b * sdq.b + q * sdq.s + h * sdq.h + (i % 8) * 8;
+    }
     const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * i];
     const float4 c = reinterpret_cast<const float4*>(dq_acc)[2 * i + 1];
     uint4 out;

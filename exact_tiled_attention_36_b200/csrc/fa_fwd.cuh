@@ -311,8 +311,9 @@ __device__ __forceinline__ void rms_normalise_row(uint8_t* tile, int r, float ep
         }
 }
 
-// MASK: kMaskNone, kMaskCausal (bottom-right, folded at compile time) or kMaskWindow
-// (the sliding window (wl, wr) of FwdArgs; fixed length only).
+// MASK: kMaskNone, kMaskCausal (bottom-right, folded at compile time), kMaskWindow
+// (the sliding window (wl, wr) of FwdArgs) or kMaskAnchor (that window plus the
+// anchor keys 0 .. n_anchor - 1); under VARLEN all of them apply within each sequence.
 // QKNORM: Q arrives raw and each softmax thread RMS-normalises its own row of Q in
 // shared memory (over d) at the start of a unit, before the tensor core reads it;
 // K arrives normalised (fa_fwd_qk_rmsnorm runs fa_rms_normalise_rows over K first:

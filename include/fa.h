@@ -147,7 +147,7 @@ fa_status fa_bwd_window_anchor(const void* q, const void* k, const void* v, cons
  * with that sequence's own lengths), over the packed layout and cu_seqlens of
  * fa_varlen_fwd / fa_varlen_bwd. Every other argument, result and error is that of
  * fa_varlen_fwd / fa_varlen_bwd (the backward takes the lse of
- * fa_varlen_fwd_window with the same window; d = 128 for the backward).
+ * fa_varlen_fwd_window with the same window).
  */
 fa_status fa_varlen_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
                                const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
@@ -327,9 +327,10 @@ fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void
 /*
  * Size in bytes of the caller-owned workspace fa_varlen_bwd needs: D
  * (float32 [Hq,total_q]) and the float32 dQ accumulator
- * (num_seqs*Hq*ceil(max_seqlen_q/4)*4*128 floats, each sequence padded to
- * max_seqlen_q), each rounded up to 256 bytes. d must be 128; returns 0 for
- * invalid sizes.
+ * (num_seqs*Hq*max_seqlen_q*64 floats for d = 64,
+ * num_seqs*Hq*ceil(max_seqlen_q/4)*4*128 floats for d = 128: each sequence padded
+ * to max_seqlen_q), each rounded up to 256 bytes. d must be 64 or 128; returns 0
+ * for invalid sizes.
  */
 size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q, int Hq, int d);
 
@@ -346,8 +347,8 @@ size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int max_seqlen_q,
  *       sequence are left as they were.
  *   workspace: device buffer of fa_varlen_bwd_workspace_size(...) bytes,
  *       16-byte aligned, owned by the caller.
- *   d must be 128 (FA_ERR_UNSUPPORTED otherwise). Causal alignment is
- *   bottom-right within each sequence.
+ *   d is 64 or 128, as for fa_varlen_fwd. Causal alignment is bottom-right
+ *   within each sequence.
  */
 fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                         const void* dout, void* dq, void* dk, void* dv, void* workspace,
@@ -363,7 +364,7 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
  * same layout. *_strides: HOST arrays {token, head} of element strides with the rules
  * of fa_varlen_fwd_strided; dq, dk and dv must not overlap each other or the inputs.
  * lse and the workspace keep their layouts. Every other argument, result and error is
- * that of fa_varlen_bwd (d = 128).
+ * that of fa_varlen_bwd.
  */
 fa_status fa_varlen_bwd_strided(const void* q, const void* k, const void* v, const void* o,
                                 const float* lse, const void* dout, void* dq, void* dk, void* dv,

@@ -143,7 +143,7 @@ def varlen_bwd(**kw):
     (dict(num_seqs=0), fb.FA_ERR_INVALID_ARG),
     (dict(max_k=-1), fb.FA_ERR_INVALID_ARG),
     (dict(Hq=3), fb.FA_ERR_INVALID_ARG),
-    (dict(d=64), fb.FA_ERR_UNSUPPORTED),  # the varlen backward is d = 128 only
+    (dict(d=96), fb.FA_ERR_UNSUPPORTED),
     (dict(cu_q=FAKE + 2), fb.FA_ERR_MISALIGNED),
     (dict(do=FAKE + 8), fb.FA_ERR_MISALIGNED),
 ])
@@ -155,7 +155,9 @@ def test_varlen_workspace_size(lib):
     r256 = lambda x: (x + 255) // 256 * 256
     # D [Hq, total_q] and a dQ accumulator padded per sequence to max_seqlen_q (groups of four)
     assert fb.fa_varlen_bwd_workspace_size(3, 100, 41, 2, 128) == r256(100 * 2 * 4) + r256(3 * 2 * 11 * 512 * 4)
-    assert fb.fa_varlen_bwd_workspace_size(3, 100, 41, 2, 64) == 0
+    # d = 64: [sequences, max_seqlen_q, Hq, 64]
+    assert fb.fa_varlen_bwd_workspace_size(3, 100, 41, 2, 64) == r256(100 * 2 * 4) + r256(3 * 41 * 2 * 64 * 4)
+    assert fb.fa_varlen_bwd_workspace_size(3, 100, 41, 2, 96) == 0
     assert fb.fa_varlen_bwd_workspace_size(0, 100, 41, 2, 128) == 0
 
 
@@ -302,8 +304,8 @@ def test_varlen_window_anchor_rejects_before_launch(lib):
     assert fb.fa_varlen_fwd_window_anchor(*no_cu, 4, fb.FA_BF16, None) == fb.FA_ERR_INVALID_ARG
     bwd = [FAKE] * 12 + [2, 256, 256, 128, 128, 4, 2, 128, 0.1, 64, 0]
     assert fb.fa_varlen_bwd_window_anchor(*bwd, -1, fb.FA_BF16, None) == fb.FA_ERR_INVALID_ARG
-    d64 = bwd[:19] + [64] + bwd[20:]
-    assert fb.fa_varlen_bwd_window_anchor(*d64, 4, fb.FA_BF16, None) == fb.FA_ERR_UNSUPPORTED
+    d96 = bwd[:19] + [96] + bwd[20:]
+    assert fb.fa_varlen_bwd_window_anchor(*d96, 4, fb.FA_BF16, None) == fb.FA_ERR_UNSUPPORTED
     assert fb.fa_varlen_bwd_window_anchor(*bwd, 4, fb.FA_BF16 + 7, None) == fb.FA_ERR_UNSUPPORTED
 
 
@@ -315,7 +317,7 @@ def test_varlen_bwd_strided_rejects_before_launch(lib):
     assert fb.fa_varlen_bwd_strided(*ptrs, *strides[:5], None, *strides[6:], *tail) == fb.FA_ERR_INVALID_ARG
     assert fb.fa_varlen_bwd_strided(*ptrs, *strides[:6], (1540, 64), st, *tail) == fb.FA_ERR_MISALIGNED
     assert fb.fa_varlen_bwd_strided(*ptrs, *strides[:7], (0, 128), *tail) == fb.FA_ERR_INVALID_ARG
-    d64 = tail[:9] + [64] + tail[10:]
-    assert fb.fa_varlen_bwd_strided(*ptrs, *strides, *d64) == fb.FA_ERR_UNSUPPORTED
+    d96 = tail[:9] + [96] + tail[10:]
+    assert fb.fa_varlen_bwd_strided(*ptrs, *strides, *d96) == fb.FA_ERR_UNSUPPORTED
     no_ws = [FAKE] * 9 + [None]
     assert fb.fa_varlen_bwd_strided(*no_ws, *strides, *tail) == fb.FA_ERR_INVALID_ARG

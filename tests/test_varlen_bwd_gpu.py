@@ -93,27 +93,33 @@ def check_sequences(vi, dq, dk, dv, causal):
 
 
 CASES = [
-    # lengths, Hq, Hkv, dtype, causal, key_pad_frac
-    ([5, 0, 130, 257, 1, 64], 4, 2, "bf16", False, 0.0),
-    ([5, 0, 130, 257, 1, 64], 4, 2, "bf16", True, 0.0),
-    ([300, 129, 128, 0, 0, 77], 2, 2, "fp16", False, 0.25),
-    ([1000, 3, 513], 6, 3, "bf16", True, 0.25),
-    ([700, 411, 129, 256], 8, 2, "fp16", True, 0.0),
+    # lengths, Hq, Hkv, dtype, causal, key_pad_frac, d
+    ([5, 0, 130, 257, 1, 64], 4, 2, "bf16", False, 0.0, 128),
+    ([5, 0, 130, 257, 1, 64], 4, 2, "bf16", True, 0.0, 128),
+    ([300, 129, 128, 0, 0, 77], 2, 2, "fp16", False, 0.25, 128),
+    ([1000, 3, 513], 6, 3, "bf16", True, 0.25, 128),
+    ([700, 411, 129, 256], 8, 2, "fp16", True, 0.0, 128),
+    ([5, 0, 130, 257, 1, 64], 4, 2, "bf16", True, 0.0, 64),
+    ([300, 129, 128, 0, 0, 77], 2, 2, "fp16", False, 0.25, 64),
+    ([1000, 3, 513], 6, 3, "bf16", True, 0.25, 64),
+    ([700, 411, 129, 256], 8, 2, "bf16", False, 0.0, 64),
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: f"{len(c[0])}seq-h{c[1]}-{c[2]}-{c[3]}-c{int(c[4])}-p{c[5]}")
+@pytest.mark.parametrize("case", CASES,
+                         ids=lambda c: f"{len(c[0])}seq-h{c[1]}-{c[2]}-{c[3]}-c{int(c[4])}-p{c[5]}-d{c[6]}")
 def test_varlen_bwd_small(case):
-    lengths, Hq, Hkv, dt, causal, pad = case
-    vi = inputs.make_varlen(inputs.VARLEN, lengths=lengths, Hq=Hq, Hkv=Hkv, d=128, dtype=dt, causal=causal,
+    lengths, Hq, Hkv, dt, causal, pad, d = case
+    vi = inputs.make_varlen(inputs.VARLEN, lengths=lengths, Hq=Hq, Hkv=Hkv, d=d, dtype=dt, causal=causal,
                             key_pad_frac=pad, seed=37, with_do=True)
     dq, dk, dv = run_varlen_fwd_bwd(vi, causal)
     check_sequences(vi, dq, dk, dv, causal)
 
 
-def test_varlen_bwd_leaves_rows_outside_sequences():
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_bwd_leaves_rows_outside_sequences(d):
     """Rows past the last sequence (total > cu[-1]) keep what they held."""
-    vi = inputs.make_varlen(inputs.VARLEN, lengths=[200, 77], Hq=4, Hkv=2, d=128, dtype="bf16", seed=41,
+    vi = inputs.make_varlen(inputs.VARLEN, lengths=[200, 77], Hq=4, Hkv=2, d=d, dtype="bf16", seed=41,
                             with_do=True)
     extra = 96
     dq, dk, dv = run_varlen_fwd_bwd(vi, True, extra_rows=extra)
@@ -124,11 +130,12 @@ def test_varlen_bwd_leaves_rows_outside_sequences():
     check_sequences(vi, dq[:n_q], dk[:n_k], dv[:n_k], True)
 
 
-def test_varlen_bwd_matches_fixed_length_path():
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_bwd_matches_fixed_length_path(d):
     """Equal lengths through the varlen path give the fixed-length path's gradients:
     dK and dV bit for bit (same products in the same order), dQ up to the order of
     its fp32 reductions."""
-    B, N, Hq, Hkv, d = 3, 200, 4, 2, 128
+    B, N, Hq, Hkv = 3, 200, 4, 2
     fi = inputs.make_fixed(inputs.CAUSAL_GQA, B=B, Nq=N, Nk=N, Hq=Hq, Hkv=Hkv, d=d, seed=43)
     q, k, v, do = (t.cuda() for t in (fi.q, fi.k, fi.v, fi.do))
     o, lse = fb.attention_fwd(q, k, v, d ** -0.5, causal=True)

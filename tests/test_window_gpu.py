@@ -130,7 +130,7 @@ VARLEN_CASES = [
 @pytest.mark.parametrize("case", VARLEN_CASES,
                          ids=lambda c: f"{len(c[0])}seq-h{c[1]}-{c[2]}-d{c[3]}-w" + "_".join(map(str, c[4])))
 def test_varlen_window(case):
-    """fa_varlen_fwd_window (and, for d = 128, fa_varlen_bwd_window), or with anchors
+    """fa_varlen_fwd_window and fa_varlen_bwd_window, or with anchors
     fa_varlen_fwd_window_anchor / fa_varlen_bwd_window_anchor: every sequence against
     the oracle with the window (and anchors) applied within that sequence."""
     lengths, Hq, Hkv, d, window, dt, pad = case
@@ -158,8 +158,6 @@ def test_varlen_window(case):
     live = ~empty
     assert np.abs(l64[live] - l_ref[live]).max() <= ATOL_L
     assert (np.abs(o64 - o_ref) <= o_bound(o_ref, q.dtype)).all()
-    if d != 128:
-        return
     ws = torch.empty(fb.fa_varlen_bwd_workspace_size(n, Tq, vi.max_seqlen_q, Hq, d), dtype=torch.uint8, device="cuda")
     dq, dk, dv = torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)
     bwd = fb.fa_varlen_bwd_window_anchor if anchors else fb.fa_varlen_bwd_window
