@@ -557,6 +557,8 @@ def run_sweep(args):
         sweep_fp8(cfg, inputs, fb, torch, stream, time_it, emit)
     if want(inputs.CAUSAL_GQA.name + "_window1024_anchor4"):
         sweep_window(inputs, fb, torch, stream, time_it, emit)
+    if want("causal_gqa_b2_n8192_hq32_hkv8_d128_noncausal") or want("causal_gqa_b2_n8192_hq32_hkv32_d128_mha"):
+        sweep_prefill_variants(inputs, fb, torch, stream, time_it, emit)
     if want(inputs.VIT_RMSNORM.name + "_packed_qkv_fused_qk_rmsnorm"):
         sweep_vit_variants(inputs, fb, torch, stream, time_it, emit)
     for cfg in (inputs.VARLEN, inputs.VARLEN_KEYPAD):
@@ -643,6 +645,26 @@ def sweep_window(inputs, fb, torch, stream, time_it, emit):
     emit(cfg.name + "_window1024_anchor4", "fwd", time_it(afwd, 30), aflops, nb)
     emit(cfg.name + "_window1024_anchor4", "bwd", time_it(abwd, 20), 2.5 * aflops,
          nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+
+
+def sweep_prefill_variants(inputs, fb, torch, stream, time_it, emit):
+    """The causal GQA prefill shape without the causal mask, and with as many KV heads
+    as query heads (Hq = Hkv = 32): the d = 128 figures beside the causal GQA ones."""
+    base = inputs.CAUSAL_GQA
+    for tag, causal, hkv in (("_noncausal", False, base.Hkv), ("_mha", True, base.Hq)):
+        fi = inputs.make_fixed(base, causal=causal, Hkv=hkv)
+        q, k, v, do = (t.cuda() for t in (fi.q, fi.k, fi.v, fi.do))
+        B, N, Hq, d = q.shape
+        flops = flops_fwd(B, N, Hq, d, causal)
+        o, lse = fb.attention_fwd(q, k, v, base.scale, causal)
+        ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, N, d), dtype=torch.uint8, device="cuda")
+        nb = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
+        emit(base.name.replace("_hkv8", f"_hkv{hkv}") + tag, "fwd",
+             time_it(lambda: fb.attention_fwd(q, k, v, base.scale, causal, out=o, lse=lse), 30), flops, nb)
+        emit(base.name.replace("_hkv8", f"_hkv{hkv}") + tag, "bwd",
+             time_it(lambda: fb.attention_bwd(q, k, v, o, lse, do, base.scale, causal, workspace=ws), 20),
+             2.5 * flops, nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+        del q, k, v, do, o, lse, ws, fi
 
 
 def sweep_vit_variants(inputs, fb, torch, stream, time_it, emit):
