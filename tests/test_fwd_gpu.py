@@ -63,6 +63,10 @@ SMALL = [
     (3, 3, 3, 384, 384, 64, True, "fp16"),
     (1, 6, 2, 640, 700, 64, False, "bf16"),
     (2, 2, 1, 1000, 1000, 128, True, "bf16"),
+    # last key tile of exactly 32 keys, a single tile of 32, and one of 33 (the narrow tail's edges)
+    (1, 2, 2, 300, 160, 64, False, "fp16"),
+    (1, 2, 2, 129, 32, 128, False, "bf16"),
+    (2, 2, 1, 200, 33, 128, False, "bf16"),
 ]
 
 

@@ -46,6 +46,7 @@ CASES = [
     (3, 200, 700, 2, 2, 64, False, "random", "bf16"),
     (3, 400, 400, 4, 2, 128, True, "blocks", "bf16"),
     (1, 129, 129, 2, 2, 64, True, "left", "fp16"),
+    (2, 160, 288, 2, 1, 128, False, "random", "bf16"),  # last key tile of 32 keys (the narrow tail)
 ]
 
 
