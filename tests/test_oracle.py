@@ -526,10 +526,11 @@ def test_fp8_dequantise_blocks_and_attention():
 
 
 def test_varlen_window_equals_numpy_per_sequence():
-    """The varlen forward with a window: every sequence is the numpy whole-matrix
-    version with the same window on that sequence alone."""
+    """The varlen forward with a window (and anchors): every sequence is the numpy
+    whole-matrix version with the same window on that sequence alone."""
     vi = inputs.make_varlen(inputs.VARLEN, lengths=[9, 1, 30, 0, 17], Hq=4, Hkv=2, d=8)
-    for window in ((3, 0), (5, 2), (-1, 4), (0, 0)):
+    # (wl, wr) windows, and (wl, wr, n_anchor) with the first keys of every sequence as anchors
+    for window in ((3, 0), (5, 2), (-1, 4), (0, 0), (3, 0, 2), (2, 1, 5), (0, -1, 1)):
         o, lse = oracle.varlen_fwd(vi.q, vi.k, vi.v, vi.cu_seqlens_q, vi.cu_seqlens_k, 0.4, window=window)
         for s, n in enumerate(vi.seqlens_q):
             a = int(vi.cu_seqlens_q[s])
