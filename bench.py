@@ -565,7 +565,7 @@ def run_sweep(args):
         if want(cfg.name):
             sweep_varlen(cfg, inputs, fb, torch, stream, time_it, emit)
     for cfg, page in ((inputs.DECODE, 0), (inputs.DECODE_RAGGED, 0), (inputs.DECODE_RAGGED, 64),
-                      (inputs.DECODE_RAGGED, 16), (inputs.DECODE_D64, 0), (inputs.DECODE_SPEC4, 0)):
+                      (inputs.DECODE_RAGGED, 32), (inputs.DECODE_RAGGED, 16), (inputs.DECODE_D64, 0), (inputs.DECODE_SPEC4, 0)):
         if want(cfg.name + (f"_paged{page}" if page else "")):
             sweep_decode(cfg, page, inputs, fb, torch, stream, time_it, emit)
     return 0

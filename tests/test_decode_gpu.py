@@ -104,6 +104,32 @@ def test_decode_paged(page_size, causal):
     assert np.abs(o - o2).max() <= 2 * 2.0 ** -8 and np.abs(np.nan_to_num(lse - lse2)).max() <= 1e-4
 
 
+@pytest.mark.parametrize("page_size", [16, 32])
+def test_decode_paged_small_pages_paired_heads(page_size):
+    """16/32-row pages with d = 64 paired KV heads (rows of two heads' 128 values)."""
+    cfg = inputs.DecodeConfig(name="t", **small(B=5, Hq=8, Hkv=4, Nq=2, Nk=1300, d=64, len_seed=21, min_len=0))
+    di = inputs.make_decode(cfg, page_size=page_size, spare_pages=7)
+    o, lse = run(di, True, paged=True)
+    check(di, o, lse, True)
+
+
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_decode_paged_out_of_pool_pages(page_size):
+    """Block-table entries outside [0, num_pages) inside a sequence's length read zero rows."""
+    cfg = inputs.DecodeConfig(name="t", **small(B=3, Nq=2, Nk=700))
+    di = inputs.make_decode(cfg, lengths=[700, 300, 650], page_size=page_size)
+    n_pages = di.k_pages.shape[0]
+    for b, i, page in ((0, 1, -1), (0, 5, n_pages), (1, 0, n_pages + 1000), (2, 650 // page_size, -7)):
+        di.block_table[b, i] = page
+        di.k[b, i * page_size:(i + 1) * page_size] = 0
+        di.v[b, i * page_size:(i + 1) * page_size] = 0
+    for b, n in enumerate(di.seqlens):  # rows past the length stay NaN
+        di.k[b, n:] = float("nan")
+        di.v[b, n:] = float("nan")
+    o, lse = run(di, True, paged=True)
+    check(di, o, lse, True)
+
+
 def test_decode_paged_fp16_d64_more_pages_than_used():
     cfg = inputs.DecodeConfig(name="t", **small(B=6, Hq=16, Hkv=4, Nq=1, Nk=900, d=64, dtype="fp16", len_seed=5))
     di = inputs.make_decode(cfg, page_size=128, spare_pages=40)
@@ -143,8 +169,10 @@ def test_decode_full_size(cfg):
     di = inputs.make_decode(cfg)
     o, lse = run(di, cfg.causal)
     check(di, o, lse, cfg.causal)
-    o_p, lse_p = run(inputs.make_decode(cfg, page_size=64), cfg.causal, paged=True) if cfg.len_seed >= 0 else (o, lse)
-    check(di, o_p, lse_p, cfg.causal)
+    if cfg.len_seed >= 0:  # the paged layouts of the benchmark: 64-row pages (TMA) and 16-row pages (cp.async)
+        for page_size in (64, 16):
+            o_p, lse_p = run(inputs.make_decode(cfg, page_size=page_size), cfg.causal, paged=True)
+            check(di, o_p, lse_p, cfg.causal)
 
 
 def test_attention_decode_wrapper():
