@@ -25,7 +25,7 @@ def _rand(rng, *shape):
 def _num(x):
     if isinstance(x, str):
         import re
-        return eval(re.sub(r"ln(\d+)", r"math.log(\1)", x), {"math": math})  # "ln3", "0.75*ln3"
+        return eval(re.sub(r"ln(\d+)", r"math.log(\1)", x), {"math": math, "inf": math.inf})  # "ln3", "-inf"
     return float(x)
 
 
@@ -48,6 +48,50 @@ def test_golden_two_key_example():
     np.testing.assert_allclose(dq[0, :, 0, :], _grid(g["dq"]), rtol=0, atol=1e-14)
     np.testing.assert_allclose(dk[0, :, 0, :], _grid(g["dk"]), rtol=0, atol=1e-14)
     np.testing.assert_allclose(dv[0, :, 0, :], _grid(g["dv"]), rtol=0, atol=1e-14)
+
+
+def _mask_cases():
+    g = json.load(open(os.path.join(GOLDEN, "mask_alignment_examples.json")))
+    return g["cases"]
+
+
+@pytest.mark.parametrize("case", _mask_cases(), ids=lambda c: c["name"])
+def test_golden_mask_alignment_examples(case):
+    """Hand-worked causal (bottom-right, Nq != Nk), window and anchor examples:
+    tests/golden/mask_alignment_examples.json. The forward, the decode wrapper
+    (the keys as a sequence's cache, NaN past its length), the packed varlen
+    wrapper and the tiled online recurrence all give the worked values."""
+    q = _grid(case["q"])[None, :, None, :]
+    k = _grid(case["k"])[None, :, None, :]
+    v = _grid(case["v"])[None, :, None, :]
+    o_ref = _grid(case["o"])
+    l_ref = np.array([_num(x) for x in case["lse"]])
+    causal, window = case["causal"], case["window"]
+    o, lse = oracle.attn_fwd(q, k, v, 1.0, causal, window=window)
+    np.testing.assert_allclose(o[0, :, 0, :], o_ref, rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(np.isneginf(lse[0, 0]), np.isneginf(l_ref))
+    live = np.isfinite(l_ref)
+    np.testing.assert_allclose(lse[0, 0][live], l_ref[live], rtol=0, atol=1e-14)
+    Nq, Nk = q.shape[1], k.shape[1]
+    if window is None:
+        # the same keys as the first Nk rows of a 3-row-longer cache, the rest NaN
+        kc = np.concatenate([k, np.full((1, 3, 1, 1), np.nan)], axis=1)
+        vc = np.concatenate([v, np.full((1, 3, 1, 1), np.nan)], axis=1)
+        od, ld = oracle.attn_decode(q, kc, vc, 1.0, [Nk], causal)
+        np.testing.assert_allclose(od[0, :, 0, :], o_ref, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(ld[0, 0][live], l_ref[live], rtol=0, atol=1e-14)
+        assert np.isneginf(ld[0, 0][~live]).all()
+        for Br, Bc in ((1, 1), (2, 2), (4, 1)):
+            O2, L2 = online.fwd_head(q[0, :, 0], k[0, :, 0], v[0, :, 0], 1.0, Br, Bc, causal=causal)
+            np.testing.assert_allclose(O2, o_ref, rtol=0, atol=1e-14)
+            np.testing.assert_allclose(L2[live], l_ref[live], rtol=0, atol=1e-14)
+    # packed after a 2-row sequence of its own: the example's rows are unchanged
+    rng = np.random.default_rng(5)
+    q0, k0, v0 = rng.standard_normal((2, 1, 1)), rng.standard_normal((2, 1, 1)), rng.standard_normal((2, 1, 1))
+    ov, lv = oracle.varlen_fwd(np.concatenate([q0, q[0]]), np.concatenate([k0, k[0]]), np.concatenate([v0, v[0]]),
+                               [0, 2, 2 + Nq], [0, 2, 2 + Nk], 1.0, causal, window=window)
+    np.testing.assert_allclose(ov[2:, 0, :], o_ref, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lv[0, 2:][live], l_ref[live], rtol=0, atol=1e-14)
 
 
 # ---------------------------------------------------------------- softmax pins
