@@ -49,3 +49,29 @@ def test_two_ranks_take_the_slowest_time_and_distinct_batches():
     # whole-job value: both ranks' work over the slowest rank's time
     assert abs(bench.job_tflops(2, 1e12, 10, 15.0) - 2 * 1e12 * 10 / 0.015 / 1e12) < 1e-9
     assert bench.max_over_ranks(3.0, 1, "cpu") == 3.0
+
+
+def test_reference_arm_prints_one_line_on_rank_zero_only(monkeypatch, capsys):
+    """`bench.py --impl reference` under torchrun: rank 0 times the oracle and prints
+    the one JSON line of the contract; every other rank exits 0 without work."""
+    import argparse
+    import json
+
+    args = argparse.Namespace(gpus=2, steps=2, warmup=1)
+    monkeypatch.setattr(bench, "REF_STEP_TOKENS", 64)  # a small sample keeps this test short
+    monkeypatch.setenv("RANK", "1")
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out == ""
+    monkeypatch.setenv("RANK", "0")
+    assert bench.run_reference(args) == 0
+    lines = capsys.readouterr().out.strip().splitlines()
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["n_gpus"] == 2 and line["steps"] == 2 and line["warmup"] == 1
+    assert line["higher_is_better"] is True and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"] == bench.WORKLOAD["name"] and line["config"]["sample_tokens"] == 64
