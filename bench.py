@@ -151,6 +151,15 @@ class ClockSampler:
 BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 
 
+def any_rank_throttled(clocks, world, device):
+    """Whether any rank's clock record (ClockSampler.stop()) shows a throttle reason
+    that rejects the measurement. Every rank gets the same answer, so all of them
+    re-measure together and take the same collective steps (one all-reduce per call
+    on every rank when world > 1)."""
+    bad = 1.0 if clocks and (set(clocks["reasons"]) & BAD_REASONS) else 0.0
+    return max_over_ranks(bad, world, device) > 0.0
+
+
 # ----------------------------------------------------------------------------- multi-rank plumbing
 def rank_seed(base_seed, rank):
     """Each rank draws its own batch: independent replicas of the workload."""
@@ -330,7 +339,7 @@ def run_ours(args):
         time.sleep(0.3)
         result = timed_region()
         clocks = sampler.stop()
-        if not clocks or not (set(clocks["reasons"]) & BAD_REASONS):
+        if not any_rank_throttled(clocks, world, "cuda"):
             break
     total_ms, fwd_ms, bwd_ms, bwd_main_ms = result
     if fb.fa_get_last_device_error(None) != fb.FA_OK:

@@ -26,7 +26,13 @@ def _worker(rank, world, port, q):
         digest = float(fi.q.float().sum())
         all_d = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
         dist.all_gather(all_d, torch.tensor([digest], dtype=torch.float64))
-        q.put((rank, m, [float(x) for x in all_d]))
+        # the re-measure decision: one rank throttled makes every rank re-measure
+        clean = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+        hot = dict(clean, reasons=["hw_thermal_slowdown", "sw_power_cap"])
+        throttled = (bench.any_rank_throttled(hot if rank == 1 else clean, world, "cpu"),
+                     bench.any_rank_throttled(clean, world, "cpu"),
+                     bench.any_rank_throttled(None if rank == 0 else clean, world, "cpu"))
+        q.put((rank, m, [float(x) for x in all_d], throttled))
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -43,12 +49,15 @@ def test_two_ranks_take_the_slowest_time_and_distinct_batches():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, m, digests in out:
+    for rank, m, digests, throttled in out:
         assert m == 15.0  # every rank sees the max
         assert digests[0] != digests[1]  # replicas draw independent batches
+        assert throttled == (True, False, False)  # the same decision on every rank
     # whole-job value: both ranks' work over the slowest rank's time
     assert abs(bench.job_tflops(2, 1e12, 10, 15.0) - 2 * 1e12 * 10 / 0.015 / 1e12) < 1e-9
     assert bench.max_over_ranks(3.0, 1, "cpu") == 3.0
+    assert bench.any_rank_throttled({"reasons": ["sw_thermal_slowdown"]}, 1, "cpu") is True
+    assert bench.any_rank_throttled({"reasons": ["sw_power_cap"]}, 1, "cpu") is False
 
 
 def test_reference_arm_prints_one_line_on_rank_zero_only(monkeypatch, capsys):
