@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "per_device.h"
 #include "fa_fwd.cuh"
 #include "fa_bwd.cuh"
 #include "fa_bwd128.cuh"
@@ -79,29 +80,55 @@ fa_status make_map_strided(CUtensorMap* m, const void* base, int d, int H, int64
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+int current_device() {
+    int dev = -1;
+    return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+// Device address of the current device's error word (every GPU has its own copy
+// of g_fa_error; a kernel must get the copy of the device it runs on). Null if
+// the lookup fails.
 int* error_word() {
-    static int* ptr = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_fa_error) == cudaSuccess) ptr = static_cast<int*>(p);
-    });
-    return ptr;
+    static fa::PerDevice<int*> ptrs;
+    int* p = nullptr;
+    ptrs.get(current_device(), [](int*& v) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_fa_error) != cudaSuccess || a == nullptr) return false;
+        v = static_cast<int*>(a);
+        return true;
+    }, &p);
+    return p;
 }
 
 // Streaming multiprocessors of the current device (the persistent forward runs at
-// most one CTA per SM); cached per device.
+// most one CTA per SM); 0 if the query fails.
 int sm_count() {
-    constexpr int kMaxDevices = 64;
-    static int counts[kMaxDevices] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-    if (counts[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        counts[dev] = n;
-    }
-    return counts[dev];
+    static fa::PerDevice<int> counts;
+    const int dev = current_device();
+    int n = 0;
+    counts.get(dev, [dev](int& v) {
+        return cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0;
+    }, &n);
+    return n;
+}
+
+// One-time set-up of a kernel on the current device: its dynamic shared memory
+// limit raised to `smem` bytes, and the registers per thread it launches with.
+// Returns that register count, or 0 if the set-up failed. `Kern` is the kernel
+// itself, so each instantiation keeps its own per-device record.
+template <auto Kern>
+int kernel_setup(int smem) {
+    static fa::PerDevice<int> regs;
+    int n = 0;
+    regs.get(current_device(), [smem](int& v) {
+        if (cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return false;
+        cudaFuncAttributes fa_attr{};
+        if (cudaFuncGetAttributes(&fa_attr, Kern) != cudaSuccess || fa_attr.numRegs <= 0) return false;
+        v = fa_attr.numRegs;
+        return true;
+    }, &n);
+    return n;
 }
 
 // Units of 256 query rows for every (batch, head) and the persistent grid over them.
@@ -130,17 +157,13 @@ fa_status common_checks(int Hq, int Hkv, int d, float scale, int causal, fa_dtyp
 template <int D, bool BF16, int MASK, bool VARLEN, bool QKNORM, bool FP8 = false, bool KEYMASK = false>
 fa_status launch_fwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdArgs& a,
                        dim3 grid, cudaStream_t stream) {
-    auto kern = fa::fa_fwd_kernel<D, BF16, MASK, VARLEN, QKNORM, FP8, KEYMASK>;
+    constexpr auto kern = fa::fa_fwd_kernel<D, BF16, MASK, VARLEN, QKNORM, FP8, KEYMASK>;
     constexpr int smem = fa::FwdCfg<D, FP8>::kSmemBytes;
-    static bool attr_ok = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-    if (!attr_ok) return FA_ERR_CUDA;
+    const int launch_regs = kernel_setup<kern>(smem);
+    if (launch_regs == 0) return FA_ERR_CUDA;
     // The kernel moves registers between warpgroups with setmaxnreg; the split
     // must fit the pool the CTA is launched with, or the increase would wait
     // for registers that never come.
-    static int launch_regs = [&] {
-        cudaFuncAttributes fa_attr{};
-        return cudaFuncGetAttributes(&fa_attr, kern) == cudaSuccess ? fa_attr.numRegs : 0;
-    }();
     if (launch_regs < fa::kFwdMinLaunchRegs) return FA_ERR_UNSUPPORTED;
     kern<<<grid, fa::kFwdThreads, smem, stream>>>(mq, mk, mv, a);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -222,25 +245,18 @@ template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 fa_status launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                        const fa::BwdArgs& a, dim3 grid, cudaStream_t stream) {
     if constexpr (D == 128) {
-        auto kern = fa::fa_bwd128_kernel<BF16, CAUSAL, VARLEN>;
+        constexpr auto kern = fa::fa_bwd128_kernel<BF16, CAUSAL, VARLEN>;
         constexpr int smem = fa::Bwd128Cfg::kSmemBytes;
-        static bool attr_ok =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-        if (!attr_ok) return FA_ERR_CUDA;
+        const int launch_regs = kernel_setup<kern>(smem);
+        if (launch_regs == 0) return FA_ERR_CUDA;
         // The kernel moves registers between warpgroups with setmaxnreg; the split
         // only fits if the launch holds enough registers per thread.
-        static int launch_regs = [&] {
-            cudaFuncAttributes fa_attr{};
-            return cudaFuncGetAttributes(&fa_attr, kern) == cudaSuccess ? fa_attr.numRegs : 0;
-        }();
         if (launch_regs < fa::kBwd128MinLaunchRegs) return FA_ERR_UNSUPPORTED;
         kern<<<grid, fa::kBwd128Threads, smem, stream>>>(mq, mk, mv, mdo, a);
     } else {
-        auto kern = fa::fa_bwd_kernel<D, BF16, CAUSAL, VARLEN>;
+        constexpr auto kern = fa::fa_bwd_kernel<D, BF16, CAUSAL, VARLEN>;
         constexpr int smem = fa::BwdCfg<D>::kSmemBytes;
-        static bool attr_ok =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-        if (!attr_ok) return FA_ERR_CUDA;
+        if (kernel_setup<kern>(smem) == 0) return FA_ERR_CUDA;
         kern<<<grid, fa::kBwdThreads, smem, stream>>>(mq, mk, mv, mdo, a);
     }
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -656,18 +672,14 @@ fa_status launch_dec_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     constexpr int DK = PAIR ? 128 : D;
     if (run_split) {
         if constexpr (RN == 0) {
-            auto kern = fa::fa_decode_kernel<D, BF16, SEQLENS, PAGED>;
+            constexpr auto kern = fa::fa_decode_kernel<D, BF16, SEQLENS, PAGED>;
             constexpr int smem = fa::DecCfg<D>::kSmemBytes;
-            static bool attr_ok =
-                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-            if (!attr_ok) return FA_ERR_CUDA;
+            if (kernel_setup<kern>(smem) == 0) return FA_ERR_CUDA;
             kern<<<a.G, fa::kDecThreads, smem, s>>>(mq, mk, mv, a, causal);
         } else {
-            auto kern = fa::fa_decode_narrow_kernel<DK, BF16, SEQLENS, PAGED, RN>;
+            constexpr auto kern = fa::fa_decode_narrow_kernel<DK, BF16, SEQLENS, PAGED, RN>;
             constexpr int smem = fa::DecNarrowCfg<DK, RN>::kSmemBytes;
-            static bool attr_ok =
-                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-            if (!attr_ok) return FA_ERR_CUDA;
+            if (kernel_setup<kern>(smem) == 0) return FA_ERR_CUDA;
             kern<<<a.G, fa::kDecThreads, smem, s>>>(mq, mk, mv, a, causal);
         }
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -1176,6 +1188,7 @@ fa_status fa_get_last_device_error(fa_stream_t stream) {
     g_last_site = v;
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_fa_error, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    if (v == fa::kErrSeqlenBound) return FA_ERR_INVALID_ARG;
     return (v >= fa::kErrTimeoutBase && v < fa::kErrSmemAlign) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
 }
 

@@ -88,6 +88,9 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         q_len = min(args.cu_q[b + 1] - q_row0, args.Nq);
         k_len = min(args.cu_k[b + 1] - k_row0, args.Nk);
         tma_b = 0;
+        // one CTA per sequence checks its lengths against the max_seqlen bounds
+        if (kt == 0 && hk == 0 && threadIdx.x == 0)
+            check_seqlens(args.cu_q, args.cu_k, b, args.Nq, args.Nk, args.err);
         if (k0 >= k_len) return;  // the tile lies past this sequence's keys
     } else {
         q_row0 = 0;

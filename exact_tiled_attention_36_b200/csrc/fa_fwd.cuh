@@ -415,6 +415,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const int u = fwd_unit_index(rnd, cta, G);
                 if (u >= args.n_units) break;
                 const FwdUnit w = fwd_unit<MASK, VARLEN>(u, args);
+                // Every sequence has exactly one unit with q0 = 0 of head 0: its lengths
+                // are checked against the max_seqlen bounds there.
+                if (VARLEN && w.q0 == 0 && w.h == 0)
+                    check_seqlens(args.cu_q, args.cu_k, w.bidx, args.Nq, args.Nk, args.err);
                 if (!w.rows || w.n_kv == 0) continue;
                 // Q of this unit once the previous unit's last S product has read Q.
                 if (!(ok = mbar_wait(q_empty, (nq & 1) ^ 1u, wc, 60))) break;

@@ -11,37 +11,32 @@
 // loads this module holds that memory until the process exits. The kernels
 // are the same as fa_bwd's: this entry point only supplies the workspace.
 //
-// The array lives in its own translation unit so that its module is loaded,
-// and its memory reserved, only when fa_bwd_noalloc is first used.
+// The array lives in its own translation unit, so it forms a module of its
+// own. Under CUDA's lazy module loading (the default) a GPU loads that module,
+// and reserves the memory, only when fa_bwd_noalloc first runs on it; with
+// CUDA_MODULE_LOADING=EAGER every GPU context the process creates loads it.
 #include <cuda_runtime.h>
 
 #include <cstddef>
-#include <mutex>
 
 #include "fa.h"
+#include "per_device.h"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_bwd_scratch[FA_BWD_NOALLOC_MAX_BYTES];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
 // Device address of g_bwd_scratch on the current device. In host code the
 // array's name is only a host-side stand-in, so the address must come from
 // cudaGetSymbolAddress, once per device, with that device current.
 fa_status scratch_on_current_device(void** out) {
+    static fa::PerDevice<void*> ptrs;
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
-    return FA_OK;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    const bool ok = ptrs.get(dev, [](void*& p) {
+        return cudaGetSymbolAddress(&p, g_bwd_scratch) == cudaSuccess && p != nullptr;
+    }, out);
+    return ok ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // namespace

@@ -12,8 +12,11 @@ namespace fa {
 
 // Device error word: the first failure of any kernel stores its code here.
 // kErrTimeoutBase + site: a bounded wait ran out; kErrSmemAlign: the dynamic
-// shared memory window was not 1024-byte aligned (the kernel did nothing).
-enum : int { kErrTimeoutBase = 0x1000, kErrSmemAlign = 0x2000 };
+// shared memory window was not 1024-byte aligned (the kernel did nothing);
+// kErrSeqlenBound: a varlen sequence was longer than the max_seqlen bound the
+// caller gave (or had a negative length), so only its first max_seqlen rows or
+// keys were processed.
+enum : int { kErrTimeoutBase = 0x1000, kErrSmemAlign = 0x2000, kErrSeqlenBound = 0x3000 };
 
 // ---------------------------------------------------------------------------
 // generic helpers
@@ -33,6 +36,14 @@ __device__ __forceinline__ bool smem_base_ok(const void* smem, int* err) {
     if ((static_cast<uint32_t>(__cvta_generic_to_shared(smem)) & 1023u) == 0) return true;
     if (threadIdx.x == 0) atomicCAS(err, 0, kErrSmemAlign);
     return false;
+}
+
+// Varlen: records kErrSeqlenBound if sequence b of cu_seqlens_q / cu_seqlens_k is
+// longer than its bound or has a negative length (the kernels clip to the bound).
+__device__ __forceinline__ void check_seqlens(const int* cu_q, const int* cu_k, int b, int max_q, int max_k,
+                                              int* err) {
+    const int lq = cu_q[b + 1] - cu_q[b], lk = cu_k[b + 1] - cu_k[b];
+    if (lq < 0 || lq > max_q || lk < 0 || lk > max_k) atomicCAS(err, 0, kErrSeqlenBound);
 }
 
 __device__ __forceinline__ int warp_id() { return static_cast<int>(threadIdx.x >> 5); }

@@ -89,8 +89,12 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  *       device, so the library cannot read them without a synchronisation).
  *       No row at or past total_q is written and no row at or past total_k
  *       is read, whatever cu_seqlens hold.
- *   max_seqlen_q, max_seqlen_k: upper bounds of the lengths (grid sizing
- *       only; a length above its bound is not processed past the bound).
+ *   max_seqlen_q, max_seqlen_k: upper bounds of the lengths (grid sizing).
+ *       A sequence longer than its bound (or with a negative length) is
+ *       processed only up to the bound, and the kernel records it in the
+ *       device error word: the next fa_get_last_device_error returns
+ *       FA_ERR_INVALID_ARG. The bounds cannot be checked before the launch,
+ *       because cu_seqlens are read on the device only.
  *   lse [Hq, total_q] float32.
  *   Causal alignment is bottom-right within each sequence.
  */
@@ -435,8 +439,12 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
  * Same arguments, results and errors as fa_bwd, minus `workspace`: the
  * workspace is a device array of FA_BWD_NOALLOC_MAX_BYTES bytes inside the
  * library, which every GPU that loads this part of the library keeps until
- * the process exits. Nothing is allocated per call: no cudaMalloc, no
- * cudaFree, no allocating library routine.
+ * the process exits. Under CUDA's lazy module loading (the default,
+ * CUDA_MODULE_LOADING=LAZY) a GPU loads it when fa_bwd_noalloc first runs
+ * there; under CUDA_MODULE_LOADING=EAGER every GPU context the process
+ * creates loads it, and holds the 64 MiB, whether or not fa_bwd_noalloc is
+ * ever called. Nothing is allocated per call: no cudaMalloc, no cudaFree,
+ * no allocating library routine.
  *   - Sizes whose fa_bwd_workspace_size(B, Hq, Nq, d) exceeds
  *     FA_BWD_NOALLOC_MAX_BYTES are rejected with FA_ERR_UNSUPPORTED before
  *     anything runs (with d = 128: B * Hq * Nq up to about 130,000 rows).
@@ -469,10 +477,12 @@ void fa_bwd_set_timing_events(void* before, void* after);
 const char* fa_status_string(fa_status s);
 
 /*
- * Synchronises `stream`, then reports and clears the device error word:
- * FA_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last call,
- * FA_ERR_CUDA if the synchronisation failed or a kernel refused to run,
- * FA_OK otherwise.
+ * Synchronises `stream`, then reports and clears the current device's error
+ * word (each GPU has its own; a kernel records into the word of the device it
+ * runs on): FA_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
+ * last call, FA_ERR_INVALID_ARG if a varlen kernel met a sequence longer than
+ * its max_seqlen bound, FA_ERR_CUDA if the synchronisation failed or a kernel
+ * refused to run, FA_OK otherwise.
  */
 fa_status fa_get_last_device_error(fa_stream_t stream);
 

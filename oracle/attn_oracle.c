@@ -166,76 +166,76 @@ int ora_attn_probs(const double* q, const double* k, int B, int Hq, int Hkv, int
     return 0;
 }
 
-/* Backward of one (batch, KV head) group over all its query heads. Writes dq
- * rows of those query heads and accumulates dk, dv of the KV head. When
- * krows != NULL only the listed key rows of dk/dv are produced and only the
- * query rows listed in qrows (may be NULL with nq == 0) get dq; query rows
- * that can see none of the listed keys are skipped, which is exact because
- * they add nothing to those keys' gradients. */
+/* Gradient terms of one query row i of query head h: recomputes the row's P and
+ * dP = dO_i V^T, D = sum_j P_ij dP_ij and dS_ij = P_ij (dP_ij - D); writes
+ * dq_i = scale sum_j dS_ij k_j when dqi != NULL, and adds scale dS_ij q_i into
+ * the dK row and P_ij dO_i into the dV row of every listed key: key krows[t]
+ * (every key t when krows == NULL) at dk_out + t * out_stride and
+ * dv_out + t * out_stride. s, p, dp are scratch rows of Nk doubles. */
+static void row_grads(const double* qi, const double* doi, const double* kb, const double* vb, long kvs,
+                      int Nq, int Nk, int d, double scale, int wl, int wr, int na,
+                      const unsigned char* key_keep, int b, int i, double* s, double* p, double* dp,
+                      double* dqi, const int* krows, int nkeys, double* dk_out, double* dv_out,
+                      long out_stride) {
+    double m, l;
+    if (dqi)
+        for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+    if (!softmax_row(qi, kb, kvs, Nk, d, scale, key_keep, b, Nq, wl, wr, na, i, s, p, &m, &l))
+        return; /* no visible key: every gradient term of this row is 0 */
+    double D = 0.0;
+    for (int j = 0; j < Nk; ++j) {
+        dp[j] = (p[j] == 0.0) ? 0.0 : dot(doi, vb + (long)j * kvs, d);
+        D += p[j] * dp[j];
+    }
+    if (dqi) {
+        for (int j = 0; j < Nk; ++j) {
+            const double ds = p[j] * (dp[j] - D);
+            if (ds == 0.0) continue;
+            const double* kj = kb + (long)j * kvs;
+            for (int c = 0; c < d; ++c) dqi[c] += scale * ds * kj[c];
+        }
+    }
+    for (int t = 0; t < nkeys; ++t) {
+        const int j = krows ? krows[t] : t;
+        if (p[j] == 0.0) continue;
+        const double ds = p[j] * (dp[j] - D);
+        double* dkj = dk_out + (long)t * out_stride;
+        double* dvj = dv_out + (long)t * out_stride;
+        for (int c = 0; c < d; ++c) {
+            dkj[c] += scale * ds * qi[c];
+            dvj[c] += p[j] * doi[c];
+        }
+    }
+}
+
+/* Backward of one (batch, KV head) group over all its query heads: writes the dq
+ * rows of those query heads and accumulates dk, dv of the KV head (every row and
+ * key; serial, callers run groups in parallel). */
 static int bwd_group(const double* q, const double* k, const double* v, const double* dout,
                      int Nq, int Nk, int Hq, int Hkv, int d, double scale, int wl, int wr, int na,
-                     const unsigned char* key_keep, int b, int hk, const int* qrows, int nq,
-                     const int* krows, int nk, double* dq, double* dk, double* dv) {
+                     const unsigned char* key_keep, int b, int hk, double* dq, double* dk, double* dv) {
     const int group = Hq / Hkv;
     const long qs = (long)Hq * d, kvs = (long)Hkv * d;
     const double* kb = k + ((long)b * Nk * Hkv + hk) * d;
     const double* vb = v + ((long)b * Nk * Hkv + hk) * d;
+    double* dkb = dk + ((long)b * Nk * Hkv + hk) * d;
+    double* dvb = dv + ((long)b * Nk * Hkv + hk) * d;
     double* s = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
     double* p = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
     double* dp = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
-    unsigned char* want_q = (unsigned char*)calloc(Nq > 0 ? Nq : 1, 1);
-    if (!s || !p || !dp || !want_q) {
-        free(s); free(p); free(dp); free(want_q);
+    if (!s || !p || !dp) {
+        free(s); free(p); free(dp);
         return 2;
-    }
-    if (krows) {
-        for (int t = 0; t < nq; ++t) want_q[qrows[t]] = 1;
     }
     for (int g = 0; g < group; ++g) {
         const int h = hk * group + g;
         for (int i = 0; i < Nq; ++i) {
-            int needed = 1;
-            if (krows) {
-                needed = want_q[i];
-                for (int t = 0; t < nk && !needed; ++t)
-                    needed = visible(key_keep, b, Nq, Nk, wl, wr, na, i, krows[t]);
-            }
-            if (!needed) continue;
-            const double* qi = q + ((long)b * Nq + i) * qs + (long)h * d;
-            const double* doi = dout + ((long)b * Nq + i) * qs + (long)h * d;
-            double m, l;
-            if (!softmax_row(qi, kb, kvs, Nk, d, scale, key_keep, b, Nq, wl, wr, na, i, s, p, &m, &l))
-                continue; /* no visible key: every gradient term of this row is 0 */
-            double D = 0.0;
-            for (int j = 0; j < Nk; ++j) {
-                dp[j] = (p[j] == 0.0) ? 0.0 : dot(doi, vb + (long)j * kvs, d);
-                D += p[j] * dp[j];
-            }
-            if (!krows || want_q[i]) {
-                double* dqi = dq + ((long)b * Nq + i) * qs + (long)h * d;
-                for (int c = 0; c < d; ++c) dqi[c] = 0.0;
-                for (int j = 0; j < Nk; ++j) {
-                    const double ds = p[j] * (dp[j] - D);
-                    if (ds == 0.0) continue;
-                    const double* kj = kb + (long)j * kvs;
-                    for (int c = 0; c < d; ++c) dqi[c] += scale * ds * kj[c];
-                }
-            }
-            const int nkeys = krows ? nk : Nk;
-            for (int t = 0; t < nkeys; ++t) {
-                const int j = krows ? krows[t] : t;
-                if (p[j] == 0.0) continue;
-                const double ds = p[j] * (dp[j] - D);
-                double* dkj = dk + ((long)b * Nk + j) * kvs + (long)hk * d;
-                double* dvj = dv + ((long)b * Nk + j) * kvs + (long)hk * d;
-                for (int c = 0; c < d; ++c) {
-                    dkj[c] += scale * ds * qi[c];
-                    dvj[c] += p[j] * doi[c];
-                }
-            }
+            const long off = ((long)b * Nq + i) * qs + (long)h * d;
+            row_grads(q + off, dout + off, kb, vb, kvs, Nq, Nk, d, scale, wl, wr, na, key_keep, b, i, s, p,
+                      dp, dq + off, NULL, Nk, dkb, dvb, kvs);
         }
     }
-    free(s); free(p); free(dp); free(want_q);
+    free(s); free(p); free(dp);
     return 0;
 }
 
@@ -251,7 +251,7 @@ int ora_attn_bwd(const double* q, const double* k, const double* v, const double
 #pragma omp parallel for schedule(dynamic, 1)
     for (long t = 0; t < (long)B * Hkv; ++t) {
         int e = bwd_group(q, k, v, dout, Nq, Nk, Hq, Hkv, d, scale, wl, wr, na, key_keep,
-                          (int)(t / Hkv), (int)(t % Hkv), NULL, 0, NULL, 0, dq, dk, dv);
+                          (int)(t / Hkv), (int)(t % Hkv), dq, dk, dv);
         if (e) {
 #pragma omp atomic write
             err = e;
@@ -263,21 +263,77 @@ int ora_attn_bwd(const double* q, const double* k, const double* v, const double
 /* Sampled backward of one (batch b, KV head hk) group: dq for the nq query
  * rows in qrows (every query head of the group), dk and dv for the nk key
  * rows in krows. Outputs use the full tensor layouts; only the sampled rows
- * are written (dk/dv rows are overwritten, not accumulated). Parallel over
- * the sampled key rows is not needed: one call is one group. */
+ * are written (dk/dv rows are overwritten, not accumulated). Query rows that
+ * are not sampled and see none of the sampled keys are skipped: they add
+ * nothing to those keys' gradients. The rows are spread over the OpenMP
+ * threads; each thread adds its rows' dk/dv terms into partial sums of its
+ * own, which are added together at the end (every row's arithmetic is that of
+ * the full backward; only the order of the final sums differs). */
 int ora_attn_bwd_sampled(const double* q, const double* k, const double* v, const double* dout,
                          int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, int wl, int wr, int na,
                          const unsigned char* key_keep, int b, int hk, const int* qrows, int nq,
                          const int* krows, int nk, double* dq, double* dk, double* dv) {
-    if (b < 0 || b >= B || hk < 0 || hk >= Hkv || Hq % Hkv) return 1;
-    for (int t = 0; t < nk; ++t) {
-        double* dkj = dk + ((long)b * Nk + krows[t]) * Hkv * d + (long)hk * d;
-        double* dvj = dv + ((long)b * Nk + krows[t]) * Hkv * d + (long)hk * d;
-        for (int c = 0; c < d; ++c) dkj[c] = dvj[c] = 0.0;
+    if (b < 0 || b >= B || hk < 0 || hk >= Hkv || Hq % Hkv || nk < 0 || nq < 0) return 1;
+    const int group = Hq / Hkv;
+    const long qs = (long)Hq * d, kvs = (long)Hkv * d;
+    const double* kb = k + ((long)b * Nk * Hkv + hk) * d;
+    const double* vb = v + ((long)b * Nk * Hkv + hk) * d;
+    unsigned char* want_q = (unsigned char*)calloc(Nq > 0 ? Nq : 1, 1);
+    double* sum_k = (double*)calloc((size_t)(nk > 0 ? nk : 1) * d, sizeof(double));
+    double* sum_v = (double*)calloc((size_t)(nk > 0 ? nk : 1) * d, sizeof(double));
+    int* rows = (int*)malloc(sizeof(int) * (Nq > 0 ? Nq : 1));
+    int err = 0;
+    if (!want_q || !sum_k || !sum_v || !rows) {
+        free(want_q); free(sum_k); free(sum_v); free(rows);
+        return 2;
     }
-    /* Split the group's query heads across threads would race on dk/dv; the
-     * speed comes from the caller sampling few rows, so this runs serially
-     * per group and callers may run several groups in parallel processes. */
-    return bwd_group(q, k, v, dout, Nq, Nk, Hq, Hkv, d, scale, wl, wr, na, key_keep, b, hk, qrows,
-                     nq, krows, nk ? nk : 0, dq, dk, dv);
+    for (int t = 0; t < nq; ++t) want_q[qrows[t]] = 1;
+    /* the query rows that take part: sampled, or seeing a sampled key */
+    int nrows = 0;
+    for (int i = 0; i < Nq; ++i) {
+        int needed = want_q[i];
+        for (int t = 0; t < nk && !needed; ++t) needed = visible(key_keep, b, Nq, Nk, wl, wr, na, i, krows[t]);
+        if (needed) rows[nrows++] = i;
+    }
+    const long work = (long)group * nrows;
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
+        double* p = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
+        double* dp = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
+        double* part_k = (double*)calloc((size_t)(nk > 0 ? nk : 1) * d, sizeof(double));
+        double* part_v = (double*)calloc((size_t)(nk > 0 ? nk : 1) * d, sizeof(double));
+        const int have = s && p && dp && part_k && part_v;
+        if (!have) {
+#pragma omp atomic write
+            err = 2;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (long w = 0; w < work; ++w) {
+            if (!have) continue;
+            const int h = hk * group + (int)(w / nrows);
+            const int i = rows[w % nrows];
+            const long off = ((long)b * Nq + i) * qs + (long)h * d;
+            row_grads(q + off, dout + off, kb, vb, kvs, Nq, Nk, d, scale, wl, wr, na, key_keep, b, i, s, p, dp,
+                      want_q[i] ? dq + off : NULL, krows, nk, part_k, part_v, d);
+        }
+        if (have) {
+#pragma omp critical
+            for (long x = 0; x < (long)nk * d; ++x) {
+                sum_k[x] += part_k[x];
+                sum_v[x] += part_v[x];
+            }
+        }
+        free(s); free(p); free(dp); free(part_k); free(part_v);
+    }
+    for (int t = 0; t < nk; ++t) {
+        double* dkj = dk + ((long)b * Nk + krows[t]) * kvs + (long)hk * d;
+        double* dvj = dv + ((long)b * Nk + krows[t]) * kvs + (long)hk * d;
+        for (int c = 0; c < d; ++c) {
+            dkj[c] = sum_k[(long)t * d + c];
+            dvj[c] = sum_v[(long)t * d + c];
+        }
+    }
+    free(want_q); free(sum_k); free(sum_v); free(rows);
+    return err;
 }

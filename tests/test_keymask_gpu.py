@@ -7,7 +7,7 @@ import torch
 import oracle
 from exact_tiled_attention_36_b200 import binding as fb
 from exact_tiled_attention_36_b200 import inputs
-from tests.gpu_util import ATOL_L, RTOL_GRAD, f64, guarded, o_bound
+from tests.gpu_util import check_grads, check_l, check_o, f64, guarded, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -19,11 +19,6 @@ def _lib():
     fb.lib()
     yield
     assert fb.fa_get_last_device_error(None) == fb.FA_OK
-
-
-def rel_l2(a, b):
-    nb = np.linalg.norm(b)
-    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
 
 
 def make_keep(kind, B, Nk, rng):
@@ -88,11 +83,11 @@ def test_keymask_fwd_bwd(case):
     empty = np.isneginf(l_ref)
     assert np.isneginf(l64[empty]).all() and (o64.transpose(0, 2, 1, 3)[empty] == 0).all()
     live = ~empty
-    assert np.abs(l64[live] - l_ref[live]).max() <= ATOL_L
-    assert (np.abs(o64 - o_ref) <= o_bound(o_ref, q.dtype)).all()
+    check_l(l64[live], l_ref[live])
+    check_o(o64, o_ref, q.dtype)
     rq, rk, rv = oracle.attn_bwd(fi.q, fi.k, fi.v, fi.do, scale, causal, key_keep=keep)
     errs = [rel_l2(f64(g), r) for g, r in ((dq, rq), (dk, rk), (dv, rv))]
-    assert max(errs) <= RTOL_GRAD, errs
+    check_grads(errs)
     # masked keys get exactly zero gradients
     masked = keep == 0
     assert (f64(dk)[masked] == 0).all() and (f64(dv)[masked] == 0).all()

@@ -7,7 +7,7 @@ import torch
 import oracle
 from exact_tiled_attention_36_b200 import binding as fb
 from exact_tiled_attention_36_b200 import inputs
-from tests.gpu_util import RTOL_GRAD, SENTINEL, f64, guarded
+from tests.gpu_util import SENTINEL, check_grads, check_rel, f64, guarded, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -19,11 +19,6 @@ def _lib():
     fb.lib()
     yield
     assert fb.fa_get_last_device_error(None) == fb.FA_OK
-
-
-def rel_l2(a, b):
-    nb = np.linalg.norm(b)
-    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
 
 
 def run_varlen_fwd_bwd(vi, causal, extra_rows=0):
@@ -84,12 +79,12 @@ def check_sequences(vi, dq, dk, dv, causal):
     got = (dq[:n_q], dk[:n_k], dv[:n_k])
     ref = (refs[0][:n_q], refs[1][:n_k], refs[2][:n_k])
     errs = [rel_l2(g, r) for g, r in zip(got, ref)]
-    assert max(errs) <= RTOL_GRAD, errs
+    check_grads(errs)
     for (qa, qb), (ka, kb) in spans:
         for g, r, (x, y) in ((dq, refs[0], (qa, qb)), (dk, refs[1], (ka, kb)), (dv, refs[2], (ka, kb))):
             nr = np.linalg.norm(r[x:y])
             if nr > 1e-3 * np.linalg.norm(r):
-                assert rel_l2(g[x:y], r[x:y]) <= RTOL_GRAD, (x, y)
+                check_rel(rel_l2(g[x:y], r[x:y]), "per-sequence rel L2")
 
 
 CASES = [
@@ -149,3 +144,34 @@ def test_varlen_bwd_matches_fixed_length_path(d):
     assert torch.equal(dk_v.reshape(B, N, Hkv, d), dk_f)
     assert torch.equal(dv_v.reshape(B, N, Hkv, d), dv_f)
     assert rel_l2(f64(dq_v.reshape(B, N, Hq, d)), f64(dq_f)) <= 1e-2
+
+
+def test_varlen_bwd_reports_a_sequence_past_max_seqlen():
+    """The backward with a max_seqlen_q below a sequence's length returns FA_OK and
+    reports FA_ERR_INVALID_ARG through the device error word; nothing is written
+    outside the gradient buffers."""
+    lengths = [64, 260, 10]
+    vi = inputs.make_varlen(inputs.VARLEN, lengths=lengths, Hq=2, Hkv=1, d=128, dtype="bf16", seed=38,
+                            with_do=True)
+    q, k, v, do = vi.q.cuda(), vi.k.cuda(), vi.v.cuda(), vi.do.cuda()
+    cu_q, cu_k = vi.cu_seqlens_q.cuda(), vi.cu_seqlens_k.cuda()
+    Tq, Hq, d = q.shape
+    Tk, Hkv, _ = k.shape
+    n, scale = len(lengths), d ** -0.5
+    o = torch.zeros_like(q)
+    lse = torch.zeros((Hq, Tq), dtype=torch.float32, device="cuda")
+    assert fb.fa_varlen_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), cu_q.data_ptr(),
+                            cu_k.data_ptr(), n, Tq, Tk, 260, 260, Hq, Hkv, d, scale, 1, fb.FA_BF16, 0) == fb.FA_OK
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    bound = 128
+    ws = torch.full((fb.fa_varlen_bwd_workspace_size(n, Tq, bound, Hq, d),), 255, dtype=torch.uint8, device="cuda")
+    dq, dq_ok = guarded((Tq, Hq, d), q.dtype)
+    dk, dk_ok = guarded((Tk, Hkv, d), q.dtype)
+    dv, dv_ok = guarded((Tk, Hkv, d), q.dtype)
+    st = fb.fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), cu_q.data_ptr(),
+                          cu_k.data_ptr(), n, Tq, Tk, bound, bound, Hq, Hkv, d, scale, 1, fb.FA_BF16, 0)
+    assert st == fb.FA_OK
+    assert fb.fa_get_last_device_error(None) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    assert dq_ok() and dk_ok() and dv_ok(), "write outside dQ / dK / dV"

@@ -6,7 +6,7 @@ import torch
 import oracle
 from exact_tiled_attention_36_b200 import binding as fb
 from exact_tiled_attention_36_b200 import inputs
-from tests.gpu_util import ATOL_L, f64, guarded, o_bound
+from tests.gpu_util import check_l, check_o, f64, guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -43,8 +43,6 @@ def check_sequences(vi, o, lse, causal, rows_per_seq=None, seed=0):
     """Per sequence, the oracle on that sequence alone (sampled rows if asked)."""
     rng = np.random.default_rng(seed)
     scale = vi.q.shape[-1] ** -0.5
-    worst_o = worst_l = 0.0
-    worst_excess = -np.inf
     for s, (Lq, Lk) in enumerate(zip(vi.seqlens_q, vi.seqlens_k)):
         if Lq == 0:
             continue
@@ -64,11 +62,8 @@ def check_sequences(vi, o, lse, causal, rows_per_seq=None, seed=0):
         assert (og.transpose(1, 0, 2)[empty] == 0).all()
         live = ~empty
         if live.any():
-            worst_l = max(worst_l, float(np.abs(lg[live] - lrf[live]).max()))
-        err = np.abs(og - orf)
-        worst_o = max(worst_o, float(err.max()))
-        worst_excess = max(worst_excess, float((err - o_bound(orf, vi.q.dtype)).max()))
-    assert worst_excess <= 0 and worst_l <= ATOL_L, (worst_o, worst_excess, worst_l)
+            check_l(lg[live], lrf[live])
+        check_o(og, orf, vi.q.dtype)
 
 
 SMALL = [
@@ -109,3 +104,35 @@ def test_varlen_matches_fixed_length_path():
     torch.cuda.synchronize()
     assert torch.equal(o_v.reshape(B, N, H, d), o_f)
     assert torch.equal(l_v.reshape(H, B, N).permute(1, 0, 2), l_f)
+
+
+@pytest.mark.parametrize("too_small", ["q", "k"])
+def test_varlen_reports_a_sequence_past_max_seqlen(too_small):
+    """A max_seqlen bound below a sequence's length cannot be caught before the launch
+    (cu_seqlens live on the device): the call returns FA_OK, processes that sequence only
+    up to the bound, and the next fa_get_last_device_error reports FA_ERR_INVALID_ARG
+    (then the word is clear again). Sequences within the bound are still exact."""
+    lengths = [100, 300, 50]
+    vi = inputs.make_varlen(inputs.VARLEN, lengths=lengths, Hq=2, Hkv=2, d=128, dtype="bf16", seed=37)
+    q, k, v = vi.q.cuda(), vi.k.cuda(), vi.v.cuda()
+    cu_q, cu_k = vi.cu_seqlens_q.cuda(), vi.cu_seqlens_k.cuda()
+    Tq, Hq, d = q.shape
+    o, o_ok = guarded((Tq, Hq, d), q.dtype)
+    lse, l_ok = guarded((Hq, Tq), torch.float32)
+    max_q, max_k = (200, 300) if too_small == "q" else (300, 200)
+    st = fb.fa_varlen_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), cu_q.data_ptr(),
+                          cu_k.data_ptr(), len(lengths), Tq, k.shape[0], max_q, max_k, Hq, 2, d, d ** -0.5, 0,
+                          fb.FA_BF16, 0)
+    assert st == fb.FA_OK
+    assert fb.fa_get_last_device_error(None) == fb.FA_ERR_INVALID_ARG
+    assert fb.fa_get_last_device_error(None) == fb.FA_OK
+    assert o_ok() and l_ok(), "write outside O / L"
+    # the sequences inside the bounds (0 and 2) are untouched by the clipping
+    o64, l64 = f64(o), f64(lse)
+    for s in (0, 2):
+        a, L = int(vi.cu_seqlens_q[s]), lengths[s]
+        o_ref, l_ref = oracle.attn_fwd(vi.q[None, a:a + L], vi.k[None, a:a + L], vi.v[None, a:a + L], d ** -0.5)
+        check_o(o64[a:a + L], o_ref[0], q.dtype)
+        check_l(l64[:, a:a + L], l_ref[0])
+    # within the bounds the word stays clear
+    run_varlen(vi, False)

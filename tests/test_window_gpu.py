@@ -7,7 +7,7 @@ import torch
 import oracle
 from exact_tiled_attention_36_b200 import binding as fb
 from exact_tiled_attention_36_b200 import inputs
-from tests.gpu_util import ATOL_L, RTOL_GRAD, f64, guarded, o_bound
+from tests.gpu_util import check_grads, check_l, check_o, check_rel, f64, guarded, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -19,11 +19,6 @@ def _lib():
     fb.lib()
     yield
     assert fb.fa_get_last_device_error(None) == fb.FA_OK
-
-
-def rel_l2(a, b):
-    nb = np.linalg.norm(b)
-    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
 
 
 def run(fi, window, backward=True):
@@ -78,11 +73,11 @@ def test_window_fwd_bwd(case):
     assert np.isneginf(lse[empty]).all()
     assert (o.transpose(0, 2, 1, 3)[empty] == 0).all()
     live = ~empty
-    assert np.abs(lse[live] - l_ref[live]).max() <= ATOL_L
-    assert (np.abs(o - o_ref) <= o_bound(o_ref, fi.q.dtype)).all()
+    check_l(lse[live], l_ref[live])
+    check_o(o, o_ref, fi.q.dtype)
     rq, rk, rv = oracle.attn_bwd(fi.q, fi.k, fi.v, fi.do, d ** -0.5, window=window)
     errs = [rel_l2(g, r) for g, r in ((dq, rq), (dk, rk), (dv, rv))]
-    assert max(errs) <= RTOL_GRAD, errs
+    check_grads(errs)
 
 
 def test_causal_window_is_the_causal_path():
@@ -108,10 +103,10 @@ def test_window_long_sequence_sampled_rows():
     o, lse, (dq, dk, dv) = run(fi, window)
     rows = [0, 1, 1023, 1024, 1025, 4000, 8191]
     o_ref, l_ref = oracle.attn_fwd(fi.q, fi.k, fi.v, d ** -0.5, window=window, rows=rows)
-    assert (np.abs(o[:, rows] - o_ref[:, rows]) <= o_bound(o_ref[:, rows], fi.q.dtype)).all()
-    assert np.abs(lse[:, :, rows] - l_ref[:, :, rows]).max() <= ATOL_L
+    check_o(o[:, rows], o_ref[:, rows], fi.q.dtype)
+    check_l(lse[:, :, rows], l_ref[:, :, rows])
     ref = f64(fi.do).sum((0, 1))  # (Hq, d) -> the single KV head sums all query heads
-    assert rel_l2(dv.sum((0, 1))[0], ref.sum(0)) <= RTOL_GRAD
+    check_rel(rel_l2(dv.sum((0, 1))[0], ref.sum(0)), "sum of dV rel L2")
 
 
 VARLEN_CASES = [
@@ -156,8 +151,8 @@ def test_varlen_window(case):
     empty = np.isneginf(l_ref)
     assert np.isneginf(l64[empty]).all() and (o64.transpose(1, 0, 2)[empty] == 0).all()
     live = ~empty
-    assert np.abs(l64[live] - l_ref[live]).max() <= ATOL_L
-    assert (np.abs(o64 - o_ref) <= o_bound(o_ref, q.dtype)).all()
+    check_l(l64[live], l_ref[live])
+    check_o(o64, o_ref, q.dtype)
     ws = torch.empty(fb.fa_varlen_bwd_workspace_size(n, Tq, vi.max_seqlen_q, Hq, d), dtype=torch.uint8, device="cuda")
     dq, dk, dv = torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)
     bwd = fb.fa_varlen_bwd_window_anchor if anchors else fb.fa_varlen_bwd_window
@@ -176,7 +171,7 @@ def test_varlen_window(case):
                                      vi.do[None, a:a + Lq], d ** -0.5, window=window)
         refs[0][a:a + Lq], refs[1][ka:ka + Lk], refs[2][ka:ka + Lk] = rq[0], rk[0], rv[0]
     errs = [rel_l2(f64(g), r) for g, r in zip((dq, dk, dv), refs)]
-    assert max(errs) <= RTOL_GRAD, errs
+    check_grads(errs)
 
 
 ANCHOR_CASES = [
@@ -217,11 +212,11 @@ def test_window_anchor_fwd_bwd(case):
     empty = np.isneginf(l_ref)
     assert np.isneginf(l64[empty]).all()
     live = ~empty
-    assert np.abs(l64[live] - l_ref[live]).max() <= ATOL_L
-    assert (np.abs(o64 - o_ref) <= o_bound(o_ref, q.dtype)).all()
+    check_l(l64[live], l_ref[live])
+    check_o(o64, o_ref, q.dtype)
     rq, rk, rv = oracle.attn_bwd(fi.q, fi.k, fi.v, fi.do, d ** -0.5, window=window)
     errs = [rel_l2(f64(g), r) for g, r in ((dq, rq), (dk, rk), (dv, rv))]
-    assert max(errs) <= RTOL_GRAD, errs
+    check_grads(errs)
 
 
 def test_window_anchor_zero_is_the_window_path():
