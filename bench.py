@@ -60,6 +60,62 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+def choose_peak(clocks, peaks, peak_src):
+    """The bf16 peak that matches the timed region's clocks: the burst figure (measured
+    with the GPU at its maximum SM clock) when the region's median SM clock under load
+    is within 5 % of the maximum or no clock record exists; the sustained figure
+    (measured over seconds at the 1 kW power cap) when the clocks sat lower."""
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if clocks and clocks.get("sm_max_mhz") and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"]:
+        return sust, (f"bf16_tflops_sustained ({peak_src}): median SM clock {clocks['sm_mhz']:.0f} MHz under "
+                      f"load, below the {clocks['sm_max_mhz']:.0f} MHz maximum")
+    why = (f"median SM clock {clocks['sm_mhz']:.0f} of {clocks['sm_max_mhz']:.0f} MHz under load" if clocks
+           else "no clock record")
+    return burst, f"bf16_tflops burst ({peak_src}): {why}"
+
+
+def algorithmic_bytes(kernel, B, N, Hq, Hkv, d):
+    """Bytes a launch must move at least: the backward main kernel reads Q, dO, K, V, L
+    and D and writes dK and dV (the fp32 dQ accumulator's reductions are implementation
+    traffic, not counted); the forward reads Q, K, V and writes O and L."""
+    q_b, kv_b, row_b = 2 * B * N * Hq * d, 2 * B * N * Hkv * d, 4 * B * Hq * N
+    if kernel == "fa_bwd128_kernel":
+        return 2 * q_b + 4 * kv_b + 2 * row_b
+    return 2 * q_b + 2 * kv_b + row_b
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def cpu_tiny_single_core():
+    """The oracle's forward of the tiny workload (B=1, H=2, N=256, d=64) on one core."""
+    import oracle
+    from exact_tiled_attention_36_b200 import inputs
+    cfg = inputs.TINY
+    fi = inputs.make_fixed(cfg)
+    args = [oracle._f64(t) for t in (fi.q, fi.k, fi.v)]
+    before = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        oracle.attn_fwd(*args, cfg.scale, cfg.causal)
+        t0 = time.perf_counter()
+        oracle.attn_fwd(*args, cfg.scale, cfg.causal)
+        dt = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(before)
+    flops = flops_fwd(cfg.B, cfg.Nq, cfg.Hq, cfg.d, cfg.causal)
+    return {"seconds": dt, "tflops": flops / dt / 1e12, "cores": 1,
+            "sample": "oracle forward of the whole tiny workload"}
+
+
 # The device code each profiled kernel is compiled from (its header and what it
 # includes; the host file only encodes descriptors and launches).
 KERNEL_SOURCES = {
@@ -444,8 +500,14 @@ def run_ours(args):
     else:
         kname, kflops, kms = "fa_fwd_kernel", f_fwd, fwd_avg
     achieved = kflops / (kms / 1e3) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak, peak_kind = choose_peak(clocks, peaks, peak_src)
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
+    clock_mhz = clocks["sm_mhz"] if clocks else peaks.get("sm_max_mhz", 1965.0)
+    f_tf, b_tf = f_fwd / (fwd_avg / 1e3) / 1e12, f_bwd / (bwd_avg / 1e3) / 1e12
+    traffic = profiled_traffic(kname)
+    alg_bytes = algorithmic_bytes(kname, B, N, Hq, Hkv, d)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -453,22 +515,32 @@ def run_ours(args):
         "config": {"workload": w["name"], "B": B, "seq_len": N, "Hq": Hq, "Hkv": Hkv, "d": d, "causal": True,
                    "parallelism": f"replicas x{world} (no exchange step)",
                    "l2": "inputs larger than L2: ~1.0 GB of tensors touched per step vs 126 MB L2"},
-        "fwd_tflops": f_fwd / (fwd_avg / 1e3) / 1e12,
-        "bwd_tflops": f_bwd / (bwd_avg / 1e3) / 1e12,
-        # both passes run inside the long step loop: the sustained peak is theirs (the burst
-        # fraction for comparison)
-        "fwd_frac_of_sustained": f_fwd / (fwd_avg / 1e3) / 1e12 / peak,
-        "fwd_frac_of_burst": f_fwd / (fwd_avg / 1e3) / 1e12 / peak_burst,
-        "bwd_frac_of_sustained": f_bwd / (bwd_avg / 1e3) / 1e12 / peak,
-        "bwd_frac_of_burst": f_bwd / (bwd_avg / 1e3) / 1e12 / peak_burst,
+        "fwd_tflops": f_tf, "bwd_tflops": b_tf,
+        # the fraction of the peak the clock record selects (roofline.peak_kind), and of both
+        "fwd_frac": f_tf / peak, "bwd_frac": b_tf / peak,
+        "fwd_frac_of_burst": f_tf / peak_burst, "bwd_frac_of_burst": b_tf / peak_burst,
+        "fwd_frac_of_sustained": f_tf / peak_sust, "bwd_frac_of_sustained": b_tf / peak_sust,
         "fwd_ms": fwd_avg, "bwd_ms": bwd_avg, "bwd_main_kernel_ms": main_avg,
         "fwd_alone": {"calls": n_fwd, "ms": fwd_alone_ms, "tflops": f_fwd / (fwd_alone_ms / 1e3) / 1e12,
                       "frac_of_burst": f_fwd / (fwd_alone_ms / 1e3) / 1e12 / peak_burst,
                       "how": "forward calls back to back after the step loop, CUDA events, max over ranks"},
         "roofline": {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "peak_kind": f"bf16_tflops_sustained ({peak_src})",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
                      "peak_burst": peak_burst, "frac_of_burst": achieved / peak_burst,
-                     "traffic": profiled_traffic(kname)},
+                     "peak_sustained": peak_sust, "frac_of_sustained": achieved / peak_sust,
+                     "traffic": traffic, "algorithmic_bytes": alg_bytes,
+                     "traffic_over_algorithmic": (traffic / alg_bytes) if traffic else None},
+        "ceilings": {
+            "how": "MUFU ex2: 16 per clock per SM x SMs x median SM clock of the timed region x FLOPs per "
+                   "score (one exponential per score; 4d FLOP forward, 10d backward)",
+            "sms": sms, "sm_mhz": clock_mhz,
+            "mufu_fwd_d128_tflops": mufu_ceiling_tflops(128, 4 * 128, sms, clock_mhz),
+            "mufu_fwd_d64_tflops": mufu_ceiling_tflops(64, 4 * 64, sms, clock_mhz),
+            "mufu_bwd_d128_tflops": mufu_ceiling_tflops(128, 10 * 128, sms, clock_mhz),
+            "fwd_frac_of_mufu": f_tf / mufu_ceiling_tflops(d, 4 * d, sms, clock_mhz),
+            "bwd_main_frac_of_mufu": (f_bwd / (main_avg / 1e3) / 1e12) / mufu_ceiling_tflops(d, 10 * d, sms,
+                                                                                              clock_mhz),
+        },
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": K_e2e, "ms_per_step": e2e_ms / K_e2e,
                 "how": "pinned host buffers; H2D of q, k, v, dO and D2H of dq, dk, dv every step on their own "
@@ -476,11 +548,21 @@ def run_ours(args):
         "gpu_launches": K * 4,  # per step: forward, preprocess, main backward, dQ convert
         "clocks": clocks,
     }
+    if world == 1 and not args.no_configs:
+        # Every workload and pass, timed after the step loop (CUDA events, inputs resident
+        # in device memory): the short-sequence shapes, varlen, the prefill variants, FP8,
+        # windows and decode.
+        del q, k, v, do, o, lse, dq, dk, dv, ws, d_in, d_out, h_out, hq, hk, hv, hdo
+        torch.cuda.empty_cache()
+        configs = {}
+        Sweep(fb, torch, peaks, configs.__setitem__, sms, clock_mhz).run()
+        line["configs"] = configs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         flops, times, cores = cpu_oracle_sample(1, CPU_SAMPLE_TOKENS)
         cpu_v = flops / times[0] / 1e12
         line["cpu_baseline"] = {"value": cpu_v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": cpu_sample_desc(CPU_SAMPLE_TOKENS), "seconds": times[0]}
+                                "cpu_model": cpu_model(), "sample": cpu_sample_desc(CPU_SAMPLE_TOKENS),
+                                "seconds": times[0], "single_core_tiny": cpu_tiny_single_core()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -490,93 +572,165 @@ def run_ours(args):
 
 
 # ----------------------------------------------------------------------------- per-workload sweep
-def run_sweep(args):
-    """Forward (and the backward where the workload has one) of every workload, and the
-    decode workloads, one JSON line each.
-    Informational: the bench line of the contract is the default mode."""
-    import torch
-    from exact_tiled_attention_36_b200 import binding as fb
-    from exact_tiled_attention_36_b200 import inputs
+EX2_PER_CLK_PER_SM = 16  # MUFU exponentials per clock per SM
 
-    peaks, peak_src = load_peaks()
-    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    stream = torch.cuda.current_stream()
 
-    def time_it(fn, iters):
+def mufu_ceiling_tflops(d, flops_per_score, sms, clock_mhz):
+    """The TFLOP/s at which the exponentials alone (one per score: the softmax of
+    "FlashAttention/zh", section "FlashAttention algorithm") would fill the MUFU pipe:
+    16 ex2 / clock / SM x SMs x clock x the FLOPs a score carries (4d forward, 10d
+    backward)."""
+    return EX2_PER_CLK_PER_SM * sms * clock_mhz * 1e6 * flops_per_score / 1e12
+
+
+class Sweep:
+    """Times the forward (and backward where the workload has one) of every workload
+    and the decode workloads. Each result goes to `sink(key, entry)`."""
+
+    def __init__(self, fb, torch, peaks, sink, sms, clock_mhz, only=None):
+        self.fb, self.torch, self.sink, self.only = fb, torch, sink, only
+        self.peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        self.hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        self.sms, self.clock = sms, clock_mhz
+        self.stream = torch.cuda.current_stream()
+
+    def time_it(self, fn, iters):
+        torch, fb = self.torch, self.fb
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        e0.record(self.stream)
         for _ in range(iters):
             fn()
-        e1.record(stream)
+        e1.record(self.stream)
         torch.cuda.synchronize()
         if fb.fa_get_last_device_error(None) != fb.FA_OK:
             raise RuntimeError("device error")
         return e0.elapsed_time(e1) / iters
 
-    def emit(name, what, ms, flops, nbytes, fp8=False):
-        line = {"kind": "config_sweep", "workload": name, "pass": what, "ms": ms,
-                "tflops": flops / (ms / 1e3) / 1e12, "frac_of_bf16_burst": flops / (ms / 1e3) / 1e12 / peak,
-                "algorithmic_gbs": nbytes / (ms / 1e3) / 1e9, "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / hbm,
-                "peaks": peak_src}
+    def emit(self, name, what, ms, flops, nbytes, d=None, fp8=False):
+        tf = flops / (ms / 1e3) / 1e12
+        e = {"workload": name, "pass": what, "ms": ms, "tflops": tf, "frac_of_burst": tf / self.peak,
+             "algorithmic_gbs": nbytes / (ms / 1e3) / 1e9, "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / self.hbm}
+        if d is not None:
+            per_score = (10 if what == "bwd" else 4) * d
+            ceil = mufu_ceiling_tflops(d, per_score, self.sms, self.clock)
+            e["mufu_ceiling_tflops"] = ceil
+            e["frac_of_mufu_ceiling"] = tf / ceil
         if fp8:  # the E4M3 tensor peak: the measured bf16 burst peak x the nominal 2x ratio
-            line["frac_of_fp8_peak"] = flops / (ms / 1e3) / 1e12 / (2.0 * peak)
-        print(json.dumps(line), flush=True)
+            e["frac_of_fp8_peak"] = tf / (2.0 * self.peak)
+        self.sink(f"{name}:{what}", e)
 
-    def want(name):
-        return args.only is None or args.only in name
+    def want(self, name):
+        return self.only is None or self.only in name
 
-    for cfg in (inputs.TINY, inputs.VISION, inputs.VIT_RMSNORM, inputs.CAUSAL_GQA):
-        if not want(cfg.name):
-            continue
-        fi = inputs.make_fixed(cfg)
-        q, k, v = (t.cuda() for t in (fi.q, fi.k, fi.v))
-        B, N, Hq, d = q.shape
+    def run(self):
+        from exact_tiled_attention_36_b200 import inputs
+        fb, torch = self.fb, self.torch
+        for cfg in (inputs.TINY, inputs.VISION, inputs.VIT_RMSNORM, inputs.CAUSAL_GQA):
+            if not self.want(cfg.name):
+                continue
+            fi = inputs.make_fixed(cfg)
+            q, k, v = (t.cuda() for t in (fi.q, fi.k, fi.v))
+            B, N, Hq, d = q.shape
+            o, lse = fb.attention_fwd(q, k, v, cfg.scale, cfg.causal)
+            flops = flops_fwd(B, N, Hq, d, cfg.causal)
+            nbytes = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
+            iters = 1000 if cfg is inputs.TINY else 30
+            ms = self.time_it(lambda: fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse), iters)
+            self.emit(cfg.name, "fwd", ms, flops, nbytes, d)
+            if cfg is inputs.TINY:
+                self.tiny_calls(fb, torch, cfg, q, k, v, o, lse, flops, nbytes, d)
+            if cfg.backward:
+                do = fi.do.cuda()
+                ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, N, d), dtype=torch.uint8, device="cuda")
+                ms = self.time_it(lambda: fb.attention_bwd(q, k, v, o, lse, do, cfg.scale, cfg.causal, workspace=ws),
+                                  20)
+                self.emit(cfg.name, "bwd", ms, 2.5 * flops,
+                          nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()), d)
+            del q, k, v, o, lse, fi
+        args = (inputs, fb, torch, self.stream, self.time_it, self.emit)
+        if self.want(inputs.CAUSAL_GQA_FP8.name):
+            sweep_fp8(inputs.CAUSAL_GQA_FP8, *args)
+        if self.want(inputs.CAUSAL_GQA.name + "_window1024_anchor4"):
+            sweep_window(*args)
+        if self.want("causal_gqa_b2_n8192_hq32_hkv8_d128_noncausal") or \
+                self.want("causal_gqa_b2_n8192_hq32_hkv32_d128_mha"):
+            sweep_prefill_variants(*args)
+        if self.want(inputs.VIT_RMSNORM.name + "_packed_qkv_fused_qk_rmsnorm"):
+            sweep_vit_variants(*args)
+        for cfg in (inputs.VARLEN, inputs.VARLEN_KEYPAD):
+            if self.want(cfg.name):
+                sweep_varlen(cfg, *args)
+        for cfg, page in ((inputs.DECODE, 0), (inputs.DECODE_RAGGED, 0), (inputs.DECODE_RAGGED, 64),
+                          (inputs.DECODE_RAGGED, 32), (inputs.DECODE_RAGGED, 16), (inputs.DECODE_D64, 0),
+                          (inputs.DECODE_SPEC4, 0)):
+            if self.want(cfg.name + (f"_paged{page}" if page else "")):
+                sweep_decode(cfg, page, *args)
+
+    def tiny_calls(self, fb, torch, cfg, q, k, v, o, lse, flops, nbytes, d):
+        """The tiny workload is bound by per-call host work when called eagerly: timed
+        through the torch-level binding, through the C ABI directly (arguments marshalled
+        once), and replayed from a CUDA graph of 100 calls (the device's time per call)."""
+        B, N, Hq, _ = q.shape
         Hkv = k.shape[2]
-        o, lse = fb.attention_fwd(q, k, v, cfg.scale, cfg.causal)
-        flops = flops_fwd(B, N, Hq, d, cfg.causal)
-        nbytes = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
-        iters = 1000 if cfg is inputs.TINY else 30
-        ms = time_it(lambda: fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse), iters)
-        emit(cfg.name, "fwd", ms, flops, nbytes)
-        if cfg is inputs.TINY:
-            # Eager calls this small are bound by the host's per-call work (Python, the C ABI
-            # call, encoding the tensor maps); 100 calls captured in a CUDA graph and replayed
-            # give the device's time per call.
-            g = torch.cuda.CUDAGraph()
-            gs = torch.cuda.Stream()
-            with torch.cuda.graph(g, stream=gs):
-                for _ in range(100):
-                    fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse, stream=gs)
-            ms = time_it(g.replay, 10) / 100
-            emit(cfg.name, "fwd_graph_replay", ms, flops, nbytes)
-            del g
-        if cfg.backward:
-            do = fi.do.cuda()
-            ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, N, d), dtype=torch.uint8, device="cuda")
-            ms = time_it(lambda: fb.attention_bwd(q, k, v, o, lse, do, cfg.scale, cfg.causal, workspace=ws), 20)
-            emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
-        del q, k, v, o, lse
-    # the causal GQA prefill shape with block-scaled E4M3 inputs (fa_fwd_fp8)
-    cfg = inputs.CAUSAL_GQA_FP8
-    if want(cfg.name):
-        sweep_fp8(cfg, inputs, fb, torch, stream, time_it, emit)
-    if want(inputs.CAUSAL_GQA.name + "_window1024_anchor4"):
-        sweep_window(inputs, fb, torch, stream, time_it, emit)
-    if want("causal_gqa_b2_n8192_hq32_hkv8_d128_noncausal") or want("causal_gqa_b2_n8192_hq32_hkv32_d128_mha"):
-        sweep_prefill_variants(inputs, fb, torch, stream, time_it, emit)
-    if want(inputs.VIT_RMSNORM.name + "_packed_qkv_fused_qk_rmsnorm"):
-        sweep_vit_variants(inputs, fb, torch, stream, time_it, emit)
-    for cfg in (inputs.VARLEN, inputs.VARLEN_KEYPAD):
-        if want(cfg.name):
-            sweep_varlen(cfg, inputs, fb, torch, stream, time_it, emit)
-    for cfg, page in ((inputs.DECODE, 0), (inputs.DECODE_RAGGED, 0), (inputs.DECODE_RAGGED, 64),
-                      (inputs.DECODE_RAGGED, 32), (inputs.DECODE_RAGGED, 16), (inputs.DECODE_D64, 0), (inputs.DECODE_SPEC4, 0)):
-        if want(cfg.name + (f"_paged{page}" if page else "")):
-            sweep_decode(cfg, page, inputs, fb, torch, stream, time_it, emit)
+        sh = self.stream.cuda_stream
+        f = fb.lib().fa_fwd
+        argv = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d,
+                float(cfg.scale), int(cfg.causal), fb.FA_BF16, sh)
+        if f(*argv) != fb.FA_OK:
+            raise RuntimeError("fa_fwd failed")
+        ms = self.time_it(lambda: f(*argv), 1000)
+        self.emit(cfg.name, "fwd_eager_c_abi", ms, flops, nbytes, d)
+        g = torch.cuda.CUDAGraph()
+        gs = torch.cuda.Stream()
+        with torch.cuda.graph(g, stream=gs):
+            for _ in range(100):
+                fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse, stream=gs)
+        ms = self.time_it(g.replay, 10) / 100
+        self.emit(cfg.name, "fwd_graph_replay", ms, flops, nbytes, d)
+        del g
+
+
+# Workloads whose forward kernel gets its own profiler capture: (input config name, calls).
+PROFILE_CASES = {"vision_fwd": ("VISION", 3), "vit_fwd": ("VIT_RMSNORM", 3), "tiny_fwd": ("TINY", 3)}
+
+
+def run_profile_case(name):
+    """A few forward calls of one workload at full size (each holds ~211 MB on the
+    device), for ncu captures of the forward kernel on that shape."""
+    import torch
+    from exact_tiled_attention_36_b200 import binding as fb
+    from exact_tiled_attention_36_b200 import inputs
+    cfg_name, calls = PROFILE_CASES[name]
+    cfg = getattr(inputs, cfg_name)
+    fi = inputs.make_fixed(cfg)
+    q, k, v = (t.cuda() for t in (fi.q, fi.k, fi.v))
+    o, lse = fb.attention_fwd(q, k, v, cfg.scale, cfg.causal)
+    for _ in range(calls - 1):
+        fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse)
+    torch.cuda.synchronize()
+    if fb.fa_get_last_device_error(None) != fb.FA_OK:
+        raise RuntimeError("device error")
+    print(f"profile case {name} ({cfg.name}): {calls} forward calls done", flush=True)
+    return 0
+
+
+def run_sweep(args):
+    """--all-configs: one JSON line per workload and pass (the same entries the default
+    bench line carries in its `configs` object)."""
+    import torch
+    from exact_tiled_attention_36_b200 import binding as fb
+    peaks, peak_src = load_peaks()
+    fb.lib()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    clock = peaks.get("sm_max_mhz", 1965.0)
+
+    def sink(key, e):
+        print(json.dumps({"kind": "config_sweep", **e, "peaks": peak_src}), flush=True)
+
+    Sweep(fb, torch, peaks, sink, sms, clock, args.only).run()
     return 0
 
 
@@ -597,7 +751,7 @@ def sweep_fp8(cfg, inputs, fb, torch, stream, time_it, emit):
             raise RuntimeError(fb.fa_status_string(r))
 
     emit(cfg.name, "fwd", time_it(ffp8, 30), flops_fwd(B, N, Hq, d, cfg.causal),
-         q8.numel() + k8.numel() + v8.numel() + 2 * o.numel() + 4 * lse.numel(), fp8=True)
+         q8.numel() + k8.numel() + v8.numel() + 2 * o.numel() + 4 * lse.numel(), d, fp8=True)
 
 
 def sweep_window(inputs, fb, torch, stream, time_it, emit):
@@ -630,9 +784,9 @@ def sweep_window(inputs, fb, torch, stream, time_it, emit):
             raise RuntimeError(fb.fa_status_string(r))
 
     nb = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
-    emit(cfg.name + "_window1024", "fwd", time_it(wfwd, 30), wflops, nb)
+    emit(cfg.name + "_window1024", "fwd", time_it(wfwd, 30), wflops, nb, d)
     emit(cfg.name + "_window1024", "bwd", time_it(wbwd, 20), 2.5 * wflops,
-         nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+         nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()), d)
     # the same window plus 4 global anchor keys (the first tokens, visible to every query)
     na = 4
     apairs = pairs + sum(max(0, min(na, i - wl)) for i in range(N))
@@ -651,9 +805,9 @@ def sweep_window(inputs, fb, torch, stream, time_it, emit):
         if r != fb.FA_OK:
             raise RuntimeError(fb.fa_status_string(r))
 
-    emit(cfg.name + "_window1024_anchor4", "fwd", time_it(afwd, 30), aflops, nb)
+    emit(cfg.name + "_window1024_anchor4", "fwd", time_it(afwd, 30), aflops, nb, d)
     emit(cfg.name + "_window1024_anchor4", "bwd", time_it(abwd, 20), 2.5 * aflops,
-         nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+         nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()), d)
 
 
 def sweep_prefill_variants(inputs, fb, torch, stream, time_it, emit):
@@ -669,10 +823,10 @@ def sweep_prefill_variants(inputs, fb, torch, stream, time_it, emit):
         ws = torch.empty(fb.fa_bwd_workspace_size(B, Hq, N, d), dtype=torch.uint8, device="cuda")
         nb = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
         emit(base.name.replace("_hkv8", f"_hkv{hkv}") + tag, "fwd",
-             time_it(lambda: fb.attention_fwd(q, k, v, base.scale, causal, out=o, lse=lse), 30), flops, nb)
+             time_it(lambda: fb.attention_fwd(q, k, v, base.scale, causal, out=o, lse=lse), 30), flops, nb, d)
         emit(base.name.replace("_hkv8", f"_hkv{hkv}") + tag, "bwd",
              time_it(lambda: fb.attention_bwd(q, k, v, o, lse, do, base.scale, causal, workspace=ws), 20),
-             2.5 * flops, nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+             2.5 * flops, nb + 2 * (do.numel() + q.numel() + k.numel() + v.numel()), d)
         del q, k, v, do, o, lse, ws, fi
 
 
@@ -697,7 +851,7 @@ def sweep_vit_variants(inputs, fb, torch, stream, time_it, emit):
 
     ms = time_it(packed, 30)
     emit(cfg.name + "_packed_qkv", "fwd", ms, flops_fwd(B, N, Hq, d, cfg.causal),
-         2 * (q.numel() + k.numel() + v.numel() + q.numel()) + 4 * lse.numel())
+         2 * (q.numel() + k.numel() + v.numel() + q.numel()) + 4 * lse.numel(), d)
     del qkv, q, k, v, o, lse
     # the ViT workload with raw Q and K, their RMS normalisation fused (fa_fwd_qk_rmsnorm)
     cfg = inputs.VIT_RMSNORM
@@ -717,7 +871,7 @@ def sweep_vit_variants(inputs, fb, torch, stream, time_it, emit):
 
     ms = time_it(fused, 30)
     emit(cfg.name + "_fused_qk_rmsnorm", "fwd", ms, flops_fwd(B, N, Hq, d, cfg.causal),
-         2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel())
+         2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel(), d)
 
 
 
@@ -730,7 +884,7 @@ def sweep_varlen(cfg, inputs, fb, torch, stream, time_it, emit):
     nbytes = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
     ms = time_it(lambda: fb.attention_varlen_fwd(q, k, v, cu_q, cu_k, vi.max_seqlen_q, vi.max_seqlen_k,
                                                  cfg.scale, cfg.causal, out=o, lse=lse), 20)
-    emit(cfg.name, "fwd", ms, flops, nbytes)
+    emit(cfg.name, "fwd", ms, flops, nbytes, cfg.d)
     if cfg is inputs.VARLEN:
         # the varlen backward on the same packed batch (dO drawn after Q, K, V)
         do = inputs.make_varlen(cfg, with_do=True).do.cuda()
@@ -750,7 +904,8 @@ def sweep_varlen(cfg, inputs, fb, torch, stream, time_it, emit):
                 raise RuntimeError(fb.fa_status_string(st))
 
         ms = time_it(vbwd, 10)
-        emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()))
+        emit(cfg.name, "bwd", ms, 2.5 * flops, nbytes + 2 * (do.numel() + q.numel() + k.numel() + v.numel()),
+             cfg.d)
 
 
 def sweep_decode(cfg, page, inputs, fb, torch, stream, time_it, emit):
@@ -790,7 +945,7 @@ def sweep_decode(cfg, page, inputs, fb, torch, stream, time_it, emit):
     vis = sum(min(n, max(0, t + n - Nq + 1)) if cfg.causal else n for n in lens for t in range(Nq))
     flops = 4.0 * d * Hq * vis
     nbytes = 2 * (2 * keys * Hkv * d + 2 * q.numel()) + 4 * lse.numel()
-    emit(cfg.name + (f"_paged{page}" if page else ""), "decode", time_it(dec, 50), flops, nbytes)
+    emit(cfg.name + (f"_paged{page}" if page else ""), "decode", time_it(dec, 50), flops, nbytes, d)
 
 
 def main():
@@ -800,14 +955,20 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="leave out the per-workload `configs` object of the bench line")
     ap.add_argument("--profile-small", action="store_true",
                     help="run only the warm-up steps on a smaller case (B=1, N=4096) for ncu captures")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
+                    help="run a few forward calls of one short-sequence workload at full size (for ncu captures)")
     ap.add_argument("--all-configs", action="store_true",
                     help="time the forward of every workload (and the causal GQA backward); one JSON line each")
     ap.add_argument("--only", default=None,
                     help="with --all-configs: only the workload groups whose name contains this text "
                          "(e.g. decode, fp8, window, varlen)")
     args = ap.parse_args()
+    if args.profile_case:
+        return run_profile_case(args.profile_case)
     if args.all_configs:
         return run_sweep(args)
     if args.impl == "reference":

@@ -310,12 +310,17 @@ def _dtype_code(t) -> int:
 def _dev(t):
     if not t.is_cuda:
         raise ValueError("tensors must be on a CUDA device")
-    return t.contiguous()
+    return t if t.is_contiguous() else t.contiguous()
 
 
 def _stream(stream):
+    """The raw CUDA stream handle: `stream` (a torch stream or a handle), or the current
+    stream of the current device."""
     import torch
     if stream is None:
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)  # the handle without a Stream object
+        if raw is not None:
+            return raw(torch.cuda.current_device())
         return torch.cuda.current_stream().cuda_stream
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
@@ -380,7 +385,7 @@ def attention_bwd(q, k, v, o, lse, dout, scale: float | None = None, causal: boo
 
 def attention_varlen_bwd(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                          scale: float | None = None, causal: bool = False, workspace=None, stream=None):
-    """dQ, dK, dV of the packed varlen forward (same layouts as q, k, v; d = 128)."""
+    """dQ, dK, dV of the packed varlen forward (same layouts as q, k, v; d = 64 or 128)."""
     import torch
     q, k, v, o, dout = _dev(q), _dev(k), _dev(v), _dev(o), _dev(dout)
     lse = _dev(lse)

@@ -40,6 +40,36 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
     return fn;
 }
 
+// Every argument of one tensor-map encoding (the key of the cache below). Built by
+// memset + assignment, so the padding bytes are zero and memcmp compares keys.
+struct MapKey {
+    const void* base;
+    int64_t rows, batches, sh, ss, sb;
+    int d, H, box_h, box_rows, elem_bytes;
+    int flags;  // bit 0: bf16, bit 1: 256-byte L2 promotion
+};
+
+// Encoded tensor maps of recent calls, per host thread (no lock): a caller that
+// repeats a call with the same tensors and shapes, as a training or decoding loop
+// does, reuses the maps instead of encoding them again. Direct-mapped on a hash of
+// the key; a map is a pure function of its key, so a stale entry is never wrong,
+// only replaced.
+struct MapCache {
+    static constexpr int kSlots = 128;
+    MapKey key[kSlots];
+    CUtensorMap map[kSlots];
+    bool used[kSlots] = {};
+};
+
+uint32_t map_key_hash(const MapKey& k) {
+    const unsigned char* p = reinterpret_cast<const unsigned char*>(&k);
+    uint32_t h = 2166136261u;  // FNV-1a
+    for (size_t i = 0; i < sizeof(MapKey); ++i) h = (h ^ p[i]) * 16777619u;
+    return h;
+}
+
+fa_status encode_map(CUtensorMap* m, const MapKey& k);
+
 // Tensor map of a [batches, rows, H, d] 16-bit tensor, box = box_rows rows x
 // box_h heads x 64 columns, 128-byte swizzle. Rows past `rows` read as zero.
 // 4-D map (d, H, rows, batches) over a tensor whose head, token and batch strides
@@ -50,10 +80,44 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 fa_status make_map_box(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t batches, bool bf16,
                        int64_t sh, int64_t ss, int64_t sb, int box_h, int box_rows, bool promote_256 = true,
                        int elem_bytes = 2) {
-    auto enc = encode_tiled();
-    if (!enc) return FA_ERR_CUDA;
     if (rows < 1) rows = 1;
     if (batches < 1) batches = 1;
+    MapKey k;
+    std::memset(&k, 0, sizeof(k));
+    k.base = base;
+    k.rows = rows;
+    k.batches = batches;
+    k.sh = sh;
+    k.ss = ss;
+    k.sb = sb;
+    k.d = d;
+    k.H = H;
+    k.box_h = box_h;
+    k.box_rows = box_rows;
+    k.elem_bytes = elem_bytes;
+    k.flags = (bf16 ? 1 : 0) | (promote_256 ? 2 : 0);
+    thread_local MapCache cache;
+    const int slot = static_cast<int>(map_key_hash(k) % MapCache::kSlots);
+    if (cache.used[slot] && std::memcmp(&cache.key[slot], &k, sizeof(k)) == 0) {
+        *m = cache.map[slot];
+        return FA_OK;
+    }
+    const fa_status st = encode_map(m, k);
+    if (st == FA_OK) {
+        cache.key[slot] = k;
+        cache.map[slot] = *m;
+        cache.used[slot] = true;
+    }
+    return st;
+}
+
+fa_status encode_map(CUtensorMap* m, const MapKey& key) {
+    auto enc = encode_tiled();
+    if (!enc) return FA_ERR_CUDA;
+    const void* base = key.base;
+    const int d = key.d, H = key.H, box_h = key.box_h, box_rows = key.box_rows, elem_bytes = key.elem_bytes;
+    const int64_t rows = key.rows, batches = key.batches, sh = key.sh, ss = key.ss, sb = key.sb;
+    const bool bf16 = (key.flags & 1) != 0, promote_256 = (key.flags & 2) != 0;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batches)};
     const cuuint64_t eb = static_cast<cuuint64_t>(elem_bytes);

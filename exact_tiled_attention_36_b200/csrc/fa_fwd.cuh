@@ -29,7 +29,9 @@
 //                 was read from with no wait in between: the tensor core executes
 //                 one thread's tcgen05.mma operations in issue order (the order
 //                 NVIDIA's own Blackwell attention example relies on; the GPU
-//                 parity tests check it).
+//                 parity tests check it). With d = 64 the order is instead: S_0 and
+//                 S_1 of key tile j + 1 as soon as each softmax has read S_t(j)
+//                 (P_t has its own TMEM columns), then P_0 V_j and P_1 V_j.
 //   warps 4-7     softmax of tile 0; warps 8-11 softmax of tile 1. Thread r owns
 //                 query row r of its tile (TMEM lane r) and keeps the whole row of
 //                 S in registers: warps 0-3 hand registers over with setmaxnreg
@@ -45,7 +47,12 @@
 //   warps 2-3     idle.
 //
 // TMEM columns: [0,128) S_0 / P_0, [128,256) S_1 / P_1, [256,256+d) O_0,
-// [256+d,256+2d) O_1.
+// [256+d,256+2d) O_1. With d = 64, P_t has its own columns [384 + 64 t, 448 + 64 t)
+// instead: the softmax frees S_t as soon as it has read it (s_free), the MMA thread
+// issues S_t of the next key tile into it at once, and the P_t V product signals
+// pv_done, which the softmax waits for before it writes the next P_t or rescales O_t.
+// The softmax of consecutive key tiles then no longer waits for the P V and S
+// products in between (at d = 64 its exponentials outweigh the products).
 #pragma once
 
 #include "sm100.cuh"
@@ -98,11 +105,16 @@ struct FwdCfg {
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 1 + 1 + 1 + 1;
+    static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 1 + 1 + 1 + 1 + 2 + 2;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0, kColO = 256;  // S_t at 128 t, O_t at 256 + d t
+    // d = 64 (16-bit): P_t has columns of its own, [384 + 64 t, 448 + 64 t), so S_t of
+    // the next key tile can be computed while the softmax still works on this one.
+    static constexpr bool kSepP = D == 64 && !FP8;
+    static constexpr uint32_t kColP = kSepP ? 384 : 0;
+    static_assert(!kSepP || kColP + 128 <= kTmemCols, "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -356,6 +368,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint64_t* sm_done = o_ready + 1;  // every softmax thread is past its last TMEM access
     uint64_t* mma_done = sm_done + 1;  // every product this CTA issued is complete
     uint64_t* q_norm = mma_done + 1;   // QKNORM: Q of the unit normalised
+    uint64_t* s_free = q_norm + 1;     // [2] kSepP: the softmax has read S_t
+    uint64_t* pv_done = s_free + 2;    // [2] kSepP: P_t V is complete
     // The barrier the MMA thread waits on before reading Q.
     uint64_t* q_ready = QKNORM ? q_norm : q_full;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
@@ -382,6 +396,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_init(sm_done, 256);
         mbar_init(mma_done, 1);
         mbar_init(q_norm, 256);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_free[i], 128);
+            mbar_init(&pv_done[i], 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -464,19 +482,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             constexpr uint32_t id_pv = FP8 ? idesc_e4m3(128, D, false, true) : idesc_f16(128, D, BF16, false, true);
             const uint32_t q_addr = smem_u32(sQ);
             // S_t = Q_t K^T with the K tile of global ring index g.
+            // Descriptors of both Q tiles and of every K / V ring slot, made once; the
+            // products step through an operand by adding to the low word.
+            SDesc qdesc[2], kdesc[S], vdesc[S];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) qdesc[i] = sdesc_sw128_split(q_addr + i * C::kTileBytes, 16, 1024);
+#pragma unroll
+            for (int i = 0; i < S; ++i) {
+                kdesc[i] = sdesc_sw128_split(smem_u32(sK + i * C::kTileBytes), 16, 1024);
+                vdesc[i] = sdesc_sw128_split(smem_u32(sV + i * C::kTileBytes), C::kSlabBytes, 1024);
+            }
             auto issue_s = [&](int t, int g) {
-                const uint32_t k_addr = smem_u32(sK + (g % S) * C::kTileBytes);
+                const SDesc kd = kdesc[g % S];
+                const SDesc qd = qdesc[t];
 #pragma unroll
                 for (int kk = 0; kk < C::kKSteps; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::kSlabBytes + (kk & 3) * 32;
-                    const uint64_t qd = sdesc_sw128(q_addr + t * C::kTileBytes + off, 16, 1024);
-                    const uint64_t kd = sdesc_sw128(k_addr + off, 16, 1024);
+                    const uint32_t step = ((kk >> 2) * C::kSlabBytes + (kk & 3) * 32) >> 4;
                     if constexpr (FP8)
-                        mma_ss_f8(tmem + C::kColS + 128 * t, qd, kd, id_qk, kk > 0 ? 1u : 0u);
+                        mma_ss_f8(tmem + C::kColS + 128 * t, (static_cast<uint64_t>(qd.hi) << 32) | (qd.lo + step),
+                                  (static_cast<uint64_t>(kd.hi) << 32) | (kd.lo + step), id_qk, kk > 0 ? 1u : 0u);
                     else
-                        mma_ss(tmem + C::kColS + 128 * t, qd, kd, id_qk, kk > 0 ? 1u : 0u);
+                        mma_ss_split(tmem + C::kColS + 128 * t, qd, step, kd, step, id_qk, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(&s_full[t]);
+            };
+            // kSepP: S_t number n (n >= 1) reuses the columns of number n - 1, which the
+            // softmax must have read first.
+            int ns[2] = {0, 0};
+            auto issue_s_sep = [&](int t, int g) -> bool {
+                if (ns[t] > 0 && !mbar_wait(&s_free[t], (ns[t] - 1) & 1, wc, 76)) return false;
+                tc_fence_after();
+                issue_s(t, g);
+                ++ns[t];
+                return true;
             };
             int gk = 0, nq = 0;
             int ps[2] = {0, 0};  // p_full phases consumed per tile
@@ -491,12 +529,55 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tc_fence_after();
                 // The first S products of this unit run while the softmax warpgroups
                 // still write the previous unit's O (they touch only the S columns).
-                for (int t = 0; t < 2; ++t)
-                    if (MASK == kMaskAnchor ? fwd_active<MASK>(w, t, 0) : (w.a(t) == 0 && w.b(t) > 0)) issue_s(t, gk);
+                for (int t = 0; ok && t < 2; ++t)
+                    if (MASK == kMaskAnchor ? fwd_active<MASK>(w, t, 0) : (w.a(t) == 0 && w.b(t) > 0)) {
+                        if constexpr (C::kSepP)
+                            ok = issue_s_sep(t, gk);
+                        else
+                            issue_s(t, gk);
+                    }
+                if (!ok) break;
                 bool started0 = false, started1 = false;  // kMaskAnchor: tile t's first P V is issued
                 if (w.n_kv == 1) tc_commit(q_empty);
                 tc_commit(&k_empty[gk % S]);
-                for (int j = 0; ok && j < w.n_kv; ++j) {
+                if constexpr (C::kSepP) {
+                    // Per key tile j: S_t(j + 1) for each tile active at j + 1 as soon as its
+                    // softmax has read S_t(j); then P_t V_j as each P_t arrives.
+                    for (int j = 0; ok && j < w.n_kv; ++j) {
+                        const int g = gk + j, st = g % S;
+                        const bool more = j + 1 < w.n_kv;
+                        if (more) {
+                            bool need[2];
+                            for (int t = 0; t < 2; ++t)
+                                need[t] = MASK == kMaskAnchor ? fwd_active<MASK>(w, t, j + 1)
+                                                              : (j + 1 >= w.a(t) && j + 1 < w.b(t));
+                            // (waited for even if no tile needs it: the slot is released below)
+                            if (!(ok = mbar_wait(&k_full[(g + 1) % S], ((g + 1) / S) & 1, wc, 66))) break;
+                            for (int t = 0; ok && t < 2; ++t)
+                                if (need[t]) ok = issue_s_sep(t, g + 1);
+                            if (!ok) break;
+                            tc_commit(&k_empty[(g + 1) % S]);
+                            if (j + 2 == w.n_kv) tc_commit(q_empty);  // the unit's last S products are issued
+                        }
+                        if (!(ok = mbar_wait(&v_full[st], (g / S) & 1, wc, 65))) break;
+                        for (int t = 0; ok && t < 2; ++t) {
+                            if (j == 0 && nq > 0 && !(ok = mbar_wait(&o_free[t], (nq - 1) & 1, wc, 67))) break;
+                            if (!fwd_active<MASK>(w, t, j)) continue;
+                            if (!(ok = mbar_wait(&p_full[t], ps[t] & 1, wc, 68))) break;
+                            ++ps[t];
+                            tc_fence_after();
+                            const bool acc0 = MASK == kMaskAnchor ? (t ? started1 : started0) : (j > w.a(t));
+                            if (t) started1 = true; else started0 = true;
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_ts_split(tmem + C::kColO + D * t, tmem + C::kColP + 64 * t + kk * 8, vdesc[st],
+                                             kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
+                            tc_commit(&pv_done[t]);
+                        }
+                        tc_commit(&v_empty[st]);
+                    }
+                }
+                for (int j = 0; !C::kSepP && ok && j < w.n_kv; ++j) {
                     const int g = gk + j, st = g % S;
                     const bool more = j + 1 < w.n_kv;
                     if (!(ok = mbar_wait(&v_full[st], (g / S) & 1, wc, 65))) break;
@@ -535,9 +616,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         } else {
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                mma_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8,
-                                       sdesc_sw128(v_addr + kk * 2048, C::kSlabBytes, 1024), id_pv,
-                                       (acc0 || kk > 0) ? 1u : 0u);
+                                mma_ts_split(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, vdesc[st],
+                                             kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
                         }
                         if (MASK == kMaskAnchor ? (more && fwd_active<MASK>(w, t, j + 1)) : (j + 1 < w.b(t)))
                             issue_s(t, g + 1);
@@ -573,8 +653,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
         const uint32_t s_addr = lane_base + C::kColS + 128 * t;
         const uint32_t o_addr = lane_base + C::kColO + D * t;
+        const uint32_t p_addr = lane_base + C::kColP + 64 * t;  // kSepP
         const float sl2_base = args.scale_log2;
         int ss = 0, nq = 0;  // s_full phases consumed; units with work done
+        int np = 0;          // kSepP: P_t written so far (each followed by one P_t V)
         bool ok = true;
         for (int rnd = 0; ok; ++rnd) {
             const int u = fwd_unit_index(rnd, cta, G);
@@ -682,6 +764,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
     #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
+                if constexpr (C::kSepP) {  // S_t is in registers: its columns may take the next S_t
+                    tc_fence_before();
+                    mbar_arrive(&s_free[t]);
+                }
                 if (need_mask) {  // masked columns read as -inf: out of the max, P = 0
     #pragma unroll
                     for (int c = 0; c < 128; ++c) {
@@ -750,8 +836,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         rsr2[i & 3] = f2_add(rsr2[i & 3], f2_pack(unpack_lo<BF16>(u), unpack_hi<BF16>(u)));
                         pk[i >> 5][i & 31] = u;
                     }
-                    tmem_st32(s_addr + 0, pk[0]);
-                    tmem_st32(s_addr + 32, pk[1]);
+                    if constexpr (C::kSepP) {
+                        // P_t's columns and O_t are free once the previous P_t V is complete.
+                        if (np > 0) {
+                            ok = warp_all(mbar_wait(&pv_done[t], (np - 1) & 1, wc, 77));
+                            if (!ok) break;
+                        }
+                        ++np;
+                        tc_fence_after();
+                        tmem_st32(p_addr + 0, pk[0]);
+                        tmem_st32(p_addr + 32, pk[1]);
+                    } else {
+                        tmem_st32(s_addr + 0, pk[0]);
+                        tmem_st32(s_addr + 32, pk[1]);
+                    }
                 }
                 const float rs = f2_sum(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])));
                 const float rsr = f2_sum(f2_add(f2_add(rsr2[0], rsr2[1]), f2_add(rsr2[2], rsr2[3])));
@@ -759,7 +857,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 lr = lr * alpha + rsr;
                 // S_t was issued after the previous key tile's P_t V and MMAs of one thread
                 // complete in order, so O_t is final for that tile here and can be
-                // rescaled in place.
+                // rescaled in place (kSepP: pv_done was waited for above).
                 if (j > 0 && __any_sync(0xffffffffu, resc)) {
     #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {

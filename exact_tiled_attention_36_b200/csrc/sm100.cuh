@@ -200,6 +200,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
+// The same descriptor as two 32-bit words: lo = start address >> 4 (bits 0-13) and
+// LBO >> 4 (bits 16-29), hi = SBO >> 4, the version and the layout type. An operand
+// that starts k x 16 bytes further on has lo + k: shared memory addresses stay below
+// 2^18, so the start-address field never carries into the LBO field. Stepping
+// through an operand then costs one 32-bit add per instruction.
+struct SDesc {
+    uint32_t lo, hi;
+};
+__device__ __forceinline__ SDesc sdesc_sw128_split(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return {((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16),
+            ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29)};
+}
+
 // Instruction descriptor of kind::f16 with fp32 accumulation: D format at
 // bit 4, A and B formats at bits 7 and 10 (0 = f16, 1 = bf16), A/B major at
 // bits 15/16 (0 = K-major, 1 = MN-major), N >> 3 at bit 17, M >> 4 at bit 24.
@@ -217,6 +230,31 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// mma_ss with split descriptors: A = {a_lo + a_step, a.hi}, B = {b_lo + b_step, b.hi}.
+__device__ __forceinline__ void mma_ss_split(uint32_t d_tmem, SDesc a, uint32_t a_step, SDesc b, uint32_t b_step,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "mov.b64 da, {%1, %2};\n\t"
+        "mov.b64 db, {%3, %4};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a.lo + a_step), "r"(a.hi), "r"(b.lo + b_step), "r"(b.hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// mma_ts with a split descriptor for B: B = {b_lo + b_step, b.hi}.
+__device__ __forceinline__ void mma_ts_split(uint32_t d_tmem, uint32_t a_tmem, SDesc b, uint32_t b_step,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b.lo + b_step), "r"(b.hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 

@@ -72,6 +72,8 @@ def _load():
                                               ctypes.c_int,
                                               _ip, ctypes.c_int, _ip, ctypes.c_int, _dp, _dp, _dp])
         lib.ora_num_threads.restype = ctypes.c_int
+        lib.ora_set_num_threads.restype = None
+        lib.ora_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -91,6 +93,11 @@ def _window(causal, window):
 
 def num_threads() -> int:
     return int(_load().ora_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads the oracle's parallel loops use from now on."""
+    _load().ora_set_num_threads(int(n))
 
 
 def _f64(x) -> np.ndarray:

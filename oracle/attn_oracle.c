@@ -98,6 +98,15 @@ int ora_num_threads(void) {
 #endif
 }
 
+/* Threads of the parallel regions that follow (the CPU baseline times one core too). */
+void ora_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Forward. rows == NULL computes every query row; otherwise only the nrows
  * listed query indices (for every batch and head) are written to o and lse. */
 int ora_attn_fwd(const double* q, const double* k, const double* v, int B, int Hq, int Hkv,
