@@ -433,6 +433,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         a.err = err;
         const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
         if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
+        // One CTA per (sequence, KV head, key tile); the causal grid dispatches the first
+        // key tiles, which see the most query tiles, first.
         const dim3 grid = causal ? dim3(Hkv, nseq, nkt) : dim3(nkt, Hkv, nseq);
         const bool timed = g_bwd_ev_before && g_bwd_ev_after;
         if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;

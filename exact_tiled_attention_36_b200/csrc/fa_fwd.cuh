@@ -482,27 +482,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             constexpr uint32_t id_pv = FP8 ? idesc_e4m3(128, D, false, true) : idesc_f16(128, D, BF16, false, true);
             const uint32_t q_addr = smem_u32(sQ);
             // S_t = Q_t K^T with the K tile of global ring index g.
-            // Descriptors of both Q tiles and of every K / V ring slot, made once; the
-            // products step through an operand by adding to the low word.
-            SDesc qdesc[2], kdesc[S], vdesc[S];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) qdesc[i] = sdesc_sw128_split(q_addr + i * C::kTileBytes, 16, 1024);
-#pragma unroll
-            for (int i = 0; i < S; ++i) {
-                kdesc[i] = sdesc_sw128_split(smem_u32(sK + i * C::kTileBytes), 16, 1024);
-                vdesc[i] = sdesc_sw128_split(smem_u32(sV + i * C::kTileBytes), C::kSlabBytes, 1024);
-            }
+            // Descriptors of the first Q tile and of the first K / V ring slot, made once:
+            // the other tiles and slots sit kTileBytes apart, and the products step through
+            // an operand, by adding to the descriptor's low word.
+            const SDesc qdesc = sdesc_sw128_split(q_addr, 16, 1024);
+            const SDesc kdesc = sdesc_sw128_split(smem_u32(sK), 16, 1024);
+            const SDesc vdesc = sdesc_sw128_split(smem_u32(sV), C::kSlabBytes, 1024);
+            constexpr uint32_t kTileStep = C::kTileBytes >> 4;
             auto issue_s = [&](int t, int g) {
-                const SDesc kd = kdesc[g % S];
-                const SDesc qd = qdesc[t];
+                const uint32_t qoff = t * kTileStep, koff = (g % S) * kTileStep;
 #pragma unroll
                 for (int kk = 0; kk < C::kKSteps; ++kk) {
                     const uint32_t step = ((kk >> 2) * C::kSlabBytes + (kk & 3) * 32) >> 4;
                     if constexpr (FP8)
-                        mma_ss_f8(tmem + C::kColS + 128 * t, (static_cast<uint64_t>(qd.hi) << 32) | (qd.lo + step),
-                                  (static_cast<uint64_t>(kd.hi) << 32) | (kd.lo + step), id_qk, kk > 0 ? 1u : 0u);
+                        mma_ss_f8(tmem + C::kColS + 128 * t,
+                                  (static_cast<uint64_t>(qdesc.hi) << 32) | (qdesc.lo + qoff + step),
+                                  (static_cast<uint64_t>(kdesc.hi) << 32) | (kdesc.lo + koff + step), id_qk,
+                                  kk > 0 ? 1u : 0u);
                     else
-                        mma_ss_split(tmem + C::kColS + 128 * t, qd, step, kd, step, id_qk, kk > 0 ? 1u : 0u);
+                        mma_ss_split(tmem + C::kColS + 128 * t, qdesc, qoff + step, kdesc, koff + step, id_qk,
+                                     kk > 0 ? 1u : 0u);
                 }
                 tc_commit(&s_full[t]);
             };
@@ -570,8 +569,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                             if (t) started1 = true; else started0 = true;
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                mma_ts_split(tmem + C::kColO + D * t, tmem + C::kColP + 64 * t + kk * 8, vdesc[st],
-                                             kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
+                                mma_ts_split(tmem + C::kColO + D * t, tmem + C::kColP + 64 * t + kk * 8, vdesc,
+                                             st * kTileStep + kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
                             tc_commit(&pv_done[t]);
                         }
                         tc_commit(&v_empty[st]);
@@ -616,8 +615,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         } else {
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                mma_ts_split(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, vdesc[st],
-                                             kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
+                                mma_ts_split(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, vdesc,
+                                             st * kTileStep + kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
                         }
                         if (MASK == kMaskAnchor ? (more && fwd_active<MASK>(w, t, j + 1)) : (j + 1 < w.b(t)))
                             issue_s(t, g + 1);
