@@ -17,21 +17,24 @@
 // in the L2; under the causal mask it runs the heaviest units (the last query
 // rows) first. The CTA keeps its barriers, TMEM and K/V ring from unit to
 // unit: the producer loads the next unit's Q as soon as the current unit's
-// last S product has been issued, and the MMA thread issues the next unit's
+// last S product has been issued, and the MMA threads issue the next unit's
 // first S products while the softmax warpgroups write the current unit's O.
 //
 // Warp roles (384 threads):
 //   warp 0        TMA producer: Q_0, Q_1 per unit, K_j, V_j into 2-stage (d = 128)
 //                 or 4-stage (d = 64) mbarrier rings that run across units.
-//   warp 1        TMEM allocation and the single MMA-issuing thread. Per key
-//                 tile j it issues O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T,
+//   warp 1        TMEM allocation and (d = 128) the single MMA-issuing thread. Per
+//                 key tile j it issues O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T,
 //                 O_1 += P_1 V_j, S_1 = Q_1 K_{j+1}^T. S_t reuses the columns P_t
 //                 was read from with no wait in between: the tensor core executes
 //                 one thread's tcgen05.mma operations in issue order (the order
 //                 NVIDIA's own Blackwell attention example relies on; the GPU
-//                 parity tests check it). With d = 64 the order is instead: S_0 and
-//                 S_1 of key tile j + 1 as soon as each softmax has read S_t(j)
-//                 (P_t has its own TMEM columns), then P_0 V_j and P_1 V_j.
+//                 parity tests check it).
+//   warps 1, 2    (d = 64) one MMA-issuing thread per query tile, each on its own SM
+//                 sub-partition: thread t issues S_t of key tile j + 1 as soon as
+//                 the softmax has read S_t(j) (P_t has its own TMEM columns), then
+//                 P_t V_j. Q and the K / V ring slots serve both tiles: their
+//                 release barriers count one commit from each thread.
 //   warps 4-7     softmax of tile 0; warps 8-11 softmax of tile 1. Thread r owns
 //                 query row r of its tile (TMEM lane r) and keeps the whole row of
 //                 S in registers: warps 0-3 hand registers over with setmaxnreg
@@ -44,7 +47,7 @@
 //                 the last rescale (exact: O and l share the reference max).
 //                 After the unit's last product each warpgroup writes its O_t
 //                 and L and releases O_t's columns for the next unit.
-//   warps 2-3     idle.
+//   warps 2-3     idle (d = 128); warp 3 idle (d = 64).
 //
 // TMEM columns: [0,128) S_0 / P_0, [128,256) S_1 / P_1, [256,256+d) O_0,
 // [256+d,256+2d) O_1. With d = 64, P_t has its own columns [384 + 64 t, 448 + 64 t)
@@ -105,7 +108,7 @@ struct FwdCfg {
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 1 + 1 + 1 + 1 + 2 + 2;
+    static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + 1 + 2 + 2;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16;
     static constexpr uint32_t kTmemCols = 512;
@@ -364,9 +367,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint64_t* s_full = v_empty + S;  // [2 tiles]
     uint64_t* p_full = s_full + 2;   // [2]
     uint64_t* o_free = p_full + 2;   // [2] the epilogue has read O_t
-    uint64_t* o_ready = o_free + 2;  // every product of the unit is complete
-    uint64_t* sm_done = o_ready + 1;  // every softmax thread is past its last TMEM access
-    uint64_t* mma_done = sm_done + 1;  // every product this CTA issued is complete
+    uint64_t* o_ready = o_free + 2;  // [2] every product of the unit's tile t is complete
+    uint64_t* sm_done = o_ready + 2;  // every softmax thread is past its last TMEM access
+    uint64_t* mma_done = sm_done + 1;  // every product this CTA issued is complete (both issuers)
     uint64_t* q_norm = mma_done + 1;   // QKNORM: Q of the unit normalised
     uint64_t* s_free = q_norm + 1;     // [2] kSepP: the softmax has read S_t
     uint64_t* pv_done = s_free + 2;    // [2] kSepP: P_t V is complete
@@ -380,21 +383,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
+        // d = 64 has two MMA-issuing threads (one per query tile); each commits once
+        constexpr uint32_t kIssuers = C::kSepP ? 2 : 1;
+        mbar_init(q_empty, kIssuers);
         for (int i = 0; i < S; ++i) {
             mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 1);
+            mbar_init(&k_empty[i], kIssuers);
             mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 1);
+            mbar_init(&v_empty[i], kIssuers);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 128);
             mbar_init(&o_free[i], 128);
         }
-        mbar_init(o_ready, 1);
+        for (int i = 0; i < 2; ++i) mbar_init(&o_ready[i], 1);
         mbar_init(sm_done, 256);
-        mbar_init(mma_done, 1);
+        mbar_init(mma_done, kIssuers);
         mbar_init(q_norm, 256);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_free[i], 128);
@@ -475,8 +480,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (v_issued > st) mbar_wait_drain(&v_full[st], ((st + S * ((v_issued - 1 - st) / S)) / S) & 1);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (!C::kSepP && warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (d = 128)
+        // One thread issues the products of both query tiles, in the order of the warp
+        // roles above: each tile's batch of products runs on the tensor core without the
+        // other tile's in between, so each tile's S is ready as early as it can be.
         if (lane == 0) {
             constexpr uint32_t id_qk = FP8 ? idesc_e4m3(128, 128, false, false) : idesc_f16(128, 128, BF16, false, false);
             constexpr uint32_t id_pv = FP8 ? idesc_e4m3(128, D, false, true) : idesc_f16(128, D, BF16, false, true);
@@ -505,16 +513,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 tc_commit(&s_full[t]);
             };
-            // kSepP: S_t number n (n >= 1) reuses the columns of number n - 1, which the
-            // softmax must have read first.
-            int ns[2] = {0, 0};
-            auto issue_s_sep = [&](int t, int g) -> bool {
-                if (ns[t] > 0 && !mbar_wait(&s_free[t], (ns[t] - 1) & 1, wc, 76)) return false;
-                tc_fence_after();
-                issue_s(t, g);
-                ++ns[t];
-                return true;
-            };
             int gk = 0, nq = 0;
             int ps[2] = {0, 0};  // p_full phases consumed per tile
             bool ok = true;
@@ -528,55 +526,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 tc_fence_after();
                 // The first S products of this unit run while the softmax warpgroups
                 // still write the previous unit's O (they touch only the S columns).
-                for (int t = 0; ok && t < 2; ++t)
-                    if (MASK == kMaskAnchor ? fwd_active<MASK>(w, t, 0) : (w.a(t) == 0 && w.b(t) > 0)) {
-                        if constexpr (C::kSepP)
-                            ok = issue_s_sep(t, gk);
-                        else
-                            issue_s(t, gk);
-                    }
-                if (!ok) break;
+                for (int t = 0; t < 2; ++t)
+                    if (MASK == kMaskAnchor ? fwd_active<MASK>(w, t, 0) : (w.a(t) == 0 && w.b(t) > 0)) issue_s(t, gk);
                 bool started0 = false, started1 = false;  // kMaskAnchor: tile t's first P V is issued
                 if (w.n_kv == 1) tc_commit(q_empty);
                 tc_commit(&k_empty[gk % S]);
-                if constexpr (C::kSepP) {
-                    // Per key tile j: S_t(j + 1) for each tile active at j + 1 as soon as its
-                    // softmax has read S_t(j); then P_t V_j as each P_t arrives.
-                    for (int j = 0; ok && j < w.n_kv; ++j) {
-                        const int g = gk + j, st = g % S;
-                        const bool more = j + 1 < w.n_kv;
-                        if (more) {
-                            bool need[2];
-                            for (int t = 0; t < 2; ++t)
-                                need[t] = MASK == kMaskAnchor ? fwd_active<MASK>(w, t, j + 1)
-                                                              : (j + 1 >= w.a(t) && j + 1 < w.b(t));
-                            // (waited for even if no tile needs it: the slot is released below)
-                            if (!(ok = mbar_wait(&k_full[(g + 1) % S], ((g + 1) / S) & 1, wc, 66))) break;
-                            for (int t = 0; ok && t < 2; ++t)
-                                if (need[t]) ok = issue_s_sep(t, g + 1);
-                            if (!ok) break;
-                            tc_commit(&k_empty[(g + 1) % S]);
-                            if (j + 2 == w.n_kv) tc_commit(q_empty);  // the unit's last S products are issued
-                        }
-                        if (!(ok = mbar_wait(&v_full[st], (g / S) & 1, wc, 65))) break;
-                        for (int t = 0; ok && t < 2; ++t) {
-                            if (j == 0 && nq > 0 && !(ok = mbar_wait(&o_free[t], (nq - 1) & 1, wc, 67))) break;
-                            if (!fwd_active<MASK>(w, t, j)) continue;
-                            if (!(ok = mbar_wait(&p_full[t], ps[t] & 1, wc, 68))) break;
-                            ++ps[t];
-                            tc_fence_after();
-                            const bool acc0 = MASK == kMaskAnchor ? (t ? started1 : started0) : (j > w.a(t));
-                            if (t) started1 = true; else started0 = true;
-#pragma unroll
-                            for (int kk = 0; kk < 8; ++kk)
-                                mma_ts_split(tmem + C::kColO + D * t, tmem + C::kColP + 64 * t + kk * 8, vdesc,
-                                             st * kTileStep + kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
-                            tc_commit(&pv_done[t]);
-                        }
-                        tc_commit(&v_empty[st]);
-                    }
-                }
-                for (int j = 0; !C::kSepP && ok && j < w.n_kv; ++j) {
+                for (int j = 0; ok && j < w.n_kv; ++j) {
                     const int g = gk + j, st = g % S;
                     const bool more = j + 1 < w.n_kv;
                     if (!(ok = mbar_wait(&v_full[st], (g / S) & 1, wc, 65))) break;
@@ -625,7 +580,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     tc_commit(&v_empty[st]);
                     if (more) tc_commit(&k_empty[(g + 1) % S]);
                 }
-                tc_commit(o_ready);
+                tc_commit(&o_ready[0]);
+                tc_commit(&o_ready[1]);
                 gk += w.n_kv;
                 ++nq;
             }
@@ -641,6 +597,130 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    } else if (C::kSepP && (warp == 1 || warp == 2)) {
+        // ------------------------------------------------------------ MMA issuers (d = 64)
+        // Warp 1 issues every product of query tile 0, warp 2 every product of tile 1
+        // (they write disjoint TMEM columns), so each thread issues half the products of a
+        // step, on its own SM sub-partition. Q and the K / V ring slots they share are
+        // released by barriers that count both threads' commits. (At d = 64 each S is
+        // issued as soon as its columns are free, well before the softmax needs it, so
+        // the two threads' products interleaving on the tensor core costs nothing; at
+        // d = 128 it delays each tile's S and the single issuer above is faster.)
+        const int t = warp - 1;
+        if (lane == 0) {
+            constexpr uint32_t id_qk = FP8 ? idesc_e4m3(128, 128, false, false) : idesc_f16(128, 128, BF16, false, false);
+            constexpr uint32_t id_pv = FP8 ? idesc_e4m3(128, D, false, true) : idesc_f16(128, D, BF16, false, true);
+            // Descriptors of this thread's Q tile and of the first K / V ring slot, made once:
+            // the other slots sit kTileBytes apart, and the products step through an operand,
+            // by adding to the descriptor's low word.
+            constexpr uint32_t kTileStep = C::kTileBytes >> 4;
+            const SDesc qdesc = sdesc_sw128_split(smem_u32(sQ + t * C::kTileBytes), 16, 1024);
+            const SDesc kdesc = sdesc_sw128_split(smem_u32(sK), 16, 1024);
+            const SDesc vdesc = sdesc_sw128_split(smem_u32(sV), C::kSlabBytes, 1024);
+            const uint32_t s_col = tmem + C::kColS + 128 * t;
+            const uint32_t o_col = tmem + C::kColO + D * t;
+            // S_t = Q_t K^T with the K tile of global ring index g.
+            auto issue_s = [&](int g) {
+                const uint32_t koff = (g % S) * kTileStep;
+#pragma unroll
+                for (int kk = 0; kk < C::kKSteps; ++kk) {
+                    const uint32_t step = ((kk >> 2) * C::kSlabBytes + (kk & 3) * 32) >> 4;
+                    if constexpr (FP8)
+                        mma_ss_f8(s_col, (static_cast<uint64_t>(qdesc.hi) << 32) | (qdesc.lo + step),
+                                  (static_cast<uint64_t>(kdesc.hi) << 32) | (kdesc.lo + koff + step), id_qk,
+                                  kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss_split(s_col, qdesc, step, kdesc, koff + step, id_qk, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&s_full[t]);
+            };
+            // kSepP: S_t number n (n >= 1) reuses the columns of number n - 1, which the
+            // softmax must have read first.
+            int ns = 0;
+            auto issue_s_sep = [&](int g) -> bool {
+                if (ns > 0 && !mbar_wait(&s_free[t], (ns - 1) & 1, wc, 76)) return false;
+                tc_fence_after();
+                issue_s(g);
+                ++ns;
+                return true;
+            };
+            int gk = 0, nq = 0;
+            int ps = 0;  // p_full phases consumed
+            bool ok = true;
+            for (int rnd = 0; ok; ++rnd) {
+                const int u = fwd_unit_index(rnd, cta, G);
+                if (u >= args.n_units) break;
+                const FwdUnit w = fwd_unit<MASK, VARLEN>(u, args);
+                if (!w.rows || w.n_kv == 0) continue;
+                if (!(ok = mbar_wait(q_ready, nq & 1, wc, 63))) break;
+                if (!(ok = mbar_wait(&k_full[gk % S], (gk / S) & 1, wc, 64))) break;
+                tc_fence_after();
+                // The first S product of this unit runs while the softmax warpgroup still
+                // writes the previous unit's O (it touches only the S columns).
+                if (MASK == kMaskAnchor ? fwd_active<MASK>(w, t, 0) : (w.a(t) == 0 && w.b(t) > 0)) {
+                    if constexpr (C::kSepP)
+                        ok = issue_s_sep(gk);
+                    else
+                        issue_s(gk);
+                }
+                if (!ok) break;
+                bool started = false;  // kMaskAnchor: the tile's first P V is issued
+                if (w.n_kv == 1) tc_commit(q_empty);
+                tc_commit(&k_empty[gk % S]);
+                if constexpr (C::kSepP) {
+                    // Per key tile j: S_t(j + 1) if the tile is active at j + 1, as soon as its
+                    // softmax has read S_t(j); then P_t V_j once P_t arrives.
+                    for (int j = 0; ok && j < w.n_kv; ++j) {
+                        const int g = gk + j, st = g % S;
+                        const bool more = j + 1 < w.n_kv;
+                        if (more) {
+                            // (waited for even if the tile does not need it: the slot is released below)
+                            if (!(ok = mbar_wait(&k_full[(g + 1) % S], ((g + 1) / S) & 1, wc, 66))) break;
+                            const bool need = MASK == kMaskAnchor ? fwd_active<MASK>(w, t, j + 1)
+                                                                  : (j + 1 >= w.a(t) && j + 1 < w.b(t));
+                            if (need && !(ok = issue_s_sep(g + 1))) break;
+                            tc_commit(&k_empty[(g + 1) % S]);
+                            if (j + 2 == w.n_kv) tc_commit(q_empty);  // the unit's last S products are issued
+                        }
+                        if (!(ok = mbar_wait(&v_full[st], (g / S) & 1, wc, 65))) break;
+                        if (j == 0 && nq > 0 && !(ok = mbar_wait(&o_free[t], (nq - 1) & 1, wc, 67))) break;
+                        if (fwd_active<MASK>(w, t, j)) {
+                            if (!(ok = mbar_wait(&p_full[t], ps & 1, wc, 68))) break;
+                            ++ps;
+                            tc_fence_after();
+                            const bool acc0 = MASK == kMaskAnchor ? started : (j > w.a(t));
+                            started = true;
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_ts_split(o_col, tmem + C::kColP + 64 * t + kk * 8, vdesc,
+                                             st * kTileStep + kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
+                            tc_commit(&pv_done[t]);
+                        }
+                        tc_commit(&v_empty[st]);
+                    }
+                }
+                tc_commit(&o_ready[t]);
+                gk += w.n_kv;
+                ++nq;
+            }
+            tc_commit(mma_done);
+            if (t == 0) {
+                // TMEM is freed once both issuers' products are complete and the softmax
+                // warpgroups are done with it. Every wait is bounded, so the arrivals come
+                // (4 s bounds here as a last resort).
+                for (uint64_t* bar : {mma_done, sm_done}) {
+                    const uint32_t a = smem_u32(bar);
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < 4000000000ull) {
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (t == 0) {
+            tc_fence_after();
+            tmem_dealloc(tmem, C::kTmemCols);
+        }
     }
         return;  // warps 0-3 end here; no code is shared with the softmax warpgroups
     } else {
@@ -873,7 +953,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 mbar_arrive(&p_full[t]);
             }
             if (!ok) break;
-            ok = warp_all(mbar_wait(o_ready, nq & 1, wc, 70));
+            ok = warp_all(mbar_wait(&o_ready[t], nq & 1, wc, 70));
             if (!ok) break;
             ++nq;
             tc_fence_after();
