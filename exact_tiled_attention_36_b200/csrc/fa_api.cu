@@ -433,9 +433,14 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         a.err = err;
         const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
         if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
-        // One CTA per (sequence, KV head, key tile); the causal grid dispatches the first
-        // key tiles, which see the most query tiles, first.
-        const dim3 grid = causal ? dim3(Hkv, nseq, nkt) : dim3(nkt, Hkv, nseq);
+        // One CTA per (sequence, KV head, key tile). The causal grid dispatches the first
+        // key tiles, which see the most query tiles, first; with d = 128 and one query head
+        // per KV head (walks a quarter as long as under 4-way grouping) it runs the key tiles
+        // of a (sequence, KV head) together instead, so their dQ reductions share the L2
+        // (measured on the causal prefill shape with Hq = Hkv = 32: 773 against 687 TFLOP/s;
+        // with 4-way grouping the heaviest-first order is faster, 785 against 767).
+        a.kt_fast = (causal && d == 128 && Hq == Hkv) ? 1 : 0;
+        const dim3 grid = (causal && !a.kt_fast) ? dim3(Hkv, nseq, nkt) : dim3(nkt, Hkv, nseq);
         const bool timed = g_bwd_ev_before && g_bwd_ev_after;
         if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;
         if (varlen)

@@ -63,6 +63,10 @@ struct BwdArgs {
     // is visible (ANDed with the window).
     const uint32_t* key_bits;
     int kb_words;
+    // d = 128 under the causal mask: 1 = the grid is (key tiles, Hkv, sequences), every key
+    // tile of a (sequence, KV head) dispatched together; 0 = (Hkv, sequences, key tiles),
+    // the first key tiles of every pair first (see fa_bwd128_kernel).
+    int kt_fast;
     int* err;
 };
 

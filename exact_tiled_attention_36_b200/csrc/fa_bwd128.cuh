@@ -75,9 +75,17 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     if (!smem_base_ok(smem, args.err)) return;
 
-    const int kt = CAUSAL ? static_cast<int>(blockIdx.z) : static_cast<int>(blockIdx.x);
-    const int hk = CAUSAL ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y);
-    const int b = CAUSAL ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
+    // Grid order. Without the causal mask, and under it when each KV head serves one
+    // query head (args.kt_fast), the grid is (key tiles, Hkv, sequences): the key tiles of a
+    // (sequence, KV head) run together, key tile kt at query tile kt + t at time t, so
+    // their dQ reductions land on neighbouring lines that stay in the L2. Under the causal
+    // mask with larger groups the walks are longer (group x query tiles), and the grid is
+    // (Hkv, sequences, key tiles): the first key tiles of every pair, the longest walks,
+    // are dispatched first, so no long walk starts near the end.
+    const bool kt_x = !CAUSAL || args.kt_fast;
+    const int kt = kt_x ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.z);
+    const int hk = kt_x ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
+    const int b = kt_x ? static_cast<int>(blockIdx.z) : static_cast<int>(blockIdx.y);
     const int k0 = kt * 128;
     // Rows of this sequence: fixed length, or varlen (b is the sequence; its rows
     // start at q_row0 / k_row0 of the packed buffers).
