@@ -438,8 +438,11 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         // per KV head (walks a quarter as long as under 4-way grouping) it runs the key tiles
         // of a (sequence, KV head) together instead, so their dQ reductions share the L2
         // (measured on the causal prefill shape with Hq = Hkv = 32: 773 against 687 TFLOP/s;
-        // with 4-way grouping the heaviest-first order is faster, 785 against 767).
-        a.kt_fast = (causal && d == 128 && Hq == Hkv) ? 1 : 0;
+        // with 4-way grouping the heaviest-first order is faster, 785 against 767). Anchor
+        // keys keep the heaviest-first order: the tile holding them is walked by every query
+        // tile, and started late it becomes the tail (window of 1024 + 4 anchors, Hq = Hkv =
+        // 32: 487 against 460 TFLOP/s; the plain window is the same either way, 585).
+        a.kt_fast = (causal && d == 128 && Hq == Hkv && n_anchor == 0) ? 1 : 0;
         const dim3 grid = (causal && !a.kt_fast) ? dim3(Hkv, nseq, nkt) : dim3(nkt, Hkv, nseq);
         const bool timed = g_bwd_ev_before && g_bwd_ev_after;
         if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;
