@@ -107,7 +107,10 @@ struct FwdCfg {
     static constexpr int kQOff = 0;                          // Q_0, Q_1
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
-    static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+    // Epilogue staging: 2 KB per softmax warp (32 rows x 32 columns of O in 16 bits).
+    static constexpr int kEpiOff = kVOff + kStages * kTileBytes;
+    static constexpr int kEpiBytesPerWarp = 32 * 32 * 2;
+    static constexpr int kBarOff = kEpiOff + 8 * kEpiBytesPerWarp;
     static constexpr int kNumBars = 2 + 4 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + 1 + 2 + 2;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16;
@@ -145,6 +148,16 @@ struct FwdUnit {
     __device__ __forceinline__ int jl(int t) const { return t ? jl1 : jl0; }
     __device__ __forceinline__ int jh(int t) const { return t ? jh1 : jh0; }
 };
+
+// 16-byte shared-memory accesses by 32-bit shared address.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+    return v;
+}
 
 // Mask kinds of the forward: none, causal (the window (-1, 0), fixed at compile
 // time), the sliding window (wl, wr) of FwdArgs, or that window plus the global
@@ -357,6 +370,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint8_t* sQ = smem + C::kQOff;
     uint8_t* sK = smem + C::kKOff;
     uint8_t* sV = smem + C::kVOff;
+    uint8_t* sEpi = smem + C::kEpiOff;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     uint64_t* q_full = bars;
     uint64_t* q_empty = bars + 1;  // the unit's last S product has read Q
@@ -961,6 +975,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const FwdUnit we = fwd_unit<MASK, VARLEN>(u, args);
             const bool out_ok = row_ok(we);
             T16* dst = out_ok ? out_row(we) : nullptr;
+            // O leaves through the warp's staging buffer, one 32-column chunk (64 bytes
+            // a row) at a time: each thread writes its row's chunk, then lane i stores
+            // bytes 16 (i % 4) .. + 16 of row 8 k + i / 4 (k = 0 .. 3), so one store
+            // instruction covers eight 64-byte row segments instead of 32 scattered 16-byte
+            // pieces. The 16-byte pieces are XOR-swizzled by row pair: both the row-wise
+            // writes and the segment-wise reads then touch each bank group once per
+            // quarter warp.
+            const uint32_t stg = smem_u32(sEpi + (warp - 4) * C::kEpiBytesPerWarp);
+            const int piece = lane & 3;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t pk[16];
@@ -975,11 +998,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pk[i] = 0u;
                 }
-                if (out_ok) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                for (int p = 0; p < 4; ++p)
+                    st_shared_v4(stg + lane * 64 + ((p ^ ((lane >> 1) & 3)) << 4), pk[4 * p], pk[4 * p + 1],
+                                 pk[4 * p + 2], pk[4 * p + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int rr = 8 * k + (lane >> 2);
+                    const uint4 val = ld_shared_v4(stg + rr * 64 + ((piece ^ ((rr >> 1) & 3)) << 4));
+                    // row rr's address and validity, from the thread that owns the row
+                    const bool seg_ok = __shfl_sync(0xffffffffu, out_ok, rr);
+                    T16* seg = reinterpret_cast<T16*>(
+                        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), rr));
+                    if (seg_ok) *reinterpret_cast<uint4*>(seg + c0 + 8 * piece) = val;
                 }
+                __syncwarp();
             }
             // O_t's columns are free for the next unit's first P_t V.
             tc_fence_before();
