@@ -543,6 +543,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int t = 0; t < 2; ++t)
                     if (MASK == kMaskAnchor ? fwd_active<MASK>(w, t, 0) : (w.a(t) == 0 && w.b(t) > 0)) issue_s(t, gk);
                 bool started0 = false, started1 = false;  // kMaskAnchor: tile t's first P V is issued
+                bool ready0 = false, ready1 = false;      // o_ready[t] committed for this unit
                 if (w.n_kv == 1) tc_commit(q_empty);
                 tc_commit(&k_empty[gk % S]);
                 for (int j = 0; ok && j < w.n_kv; ++j) {
@@ -587,15 +588,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                 mma_ts_split(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, vdesc,
                                              st * kTileStep + kk * 128, id_pv, (acc0 || kk > 0) ? 1u : 0u);
                         }
-                        if (MASK == kMaskAnchor ? (more && fwd_active<MASK>(w, t, j + 1)) : (j + 1 < w.b(t)))
+                        if (MASK == kMaskAnchor ? (more && fwd_active<MASK>(w, t, j + 1)) : (j + 1 < w.b(t))) {
                             issue_s(t, g + 1);
+                        } else if (MASK != kMaskAnchor) {
+                            // tile t's last P V of the unit: its epilogue need not wait for the
+                            // other tile's last softmax and P V
+                            tc_commit(&o_ready[t]);
+                            if (t) ready1 = true; else ready0 = true;
+                        }
                     }
                     if (j + 2 == w.n_kv) tc_commit(q_empty);  // the unit's last S products are issued
                     tc_commit(&v_empty[st]);
                     if (more) tc_commit(&k_empty[(g + 1) % S]);
                 }
-                tc_commit(&o_ready[0]);
-                tc_commit(&o_ready[1]);
+                if (!ready0) tc_commit(&o_ready[0]);
+                if (!ready1) tc_commit(&o_ready[1]);
                 gk += w.n_kv;
                 ++nq;
             }
@@ -967,14 +974,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 mbar_arrive(&p_full[t]);
             }
             if (!ok) break;
+            // (decoded again while the last P V runs)
+            const FwdUnit we = fwd_unit<MASK, VARLEN>(u, args);
+            const bool out_ok = row_ok(we);
+            T16* dst = out_ok ? out_row(we) : nullptr;
+            const float inv_l = FP8 ? (l > 0.f ? v_max / l : 0.f) : ((lr > 0.f) ? 1.f / lr : 0.f);
             ok = warp_all(mbar_wait(&o_ready[t], nq & 1, wc, 70));
             if (!ok) break;
             ++nq;
             tc_fence_after();
-            const float inv_l = FP8 ? (l > 0.f ? v_max / l : 0.f) : ((lr > 0.f) ? 1.f / lr : 0.f);
-            const FwdUnit we = fwd_unit<MASK, VARLEN>(u, args);
-            const bool out_ok = row_ok(we);
-            T16* dst = out_ok ? out_row(we) : nullptr;
             // O leaves through the warp's staging buffer, one 32-column chunk (64 bytes
             // a row) at a time: each thread writes its row's chunk, then lane i stores
             // bytes 16 (i % 4) .. + 16 of row 8 k + i / 4 (k = 0 .. 3), so one store
