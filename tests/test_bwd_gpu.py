@@ -109,3 +109,40 @@ def test_bwd_causal_gqa_full_size():
             sdv = dv[b, :, hk].sum(0)
             ref = do[b, :, hk * g:(hk + 1) * g].sum((0, 1))
             check_rel(rel_l2(sdv, ref), "sum of dV over keys rel L2")
+
+
+@pytest.mark.parametrize("hkv,causal", [(32, True), (8, False)], ids=["causal-hq32-hkv32", "noncausal-hq32-hkv8"])
+def test_bwd_full_size_other_grids(hkv, causal):
+    """The prefill shape in the two other backward grids, element-wise against the oracle:
+    - one query head per KV head, causal (Hq = Hkv = 32): the key tiles of a (batch, head)
+      run next to each other (key tile fastest) instead of heaviest first, 4096 CTAs;
+    - without the mask (Hq = 32, Hkv = 8): every key tile walks all 64 query tiles of its
+      4 heads, starting at a query tile rotated by its key tile.
+    dK and dV of keys on the first, middle and last key tiles and dQ of one row in each
+    query tile, in four (batch, KV head) groups; on every row of dK and dV the two
+    identities that hold at any size."""
+    cfg = inputs.CAUSAL_GQA
+    fi = inputs.make_fixed(cfg, Hkv=hkv, causal=causal)
+    dq, dk, dv = run_fwd_bwd(fi, causal, cfg.scale)
+    dq, dk, dv = f64(dq), f64(dk), f64(dv)
+    g = cfg.Hq // hkv
+    N = cfg.Nq
+    qrows = sorted({0, N - 1} | {t * 128 + (53 * t) % 128 for t in range(N // 128)})
+    krows = [0, 1, 127, 128, 2048, 4095, 6000, 8191]
+    q64, k64, v64, do64 = (oracle._f64(t) for t in (fi.q, fi.k, fi.v, fi.do))
+    for (b, hk) in [(0, 0), (0, hkv // 2 + 1), (1, hkv // 4 + 1), (1, hkv - 1)]:
+        sq, sk, sv = oracle.attn_bwd_sampled(q64, k64, v64, do64, cfg.scale, b, hk, qrows, krows, causal)
+        gq = dq[b][qrows][:, hk * g:(hk + 1) * g]
+        check_rel(rel_l2(gq, sq), "dQ sampled rows rel L2 (other grids)")
+        for name, got, ref in (("dk", dk[b, krows, hk], sk), ("dv", dv[b, krows, hk], sv)):
+            for t in range(len(krows)):
+                check_rel(rel_l2(got[t], ref[t]), f"{name} per sampled row rel L2 (other grids)")
+        for t in range(len(qrows)):
+            check_rel(rel_l2(gq[t], sq[t]), "dQ per sampled row rel L2 (other grids)")
+    do = f64(fi.do)
+    for b in range(cfg.B):
+        for hk in range(hkv):
+            sdk = dk[b, :, hk].sum(0)
+            assert np.abs(sdk).max() <= 2e-2 * np.abs(dk[b, :, hk]).sum(0).max() + 1e-3
+            ref = do[b, :, hk * g:(hk + 1) * g].sum((0, 1))
+            check_rel(rel_l2(dv[b, :, hk].sum(0), ref), "sum of dV over keys rel L2 (other grids)")
