@@ -96,7 +96,17 @@ def sample_rows(N, n, seed):
     return sorted(r for r in rows if 0 <= r < N)
 
 
-@pytest.mark.parametrize("cfg", [inputs.VISION, inputs.VIT_RMSNORM, inputs.CAUSAL_GQA], ids=lambda c: c.name)
+# The prefill shape's other variants the benchmark times: without the mask (the persistent
+# grid keeps a (batch, head)'s units together instead of heaviest first) and with one query
+# head per KV head.
+_PREFILL_NONCAUSAL = inputs.FixedConfig(**{**inputs.CAUSAL_GQA.__dict__, "causal": False,
+                                           "name": inputs.CAUSAL_GQA.name + "_noncausal"})
+_PREFILL_MHA = inputs.FixedConfig(**{**inputs.CAUSAL_GQA.__dict__, "Hkv": inputs.CAUSAL_GQA.Hq,
+                                     "name": inputs.CAUSAL_GQA.name + "_hkv32"})
+
+
+@pytest.mark.parametrize("cfg", [inputs.VISION, inputs.VIT_RMSNORM, inputs.CAUSAL_GQA, _PREFILL_NONCAUSAL, _PREFILL_MHA],
+                         ids=lambda c: c.name)
 def test_fwd_full_size_sampled_rows(cfg):
     fi = inputs.make_fixed(cfg, with_do=False)
     o, lse = run_fwd(fi, cfg.causal, cfg.scale)

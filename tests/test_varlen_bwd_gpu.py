@@ -175,3 +175,40 @@ def test_varlen_bwd_reports_a_sequence_past_max_seqlen():
     assert fb.fa_get_last_device_error(None) == fb.FA_ERR_INVALID_ARG
     assert fb.fa_get_last_device_error(None) == fb.FA_OK
     assert dq_ok() and dk_ok() and dv_ok(), "write outside dQ / dK / dV"
+
+
+def test_varlen_bwd_workload_sampled_rows():
+    """The varlen workload at full size (32 sequences of U[64, 4096] tokens, Hq = Hkv = 32,
+    d = 128, fp16, no mask), in the configuration the benchmark times. Each sequence is an
+    attention problem of its own, so the oracle takes it alone: for the longest, the shortest
+    and a middle sequence, in three heads each, dQ, dK and dV of sampled rows element-wise.
+    Over every sequence and head, the two identities: the keys' dK sum to zero and their dV
+    to the sum of dO over the sequence's queries."""
+    cfg = inputs.VARLEN
+    vi = inputs.make_varlen(cfg, with_do=True)
+    dq, dk, dv = run_varlen_fwd_bwd(vi, cfg.causal)
+    scale = cfg.d ** -0.5
+    lens = list(vi.seqlens_q)
+    order = sorted(range(len(lens)), key=lambda s: lens[s])
+    for s in (order[-1], order[0], order[len(order) // 2]):
+        a, ka = int(vi.cu_seqlens_q[s]), int(vi.cu_seqlens_k[s])
+        L, Lk = vi.seqlens_q[s], vi.seqlens_k[s]
+        q1, k1, v1, do1 = (oracle._f64(t) for t in (vi.q[None, a:a + L], vi.k[None, ka:ka + Lk],
+                                                      vi.v[None, ka:ka + Lk], vi.do[None, a:a + L]))
+        qrows = sorted({0, L - 1} | set(range(0, L, max(1, L // 24))))
+        krows = sorted({0, Lk - 1, Lk // 2, min(127, Lk - 1), min(128, Lk - 1)})
+        for h in (0, 13, cfg.Hq - 1):
+            sq, sk, sv = oracle.attn_bwd_sampled(q1, k1, v1, do1, scale, 0, h, qrows, krows, cfg.causal)
+            gq = dq[a + np.asarray(qrows)][:, h:h + 1]
+            for t in range(len(qrows)):
+                check_rel(rel_l2(gq[t], sq[t]), "varlen dQ per sampled row rel L2")
+            for name, got, ref in (("dk", dk[ka + np.asarray(krows), h], sk), ("dv", dv[ka + np.asarray(krows), h], sv)):
+                for t in range(len(krows)):
+                    check_rel(rel_l2(got[t], ref[t]), f"varlen {name} per sampled row rel L2")
+    do = f64(vi.do)
+    for s, (L, Lk) in enumerate(zip(vi.seqlens_q, vi.seqlens_k)):
+        a, ka = int(vi.cu_seqlens_q[s]), int(vi.cu_seqlens_k[s])
+        sdk = dk[ka:ka + Lk].sum(0)
+        assert np.abs(sdk).max() <= 2e-2 * np.abs(dk[ka:ka + Lk]).sum(0).max() + 1e-3
+        check_rel(rel_l2(dv[ka:ka + Lk].sum(0), do[a:a + L].sum(0)), "varlen sum of dV over keys rel L2")
+
