@@ -70,6 +70,9 @@ def fwd(**kw):
     (dict(k=FAKE + 8), fb.FA_ERR_MISALIGNED),
     (dict(lse=FAKE + 4), fb.FA_ERR_MISALIGNED),
     (dict(Nq=0), fb.FA_OK),  # no work: nothing is launched
+    # past the grid's per-dimension limit (65535): refused, not truncated
+    (dict(Hq=65536, Hkv=1), fb.FA_ERR_UNSUPPORTED),
+    (dict(B=65536), fb.FA_ERR_UNSUPPORTED),
 ])
 def test_fwd_rejects_before_launch(lib, kw, code):
     assert fwd(**kw) == code
@@ -111,6 +114,8 @@ def bwd(**kw):
     (dict(d=80), fb.FA_ERR_UNSUPPORTED),
     (dict(ws=FAKE + 8), fb.FA_ERR_MISALIGNED),
     (dict(dv=FAKE + 1), fb.FA_ERR_MISALIGNED),
+    (dict(B=65536), fb.FA_ERR_UNSUPPORTED),
+    (dict(Hq=65536, Hkv=65536), fb.FA_ERR_UNSUPPORTED),
 ])
 def test_bwd_rejects_before_launch(lib, kw, code):
     assert bwd(**kw) == code
