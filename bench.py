@@ -694,26 +694,40 @@ class Sweep:
 
 
 # Workloads whose forward kernel gets its own profiler capture: (input config name, calls).
-PROFILE_CASES = {"vision_fwd": ("VISION", 3), "vit_fwd": ("VIT_RMSNORM", 3), "tiny_fwd": ("TINY", 3)}
+# name -> (workload, calls, overrides of its shape); cases ending in "_bwd_small" run the
+# backward after each forward
+PROFILE_CASES = {"vision_fwd": ("VISION", 3, {}), "vit_fwd": ("VIT_RMSNORM", 3, {}), "tiny_fwd": ("TINY", 3, {}),
+                 "mha_bwd_small": ("CAUSAL_GQA", 3, dict(B=1, Nq=4096, Nk=4096, Hkv=32))}
 
 
 def run_profile_case(name):
     """A few forward calls of one workload at full size (each holds ~211 MB on the
-    device), for ncu captures of the forward kernel on that shape."""
+    device), for ncu captures of the forward kernel on that shape; or, for a backward
+    case, a few forward + backward calls of a small prefill shape (~0.3 GB)."""
     import torch
     from exact_tiled_attention_36_b200 import binding as fb
     from exact_tiled_attention_36_b200 import inputs
-    cfg_name, calls = PROFILE_CASES[name]
+    cfg_name, calls, over = PROFILE_CASES[name]
     cfg = getattr(inputs, cfg_name)
-    fi = inputs.make_fixed(cfg)
+    backward = name.endswith("_bwd_small")
+    fi = inputs.make_fixed(cfg, with_do=backward, **over)
     q, k, v = (t.cuda() for t in (fi.q, fi.k, fi.v))
+    do = fi.do.cuda() if backward else None
     o, lse = fb.attention_fwd(q, k, v, cfg.scale, cfg.causal)
-    for _ in range(calls - 1):
-        fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse)
+    ws = None
+    for i in range(calls):
+        if i:
+            fb.attention_fwd(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse)
+        if backward:
+            if ws is None:
+                ws = torch.empty(fb.fa_bwd_workspace_size(q.shape[0], q.shape[2], q.shape[1], q.shape[3]),
+                                 dtype=torch.uint8, device="cuda")
+            fb.attention_bwd(q, k, v, o, lse, do, cfg.scale, cfg.causal, workspace=ws)
     torch.cuda.synchronize()
     if fb.fa_get_last_device_error(None) != fb.FA_OK:
         raise RuntimeError("device error")
-    print(f"profile case {name} ({cfg.name}): {calls} forward calls done", flush=True)
+    what = "forward + backward" if backward else "forward"
+    print(f"profile case {name} ({cfg.name}, {over or 'full size'}): {calls} {what} calls done", flush=True)
     return 0
 
 
@@ -960,7 +974,8 @@ def main():
     ap.add_argument("--profile-small", action="store_true",
                     help="run only the warm-up steps on a smaller case (B=1, N=4096) for ncu captures")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
-                    help="run a few forward calls of one short-sequence workload at full size (for ncu captures)")
+                    help="run a few forward calls of one short-sequence workload at full size, or forward + "
+                         "backward calls of a small prefill case (for ncu captures)")
     ap.add_argument("--all-configs", action="store_true",
                     help="time the forward of every workload (and the causal GQA backward); one JSON line each")
     ap.add_argument("--only", default=None,
