@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "bwd_grid.h"
 #include "per_device.h"
 #include "fa_fwd.cuh"
 #include "fa_bwd.cuh"
@@ -433,23 +434,11 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
         a.err = err;
         const unsigned nkt = static_cast<unsigned>((Nk + 127) / 128);
         if (nkt > 65535u) return FA_ERR_UNSUPPORTED;
-        // One CTA per (sequence, KV head, key tile). The causal grid dispatches the first
-        // key tiles, which see the most query tiles, first. With d = 128, one query head per
-        // KV head (walks a quarter as long as under 4-way grouping) and a grid of at least 12
-        // waves, it runs the key tiles of a (sequence, KV head) together instead: the CTAs
-        // then read the same Q and dO tiles and reduce into the same dQ lines (B=1 N=4096,
-        // Hq = Hkv = 32: DRAM reads 202 against 447 MB, reduction hit rate 63 against 55 %).
-        // That pays once the grid is long enough for the late start of each head's longest
-        // walk not to matter (Hq = Hkv = 32, causal, TFLOP/s key-tile-first against heaviest
-        // first: 512 CTAs 469 / 552, 1024 CTAs 658-664 / 661-689, 2048 CTAs 575-766 / 529-732,
-        // 4096 CTAs 761-765 / 676-677); with 4-way grouping the heaviest-first order is faster
-        // (785 against 767). Anchor keys keep the heaviest-first order: the tile holding them is
-        // walked by every query tile, and started late it becomes the tail (window of 1024 + 4
-        // anchors, Hq = Hkv = 32: 487 against 460 TFLOP/s; the plain window: 585 either way).
+        // One CTA per (sequence, KV head, key tile), in the order bwd_key_tile_fastest picks.
         const long long n_ctas = static_cast<long long>(nkt) * Hkv * nseq;
         const int sms = sm_count();
         if (sms <= 0) return FA_ERR_CUDA;
-        a.kt_fast = (causal && d == 128 && Hq == Hkv && n_anchor == 0 && n_ctas >= 12LL * sms) ? 1 : 0;
+        a.kt_fast = fa::bwd_key_tile_fastest(causal, d, Hq, Hkv, n_anchor, n_ctas, sms) ? 1 : 0;
         const dim3 grid = (causal && !a.kt_fast) ? dim3(Hkv, nseq, nkt) : dim3(nkt, Hkv, nseq);
         const bool timed = g_bwd_ev_before && g_bwd_ev_after;
         if (timed && cudaEventRecord(g_bwd_ev_before, s) != cudaSuccess) return FA_ERR_CUDA;
